@@ -1,0 +1,381 @@
+"""GDLA forward oracle: a plain, slow, float64 CPU statement of the layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or execute this
+module; only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` / reference leg
+of ``bench.py`` use it.  It shares no code with the CUDA path (it does not import the
+``differential_latent_attention_fwd_b200`` package; callers hand it plain arrays).
+
+Source of every step: "Motif 3: Technical Report", picx.dev summary page, section 2.2
+"Grouped Differential Latent Attention (GDLA)" (equations for c^Q, [q^C; q^R], [c^KV; k^R],
+the normalised latent, [K^C; V], the head split n_N = n_H/(g+1), lambda_t, D_t, G_t and the
+gated output), plus the paperglide.net page ("Model Architecture" worked example and the
+Figure 1 caption: one lambda per signal head, gate from the normalised query latent, one
+rotary key shared by all KV heads, 16 KV heads shared by the signal and noise paths).
+
+Every floating-point step is float64.  Matrix products use numpy's BLAS (a library
+primitive); there is no blocking, fusion or reordering beyond the equations, except the
+weight-absorbed decode route, which is a second, independent statement of the same algebra
+and is checked against the literal one.
+
+Readings where the pages are silent (each also listed in the design notes):
+  * weights are [in, out] (the pages write x W);
+  * [q^C; q^R]: the first n_H*d_nope columns are q^C (head-major), the rest q^R (head-major);
+  * [c^KV; k^R]: the first kv_rank columns are c^KV, the last d_rope are k^R;
+  * Reshape_heads(c W_b^KV): head j owns columns j*(d_nope+d_v) ..., K^C first then V;
+  * heads 0..n_S-1 are the signal heads, n_S..n_H-1 the noise heads; signal head s reads
+    KV head s // (n_S/n_KV), noise head n reads KV head n // (n_N/n_KV);
+  * Repeat_g pairs signal head s with noise head s // g ("grouped"); the paperglide worked
+    example lists the noise outputs tiled (s mod n_N), available as noise_map="tiled";
+  * softmax scale 1/sqrt(d_nope + d_rope); RMSNorm eps 1e-6 with a gain vector;
+  * RoPE: rotate-half on the d_rope part, pairs (i, i + d_rope/2), angle pos * theta^(-2i/d_rope),
+    theta 10000, pos = 0-based token index (decode: the number of cached keys);
+  * masks: causal s <= t; sliding window t - W < s <= t (W keys, self included);
+  * no biases, no per-head normalisation after the subtraction; vec() is head-major.
+
+Parity: every function here is pinned by tests/test_oracle_pins.py (worked example, closed
+forms, library routines, invariants, brute force) except where a docstring says otherwise.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+
+# --------------------------------------------------------------------------------------
+# configuration
+# --------------------------------------------------------------------------------------
+@dataclass(frozen=True)
+class OracleConfig:
+    d_model: int
+    q_rank: int
+    kv_rank: int
+    n_signal: int
+    n_noise: int
+    n_kv_heads: int
+    d_nope: int
+    d_rope: int
+    d_v: int
+    window: int = 0
+    rope_theta: float = 10000.0
+    rms_eps: float = 1e-6
+    noise_map: str = "grouped"      # Repeat_g order: "grouped" (s // g) or "tiled" (s % n_N)
+
+    @property
+    def n_heads(self) -> int:
+        return self.n_signal + self.n_noise
+
+    @property
+    def g(self) -> int:
+        """Grouped ratio: n_N = n_H / (g + 1), n_S = g n_N (picx.dev page, section 2.2)."""
+        assert self.n_heads % (self.n_noise) == 0
+        g = self.n_heads // self.n_noise - 1
+        assert self.n_signal == g * self.n_noise
+        return g
+
+    @staticmethod
+    def from_shape(s, noise_map: str = "grouped") -> "OracleConfig":
+        """Build from any object with the same attribute names (e.g. synth.GdlaShape)."""
+        return OracleConfig(s.d_model, s.q_rank, s.kv_rank, s.n_signal, s.n_noise, s.n_kv_heads,
+                            s.d_nope, s.d_rope, s.d_v, s.window, s.rope_theta, s.rms_eps,
+                            noise_map)
+
+
+def f64(a) -> np.ndarray:
+    """Exact upcast of a torch tensor (any dtype, incl. bf16) or array-like to float64."""
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu")
+        import torch  # local: the oracle needs torch only to read tensors it is handed
+        return a.to(torch.float64).numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------------------
+# element-wise building blocks
+# --------------------------------------------------------------------------------------
+def rms_norm(v: np.ndarray, gain: np.ndarray | None, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis: v / sqrt(mean(v^2) + eps) * gain."""
+    r = v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
+    return r if gain is None else r * gain
+
+
+def rope(v: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half rotary embedding of the decoupled rope part (last axis, even length).
+
+    Pair (i, i + d/2) is rotated by angle pos * theta^(-2i/d).  ``pos`` broadcasts against
+    ``v[..., 0]``.
+    """
+    d = v.shape[-1]
+    half = d // 2
+    inv_freq = theta ** (-2.0 * np.arange(half, dtype=np.float64) / d)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * inv_freq
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = v[..., :half], v[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def sigmoid(z: np.ndarray) -> np.ndarray:
+    """Logistic function, evaluated without overflow for either sign."""
+    z = np.asarray(z, dtype=np.float64)
+    e = np.exp(-np.abs(z))
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+# --------------------------------------------------------------------------------------
+# head bookkeeping
+# --------------------------------------------------------------------------------------
+def kv_head_of(cfg: OracleConfig) -> np.ndarray:
+    """KV head read by each of the n_H query heads (signal heads first, then noise heads)."""
+    assert cfg.n_signal % cfg.n_kv_heads == 0 and cfg.n_noise % cfg.n_kv_heads == 0
+    sig = np.arange(cfg.n_signal) // (cfg.n_signal // cfg.n_kv_heads)
+    noi = np.arange(cfg.n_noise) // (cfg.n_noise // cfg.n_kv_heads)
+    return np.concatenate([sig, noi])
+
+
+def noise_of_signal(cfg: OracleConfig) -> np.ndarray:
+    """Repeat_g: the noise head whose output signal head s subtracts."""
+    s = np.arange(cfg.n_signal)
+    if cfg.noise_map == "grouped":
+        return s // cfg.g
+    if cfg.noise_map == "tiled":
+        return s % cfg.n_noise
+    raise ValueError(cfg.noise_map)
+
+
+def key_range(t: int, window: int) -> tuple[int, int]:
+    """Keys visible to query position t: [lo, t] (causal, or the last ``window`` keys)."""
+    lo = 0 if window <= 0 else max(0, t - window + 1)
+    return lo, t
+
+
+# --------------------------------------------------------------------------------------
+# projections (picx.dev page, section 2.2, first five equations)
+# --------------------------------------------------------------------------------------
+def query_path(x: np.ndarray, W_aQ, W_bQ, g_q, pos, cfg: OracleConfig):
+    """c^Q = RMSNorm(x W_aQ); [q^C; q^R] = c^Q W_bQ; RoPE on q^R.
+
+    x: [N, d].  Returns (c^Q [N, r_q], q^C [N, n_H, d_nope], rotated q^R [N, n_H, d_rope]).
+    """
+    cQ = rms_norm(x @ W_aQ, g_q, cfg.rms_eps)
+    qq = cQ @ W_bQ
+    nc = cfg.n_heads * cfg.d_nope
+    qC = qq[:, :nc].reshape(-1, cfg.n_heads, cfg.d_nope)
+    qR = qq[:, nc:].reshape(-1, cfg.n_heads, cfg.d_rope)
+    qR = rope(qR, np.asarray(pos)[:, None], cfg.rope_theta)
+    return cQ, qC, qR
+
+
+def kv_latent(x: np.ndarray, W_aKV, g_kv, pos, cfg: OracleConfig):
+    """[c^KV; k^R] = x W_aKV; normalised latent = RMSNorm(c^KV); RoPE on k^R (not normalised).
+
+    Returns (c_bar [N, kv_rank], rotated k^R [N, d_rope]); together they are one latent-cache row.
+    """
+    ck = x @ W_aKV
+    cbar = rms_norm(ck[:, : cfg.kv_rank], g_kv, cfg.rms_eps)
+    kR = rope(ck[:, cfg.kv_rank:], np.asarray(pos), cfg.rope_theta)
+    return cbar, kR
+
+
+def kv_heads(cbar: np.ndarray, W_bKV, cfg: OracleConfig):
+    """[K^C; V] = Reshape_heads(c_bar W_bKV) -> K^C [N, n_KV, d_nope], V [N, n_KV, d_v]."""
+    kv = (cbar @ W_bKV).reshape(-1, cfg.n_kv_heads, cfg.d_nope + cfg.d_v)
+    return kv[..., : cfg.d_nope], kv[..., cfg.d_nope:]
+
+
+def lambda_coeff(x: np.ndarray, W_lambda) -> np.ndarray:
+    """lambda_t = sigmoid(x_t W^lambda), one value per signal head."""
+    return sigmoid(x @ W_lambda)
+
+
+def gate_logits(cQ: np.ndarray, W_G, cfg: OracleConfig) -> np.ndarray:
+    """G_t = Reshape_heads(c^Q_t W^G) -> [N, n_S, d_v] (the sigmoid is applied in the combine)."""
+    return (cQ @ W_G).reshape(-1, cfg.n_signal, cfg.d_v)
+
+
+# --------------------------------------------------------------------------------------
+# attention, combine, output
+# --------------------------------------------------------------------------------------
+def softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
+    """Textbook softmax attention of a few queries over one key set.
+
+    q [h, dk], k [S, dk], v [S, dv] -> [h, dv] = softmax(q k^T * scale) v.
+    """
+    s = (q @ k.T) * scale
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=-1, keepdims=True)
+    return p @ v
+
+
+def differential_combine(H_S: np.ndarray, H_N: np.ndarray, lam: np.ndarray,
+                         gate: np.ndarray, noise_map: np.ndarray, gate_is_logit: bool = True):
+    """D = H_S - lambda (.) Repeat_g(H_N); returns (D, sigmoid(G) (.) D).
+
+    H_S [n_S, dv], H_N [n_N, dv], lam [n_S], gate [n_S, dv] (logits G, or already-sigmoided
+    values when ``gate_is_logit`` is False), noise_map [n_S] = noise head of each signal head.
+    """
+    D = H_S - lam[:, None] * H_N[noise_map]
+    sg = sigmoid(gate) if gate_is_logit else gate
+    return D, sg * D
+
+
+def attend_row(qC_t, qR_t, KC, kR, V, lo: int, hi: int, cfg: OracleConfig) -> np.ndarray:
+    """Per-head attention outputs H [n_H, d_v] of one query over keys lo..hi (inclusive).
+
+    q_h = [q^C_h; q^R_h], k_{j,s} = [K^C_{j,s}; k^R_s] (one rotary key for all KV heads).
+    """
+    scale = 1.0 / np.sqrt(cfg.d_nope + cfg.d_rope)
+    kvh = kv_head_of(cfg)
+    H = np.empty((cfg.n_heads, cfg.d_v))
+    kR_keys = kR[lo: hi + 1]
+    for j in range(cfg.n_kv_heads):
+        heads = np.nonzero(kvh == j)[0]
+        q = np.concatenate([qC_t[heads], qR_t[heads]], axis=-1)
+        k = np.concatenate([KC[lo: hi + 1, j], kR_keys], axis=-1)
+        H[heads] = softmax_attention(q, k, V[lo: hi + 1, j], scale)
+    return H
+
+
+def combine_row(H: np.ndarray, lam_t: np.ndarray, G_t: np.ndarray, W_O, cfg: OracleConfig):
+    """Differential combine + sigmoid gate + output projection of one token: returns (Dg, y)."""
+    _, Dg = differential_combine(H[: cfg.n_signal], H[cfg.n_signal:], lam_t, G_t,
+                                 noise_of_signal(cfg))
+    return Dg, Dg.reshape(-1) @ W_O
+
+
+# --------------------------------------------------------------------------------------
+# full layer: prefill
+# --------------------------------------------------------------------------------------
+def _weights64(w: dict) -> dict:
+    return {k: f64(v) for k, v in w.items()}
+
+
+def gdla_prefill(x, weights: dict, cfg: OracleConfig, rows=None, g_q=None, g_kv=None,
+                 pos_offset: int = 0, return_parts: bool = False, chunk: int = 8192):
+    """GDLA(x_t) for every sequence of a batch, at the requested query rows.
+
+    x [B, T, d]; ``rows`` = list of query positions (default: all).  Position of token t is
+    pos_offset + t.  Returns y [B, len(rows), d] (and a dict of per-row intermediates when
+    ``return_parts``: c^Q, q^C, q^R, lambda, G, Dg and, for all tokens, the latent cache rows).
+    """
+    W = _weights64(weights)
+    gq = None if g_q is None else f64(g_q)
+    gkv = None if g_kv is None else f64(g_kv)
+    B, T, _ = x.shape
+    rows = list(range(T)) if rows is None else [int(r) for r in rows]
+    t_hi = max(rows) + 1
+    ys, parts = [], []
+    for b in range(B):
+        # latent rows (c_bar, k^R) of every token a requested query can see
+        cbar = np.empty((t_hi, cfg.kv_rank))
+        kR = np.empty((t_hi, cfg.d_rope))
+        for c0 in range(0, t_hi, chunk):
+            c1 = min(t_hi, c0 + chunk)
+            xb = f64(x[b, c0:c1])
+            cbar[c0:c1], kR[c0:c1] = kv_latent(xb, W["W_aKV"], gkv,
+                                               pos_offset + np.arange(c0, c1), cfg)
+        KC, V = kv_heads(cbar, W["W_bKV"], cfg)
+        xr = f64(x[b, rows])
+        pos_r = pos_offset + np.asarray(rows)
+        cQ, qC, qR = query_path(xr, W["W_aQ"], W["W_bQ"], gq, pos_r, cfg)
+        lam = lambda_coeff(xr, W["W_lambda"])
+        G = gate_logits(cQ, W["W_G"], cfg)
+        y = np.empty((len(rows), cfg.d_model))
+        Dg_all = np.empty((len(rows), cfg.n_signal, cfg.d_v))
+        for i, t in enumerate(rows):
+            lo, hi = key_range(t, cfg.window)
+            H = attend_row(qC[i], qR[i], KC, kR, V, lo, hi, cfg)
+            Dg_all[i], y[i] = combine_row(H, lam[i], G[i], W["W_O"], cfg)
+        ys.append(y)
+        if return_parts:
+            parts.append(dict(cQ=cQ, qC=qC, qR=qR, lam=lam, G=G, Dg=Dg_all,
+                              cbar=cbar, kR=kR, KC=KC, V=V))
+    y = np.stack(ys)
+    return (y, parts) if return_parts else y
+
+
+# --------------------------------------------------------------------------------------
+# full layer: decode (one new token per sequence, keys = cached latent rows + itself)
+# --------------------------------------------------------------------------------------
+def _decode_common(x_new, weights, cache, cache_len, cfg, g_q, g_kv):
+    W = _weights64(weights)
+    gq = None if g_q is None else f64(g_q)
+    gkv = None if g_kv is None else f64(g_kv)
+    xn = f64(x_new)
+    lens = [int(v) for v in (cache_len.tolist() if hasattr(cache_len, "tolist") else cache_len)]
+    pos = np.asarray(lens)
+    cQ, qC, qR = query_path(xn, W["W_aQ"], W["W_bQ"], gq, pos, cfg)
+    cbar_new, kR_new = kv_latent(xn, W["W_aKV"], gkv, pos, cfg)
+    lam = lambda_coeff(xn, W["W_lambda"])
+    G = gate_logits(cQ, W["W_G"], cfg)
+    return W, lens, cQ, qC, qR, cbar_new, kR_new, lam, G
+
+
+def _keys_of(cache, b, p, cbar_new, kR_new, cfg):
+    """Latent rows 0..p of sequence b: the p cached rows followed by the new token's row."""
+    rows = f64(cache[b, :p]) if p else np.zeros((0, cfg.kv_rank + cfg.d_rope))
+    cbar = np.concatenate([rows[:, : cfg.kv_rank], cbar_new[b][None]], axis=0)
+    kR = np.concatenate([rows[:, cfg.kv_rank:], kR_new[b][None]], axis=0)
+    return cbar, kR
+
+
+def gdla_decode(x_new, weights: dict, cache, cache_len, cfg: OracleConfig, g_q=None, g_kv=None,
+                return_parts: bool = False):
+    """Literal decode: the prefill definition applied to the new token at position cache_len[b].
+
+    cache [B, cap, kv_rank + d_rope] holds (normalised c^KV | rotated k^R) per cached token.
+    K^C and V are re-expanded from the latent rows with W_bKV exactly as in prefill.
+    Returns y [B, d] (and the new latent rows when ``return_parts``).
+    """
+    W, lens, cQ, qC, qR, cbar_new, kR_new, lam, G = _decode_common(
+        x_new, weights, cache, cache_len, cfg, g_q, g_kv)
+    y = np.empty((len(lens), cfg.d_model))
+    Dgs = []
+    for b, p in enumerate(lens):
+        cbar, kR = _keys_of(cache, b, p, cbar_new, kR_new, cfg)
+        KC, V = kv_heads(cbar, W["W_bKV"], cfg)
+        lo, hi = key_range(p, cfg.window)
+        H = attend_row(qC[b], qR[b], KC, kR, V, lo, hi, cfg)
+        Dg, y[b] = combine_row(H, lam[b], G[b], W["W_O"], cfg)
+        Dgs.append(Dg)
+    if return_parts:
+        return y, dict(cbar_new=cbar_new, kR_new=kR_new, Dg=np.stack(Dgs), lam=lam, G=G)
+    return y
+
+
+def gdla_decode_absorbed(x_new, weights: dict, cache, cache_len, cfg: OracleConfig, g_q=None,
+                         g_kv=None):
+    """Weight-absorbed decode: attention runs in the latent space, K^C and V are never formed.
+
+    With W_UK_j / W_UV_j the K^C / V column blocks of W_bKV for KV head j:
+      score_{h,s} = (W_UK_j q^C_h) . c_bar_s + q^R_h . k^R_s            (q^C_h . K^C_{j,s} regrouped)
+      l_h        = sum_s p_{h,s} c_bar_s                               (latent attention output)
+      D_s        = (l_s - lambda_s l_{n(s)}) W_UV_j                    (H = l W_UV, linear in l)
+    Same result as ``gdla_decode`` up to rounding order; used for sizes where re-expanding
+    every cached row is too slow.
+    """
+    W, lens, cQ, qC, qR, cbar_new, kR_new, lam, G = _decode_common(
+        x_new, weights, cache, cache_len, cfg, g_q, g_kv)
+    scale = 1.0 / np.sqrt(cfg.d_nope + cfg.d_rope)
+    kvh = kv_head_of(cfg)
+    nmap = noise_of_signal(cfg)
+    blk = cfg.d_nope + cfg.d_v
+    W_UK = [W["W_bKV"][:, j * blk: j * blk + cfg.d_nope] for j in range(cfg.n_kv_heads)]
+    W_UV = [W["W_bKV"][:, j * blk + cfg.d_nope: (j + 1) * blk] for j in range(cfg.n_kv_heads)]
+    y = np.empty((len(lens), cfg.d_model))
+    for b, p in enumerate(lens):
+        cbar, kR = _keys_of(cache, b, p, cbar_new, kR_new, cfg)
+        lo, hi = key_range(p, cfg.window)
+        cbar, kR = cbar[lo: hi + 1], kR[lo: hi + 1]
+        qt = np.stack([W_UK[kvh[h]] @ qC[b, h] for h in range(cfg.n_heads)])   # [n_H, kv_rank]
+        s = (qt @ cbar.T + qR[b] @ kR.T) * scale
+        s = s - s.max(axis=-1, keepdims=True)
+        pr = np.exp(s)
+        pr = pr / pr.sum(axis=-1, keepdims=True)
+        lat = pr @ cbar                                                          # [n_H, kv_rank]
+        lat_S, lat_N = lat[: cfg.n_signal], lat[cfg.n_signal:]
+        Dlat = lat_S - lam[b][:, None] * lat_N[nmap]
+        D = np.stack([Dlat[s_] @ W_UV[kvh[s_]] for s_ in range(cfg.n_signal)])
+        Dg = sigmoid(G[b]) * D
+        y[b] = Dg.reshape(-1) @ W["W_O"]
+    return y
