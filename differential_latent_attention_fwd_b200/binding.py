@@ -1,0 +1,198 @@
+"""ctypes binding of libgdla.so (include/gdla.h): argument marshalling only.
+
+Every function here has the name of the C entry point it wraps, takes torch tensors (device
+memory owned by the caller) or plain integers, checks dtype/device/contiguity, and forwards raw
+pointers.  All arithmetic happens in the CUDA kernels behind the C ABI; if the library is
+missing this module raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgdla.so")
+HEADER = os.path.join(HERE, "..", "include", "gdla.h")
+
+GDLA_MODE_PREFILL = 0
+GDLA_MODE_DECODE = 1
+STATUS = {0: "GDLA_OK", -1: "GDLA_ERR_INVALID_ARG", -2: "GDLA_ERR_UNSUPPORTED_SHAPE",
+          -3: "GDLA_ERR_WORKSPACE_TOO_SMALL", -4: "GDLA_ERR_LAUNCH",
+          -5: "GDLA_ERR_DEVICE_TIMEOUT", -6: "GDLA_ERR_CUDA"}
+
+
+class GdlaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} -> {status} ({STATUS.get(status, '?')})")
+        self.status = status
+
+
+class gdla_config_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("d_model", "q_rank", "kv_rank", "n_signal", "n_noise",
+                                             "n_kv_heads", "d_nope", "d_rope", "d_v", "window")] + \
+               [("rope_theta", ctypes.c_float), ("rms_eps", ctypes.c_float)]
+
+
+class gdla_weights_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W_aQ", "W_bQ", "W_aKV", "W_bKV", "W_lambda", "W_G",
+                                                "W_O", "g_q", "g_kv")]
+
+
+class gdla_absorbed_t(ctypes.Structure):
+    _fields_ = [("w", gdla_weights_t), ("W_UKt", ctypes.c_void_p), ("cfg", gdla_config_t),
+                ("magic", ctypes.c_uint32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdla.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m differential_latent_attention_fwd_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, SZ, ULL = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_ulonglong
+        cfgp, wp, abp = (ctypes.POINTER(gdla_config_t), ctypes.POINTER(gdla_weights_t),
+                         ctypes.POINTER(gdla_absorbed_t))
+        sig = {
+            "gdla_workspace_size": [cfgp, I, I, I, ctypes.POINTER(SZ)],
+            "gdla_absorbed_size": [cfgp, ctypes.POINTER(SZ)],
+            "gdla_prefill_fwd": [cfgp, wp, P, I, I, P, P, I, P, SZ, P],
+            "gdla_absorb_weights": [cfgp, wp, P, SZ, abp, P],
+            "gdla_decode_fwd": [cfgp, abp, P, P, P, I, I, P, P, SZ, P],
+            "gdla_device_error": [P, ctypes.POINTER(I), I],
+            "gdla_set_wait_limit_ns": [ULL],
+            "gdla_selftest_wait_timeout": [ULL, P, ctypes.POINTER(I)],
+            "gdla_workspace_offset": [cfgp, I, I, I, I, ctypes.POINTER(SZ)],
+            "gdla_status_string": [I],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_char_p if name == "gdla_status_string" else I
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the entry points declared in include/gdla.h."""
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(gdla_\w+)\s*\(", src, re.M)))
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise GdlaError(fn, rc)
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def make_config(shape) -> gdla_config_t:
+    """gdla_config_t from any object with the GdlaShape attribute names."""
+    return gdla_config_t(shape.d_model, shape.q_rank, shape.kv_rank, shape.n_signal, shape.n_noise,
+                         shape.n_kv_heads, shape.d_nope, shape.d_rope, shape.d_v, shape.window,
+                         float(shape.rope_theta), float(shape.rms_eps))
+
+
+def make_weights(w: dict, g_q=None, g_kv=None) -> gdla_weights_t:
+    names = ("W_aQ", "W_bQ", "W_aKV", "W_bKV", "W_lambda", "W_G", "W_O")
+    ptrs = [_ptr(w[n], torch.bfloat16, n) for n in names]
+    return gdla_weights_t(*ptrs, _ptr(g_q, torch.bfloat16, "g_q"), _ptr(g_kv, torch.bfloat16, "g_kv"))
+
+
+# ----------------------------------------------------------------------------- entry points
+def gdla_status_string(status: int) -> str:
+    return lib().gdla_status_string(status).decode()
+
+
+def gdla_workspace_size(cfg: gdla_config_t, B: int, T: int, mode: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check("gdla_workspace_size", lib().gdla_workspace_size(ctypes.byref(cfg), B, T, mode,
+                                                            ctypes.byref(out)))
+    return out.value
+
+
+def gdla_workspace_offset(cfg: gdla_config_t, B: int, T: int, mode: int, which: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check("gdla_workspace_offset", lib().gdla_workspace_offset(ctypes.byref(cfg), B, T, mode, which,
+                                                                ctypes.byref(out)))
+    return out.value
+
+
+def gdla_absorbed_size(cfg: gdla_config_t) -> int:
+    out = ctypes.c_size_t(0)
+    _check("gdla_absorbed_size", lib().gdla_absorbed_size(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def gdla_prefill_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, y: torch.Tensor,
+                     workspace: torch.Tensor, kv_cache_out: torch.Tensor | None = None,
+                     cache_cap: int = 0, stream=None) -> None:
+    B, T, _ = x.shape
+    _check("gdla_prefill_fwd", lib().gdla_prefill_fwd(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(x, torch.bfloat16, "x"), B, T,
+        _ptr(y, torch.bfloat16, "y"), _ptr(kv_cache_out, torch.bfloat16, "kv_cache_out"),
+        int(cache_cap), _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def gdla_absorb_weights(cfg, w: gdla_weights_t, dst: torch.Tensor, stream=None) -> gdla_absorbed_t:
+    out = gdla_absorbed_t()
+    _check("gdla_absorb_weights", lib().gdla_absorb_weights(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(dst, None, "dst"), dst.numel() * dst.element_size(),
+        ctypes.byref(out), _stream(stream)))
+    return out
+
+
+def gdla_decode_fwd(cfg, absorbed: gdla_absorbed_t, x_new: torch.Tensor, kv_cache: torch.Tensor,
+                    cache_len: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor,
+                    stream=None) -> None:
+    B = x_new.shape[0]
+    cap = kv_cache.shape[1]
+    _check("gdla_decode_fwd", lib().gdla_decode_fwd(
+        ctypes.byref(cfg), ctypes.byref(absorbed), _ptr(x_new, torch.bfloat16, "x_new"),
+        _ptr(kv_cache, torch.bfloat16, "kv_cache"), _ptr(cache_len, torch.int32, "cache_len"), cap, B,
+        _ptr(y, torch.bfloat16, "y"), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gdla_device_error(stream=None, clear: bool = True) -> int:
+    site = ctypes.c_int(0)
+    rc = lib().gdla_device_error(_stream(stream), ctypes.byref(site), int(clear))
+    if rc not in (0, -5):
+        _check("gdla_device_error", rc)
+    return site.value
+
+
+def gdla_set_wait_limit_ns(ns: int) -> None:
+    _check("gdla_set_wait_limit_ns", lib().gdla_set_wait_limit_ns(int(ns)))
+
+
+def gdla_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    site = ctypes.c_int(0)
+    rc = lib().gdla_selftest_wait_timeout(int(limit_ns), _stream(stream), ctypes.byref(site))
+    if rc not in (0, -5):
+        _check("gdla_selftest_wait_timeout", rc)
+    return site.value

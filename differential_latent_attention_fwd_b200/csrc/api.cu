@@ -1,0 +1,397 @@
+// C ABI of the GDLA forward pass: argument validation, workspace carving and the launch
+// sequence of the prefill and absorbed-decode paths (declared in include/gdla.h).
+#include "../../include/gdla.h"
+#include "gdla_common.cuh"
+#include "gdla_decode.h"
+#include "gdla_internal.h"
+
+#include <math.h>
+#include <string.h>
+
+namespace gdla {
+
+// Device error word written by bounded waits (one instance per device that loads the library).
+__device__ int g_device_error = 0;
+
+static unsigned long long g_wait_limit_ns = 2000000000ull;
+static const uint32_t kAbsorbedMagic = 0x47444C41u;  // "GDLA"
+
+static int error_word(int** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return GDLA_ERR_CUDA;
+  *out = static_cast<int*>(p);
+  return GDLA_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_config(const gdla_config_t* c) {
+  if (!c) return GDLA_ERR_INVALID_ARG;
+  if (c->d_nope != 128 || c->d_rope != 64 || c->d_v != 128) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  if (c->q_rank != 1024 || c->kv_rank != 512) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  if (c->n_noise <= 0 || c->n_signal != 4 * c->n_noise || c->n_kv_heads != c->n_noise)
+    return GDLA_ERR_UNSUPPORTED_SHAPE;
+  if (c->n_noise > 16) return GDLA_ERR_UNSUPPORTED_SHAPE;  // decode keeps 80 heads per CTA
+  if (c->d_model <= 0 || c->d_model % 64 != 0) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  if (c->window < 0 || !(c->rope_theta > 0.f) || !(c->rms_eps >= 0.f)) return GDLA_ERR_INVALID_ARG;
+  return GDLA_OK;
+}
+
+static int check_weights(const gdla_weights_t* w) {
+  if (!w || !w->W_aQ || !w->W_bQ || !w->W_aKV || !w->W_bKV || !w->W_lambda || !w->W_G || !w->W_O)
+    return GDLA_ERR_INVALID_ARG;
+  const void* ps[] = {w->W_aQ, w->W_bQ, w->W_aKV, w->W_bKV, w->W_lambda, w->W_G, w->W_O};
+  for (const void* p : ps)
+    if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
+  if ((w->g_q && !aligned16(w->g_q)) || (w->g_kv && !aligned16(w->g_kv))) return GDLA_ERR_INVALID_ARG;
+  return GDLA_OK;
+}
+
+// ---------------------------------------------------------------- workspace layout
+enum { WS_D1, WS_CQ, WS_LATENT, WS_LAM, WS_QQ, WS_G, WS_KV, WS_ONOISE, WS_DG, WS_KR16, WS_N };
+
+static int decode_splits(int B) {
+  int s = (2 * 148 + B - 1) / B;
+  return s < 1 ? 1 : (s > 64 ? 64 : s);
+}
+
+static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS_N + 1]) {
+  const long long M = mode == GDLA_MODE_PREFILL ? (long long)B * T : (long long)B;
+  const int nH = c->n_signal + c->n_noise;
+  const long long qq = (long long)nH * (c->d_nope + c->d_rope);
+  const long long d1 = c->q_rank + c->kv_rank + c->d_rope + c->n_signal;
+  size_t sz[WS_N];
+  sz[WS_D1] = M * d1 * 4;
+  sz[WS_CQ] = M * c->q_rank * 2;
+  sz[WS_LAM] = M * c->n_signal * 4;
+  sz[WS_G] = M * (long long)c->n_signal * c->d_v * 2;
+  sz[WS_DG] = M * (long long)c->n_signal * c->d_v * 2;
+  if (mode == GDLA_MODE_PREFILL) {
+    sz[WS_LATENT] = M * (c->kv_rank + c->d_rope) * 2;
+    sz[WS_QQ] = M * qq * 2;
+    sz[WS_KV] = M * (long long)c->n_kv_heads * (c->d_nope + c->d_v) * 2;
+    sz[WS_ONOISE] = M * (long long)c->n_noise * c->d_v * 4;
+    sz[WS_KR16] = M * c->d_rope * 2;
+  } else {
+    const int ns = decode_splits(B);
+    sz[WS_LATENT] = 0;
+    sz[WS_QQ] = M * qq * 4;                                          // fp32 q^C | q^R
+    sz[WS_KV] = M * (long long)nH * (c->kv_rank + c->d_rope) * 2;    // q~ rows
+    sz[WS_ONOISE] = M * (long long)ns * nH * c->kv_rank * 4;         // split partials
+    sz[WS_KR16] = M * (long long)ns * nH * 2 * 4;                    // split (max, sum)
+  }
+  size_t o = 0;
+  for (int i = 0; i < WS_N; ++i) {
+    off[i] = o;
+    o += (sz[i] + 255) & ~size_t(255);
+  }
+  off[WS_N] = o;
+}
+
+}  // namespace gdla
+
+using namespace gdla;
+
+extern "C" {
+
+const char* gdla_status_string(int s) {
+  switch (s) {
+    case GDLA_OK: return "ok";
+    case GDLA_ERR_INVALID_ARG: return "invalid argument";
+    case GDLA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case GDLA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case GDLA_ERR_LAUNCH: return "kernel launch failed";
+    case GDLA_ERR_DEVICE_TIMEOUT: return "bounded in-kernel wait expired";
+    case GDLA_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+int gdla_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_limit_ns = ns < 1000ull ? 1000ull : ns;
+  return GDLA_OK;
+}
+
+int gdla_workspace_size(const gdla_config_t* cfg, int B, int T, int mode, size_t* bytes) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!bytes || B <= 0 || (mode == GDLA_MODE_PREFILL && T <= 0) ||
+      (mode != GDLA_MODE_PREFILL && mode != GDLA_MODE_DECODE))
+    return GDLA_ERR_INVALID_ARG;
+  size_t off[WS_N + 1];
+  layout(cfg, B, T, mode, off);
+  *bytes = off[WS_N];
+  return GDLA_OK;
+}
+
+int gdla_workspace_offset(const gdla_config_t* cfg, int B, int T, int mode, int which,
+                          size_t* offset) {
+  size_t total;
+  int rc = gdla_workspace_size(cfg, B, T, mode, &total);
+  if (rc) return rc;
+  if (!offset || which < 0 || which >= WS_N) return GDLA_ERR_INVALID_ARG;
+  size_t off[WS_N + 1];
+  layout(cfg, B, T, mode, off);
+  *offset = off[which];
+  return GDLA_OK;
+}
+
+int gdla_absorbed_size(const gdla_config_t* cfg, size_t* bytes) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!bytes) return GDLA_ERR_INVALID_ARG;
+  *bytes = (size_t)cfg->n_kv_heads * cfg->d_nope * cfg->kv_rank * 2;
+  return GDLA_OK;
+}
+
+int gdla_prefill_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int B,
+                     int T, void* y, void* kv_cache_out, int cache_cap, void* workspace,
+                     size_t ws_bytes, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_weights(w))) return rc;
+  if (!x || !y || !workspace || B <= 0 || T <= 0) return GDLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(workspace)) return GDLA_ERR_INVALID_ARG;
+  if ((long long)B * T > (1ll << 30)) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  if (kv_cache_out && (cache_cap < T || !aligned16(kv_cache_out))) return GDLA_ERR_INVALID_ARG;
+  size_t off[WS_N + 1];
+  layout(cfg, B, T, GDLA_MODE_PREFILL, off);
+  if (ws_bytes < off[WS_N]) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* err;
+  if ((rc = error_word(&err))) return rc;
+  KernelCtlHost ctl{err, g_wait_limit_ns};
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* D1 = reinterpret_cast<float*>(ws + off[WS_D1]);
+  void* cQ = ws + off[WS_CQ];
+  void* latent = ws + off[WS_LATENT];
+  float* lam = reinterpret_cast<float*>(ws + off[WS_LAM]);
+  void* QQ = ws + off[WS_QQ];
+  void* G = ws + off[WS_G];
+  void* KV = ws + off[WS_KV];
+  float* On = reinterpret_cast<float*>(ws + off[WS_ONOISE]);
+  void* Dg = ws + off[WS_DG];
+  void* kR16 = ws + off[WS_KR16];
+  const int M = B * T;
+  const int nH = cfg->n_signal + cfg->n_noise;
+  const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
+  RopeTable rope;
+  fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
+
+  // a1: [x W_aQ | x W_aKV | x W_lambda] in fp32
+  GemmEpi ep{};
+  ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = M; ep.rope_lo = ep.rope_hi = 0; ep.pos_T = T;
+  ep.rope = rope;
+  ep.C = D1; ep.N = cfg->q_rank;
+  if (launch_gemm(x, cfg->d_model, w->W_aQ, cfg->q_rank, false, M, cfg->q_rank, cfg->d_model, ep, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  ep.C = D1 + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
+  if (launch_gemm(x, cfg->d_model, w->W_aKV, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  ep.C = D1 + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
+  if (launch_gemm(x, cfg->d_model, w->W_lambda, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st))
+    return GDLA_ERR_LAUNCH;
+
+  // a2: norms, rotary key, lambda, latent rows
+  NormParams np{};
+  np.D1 = D1; np.ld1 = ld1; np.M = M; np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank;
+  np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
+  np.cQ = cQ; np.latent = latent; np.kR16 = kR16; np.lam = lam; np.pos_T = T; np.pos_ptr = nullptr;
+  np.cache = kv_cache_out; np.cache_cap = cache_cap; np.rope = rope; np.err = err;
+  if (launch_norm_rope(np, st)) return GDLA_ERR_LAUNCH;
+
+  // a3: up-projections (q^C | rotated q^R), gate logits, K^C | V
+  const int nqq = nH * (cfg->d_nope + cfg->d_rope);
+  GemmEpi eq{};
+  eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F16; eq.M = M; eq.N = nqq;
+  eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = T; eq.rope = rope;
+  if (launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, M, nqq, cfg->q_rank, eq, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  GemmEpi eg{};
+  eg.C = G; eg.ldc = cfg->n_signal * cfg->d_v; eg.out_type = OUT_BF16; eg.M = M; eg.N = eg.ldc;
+  eg.pos_T = T;
+  if (launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, M, eg.N, cfg->q_rank, eg, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  GemmEpi ekv{};
+  const int nkv = cfg->n_kv_heads * (cfg->d_nope + cfg->d_v);
+  ekv.C = KV; ekv.ldc = nkv; ekv.out_type = OUT_F16; ekv.M = M; ekv.N = nkv; ekv.pos_T = T;
+  if (launch_gemm(latent, cfg->kv_rank + cfg->d_rope, w->W_bKV, nkv, false, M, nkv, cfg->kv_rank,
+                  ekv, ctl, st))
+    return GDLA_ERR_LAUNCH;
+
+  // a4: fused attention + differential combine + gate
+  AttnParams ap{};
+  ap.B = B; ap.T = T; ap.window = cfg->window; ap.n_groups = cfg->n_noise;
+  ap.n_signal = cfg->n_signal; ap.rope_col0 = nH * cfg->d_nope;
+  ap.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
+  ap.lam = lam; ap.G = G; ap.O_noise = On; ap.Dg = Dg;
+  if (launch_attn_prefill(QQ, nqq, KV, kR16, ap, ctl, st)) return GDLA_ERR_LAUNCH;
+
+  // a5: output projection
+  GemmEpi eo{};
+  eo.C = y; eo.ldc = cfg->d_model; eo.out_type = OUT_BF16; eo.M = M; eo.N = cfg->d_model;
+  eo.pos_T = T;
+  if (launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, M, cfg->d_model,
+                  cfg->n_signal * cfg->d_v, eo, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  return GDLA_OK;
+}
+
+int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void* dst,
+                        size_t dst_bytes, gdla_absorbed_t* out, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_weights(w))) return rc;
+  if (!dst || !out || !aligned16(dst)) return GDLA_ERR_INVALID_ARG;
+  size_t need;
+  gdla_absorbed_size(cfg, &need);
+  if (dst_bytes < need) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  if (launch_absorb_uk(w->W_bKV, dst, cfg->kv_rank, cfg->n_kv_heads, cfg->d_nope, cfg->d_v,
+                       static_cast<cudaStream_t>(stream)))
+    return GDLA_ERR_LAUNCH;
+  out->w = *w;
+  out->W_UKt = dst;
+  out->cfg = *cfg;
+  out->magic = kAbsorbedMagic;
+  return GDLA_OK;
+}
+
+int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const void* x_new,
+                    void* kv_cache, const int* cache_len, int cap, int B, void* y, void* workspace,
+                    size_t ws_bytes, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!ab || ab->magic != kAbsorbedMagic || !ab->W_UKt) return GDLA_ERR_INVALID_ARG;
+  if (ab->cfg.d_model != cfg->d_model || ab->cfg.n_noise != cfg->n_noise)
+    return GDLA_ERR_INVALID_ARG;  // absorbed for another layer shape (the window may differ)
+  const gdla_weights_t* w = &ab->w;
+  if ((rc = check_weights(w))) return rc;
+  if (!x_new || !kv_cache || !cache_len || !y || !workspace || B <= 0 || cap <= 0)
+    return GDLA_ERR_INVALID_ARG;
+  if (!aligned16(x_new) || !aligned16(kv_cache) || !aligned16(y) || !aligned16(workspace))
+    return GDLA_ERR_INVALID_ARG;
+  size_t off[WS_N + 1];
+  layout(cfg, B, 1, GDLA_MODE_DECODE, off);
+  if (ws_bytes < off[WS_N]) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* err;
+  if ((rc = error_word(&err))) return rc;
+  KernelCtlHost ctl{err, g_wait_limit_ns};
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* D1 = reinterpret_cast<float*>(ws + off[WS_D1]);
+  void* cQ = ws + off[WS_CQ];
+  float* lam = reinterpret_cast<float*>(ws + off[WS_LAM]);
+  float* QQ = reinterpret_cast<float*>(ws + off[WS_QQ]);
+  void* G = ws + off[WS_G];
+  void* qt = ws + off[WS_KV];
+  float* part = reinterpret_cast<float*>(ws + off[WS_ONOISE]);
+  float* ml = reinterpret_cast<float*>(ws + off[WS_KR16]);
+  void* Dg = ws + off[WS_DG];
+  const int nH = cfg->n_signal + cfg->n_noise;
+  const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
+  const int nsplit = decode_splits(B);
+  RopeTable rope;
+  fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
+
+  GemmEpi ep{};
+  ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = B; ep.pos_T = 1; ep.rope = rope;
+  ep.C = D1; ep.N = cfg->q_rank;
+  if (launch_gemm(x_new, cfg->d_model, w->W_aQ, cfg->q_rank, false, B, ep.N, cfg->d_model, ep, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  ep.C = D1 + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
+  if (launch_gemm(x_new, cfg->d_model, w->W_aKV, ep.N, false, B, ep.N, cfg->d_model, ep, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  ep.C = D1 + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
+  if (launch_gemm(x_new, cfg->d_model, w->W_lambda, ep.N, false, B, ep.N, cfg->d_model, ep, ctl, st))
+    return GDLA_ERR_LAUNCH;
+
+  NormParams np{};
+  np.D1 = D1; np.ld1 = ld1; np.M = B; np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank;
+  np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
+  np.cQ = cQ; np.latent = nullptr; np.kR16 = nullptr; np.lam = lam; np.pos_T = 1;
+  np.pos_ptr = cache_len; np.cache = kv_cache; np.cache_cap = cap; np.rope = rope; np.err = err;
+  if (launch_norm_rope(np, st)) return GDLA_ERR_LAUNCH;
+
+  const int nqq = nH * (cfg->d_nope + cfg->d_rope);
+  GemmEpi eq{};
+  eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F32; eq.M = B; eq.N = nqq;
+  eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = 1; eq.pos_ptr = cache_len;
+  eq.rope = rope;
+  if (launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, B, nqq, cfg->q_rank, eq, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  GemmEpi eg{};
+  eg.C = G; eg.ldc = cfg->n_signal * cfg->d_v; eg.out_type = OUT_BF16; eg.M = B; eg.N = eg.ldc;
+  eg.pos_T = 1;
+  if (launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, B, eg.N, cfg->q_rank, eg, ctl, st))
+    return GDLA_ERR_LAUNCH;
+
+  DecQParams qp{};
+  qp.B = B; qp.n_groups = cfg->n_noise; qp.n_signal = cfg->n_signal; qp.n_heads = nH;
+  qp.QQ = QQ; qp.qq_ld = nqq; qp.rope_col0 = nH * cfg->d_nope; qp.W_UKt = ab->W_UKt; qp.qt = qt;
+  if (launch_qtilde(qp, st)) return GDLA_ERR_LAUNCH;
+
+  DecAttnParams dp{};
+  dp.B = B; dp.cap = cap; dp.window = cfg->window; dp.n_split = nsplit; dp.cache_len = cache_len;
+  dp.cache = kv_cache; dp.qt = qt;
+  dp.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
+  dp.part = part; dp.ml = ml; dp.err = err;
+  if (nH != 80) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  if (launch_dec_attn_simt(dp, st)) return GDLA_ERR_LAUNCH;
+
+  DecCombParams cp{};
+  cp.B = B; cp.n_groups = cfg->n_noise; cp.n_signal = cfg->n_signal; cp.n_split = nsplit;
+  cp.part = part; cp.ml = ml; cp.lam = lam; cp.G = G; cp.W_bKV = w->W_bKV; cp.Dg = Dg;
+  if (launch_dec_combine(cp, st)) return GDLA_ERR_LAUNCH;
+
+  GemmEpi eo{};
+  eo.C = y; eo.ldc = cfg->d_model; eo.out_type = OUT_BF16; eo.M = B; eo.N = cfg->d_model;
+  eo.pos_T = 1;
+  if (launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, B, cfg->d_model,
+                  cfg->n_signal * cfg->d_v, eo, ctl, st))
+    return GDLA_ERR_LAUNCH;
+  return GDLA_OK;
+}
+
+int gdla_device_error(void* stream, int* site, int clear) {
+  if (!site) return GDLA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDLA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return GDLA_ERR_CUDA;
+  if (clear && v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return GDLA_ERR_CUDA;
+  }
+  *site = v;
+  return v ? GDLA_ERR_DEVICE_TIMEOUT : GDLA_OK;
+}
+
+}  // extern "C"
+
+namespace gdla {
+// One CTA waits on an mbarrier that nothing ever arrives on: the bounded wait must expire,
+// record its site code and return, and the kernel must then exit normally.
+__global__ void selftest_wait_kernel(KernelCtl ctl) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, ctl, SITE_SELFTEST);
+}
+}  // namespace gdla
+
+extern "C" int gdla_selftest_wait_timeout(unsigned long long limit_ns, void* stream, int* site) {
+  if (!site) return GDLA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* err;
+  int rc = error_word(&err);
+  if (rc) return rc;
+  KernelCtl kc{err, limit_ns < 1000ull ? 1000ull : limit_ns};
+  int prev = 0;
+  if (cudaMemcpyFromSymbol(&prev, g_device_error, sizeof(int)) != cudaSuccess) return GDLA_ERR_CUDA;
+  if (prev) return GDLA_ERR_DEVICE_TIMEOUT;  // an earlier failure is still unread
+  selftest_wait_kernel<<<1, 32, 0, st>>>(kc);
+  if (cudaPeekAtLastError() != cudaSuccess) return GDLA_ERR_LAUNCH;
+  return gdla_device_error(stream, site, 1);
+}

@@ -1,0 +1,43 @@
+// Host-side declarations of the absorbed-form decode kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace gdla {
+
+struct DecQParams {
+  int B, n_groups, n_signal, n_heads;
+  const float* QQ;        // [B, qq_ld] fp32: q^C (head-major) | rotated q^R (head-major)
+  int qq_ld, rope_col0;
+  const void* W_UKt;      // bf16 [n_groups][128][512]
+  void* qt;               // bf16 [B][n_heads][576]
+};
+
+struct DecAttnParams {
+  int B, cap, window, n_split;
+  const int* cache_len;   // [B] keys before the new token (its row sits at cache_len[b])
+  const void* cache;      // bf16 [B][cap][576]
+  const void* qt;         // bf16 [B][80][576]
+  float scale_log2;
+  float* part;            // [B][n_split][80][512] latent accumulators
+  float* ml;              // [B][n_split][80][2]  (running max in log2 units, row sum)
+  int* err;               // device error word
+};
+
+struct DecCombParams {
+  int B, n_groups, n_signal, n_split;
+  const float* part;
+  const float* ml;
+  const float* lam;       // [B][n_signal]
+  const void* G;          // bf16 [B][n_signal * 128]
+  const void* W_bKV;      // bf16 [kv_rank][n_groups * 256]
+  void* Dg;               // bf16 [B][n_signal * 128]
+};
+
+int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int d_nope, int d_v,
+                     cudaStream_t st);
+int launch_qtilde(const DecQParams& p, cudaStream_t st);
+int launch_dec_attn_simt(const DecAttnParams& p, cudaStream_t st);
+int launch_dec_combine(const DecCombParams& p, cudaStream_t st);
+
+}  // namespace gdla

@@ -1,0 +1,85 @@
+// Host-side declarations shared by the GDLA translation units (not part of the public ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdla {
+
+enum OutType : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_F16 = 2 };
+
+// Rotary-embedding frequency table, theta^(-2i/d_rope) for i < d_rope/2, in double.
+struct RopeTable {
+  double inv_freq[32];
+  int d_rope;
+};
+
+// Epilogue of the projection GEMM C[M, N] = A[M, K] B[K, N].
+struct GemmEpi {
+  void* C;               // output base (row-major, leading dimension ldc elements)
+  long long ldc;
+  int out_type;          // OutType
+  int M, N;
+  int rope_lo, rope_hi;  // columns [rope_lo, rope_hi) (multiples of 64) hold 64-wide rope heads
+  int pos_T;             // row position = row % pos_T (used when pos_ptr is null)
+  const int* pos_ptr;    // row position = pos_ptr[row]
+  RopeTable rope;
+};
+
+struct KernelCtlHost {
+  int* err;
+  unsigned long long limit_ns;
+};
+
+// Tensor-map encoding through the driver entry point (no libcuda link dependency).
+// Returns 0 on success.  dims/strides as cuTensorMapEncodeTiled: 2-D, innermost first.
+int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                 uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                 CUtensorMapSwizzle swz);
+
+// C = A * B.  A: [M, K] row-major bf16 (lda elements).  B: bf16, either [K, N] row-major
+// (b_kmajor = false, ldb elements) or [N, K] row-major (b_kmajor = true).  K % 64 == 0.
+int launch_gemm(const void* A, long long lda, const void* B, long long ldb, bool b_kmajor, int M,
+                int N, int K, const GemmEpi& ep, KernelCtlHost ctl, cudaStream_t st);
+
+void fill_rope_table(RopeTable* t, int d_rope, double theta);
+
+// Row-wise epilogue of the down-projection (norms, rotary key, lambda, latent-cache rows).
+struct NormParams {
+  const float* D1;            // [M, ld1] fp32: x W_a^Q | x W_a^KV | x W^lambda
+  int ld1, M;
+  int q_rank, kv_rank, n_signal;
+  const void* g_q;            // bf16 [q_rank] or null (ones)
+  const void* g_kv;           // bf16 [kv_rank] or null
+  float eps;
+  void* cQ;                   // bf16 [M, q_rank]
+  void* latent;               // bf16 [M, kv_rank + 64] or null
+  void* kR16;                 // fp16 [M, 64] or null
+  float* lam;                 // [M, n_signal]
+  int pos_T;                  // prefill: pos = m % pos_T, sequence = m / pos_T
+  const int* pos_ptr;         // decode: pos = pos_ptr[m], sequence = m
+  void* cache;                // optional bf16 [n_seq, cache_cap, kv_rank + 64]
+  long long cache_cap;
+  int* err;                   // device error word (bad cache_len is reported here)
+  RopeTable rope;
+};
+int launch_norm_rope(const NormParams& p, cudaStream_t st);
+
+// Fused prefill attention (QK^T, online softmax, PV, differential combine and gate).
+struct AttnParams {
+  int B, T, window;
+  int n_groups;               // KV heads = noise heads
+  int n_signal;               // 4 * n_groups
+  int rope_col0;              // first q^R column of QQ (n_heads * 128)
+  float scale_log2;           // log2(e) / sqrt(d_qk)
+  const float* lam;           // [B*T, n_signal]
+  const void* G;              // bf16 [B*T, n_signal*128] gate logits
+  float* O_noise;             // [B*T, n_groups, 128] fp32 scratch
+  void* Dg;                   // bf16 [B*T, n_signal*128]
+};
+int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* kR16,
+                        const AttnParams& p, KernelCtlHost ctl, cudaStream_t st);
+
+}  // namespace gdla

@@ -1,0 +1,255 @@
+// Projection GEMM on the 5th-generation tensor cores: C[M, N] = A[M, K] * B[K, N].
+//
+// Used for every linear map of the GDLA layer (picx.dev "Motif 3" summary, section 2.2:
+// x W_a^Q, c^Q W_b^Q, x W_a^KV, c W_b^KV, x W^lambda, c^Q W^G and the output projection W^O).
+//
+// One CTA computes one 128 x BN tile.  Warp 0 streams A (K-major, 128-byte swizzle) and B
+// (the [in, out] weight: M/N-major, or a [N, K] matrix: K-major) with TMA into a STAGES-deep
+// shared-memory ring; one thread of warp 1 issues tcgen05.mma (M = 128, N = BN, K = 16) into a
+// TMEM accumulator; all four warps then drain TMEM row-per-thread, apply the fused epilogue
+// (rotary embedding on the rope column range, dtype conversion) and store.
+#include "gdla_common.cuh"
+#include "gdla_internal.h"
+
+#include <math.h>
+#include <string.h>
+
+namespace gdla {
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+
+template <int BN, int STAGES, bool B_KMAJOR>
+__global__ void __launch_bounds__(128, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                   int K, const __grid_constant__ GemmEpi ep, KernelCtl ctl) {
+  constexpr int A_BYTES = 128 * 64 * 2;
+  constexpr int B_BYTES = BN * 64 * 2;
+  constexpr int STAGE = A_BYTES + B_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* done = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN;
+  const int nk = K / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    uint32_t issued_mask = 0, last_par = 0;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (kb / STAGES) & 1;
+      if (kb >= STAGES && !mbar_wait(&empty[s], ph ^ 1, ctl, SITE_GEMM_PRODUCER)) break;
+      uint8_t* st = smem + s * STAGE;
+      mbar_expect_tx(&full[s], STAGE);
+      tma_load_2d(st, &mapA, &full[s], kb * 64, m0);
+      if (B_KMAJOR) {
+        tma_load_2d(st + A_BYTES, &mapB, &full[s], kb * 64, n0);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c)
+          tma_load_2d(st + A_BYTES + c * 8192, &mapB, &full[s], n0 + c * 64, kb * 64);
+      }
+      issued_mask |= 1u << s;
+      last_par = (last_par & ~(1u << s)) | (ph << s);
+    }
+    // let every copy we issued land before this CTA can retire
+    for (int s = 0; s < STAGES; ++s)
+      if (issued_mask & (1u << s)) mbar_drain(&full[s], (last_par >> s) & 1, ctl.err);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = make_idesc(128, BN, 1, 0, B_KMAJOR ? 0 : 1);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (kb / STAGES) & 1;
+      if (!mbar_wait(&full[s], ph, ctl, SITE_GEMM_MMA)) break;
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(smem + s * STAGE);
+      const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
+        const uint64_t bd = B_KMAJOR ? sdesc_sw128(b_base + k * 32, 16, 1024)
+                                     : sdesc_sw128(b_base + k * 2048, 8192, 1024);
+        mma_ss(tmem, ad, bd, idesc, (kb | k) != 0);
+      }
+      mma_commit(&empty[s]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: thread = accumulator row
+  const bool ok = mbar_wait(done, 0, ctl, SITE_GEMM_EPI) || mbar_drain(done, 0, ctl.err);
+  tc_fence_after();
+  const int row = m0 + warp * 32 + lane;
+  const bool row_ok = ok && row < ep.M && *reinterpret_cast<volatile int*>(ctl.err) == 0;
+  int pos = 0;
+  if (ep.rope_hi > ep.rope_lo && row < ep.M) pos = ep.pos_ptr ? ep.pos_ptr[row] : (row % ep.pos_T);
+  const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    if (n0 + c0 >= ep.N) break;  // uniform across the CTA
+    uint32_t r[64];
+    GDLA_TMEM_LD32(t_row + c0, r);
+    GDLA_TMEM_LD32(t_row + c0 + 32, (r + 32));
+    tmem_ld_wait();
+    float v[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+    const int col = n0 + c0;
+    if (col >= ep.rope_lo && col < ep.rope_hi) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float cs, sn;
+        rope_cs(pos, ep.rope.inv_freq[i], &cs, &sn);
+        const float x1 = v[i], x2 = v[i + 32];
+        v[i] = x1 * cs - x2 * sn;
+        v[i + 32] = x2 * cs + x1 * sn;
+      }
+    }
+    if (!row_ok) continue;
+    const int ncols = min(64, ep.N - col);
+    if (ep.out_type == OUT_F32) {
+      float* dst = reinterpret_cast<float*>(ep.C) + (long long)row * ep.ldc + col;
+      if (ncols == 64) {
+#pragma unroll
+        for (int i = 0; i < 64; i += 4)
+          *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i < ncols) dst[i] = v[i];
+      }
+    } else {
+      uint32_t p[32];
+      if (ep.out_type == OUT_BF16) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p[i] = pack_bf162(v[2 * i], v[2 * i + 1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p[i] = pack_half2(v[2 * i], v[2 * i + 1]);
+      }
+      uint16_t* dst = reinterpret_cast<uint16_t*>(ep.C) + (long long)row * ep.ldc + col;
+      if (ncols == 64) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(p[i], p[i + 1], p[i + 2], p[i + 3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i < ncols) dst[i] = uint16_t(p[i >> 1] >> ((i & 1) * 16));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, BN);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                 uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                 CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return -1;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -2;
+}
+
+void fill_rope_table(RopeTable* t, int d_rope, double theta) {
+  memset(t, 0, sizeof(*t));
+  t->d_rope = d_rope;
+  for (int i = 0; i < d_rope / 2 && i < 32; ++i) t->inv_freq[i] = pow(theta, -2.0 * i / d_rope);
+}
+
+template <int BN, int STAGES, bool BK>
+static int run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K,
+                    const GemmEpi& ep, KernelCtlHost ctl, cudaStream_t st) {
+  constexpr int STAGE = 128 * 64 * 2 + BN * 64 * 2;
+  const int smem = STAGES * STAGE + 1024 + 256;
+  auto kfn = gemm_tc_kernel<BN, STAGES, BK>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return -4;
+  dim3 grid((M + 127) / 128, (N + BN - 1) / BN);
+  KernelCtl kc{ctl.err, ctl.limit_ns};
+  kfn<<<grid, 128, smem, st>>>(ma, mb, K, ep, kc);
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
+}
+
+int launch_gemm(const void* A, long long lda, const void* B, long long ldb, bool b_kmajor, int M,
+                int N, int K, const GemmEpi& ep, KernelCtlHost ctl, cudaStream_t st) {
+  if (M <= 0 || N <= 0) return 0;
+  if (K <= 0 || K % 64 != 0) return -1;
+  const int BN = N >= 256 ? 256 : (N > 64 ? 128 : 64);
+  CUtensorMap ma, mb;
+  if (make_tmap_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return -3;
+  int rc;
+  if (b_kmajor)
+    rc = make_tmap_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, N, ldb * 2, 64, BN,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    rc = make_tmap_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, K, ldb * 2, 64, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return -3;
+  if (b_kmajor) {
+    if (BN == 256) return run_gemm<256, 4, true>(ma, mb, M, N, K, ep, ctl, st);
+    if (BN == 128) return run_gemm<128, 6, true>(ma, mb, M, N, K, ep, ctl, st);
+    return run_gemm<64, 8, true>(ma, mb, M, N, K, ep, ctl, st);
+  }
+  if (BN == 256) return run_gemm<256, 4, false>(ma, mb, M, N, K, ep, ctl, st);
+  if (BN == 128) return run_gemm<128, 6, false>(ma, mb, M, N, K, ep, ctl, st);
+  return run_gemm<64, 8, false>(ma, mb, M, N, K, ep, ctl, st);
+}
+
+}  // namespace gdla

@@ -1,0 +1,135 @@
+// Down-projection epilogue of GDLA: one warp per token.
+//
+// From the fp32 row [x W_a^Q | x W_a^KV | x W^lambda] it forms (picx.dev "Motif 3" summary,
+// section 2.2; paperglide.net Figure 1 caption):
+//   c^Q      = RMSNorm(x W_a^Q)                          -> bf16 (operand of the up-projections)
+//   c_bar^KV = RMSNorm(c^KV)                             -> bf16 latent-cache row, columns 0..kv_rank-1
+//   k^R      = RoPE(k^R, pos) (not normalised)           -> bf16 latent-cache row, last d_rope columns
+//                                                           (+ an fp16 copy for the prefill attention)
+//   lambda   = sigmoid(x W^lambda), one per signal head  -> fp32
+// Position: prefill row m is token m % T of sequence m / T; decode row b is at pos_ptr[b].
+#include "gdla_common.cuh"
+#include "gdla_internal.h"
+
+namespace gdla {
+
+
+template <int NQ, int NKV>  // per-lane element counts: q_rank / 32, kv_rank / 32
+__global__ void __launch_bounds__(256) norm_rope_kernel(const __grid_constant__ NormParams p) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= p.M) return;
+  const int m = warp;
+  const float* row = p.D1 + (long long)m * p.ld1;
+  const __nv_bfloat16* g_q = static_cast<const __nv_bfloat16*>(p.g_q);
+  const __nv_bfloat16* g_kv = static_cast<const __nv_bfloat16*>(p.g_kv);
+  __nv_bfloat16* cQ = static_cast<__nv_bfloat16*>(p.cQ);
+  __nv_bfloat16* latent = static_cast<__nv_bfloat16*>(p.latent);
+  __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(p.cache);
+  __half* kR16 = static_cast<__half*>(p.kR16);
+  const int row_w = p.kv_rank + 64;
+
+  // ---- c^Q: lane owns float4 groups lane, lane + 32, ...
+  float q[NQ];
+#pragma unroll
+  for (int k = 0; k < NQ / 4; ++k) {
+    const float4 v = *reinterpret_cast<const float4*>(row + 4 * (lane + 32 * k));
+    q[4 * k] = v.x; q[4 * k + 1] = v.y; q[4 * k + 2] = v.z; q[4 * k + 3] = v.w;
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NQ; ++i) ss += q[i] * q[i];
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rq = rsqrtf(ss / float(p.q_rank) + p.eps);
+#pragma unroll
+  for (int k = 0; k < NQ / 4; ++k) {
+    const int c = 4 * (lane + 32 * k);
+    float g[4] = {1.f, 1.f, 1.f, 1.f};
+    if (g_q) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) g[e] = __bfloat162float(g_q[c + e]);
+    }
+    uint2 pk;
+    pk.x = pack_bf162(q[4 * k] * rq * g[0], q[4 * k + 1] * rq * g[1]);
+    pk.y = pack_bf162(q[4 * k + 2] * rq * g[2], q[4 * k + 3] * rq * g[3]);
+    *reinterpret_cast<uint2*>(cQ + (long long)m * p.q_rank + c) = pk;
+  }
+
+  // ---- c^KV
+  const float* rkv = row + p.q_rank;
+  float kv[NKV];
+#pragma unroll
+  for (int k = 0; k < NKV / 4; ++k) {
+    const float4 v = *reinterpret_cast<const float4*>(rkv + 4 * (lane + 32 * k));
+    kv[4 * k] = v.x; kv[4 * k + 1] = v.y; kv[4 * k + 2] = v.z; kv[4 * k + 3] = v.w;
+  }
+  ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NKV; ++i) ss += kv[i] * kv[i];
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rkvn = rsqrtf(ss / float(p.kv_rank) + p.eps);
+
+  // ---- k^R rotation: lane owns the pair (lane, lane + 32)
+  int pos = p.pos_ptr ? p.pos_ptr[m] : (m % p.pos_T);
+  const int seq = p.pos_ptr ? m : (m / p.pos_T);
+  bool cache_ok = p.cache != nullptr;
+  if (cache_ok && (pos < 0 || pos >= p.cache_cap)) {
+    if (lane == 0 && p.err) atomicCAS(p.err, 0, SITE_BAD_CACHE_LEN);
+    cache_ok = false;
+    pos = 0;
+  }
+  const float* rkr = rkv + p.kv_rank;
+  float cs, sn;
+  rope_cs(pos, p.rope.inv_freq[lane], &cs, &sn);
+  const float x1 = rkr[lane], x2 = rkr[lane + 32];
+  const float k1 = x1 * cs - x2 * sn, k2 = x2 * cs + x1 * sn;
+
+  __nv_bfloat16* dsts[2] = {latent ? latent + (long long)m * row_w : nullptr,
+                            cache_ok ? cache + ((long long)seq * p.cache_cap + pos) * row_w : nullptr};
+#pragma unroll
+  for (int d = 0; d < 2; ++d) {
+    __nv_bfloat16* dst = dsts[d];
+    if (!dst) continue;
+#pragma unroll
+    for (int k = 0; k < NKV / 4; ++k) {
+      const int c = 4 * (lane + 32 * k);
+      float g[4] = {1.f, 1.f, 1.f, 1.f};
+      if (g_kv) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) g[e] = __bfloat162float(g_kv[c + e]);
+      }
+      uint2 pk;
+      pk.x = pack_bf162(kv[4 * k] * rkvn * g[0], kv[4 * k + 1] * rkvn * g[1]);
+      pk.y = pack_bf162(kv[4 * k + 2] * rkvn * g[2], kv[4 * k + 3] * rkvn * g[3]);
+      *reinterpret_cast<uint2*>(dst + c) = pk;
+    }
+    dst[p.kv_rank + lane] = __float2bfloat16_rn(k1);
+    dst[p.kv_rank + lane + 32] = __float2bfloat16_rn(k2);
+  }
+  if (kR16) {
+    kR16[(long long)m * 64 + lane] = __float2half_rn(k1);
+    kR16[(long long)m * 64 + lane + 32] = __float2half_rn(k2);
+  }
+
+  // ---- lambda
+  const float* rl = rkr + 64;
+  for (int c = lane; c < p.n_signal; c += 32)
+    p.lam[(long long)m * p.n_signal + c] = 1.0f / (1.0f + expf(-rl[c]));
+}
+
+int launch_norm_rope(const NormParams& p, cudaStream_t st) {
+  if (p.M <= 0) return 0;
+  const int threads = 256;
+  const int blocks = (p.M * 32 + threads - 1) / threads;
+  if (p.q_rank == 1024 && p.kv_rank == 512)
+    norm_rope_kernel<32, 16><<<blocks, threads, 0, st>>>(p);
+  else if (p.q_rank == 128 && p.kv_rank == 128)
+    norm_rope_kernel<4, 4><<<blocks, threads, 0, st>>>(p);
+  else
+    return -2;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
+}
+
+}  // namespace gdla

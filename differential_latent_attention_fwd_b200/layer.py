@@ -1,0 +1,58 @@
+"""GdlaLayer: device-resident weights + caller-side buffers around the C ABI.
+
+A convenience for Python users: it owns the layer's bf16 weights on one CUDA device, the
+decode-ready absorbed weights, and a reusable workspace (allocated with torch, which is only
+the memory/stream plumbing here), and forwards to the C entry points in ``binding``.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as gb
+from .synth import GdlaShape, WEIGHT_NAMES
+
+
+class GdlaLayer:
+    def __init__(self, shape: GdlaShape, weights: dict, g_q=None, g_kv=None, device="cuda"):
+        self.shape = shape
+        self.device = torch.device(device)
+        self.w = {n: weights[n].to(self.device, torch.bfloat16).contiguous() for n in WEIGHT_NAMES}
+        self.g_q = None if g_q is None else g_q.to(self.device, torch.bfloat16).contiguous()
+        self.g_kv = None if g_kv is None else g_kv.to(self.device, torch.bfloat16).contiguous()
+        self.cfg = gb.make_config(shape)
+        self.cw = gb.make_weights(self.w, self.g_q, self.g_kv)
+        self._ws = None
+        self._absorbed = None
+        self._absorbed_buf = None
+
+    def workspace(self, B: int, T: int, mode: int) -> torch.Tensor:
+        need = gb.gdla_workspace_size(self.cfg, B, T, mode)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def prefill(self, x: torch.Tensor, y: torch.Tensor | None = None,
+                kv_cache_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        B, T, d = x.shape
+        if y is None:
+            y = torch.empty((B, T, d), dtype=torch.bfloat16, device=self.device)
+        ws = self.workspace(B, T, gb.GDLA_MODE_PREFILL)
+        cap = 0 if kv_cache_out is None else kv_cache_out.shape[1]
+        gb.gdla_prefill_fwd(self.cfg, self.cw, x, y, ws, kv_cache_out, cap, stream)
+        return y
+
+    def absorbed(self, stream=None) -> gb.gdla_absorbed_t:
+        if self._absorbed is None:
+            n = gb.gdla_absorbed_size(self.cfg)
+            self._absorbed_buf = torch.empty(n, dtype=torch.uint8, device=self.device)
+            self._absorbed = gb.gdla_absorb_weights(self.cfg, self.cw, self._absorbed_buf, stream)
+        return self._absorbed
+
+    def decode(self, x_new: torch.Tensor, kv_cache: torch.Tensor, cache_len: torch.Tensor,
+               y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        B, d = x_new.shape
+        if y is None:
+            y = torch.empty((B, d), dtype=torch.bfloat16, device=self.device)
+        ws = self.workspace(B, 1, gb.GDLA_MODE_DECODE)
+        gb.gdla_decode_fwd(self.cfg, self.absorbed(stream), x_new, kv_cache, cache_len, y, ws, stream)
+        return y

@@ -1,0 +1,151 @@
+/*
+ * gdla.h -- C ABI of the B200 (sm_100a) Grouped Differential Latent Attention forward pass.
+ *
+ * Operation (source: "Motif 3: Technical Report"; picx.dev summary page, section 2.2
+ * "Grouped Differential Latent Attention (GDLA)", all equations; paperglide.net page,
+ * section "Model Architecture" and the Figure 1 caption):
+ *
+ *   c^Q_t        = RMSNorm(x_t W_a^Q)                   [q^C_t; q^R_t] = c^Q_t W_b^Q
+ *   [c^KV_t; k^R_t] = x_t W_a^KV                        c_bar_t = RMSNorm(c^KV_t)
+ *   [K^C_t; V_t] = Reshape_heads(c_bar_t W_b^KV)         (16 KV heads, shared by both paths)
+ *   lambda_t     = sigmoid(x_t W^lambda) in (0,1)^{n_S}   (one value per signal head)
+ *   H_h          = softmax attention of head h over keys [K^C; RoPE(k^R)] (one rotary key
+ *                  shared by every KV head) under a causal or sliding-window mask
+ *   D_t          = H_{S,t} - lambda_t (.) Repeat_g(H_{N,t}),  n_N = n_H/(g+1), n_S = g n_N
+ *   G_t          = Reshape_heads(c^Q_t W^G)
+ *   GDLA(x_t)    = vec(sigmoid(G_t) (.) D_t) W^O
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - weights are [in, out] row-major bf16 (the pages' x W);
+ *   - W_b^Q columns: q^C of every head (head-major, d_nope each), then q^R of every head;
+ *   - W_a^KV columns: c^KV (kv_rank), then k^R (d_rope);
+ *   - W_b^KV columns: per KV head j, d_nope K^C columns then d_v V columns;
+ *   - heads 0..n_S-1 are signal heads, n_S..n_H-1 noise heads; signal head s and noise head
+ *     s / g read KV head s / g (Repeat_g pairs signal s with noise s / g);
+ *   - softmax scale 1/sqrt(d_nope + d_rope); RMSNorm eps from the config, gains optional;
+ *   - RoPE: rotate-half over the d_rope part, pairs (i, i + d_rope/2), angle pos*theta^(-2i/d_rope),
+ *     pos = 0-based position in the sequence (decode: the cache length);
+ *   - masks: causal keys s <= t; sliding window keys t - W < s <= t (W keys incl. self).
+ *
+ * Compiled specialisation: d_nope = 128, d_rope = 64, d_v = 128, g = n_signal / n_noise = 4,
+ * n_kv_heads = n_noise, q_rank = 1024, kv_rank = 512, d_model a multiple of 64.
+ * Other shapes return GDLA_ERR_UNSUPPORTED_SHAPE.
+ *
+ * Memory and streams: every buffer is allocated by the caller (device memory unless stated);
+ * the library never allocates, frees or synchronises device memory on these paths.  All
+ * calls are asynchronous on the given stream.  Pointer arguments must be 16-byte aligned.
+ *
+ * Errors: every entry point returns 0 (GDLA_OK) or a negative gdla_status_t.  Argument
+ * problems are detected on the host before anything is launched.  Kernels never trap: every
+ * wait inside a kernel is bounded, and on expiry the kernel records a site code in a device
+ * error word, drains its own copies and exits; gdla_device_error() reads that word.
+ */
+#ifndef GDLA_H_
+#define GDLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDLA_OK = 0,
+  GDLA_ERR_INVALID_ARG = -1,        /* null pointer, non-positive size, misaligned buffer */
+  GDLA_ERR_UNSUPPORTED_SHAPE = -2,  /* config outside the compiled specialisation */
+  GDLA_ERR_WORKSPACE_TOO_SMALL = -3,
+  GDLA_ERR_LAUNCH = -4,             /* a kernel launch or tensor-map encode failed */
+  GDLA_ERR_DEVICE_TIMEOUT = -5,     /* a bounded in-kernel wait expired (see gdla_device_error) */
+  GDLA_ERR_CUDA = -6                /* a CUDA runtime call failed */
+} gdla_status_t;
+
+/* Layer shape.  window: 0 = full causal attention, W > 0 = sliding window of W keys. */
+typedef struct {
+  int d_model, q_rank, kv_rank, n_signal, n_noise, n_kv_heads, d_nope, d_rope, d_v;
+  int window;
+  float rope_theta, rms_eps;
+} gdla_config_t;
+
+/* Layer weights: device pointers, bf16, row-major [in, out]:
+ *   W_aQ [d_model, q_rank]; W_bQ [q_rank, n_H*(d_nope+d_rope)]; W_aKV [d_model, kv_rank+d_rope];
+ *   W_bKV [kv_rank, n_kv_heads*(d_nope+d_v)]; W_lambda [d_model, n_signal];
+ *   W_G [q_rank, n_signal*d_v]; W_O [n_signal*d_v, d_model];
+ *   g_q [q_rank], g_kv [kv_rank]: RMSNorm gains, or NULL for ones.
+ * The library reads them; the caller keeps them alive while calls that use them run. */
+typedef struct {
+  const void *W_aQ, *W_bQ, *W_aKV, *W_bKV, *W_lambda, *W_G, *W_O;
+  const void *g_q, *g_kv;
+} gdla_weights_t;
+
+/* Weights prepared for decode by gdla_absorb_weights.  The struct is plain data owned by
+ * the caller; `base` is the caller's device buffer holding the derived tensors. */
+typedef struct {
+  gdla_weights_t w;          /* the original weights (pointers copied, not the data) */
+  void* W_UKt;               /* bf16 [n_kv_heads][d_nope][kv_rank]: K^C blocks of W_b^KV, transposed */
+  gdla_config_t cfg;
+  uint32_t magic;
+} gdla_absorbed_t;
+
+enum { GDLA_MODE_PREFILL = 0, GDLA_MODE_DECODE = 1 };
+
+/* Bytes of workspace that gdla_prefill_fwd (mode 0: B sequences of T tokens) or
+ * gdla_decode_fwd (mode 1: B sequences; T ignored) needs. */
+int gdla_workspace_size(const gdla_config_t* cfg, int B, int T, int mode, size_t* bytes);
+
+/* Bytes of device memory gdla_absorb_weights writes. */
+int gdla_absorbed_size(const gdla_config_t* cfg, size_t* bytes);
+
+/* Prefill: y[b, t, :] = GDLA(x[b, t, :]) for B independent sequences of T tokens.
+ *   x  [B, T, d_model] bf16 (device)       y [B, T, d_model] bf16 (device, written)
+ *   kv_cache_out: NULL, or bf16 [B, cache_cap, kv_rank + d_rope]; row (b, t) receives the
+ *     latent-cache entry (RMSNorm'd c^KV | rotated k^R) of token t, for later decode calls.
+ *   workspace: >= gdla_workspace_size(cfg, B, T, GDLA_MODE_PREFILL) bytes of device memory.
+ * Any T >= 1 is allowed (tails are masked).  Returns after enqueueing on `stream`. */
+int gdla_prefill_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int B,
+                     int T, void* y, void* kv_cache_out, int cache_cap, void* workspace,
+                     size_t ws_bytes, void* stream);
+
+/* One-time weight preparation for the absorbed-form decode (MLA-style weight absorption:
+ * attention runs in the latent space and K/V are never materialised; the pages note that
+ * MLA rebuilds the keys/values only inside the attention computation).
+ *   dst: >= gdla_absorbed_size(cfg) bytes of device memory, kept alive by the caller.
+ *   out: filled on success (host struct). */
+int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void* dst,
+                        size_t dst_bytes, gdla_absorbed_t* out, void* stream);
+
+/* Decode one new token per sequence.
+ *   x_new [B, d_model] bf16.  kv_cache [B, cap, kv_rank + d_rope] bf16: rows 0..len[b]-1 hold
+ *   the cached latent entries; the new token's entry is written at row len[b] (so
+ *   len[b] < cap) and it attends to rows 0..len[b] (or the last `window` of them).
+ *   cache_len [B] int32 (device).  y [B, d_model] bf16 (written). */
+int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* absorbed, const void* x_new,
+                    void* kv_cache, const int* cache_len, int cap, int B, void* y,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/* Reads (and with clear != 0 resets) the device error word after synchronising `stream`:
+ * *site = 0 when every kernel finished normally, else the site code of the first bounded wait
+ * that expired.  Returns GDLA_OK, or GDLA_ERR_DEVICE_TIMEOUT when *site != 0. */
+int gdla_device_error(void* stream, int* site, int clear);
+
+/* Bound of one in-kernel wait, in nanoseconds (default 2e9).  Values < 1000 are clamped. */
+int gdla_set_wait_limit_ns(unsigned long long ns);
+
+/* Self-test of the bounded-wait path: launches one CTA that waits on an mbarrier nothing
+ * arrives on, with a wait bound of `limit_ns`; writes the kernel's report to *site
+ * (the self-test site code when the wait expired as intended).  Synchronises `stream`. */
+int gdla_selftest_wait_timeout(unsigned long long limit_ns, void* stream, int* site);
+
+/* Byte offset, inside a prefill or decode workspace, of a named intermediate (for
+ * inspection in tests): 0 D1 (fp32 down-projection), 1 c^Q, 2 latent rows, 3 lambda, 4 QQ
+ * (q^C | rotated q^R), 5 G, 6 KV, 7 noise-head outputs, 8 Dg, 9 kR16. */
+int gdla_workspace_offset(const gdla_config_t* cfg, int B, int T, int mode, int which,
+                          size_t* offset);
+
+const char* gdla_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDLA_H_ */

@@ -1,0 +1,83 @@
+"""The C ABI library loads and exports every entry point declared in include/gdla.h, and its
+host-side validation answers without a GPU (no kernel is launched here)."""
+import ctypes
+
+import pytest
+
+from differential_latent_attention_fwd_b200 import binding as gb
+from differential_latent_attention_fwd_b200 import build as gbuild
+from differential_latent_attention_fwd_b200.synth import GdlaShape
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gb.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = gb.header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in gdla.h but not exported"
+
+
+def test_status_strings(L):
+    for code in range(0, -7, -1):
+        assert gb.gdla_status_string(code) not in ("", "unknown status")
+    assert gb.gdla_status_string(-99) == "unknown status"
+
+
+def test_workspace_size_and_offsets(L):
+    cfg = gb.make_config(GdlaShape())
+    n = gb.gdla_workspace_size(cfg, 1, 256, gb.GDLA_MODE_PREFILL)
+    M = 256
+    # dominant buffers: q^C|q^R (fp16), gate, Dg, K|V, noise outputs, fp32 down-projection
+    assert n >= M * (80 * 192 * 2 + 8192 * 2 * 2 + 4096 * 2 + 16 * 128 * 4 + 1664 * 4)
+    offs = [gb.gdla_workspace_offset(cfg, 1, 256, 0, i) for i in range(10)]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs) and offs[-1] < n
+    assert gb.gdla_workspace_size(cfg, 2, 256, 0) > n
+    d = gb.gdla_workspace_size(cfg, 64, 1, gb.GDLA_MODE_DECODE)
+    assert d > 64 * 80 * 576 * 2
+    assert gb.gdla_absorbed_size(cfg) == 16 * 128 * 512 * 2
+
+
+def test_host_validation_without_gpu(L):
+    cfg = gb.make_config(GdlaShape())
+    bad = gb.make_config(GdlaShape(d_nope=64))
+    with pytest.raises(gb.GdlaError) as e:
+        gb.gdla_workspace_size(bad, 1, 16, 0)
+    assert e.value.status == -2
+    with pytest.raises(gb.GdlaError) as e:
+        gb.gdla_workspace_size(cfg, 0, 16, 0)
+    assert e.value.status == -1
+    with pytest.raises(gb.GdlaError) as e:
+        gb.gdla_workspace_size(cfg, 1, 16, 7)
+    assert e.value.status == -1
+    # null weights / buffers are rejected before any launch
+    w = gb.gdla_weights_t()
+    rc = L.gdla_prefill_fwd(ctypes.byref(cfg), ctypes.byref(w), None, 1, 16, None, None, 0, None, 0, None)
+    assert rc == -1
+    rc = L.gdla_decode_fwd(ctypes.byref(cfg), None, None, None, None, 1, 1, None, None, 0, None)
+    assert rc == -1
+    # an absorbed handle that was never filled is rejected
+    ab = gb.gdla_absorbed_t()
+    rc = L.gdla_decode_fwd(ctypes.byref(cfg), ctypes.byref(ab), None, None, None, 1, 1, None, None, 0, None)
+    assert rc == -1
+    # GDA-style config (g = 1) is outside the compiled specialisation
+    gda = gb.make_config(GdlaShape(n_signal=16, n_noise=16))
+    with pytest.raises(gb.GdlaError) as e:
+        gb.gdla_workspace_size(gda, 1, 16, 0)
+    assert e.value.status == -2
+
+
+def test_misaligned_pointer_rejected(L):
+    cfg = gb.make_config(GdlaShape())
+    fake = ctypes.c_void_p(0x1000)
+    w = gb.gdla_weights_t(fake, fake, fake, fake, fake, fake, fake, None, None)
+    rc = L.gdla_prefill_fwd(ctypes.byref(cfg), ctypes.byref(w), ctypes.c_void_p(0x1008), 1, 16,
+                            fake, None, 0, fake, 1 << 40, None)
+    assert rc == -1
+    # workspace too small is reported before anything touches the device
+    rc = L.gdla_prefill_fwd(ctypes.byref(cfg), ctypes.byref(w), fake, 1, 16, fake, None, 0, fake, 16, None)
+    assert rc == -3

@@ -1,0 +1,135 @@
+"""GPU prefill parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerance of the layer output y: max-abs 2e-2 and relative L2 5e-3.  Intermediates are checked
+stage by stage first, with a bound derived from the storage precision of each stage (one bf16
+rounding ~1.6e-3 rms relative, fp16 ~2e-4), so that a failure names the kernel at fault.
+"""
+import numpy as np
+import pytest
+import torch
+
+from differential_latent_attention_fwd_b200 import binding as gb
+from differential_latent_attention_fwd_b200 import synth
+from tests.gpu_helpers import (MAX_ABS, REL_L2, WS_CQ, WS_D1, WS_DG, WS_G, WS_KV, WS_LAM,
+                               WS_LATENT, WS_ONOISE, WS_QQ, check, oracle_prefill, prefill_case,
+                               to_np, ws_view)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(layer, x, kv_cache_out=None):
+    y = layer.prefill(x, kv_cache_out=kv_cache_out)
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
+    return y
+
+
+def test_stagewise_intermediates_t256(cuda_ok):
+    """Every stage of the T=256 causal layer against the oracle's intermediates."""
+    B, T = 1, 256
+    shape, inp, layer, x = prefill_case(B, T, 0, seed=0)
+    y = _run(layer, x)
+    ws = layer._ws
+    cfg = layer.cfg
+    yo, parts = oracle_prefill(inp, parts=True)
+    p = parts[0]
+    nH = shape.n_heads
+    errs = []
+    # fp32 down-projection, before the norms
+    x64 = to_np(inp.x[0])
+    W = {k: to_np(v) for k, v in inp.weights.items()}
+    d1 = to_np(ws_view(ws, cfg, B, T, 0, WS_D1, torch.float32, (T, 1664)))
+    check("x W_aQ (fp32)", d1[:, :1024], x64 @ W["W_aQ"], rel=1e-4, mabs=1e-2, errors=errs)
+    check("x W_aKV (fp32)", d1[:, 1024:1600], x64 @ W["W_aKV"], rel=1e-4, mabs=1e-2, errors=errs)
+    check("x W_lambda (fp32)", d1[:, 1600:], x64 @ W["W_lambda"], rel=1e-4, mabs=1e-2, errors=errs)
+    cq = to_np(ws_view(ws, cfg, B, T, 0, WS_CQ, torch.bfloat16, (T, 1024)))
+    check("c^Q (bf16)", cq, p["cQ"], rel=4e-3, mabs=5e-2, errors=errs)
+    lat = to_np(ws_view(ws, cfg, B, T, 0, WS_LATENT, torch.bfloat16, (T, 576)))
+    check("c_bar^KV (bf16)", lat[:, :512], p["cbar"], rel=4e-3, mabs=5e-2, errors=errs)
+    check("rotated k^R (bf16)", lat[:, 512:], p["kR"], rel=4e-3, mabs=5e-2, errors=errs)
+    lam = to_np(ws_view(ws, cfg, B, T, 0, WS_LAM, torch.float32, (T, 64)))
+    check("lambda (fp32)", lam, p["lam"], rel=1e-4, mabs=1e-4, errors=errs)
+    qq = to_np(ws_view(ws, cfg, B, T, 0, WS_QQ, torch.float16, (T, nH * 192)))
+    check("q^C (fp16)", qq[:, : nH * 128].reshape(T, nH, 128), p["qC"], rel=6e-3, mabs=5e-2, errors=errs)
+    check("rotated q^R (fp16)", qq[:, nH * 128:].reshape(T, nH, 64), p["qR"], rel=6e-3, mabs=5e-2,
+          errors=errs)
+    g = to_np(ws_view(ws, cfg, B, T, 0, WS_G, torch.bfloat16, (T, 64, 128)))
+    check("G (bf16)", g, p["G"], rel=6e-3, mabs=5e-2, errors=errs)
+    kv = to_np(ws_view(ws, cfg, B, T, 0, WS_KV, torch.float16, (T, 16, 256)))
+    check("K^C (fp16)", kv[..., :128], p["KC"], rel=6e-3, mabs=5e-2, errors=errs)
+    check("V (fp16)", kv[..., 128:], p["V"], rel=6e-3, mabs=5e-2, errors=errs)
+    dg = to_np(ws_view(ws, cfg, B, T, 0, WS_DG, torch.bfloat16, (T, 64, 128)))
+    check("Dg (bf16)", dg, p["Dg"], rel=REL_L2, mabs=MAX_ABS, errors=errs)
+    check("y (bf16)", to_np(y[0]), yo[0], errors=errs)
+    assert not errs, "\n".join(errs)
+
+
+@pytest.mark.parametrize("B,T,window", [
+    (1, 1, 0), (1, 100, 0), (1, 129, 0), (1, 300, 0), (2, 200, 64), (1, 700, 128),
+    (1, 384, 1), (1, 257, 256), (3, 130, 0),
+])
+def test_prefill_edge_shapes(cuda_ok, B, T, window):
+    shape, inp, layer, x = prefill_case(B, T, window, seed=11)
+    y = _run(layer, x)
+    yo = oracle_prefill(inp)
+    errs = []
+    for b in range(B):
+        check(f"y[b={b}] B={B} T={T} W={window}", to_np(y[b]), yo[b], errors=errs)
+    assert not errs, "\n".join(errs)
+
+
+def test_prefill_writes_latent_cache(cuda_ok):
+    B, T, cap = 2, 150, 160
+    shape, inp, layer, x = prefill_case(B, T, 0, seed=5)
+    cache = torch.zeros((B, cap, 576), dtype=torch.bfloat16, device="cuda")
+    _run(layer, x, kv_cache_out=cache)
+    _, parts = oracle_prefill(inp, parts=True)
+    for b in range(B):
+        want = np.concatenate([parts[b]["cbar"], parts[b]["kR"]], -1)
+        check(f"cache rows b={b}", to_np(cache[b, :T]), want, rel=4e-3, mabs=5e-2)
+    assert float(cache[:, T:].abs().max()) == 0.0
+
+
+def test_prefill_deterministic(cuda_ok):
+    shape, inp, layer, x = prefill_case(1, 300, 0, seed=3)
+    y1 = _run(layer, x).clone()
+    y2 = _run(layer, x)
+    assert torch.equal(y1, y2)
+
+
+def _sampled_workload(name, n_rows=512):
+    wl = synth.WORKLOADS[name]
+    B, T, window, seed = wl["B"], wl["T"], wl["window"], wl["seed"]
+    shape, inp, layer, x = prefill_case(B, T, window, seed)
+    y = _run(layer, x)
+    rows = synth.sample_rows(T, window, n_rows, seed)
+    yo = oracle_prefill(inp, rows=rows)
+    errs = []
+    for b in range(B):
+        check(f"{name} b={b} ({len(rows)} sampled rows)", to_np(y[b, rows]), yo[b], errors=errs)
+    del layer, x, y
+    torch.cuda.empty_cache()
+    assert not errs, "\n".join(errs)
+
+
+def test_workload_t256_causal_all_rows(cuda_ok):
+    wl = synth.WORKLOADS["prefill_b1_t256_causal"]
+    shape, inp, layer, x = prefill_case(wl["B"], wl["T"], wl["window"], wl["seed"])
+    y = _run(layer, x)
+    check("T=256 causal, all rows", to_np(y[0]), oracle_prefill(inp)[0])
+
+
+def test_workload_b2_t8192_swa2048_sampled(cuda_ok):
+    _sampled_workload("prefill_b2_t8192_swa2048")
+
+
+def test_workload_t32768_causal_sampled(cuda_ok):
+    _sampled_workload("prefill_b1_t32768_causal")
+
+
+def test_workload_t262144_swa2048_sampled(cuda_ok):
+    _sampled_workload("prefill_b1_t262144_swa2048")
+
+
+def test_workload_t262144_causal_sampled(cuda_ok):
+    _sampled_workload("prefill_b1_t262144_causal")
