@@ -12,10 +12,11 @@ gated output), plus the paperglide.net page ("Model Architecture" worked example
 Figure 1 caption: one lambda per signal head, gate from the normalised query latent, one
 rotary key shared by all KV heads, 16 KV heads shared by the signal and noise paths).
 
-Every floating-point step is float64.  Matrix products use numpy's BLAS (a library
-primitive); there is no blocking, fusion or reordering beyond the equations, except the
-weight-absorbed decode route, which is a second, independent statement of the same algebra
-and is checked against the literal one.
+Every floating-point step is float64.  Matrix products use numpy's BLAS or torch's CPU
+matmul (library primitives); the masked softmax uses torch.softmax (a library routine).  The only grouping beyond the equations: prefill evaluates the masked softmax
+attention of several query rows as one product over a shared key block (each row still
+normalises over exactly its own visible keys), and the weight-absorbed decode route is a
+second, independent statement of the same algebra, checked against the literal one.
 
 Readings where the pages are silent (each also listed in the design notes):
   * weights are [in, out] (the pages write x W);
@@ -250,20 +251,65 @@ def _weights64(w: dict) -> dict:
     return {k: f64(v) for k, v in w.items()}
 
 
+def masked_softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                             allowed: np.ndarray) -> np.ndarray:
+    """Masked softmax attention of several query rows over one shared key block.
+
+    q [r, h, dk] (r query positions, h heads reading the same keys), k [S, dk], v [S, dv],
+    allowed [r, S] bool (key s visible to row r) -> [r, h, dv] = softmax(q k^T scale + mask) v.
+    Every row must see at least one key.  Evaluated with float64 torch CPU ops (matmul,
+    masked fill, softmax), which run multithreaded on large blocks.
+    """
+    import torch
+    r, h, dk = q.shape
+    tq, tk, tv = torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v)
+    s = (tq.reshape(r * h, dk) @ tk.T).reshape(r, h, -1) * scale
+    s.masked_fill_(~torch.from_numpy(allowed)[:, None, :], float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    return (p.reshape(r * h, -1) @ tv).reshape(r, h, -1).numpy()
+
+
+def _row_chunks(rows, window: int, max_rows: int = 64):
+    """Split sorted query rows into runs whose shared key span stays near what each row needs."""
+    out, i = [], 0
+    while i < len(rows):
+        lo0 = key_range(rows[i], window)[0]
+        k = i + 1
+        while k < len(rows) and k - i < max_rows:
+            t = rows[k]
+            need = t - key_range(t, window)[0] + 1
+            if t - lo0 + 1 > 2 * need + 1024:
+                break
+            k += 1
+        out.append((i, k))
+        i = k
+    return out
+
+
 def gdla_prefill(x, weights: dict, cfg: OracleConfig, rows=None, g_q=None, g_kv=None,
                  pos_offset: int = 0, return_parts: bool = False, chunk: int = 8192):
     """GDLA(x_t) for every sequence of a batch, at the requested query rows.
 
     x [B, T, d]; ``rows`` = list of query positions (default: all).  Position of token t is
     pos_offset + t.  Returns y [B, len(rows), d] (and a dict of per-row intermediates when
-    ``return_parts``: c^Q, q^C, q^R, lambda, G, Dg and, for all tokens, the latent cache rows).
+    ``return_parts``: c^Q, q^C, q^R, lambda, G, Dg and, for all tokens, c_bar, k^R, K^C, V).
+    Attention is evaluated one KV head at a time for all requested rows (signal and noise
+    heads of that KV head together), rows batched into masked products over a shared key
+    block; each row's softmax still runs over exactly its own visible keys.
     """
     W = _weights64(weights)
     gq = None if g_q is None else f64(g_q)
     gkv = None if g_kv is None else f64(g_kv)
     B, T, _ = x.shape
     rows = list(range(T)) if rows is None else [int(r) for r in rows]
-    t_hi = max(rows) + 1
+    rows_a = np.asarray(rows)
+    order = np.argsort(rows_a, kind="stable")
+    srows = rows_a[order]
+    t_hi = int(srows[-1]) + 1
+    scale = 1.0 / np.sqrt(cfg.d_nope + cfg.d_rope)
+    kvh = kv_head_of(cfg)
+    blk = cfg.d_nope + cfg.d_v
+    chunks = _row_chunks(srows.tolist(), cfg.window)
     ys, parts = [], []
     for b in range(B):
         # latent rows (c_bar, k^R) of every token a requested query can see
@@ -274,22 +320,41 @@ def gdla_prefill(x, weights: dict, cfg: OracleConfig, rows=None, g_q=None, g_kv=
             xb = f64(x[b, c0:c1])
             cbar[c0:c1], kR[c0:c1] = kv_latent(xb, W["W_aKV"], gkv,
                                                pos_offset + np.arange(c0, c1), cfg)
-        KC, V = kv_heads(cbar, W["W_bKV"], cfg)
         xr = f64(x[b, rows])
-        pos_r = pos_offset + np.asarray(rows)
+        pos_r = pos_offset + rows_a
         cQ, qC, qR = query_path(xr, W["W_aQ"], W["W_bQ"], gq, pos_r, cfg)
         lam = lambda_coeff(xr, W["W_lambda"])
         G = gate_logits(cQ, W["W_G"], cfg)
+        H = np.empty((len(rows), cfg.n_heads, cfg.d_v))
+        if return_parts:
+            KC_all = np.empty((t_hi, cfg.n_kv_heads, cfg.d_nope))
+            V_all = np.empty((t_hi, cfg.n_kv_heads, cfg.d_v))
+        for j in range(cfg.n_kv_heads):
+            heads = np.nonzero(kvh == j)[0]
+            # [K^C_j; V_j] = c_bar W_b^KV restricted to KV head j's column block
+            KC_j = cbar @ W["W_bKV"][:, j * blk: j * blk + cfg.d_nope]
+            V_j = cbar @ W["W_bKV"][:, j * blk + cfg.d_nope: (j + 1) * blk]
+            if return_parts:
+                KC_all[:, j], V_all[:, j] = KC_j, V_j
+            K_j = np.concatenate([KC_j, kR], axis=-1)           # k_{j,s} = [K^C_{j,s}; k^R_s]
+            q_j = np.concatenate([qC[:, heads], qR[:, heads]], axis=-1)
+            for i0, i1 in chunks:
+                rr = srows[i0:i1]
+                idx = order[i0:i1]
+                los = np.array([key_range(int(t), cfg.window)[0] for t in rr])
+                lo, hi = int(los.min()), int(rr.max())
+                keys = np.arange(lo, hi + 1)
+                allowed = (keys[None, :] >= los[:, None]) & (keys[None, :] <= rr[:, None])
+                H[idx[:, None], heads[None, :]] = masked_softmax_attention(
+                    q_j[idx], K_j[lo: hi + 1], V_j[lo: hi + 1], scale, allowed)
         y = np.empty((len(rows), cfg.d_model))
         Dg_all = np.empty((len(rows), cfg.n_signal, cfg.d_v))
-        for i, t in enumerate(rows):
-            lo, hi = key_range(t, cfg.window)
-            H = attend_row(qC[i], qR[i], KC, kR, V, lo, hi, cfg)
-            Dg_all[i], y[i] = combine_row(H, lam[i], G[i], W["W_O"], cfg)
+        for i in range(len(rows)):
+            Dg_all[i], y[i] = combine_row(H[i], lam[i], G[i], W["W_O"], cfg)
         ys.append(y)
         if return_parts:
             parts.append(dict(cQ=cQ, qC=qC, qR=qR, lam=lam, G=G, Dg=Dg_all,
-                              cbar=cbar, kR=kR, KC=KC, V=V))
+                              cbar=cbar, kR=kR, KC=KC_all, V=V_all))
     y = np.stack(ys)
     return (y, parts) if return_parts else y
 

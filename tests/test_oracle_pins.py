@@ -374,3 +374,28 @@ def test_brute_force_tiny(window):
     x = tiny_x(cfg, 1, 6, seed=12)
     np.testing.assert_allclose(O.gdla_prefill(x, W, cfg)[0], _brute_prefill(x[0], W, cfg),
                                rtol=1e-11, atol=1e-12)
+
+
+def test_masked_softmax_attention_is_sdpa_with_mask():
+    r = np.random.default_rng(13)
+    q, k, v = r.normal(size=(6, 3, 10)), r.normal(size=(17, 10)), r.normal(size=(17, 4))
+    allowed = r.random((6, 17)) < 0.6
+    allowed[:, 0] = True
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).transpose(0, 1), torch.from_numpy(k)[None].expand(3, 17, 10),
+        torch.from_numpy(v)[None].expand(3, 17, 4), attn_mask=torch.from_numpy(allowed)[None],
+        scale=0.29).transpose(0, 1).numpy()
+    np.testing.assert_allclose(O.masked_softmax_attention(q, k, v, 0.29, allowed), ref,
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_row_subsets_and_order_agree():
+    """Sampled rows (any order, any chunking) equal the same rows of the all-rows run."""
+    for window in (0, 5):
+        cfg = tiny_cfg(window=window)
+        W = tiny_weights(cfg)
+        x = tiny_x(cfg, 2, 40)
+        full = O.gdla_prefill(x, W, cfg)
+        rows = [39, 3, 17, 0, 25, 26, 8]
+        sub = O.gdla_prefill(x, W, cfg, rows=rows)
+        np.testing.assert_allclose(sub, full[:, rows], rtol=1e-12, atol=1e-13)
