@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""GDLA forward benchmark on B200: one JSON line on rank 0.
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+  * prefill of B=1 x T=32768 tokens, full causal (the layer's headline workload), and
+  * absorbed-form decode of B=64 sequences with 32768 cached positions, causal and SWA W=2048.
+`value` is the prefill throughput of the whole layer (algorithmic FLOPs / time); decode
+figures ride along under "decode".  Inputs are resident in HBM when the timed region starts;
+"e2e" repeats the prefill through the C ABI with host buffers (pinned H2D of x, D2H of y).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+       (N > 1: launch under torch.distributed.run; every rank runs the same per-GPU workload.)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDLA prefill TFLOP/s (% BF16 peak) at 32K; decode tok/s & KV GB/s vs HBM"
+PREFILL = dict(name="prefill_b1_t32768_causal", B=1, T=32768, window=0, seed=2)
+DECODE = dict(B=64, L=32768, cap=32769, seed=4, windows=(0, 2048))
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- work accounting
+def layer_dims():
+    from differential_latent_attention_fwd_b200.synth import GdlaShape
+    return GdlaShape()
+
+
+def valid_pairs(T: int, window: int) -> int:
+    if window <= 0 or window >= T:
+        return T * (T + 1) // 2
+    return window * (window + 1) // 2 + (T - window) * window
+
+
+def attn_flops_per_pair(s) -> int:
+    return s.n_heads * 2 * (s.d_qk + s.d_v)          # QK^T and PV over every head
+
+
+def proj_flops_per_token(s) -> int:
+    nqq = s.n_heads * s.d_qk
+    return 2 * (s.d_model * s.q_rank + s.d_model * (s.kv_rank + s.d_rope) + s.d_model * s.n_signal
+                + s.q_rank * nqq + s.q_rank * s.n_signal * s.d_v + s.kv_rank * s.n_kv_heads * (s.d_nope + s.d_v)
+                + s.n_signal * s.d_v * s.d_model)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured (MEASURED_PEAKS.json)"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons, n = [], [], set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            n += 1
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        loaded = [v for v in sm if v >= 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "samples": n,
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+def oracle_prefill_sample(inp, n_rows: int, seed: int):
+    """Time the fp64 oracle on n_rows query rows of the prefill workload (it still forms the
+    latent/K/V rows of every earlier token).  Returns (seconds, flops of the work done)."""
+    import numpy as np
+    from oracle import gdla_oracle as O
+    s = inp.shape
+    T = inp.x.shape[1]
+    rng = np.random.default_rng(seed)
+    rows = sorted(set(int(r) for r in rng.integers(0, T, n_rows)))
+    cfg = O.OracleConfig.from_shape(s)
+    t0 = time.perf_counter()
+    O.gdla_prefill(inp.x, inp.weights, cfg, rows=rows, g_q=inp.g_q, g_kv=inp.g_kv)
+    dt = time.perf_counter() - t0
+    t_hi = max(rows) + 1
+    kv_flops = 2 * t_hi * (s.d_model * (s.kv_rank + s.d_rope) + s.kv_rank * s.n_kv_heads * (s.d_nope + s.d_v))
+    row_flops = len(rows) * (proj_flops_per_token(s) - 2 * (s.d_model * (s.kv_rank + s.d_rope)
+                                                           + s.kv_rank * s.n_kv_heads * (s.d_nope + s.d_v)))
+    attn = sum(min(r + 1, s.window if s.window else r + 1) for r in rows) * attn_flops_per_pair(s)
+    return dt, kv_flops + row_flops + attn, rows
+
+
+def threads_used() -> int:
+    for v in ("OPENBLAS_NUM_THREADS", "OMP_NUM_THREADS"):
+        if os.environ.get(v, "").isdigit():
+            return int(os.environ[v])
+    return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The oracle, as it stands, on host cores: each step = a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from differential_latent_attention_fwd_b200 import synth
+    s = layer_dims()
+    inp = synth.make_prefill_inputs(s, PREFILL["B"], PREFILL["T"], PREFILL["seed"])
+    times, flops = [], []
+    for i in range(args.warmup + args.steps):
+        dt, fl, rows = oracle_prefill_sample(inp, 2, seed=100 + i)
+        if i >= args.warmup:
+            times.append(dt)
+            flops.append(fl)
+    tf = sum(flops) / sum(times) / 1e12
+    sample = (f"per step: 2 uniformly drawn query rows of {PREFILL['name']} (all 80 heads), "
+              "with the latent/K/V rows of every earlier token; fp64 numpy")
+    line = {"impl": "reference", "metric": METRIC, "value": tf, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PREFILL["name"], "B": PREFILL["B"], "seq_len": PREFILL["T"],
+                       "mask": "causal"},
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": threads_used(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from differential_latent_attention_fwd_b200 import binding as gb
+    from differential_latent_attention_fwd_b200 import synth
+    from differential_latent_attention_fwd_b200.layer import GdlaLayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+
+    s = layer_dims()
+    B, T = PREFILL["B"], args.T
+    inp = synth.make_prefill_inputs(s, B, T, PREFILL["seed"])
+    layer = GdlaLayer(s, inp.weights, inp.g_q, inp.g_kv, device=dev)
+    x_host = inp.x.pin_memory()
+    x = x_host.to(dev, non_blocking=True)
+    y = torch.empty_like(x)
+    ws = layer.workspace(B, T, gb.GDLA_MODE_PREFILL)
+    windows = () if args.skip_decode else DECODE["windows"]
+    dinp = synth.make_decode_inputs(synth.GdlaShape(), DECODE["B"], 1 if args.skip_decode else DECODE["L"],
+                                    2 if args.skip_decode else DECODE["cap"], DECODE["seed"])
+    cache = dinp.cache.to(dev)
+    lens = dinp.cache_len.to(dev)
+    x_new = dinp.x_new.to(dev)
+    y_new = torch.empty_like(x_new)
+    absorbed = layer.absorbed()
+    dcfg = {w: gb.make_config(s.with_window(w)) for w in (0, 2048)}
+    dws = torch.empty(gb.gdla_workspace_size(dcfg[0], DECODE["B"], 1, gb.GDLA_MODE_DECODE),
+                      dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+    pev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    dev_ev = {w: [torch.cuda.Event(enable_timing=True) for _ in range(5)] for w in windows}
+
+    def prefill_once():
+        gb.gdla_set_stage_events(pev)
+        gb.gdla_prefill_fwd(layer.cfg, layer.cw, x, y, ws, stream=stream)
+
+    def decode_once(w):
+        gb.gdla_set_stage_events(dev_ev[w])
+        gb.gdla_decode_fwd(dcfg[w], absorbed, x_new, cache, lens, y_new, dws, stream=stream)
+
+    def step():
+        flush.fill_(1)
+        prefill_once()
+        torch.cuda.synchronize(dev)
+        rec = {"prefill_ms": pev[0].elapsed_time(pev[5]), "attn_ms": pev[3].elapsed_time(pev[4]),
+               "down_ms": pev[0].elapsed_time(pev[1]), "norm_ms": pev[1].elapsed_time(pev[2]),
+               "up_ms": pev[2].elapsed_time(pev[3]), "out_ms": pev[4].elapsed_time(pev[5])}
+        for w in windows:
+            flush.fill_(1)
+            decode_once(w)
+            torch.cuda.synchronize(dev)
+            e = dev_ev[w]
+            rec[f"dec{w}_ms"] = e[0].elapsed_time(e[4])
+            rec[f"dec{w}_attn_ms"] = e[1].elapsed_time(e[2])
+            rec[f"dec{w}_q_ms"] = e[0].elapsed_time(e[1])
+            rec[f"dec{w}_comb_ms"] = e[2].elapsed_time(e[3])
+        return rec
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    assert gb.gdla_device_error(stream) == 0, "device error during warm-up"
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    barrier()
+    launches0 = gb.gdla_kernel_launches()
+    recs = []
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            recs.append(step())
+        barrier()
+    launches = gb.gdla_kernel_launches() - launches0
+    gb.gdla_set_stage_events([])
+    site = gb.gdla_device_error(stream)
+    assert site == 0, f"device error site {site:#x} in the timed region"
+
+    def mean(k):
+        return statistics.mean(r[k] for r in recs)
+
+    keys = list(recs[0].keys())
+    local_stats = torch.tensor([mean(k) for k in keys], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(local_stats, op=dist.ReduceOp.MAX)
+    st = dict(zip(keys, local_stats.tolist()))
+
+    # ---- end to end through the C ABI with host buffers (pinned H2D of x, D2H of y)
+    y_host = torch.empty_like(x_host).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for i in range(0 if args.skip_e2e else max(2, min(args.steps, 5)) + 1):
+        flush.fill_(1)
+        barrier()
+        e0.record(stream)
+        x.copy_(x_host, non_blocking=True)
+        gb.gdla_prefill_fwd(layer.cfg, layer.cw, x, y, ws, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if i > 0:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_t = torch.tensor([statistics.mean(e2e_ms) if e2e_ms else float("nan")], dtype=torch.float64,
+                         device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+
+    peaks, peak_src = load_peaks()
+    pairs = valid_pairs(T, 0)
+    attn_flop = B * pairs * attn_flops_per_pair(s)
+    layer_flop = attn_flop + B * T * proj_flops_per_token(s)
+    value = world * layer_flop / (st["prefill_ms"] * 1e-3) / 1e12
+    attn_tf = attn_flop / (st["attn_ms"] * 1e-3) / 1e12
+    e2e_val = world * layer_flop / (e2e_t.item() * 1e-3) / 1e12
+
+    decode = {}
+    for w in windows:
+        keys_read = DECODE["L"] + 1 if w == 0 else min(w, DECODE["L"] + 1)
+        kv_bytes = DECODE["B"] * keys_read * s.latent_row * 2
+        t_att = st[f"dec{w}_attn_ms"] * 1e-3
+        t_all = st[f"dec{w}_ms"] * 1e-3
+        decode["causal" if w == 0 else f"swa{w}"] = {
+            "B": DECODE["B"], "cache_len": DECODE["L"], "window": w,
+            "tok_per_s": world * DECODE["B"] / t_all, "ms": st[f"dec{w}_ms"],
+            "latent_attention_ms": st[f"dec{w}_attn_ms"], "query_path_ms": st[f"dec{w}_q_ms"],
+            "combine_ms": st[f"dec{w}_comb_ms"],
+            "kv_bytes": kv_bytes, "kv_gbs": kv_bytes / t_att / 1e9,
+            "kv_frac_of_hbm": kv_bytes / t_att / 1e9 / peaks["hbm_gbs"],
+        }
+
+    traffic = None
+    tf_path = os.path.join(ROOT, "profiles", "attn_prefill_t32768_causal.traffic.json")
+    try:
+        with open(tf_path) as f:
+            tr = json.load(f)
+        if tr.get("kernel_source_sha256") == kernel_source_digest():
+            traffic = tr.get("dram_bytes_per_launch")
+    except Exception:
+        traffic = None
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": st["prefill_ms"] + sum(
+            st[f"dec{w}_ms"] for w in windows),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": (f"prefill_b1_t{T}_causal" + ("" if args.skip_decode else
+                                " (+ decode_b64_l32768 causal and swa2048)")),
+                   "B": B, "seq_len": T, "mask": "causal", "d_model": s.d_model,
+                   "heads": f"{s.n_signal} signal + {s.n_noise} noise, {s.n_kv_heads} KV",
+                   "attn_operands": "fp16 (q, K^C, V, k^R, P); projections bf16; fp32 accumulate",
+                   "l2": "flushed (256 MiB write) before every timed call",
+                   "parallelism": f"replicas x{world}"},
+        "prefill": {"layer_ms": st["prefill_ms"], "attention_ms": st["attn_ms"],
+                    "down_proj_ms": st["down_ms"], "norm_rope_ms": st["norm_ms"],
+                    "up_proj_ms": st["up_ms"], "out_proj_ms": st["out_ms"],
+                    "layer_flop": layer_flop, "attention_flop": attn_flop,
+                    "attention_tflops": attn_tf, "tok_per_s": world * B * T / (st["prefill_ms"] * 1e-3),
+                    "layer_frac_of_bf16_peak": value / world / peaks["bf16_tflops_sustained"]},
+        "decode": decode,
+        "roofline": {"kernel": "attn_prefill_kernel", "bound": "tensor", "achieved": attn_tf,
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": attn_tf / peaks["bf16_tflops_sustained"],
+                     "frac_of_burst_peak": attn_tf / peaks["bf16_tflops"],
+                     "peak_source": peak_src + ", sustained bf16 (fp16 has the same dense rate)",
+                     "traffic": traffic},
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": x.numel() * 2,
+                "d2h_bytes_per_step": y.numel() * 2, "ms": e2e_t.item()},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, rows = oracle_prefill_sample(inp, 8, seed=7)
+        line["cpu_baseline"] = {
+            "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads_used(), "kind": "oracle",
+            "sample": f"{len(rows)} uniformly drawn query rows of {PREFILL['name']} (all 80 heads) "
+                      f"plus the latent/K/V rows of tokens 0..{max(rows)}; fp64 numpy; {dt:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("attn_prefill.cu", "gdla_common.cuh"):
+        with open(os.path.join(ROOT, "differential_latent_attention_fwd_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="gdla", choices=["gdla", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=PREFILL["T"], help="prefill length (profiling runs)")
+    ap.add_argument("--skip-decode", action="store_true", help="profiling runs: prefill only")
+    ap.add_argument("--skip-e2e", action="store_true", help="profiling runs: no host-buffer pass")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -71,19 +71,22 @@ def lib() -> ctypes.CDLL:
             "gdla_selftest_wait_timeout": [ULL, P, ctypes.POINTER(I)],
             "gdla_workspace_offset": [cfgp, I, I, I, I, ctypes.POINTER(SZ)],
             "gdla_status_string": [I],
+            "gdla_set_stage_events": [ctypes.POINTER(P), I],
+            "gdla_kernel_launches": [],
         }
         for name, args in sig.items():
             f = getattr(L, name)
             f.argtypes = args
-            f.restype = ctypes.c_char_p if name == "gdla_status_string" else I
+            f.restype = {"gdla_status_string": ctypes.c_char_p,
+                         "gdla_kernel_launches": ctypes.c_ulonglong}.get(name, I)
         _lib = L
     return _lib
 
 
 def header_functions() -> list:
     """Names of the entry points declared in include/gdla.h."""
-    src = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(gdla_\w+)\s*\(", src, re.M)))
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    return sorted(set(re.findall(r"\b(gdla_\w+)\s*\(", src)))
 
 
 def _check(fn: str, rc: int) -> None:
@@ -196,3 +199,16 @@ def gdla_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     if rc not in (0, -5):
         _check("gdla_selftest_wait_timeout", rc)
     return site.value
+
+
+def gdla_set_stage_events(events) -> None:
+    """events: list of torch.cuda.Event (created with enable_timing=True), or [] to disable."""
+    for e in events:            # torch creates the CUDA event on its first record
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * max(1, len(events)))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check("gdla_set_stage_events", lib().gdla_set_stage_events(arr, len(events)))
+
+
+def gdla_kernel_launches() -> int:
+    return int(lib().gdla_kernel_launches())
