@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "gdla_status_string": [I],
             "gdla_set_stage_events": [ctypes.POINTER(P), I],
             "gdla_kernel_launches": [],
+            "gdla_attn_prefill_noalloc": [cfgp, P, P, P, P, P, P, I, I, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -212,3 +213,17 @@ def gdla_set_stage_events(events) -> None:
 
 def gdla_kernel_launches() -> int:
     return int(lib().gdla_kernel_launches())
+
+
+GDLA_NOALLOC_MAX_TOKENS = 4096
+
+
+def gdla_attn_prefill_noalloc(cfg, qq: torch.Tensor, kv: torch.Tensor, kr16: torch.Tensor,
+                              lam: torch.Tensor, gate: torch.Tensor, dg: torch.Tensor, B: int, T: int,
+                              stream=None) -> None:
+    """Fused attention stage without a workspace (its scratch is a fixed array in the library)."""
+    _check("gdla_attn_prefill_noalloc", lib().gdla_attn_prefill_noalloc(
+        ctypes.byref(cfg), _ptr(qq, torch.float16, "qq"), _ptr(kv, torch.float16, "kv"),
+        _ptr(kr16, torch.float16, "kr16"), _ptr(lam, torch.float32, "lam"),
+        _ptr(gate, torch.bfloat16, "gate"), _ptr(dg, torch.bfloat16, "dg"), int(B), int(T),
+        _stream(stream)))

@@ -14,6 +14,18 @@ namespace gdla {
 __device__ int g_device_error = 0;
 
 static unsigned long long g_wait_limit_ns = 2000000000ull;
+static cudaEvent_t g_stage_ev[8];
+static int g_n_stage_ev = 0;
+static unsigned long long g_launches = 0;
+
+static void stage(int i, cudaStream_t st) {
+  if (i < g_n_stage_ev) cudaEventRecord(g_stage_ev[i], st);
+}
+// Every launch_* helper enqueues exactly one kernel; returns true on failure.
+static bool launch_failed(int rc) {
+  if (rc == 0) ++g_launches;
+  return rc != 0;
+}
 static const uint32_t kAbsorbedMagic = 0x47444C41u;  // "GDLA"
 
 static int error_word(int** out) {
@@ -86,6 +98,16 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
     o += (sz[i] + 255) & ~size_t(255);
   }
   off[WS_N] = o;
+}
+
+// Shared with the other translation units of the library (same error word, same bound).
+int shared_kernel_ctl(KernelCtlHost* out) {
+  int* err;
+  const int rc = error_word(&err);
+  if (rc) return rc;
+  out->err = err;
+  out->limit_ns = g_wait_limit_ns;
+  return GDLA_OK;
 }
 
 }  // namespace gdla
@@ -179,61 +201,67 @@ int gdla_prefill_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const vo
   fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
 
   // a1: [x W_aQ | x W_aKV | x W_lambda] in fp32
+  stage(0, st);
   GemmEpi ep{};
   ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = M; ep.rope_lo = ep.rope_hi = 0; ep.pos_T = T;
   ep.rope = rope;
   ep.C = D1; ep.N = cfg->q_rank;
-  if (launch_gemm(x, cfg->d_model, w->W_aQ, cfg->q_rank, false, M, cfg->q_rank, cfg->d_model, ep, ctl, st))
+  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_aQ, cfg->q_rank, false, M, cfg->q_rank, cfg->d_model, ep, ctl, st)))
     return GDLA_ERR_LAUNCH;
   ep.C = D1 + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
-  if (launch_gemm(x, cfg->d_model, w->W_aKV, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st))
+  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_aKV, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
     return GDLA_ERR_LAUNCH;
   ep.C = D1 + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
-  if (launch_gemm(x, cfg->d_model, w->W_lambda, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st))
+  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_lambda, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
     return GDLA_ERR_LAUNCH;
 
+  stage(1, st);
   // a2: norms, rotary key, lambda, latent rows
   NormParams np{};
   np.D1 = D1; np.ld1 = ld1; np.M = M; np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank;
   np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
   np.cQ = cQ; np.latent = latent; np.kR16 = kR16; np.lam = lam; np.pos_T = T; np.pos_ptr = nullptr;
   np.cache = kv_cache_out; np.cache_cap = cache_cap; np.rope = rope; np.err = err;
-  if (launch_norm_rope(np, st)) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
 
+  stage(2, st);
   // a3: up-projections (q^C | rotated q^R), gate logits, K^C | V
   const int nqq = nH * (cfg->d_nope + cfg->d_rope);
   GemmEpi eq{};
   eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F16; eq.M = M; eq.N = nqq;
   eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = T; eq.rope = rope;
-  if (launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, M, nqq, cfg->q_rank, eq, ctl, st))
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, M, nqq, cfg->q_rank, eq, ctl, st)))
     return GDLA_ERR_LAUNCH;
   GemmEpi eg{};
   eg.C = G; eg.ldc = cfg->n_signal * cfg->d_v; eg.out_type = OUT_BF16; eg.M = M; eg.N = eg.ldc;
   eg.pos_T = T;
-  if (launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, M, eg.N, cfg->q_rank, eg, ctl, st))
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, M, eg.N, cfg->q_rank, eg, ctl, st)))
     return GDLA_ERR_LAUNCH;
   GemmEpi ekv{};
   const int nkv = cfg->n_kv_heads * (cfg->d_nope + cfg->d_v);
   ekv.C = KV; ekv.ldc = nkv; ekv.out_type = OUT_F16; ekv.M = M; ekv.N = nkv; ekv.pos_T = T;
-  if (launch_gemm(latent, cfg->kv_rank + cfg->d_rope, w->W_bKV, nkv, false, M, nkv, cfg->kv_rank,
-                  ekv, ctl, st))
+  if (launch_failed(launch_gemm(latent, cfg->kv_rank + cfg->d_rope, w->W_bKV, nkv, false, M, nkv, cfg->kv_rank,
+                  ekv, ctl, st)))
     return GDLA_ERR_LAUNCH;
 
+  stage(3, st);
   // a4: fused attention + differential combine + gate
   AttnParams ap{};
   ap.B = B; ap.T = T; ap.window = cfg->window; ap.n_groups = cfg->n_noise;
   ap.n_signal = cfg->n_signal; ap.rope_col0 = nH * cfg->d_nope;
   ap.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
   ap.lam = lam; ap.G = G; ap.O_noise = On; ap.Dg = Dg;
-  if (launch_attn_prefill(QQ, nqq, KV, kR16, ap, ctl, st)) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_attn_prefill(QQ, nqq, KV, kR16, ap, ctl, st))) return GDLA_ERR_LAUNCH;
 
+  stage(4, st);
   // a5: output projection
   GemmEpi eo{};
   eo.C = y; eo.ldc = cfg->d_model; eo.out_type = OUT_BF16; eo.M = M; eo.N = cfg->d_model;
   eo.pos_T = T;
-  if (launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, M, cfg->d_model,
-                  cfg->n_signal * cfg->d_v, eo, ctl, st))
+  if (launch_failed(launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, M, cfg->d_model,
+                  cfg->n_signal * cfg->d_v, eo, ctl, st)))
     return GDLA_ERR_LAUNCH;
+  stage(5, st);
   return GDLA_OK;
 }
 
@@ -246,8 +274,8 @@ int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void*
   size_t need;
   gdla_absorbed_size(cfg, &need);
   if (dst_bytes < need) return GDLA_ERR_WORKSPACE_TOO_SMALL;
-  if (launch_absorb_uk(w->W_bKV, dst, cfg->kv_rank, cfg->n_kv_heads, cfg->d_nope, cfg->d_v,
-                       static_cast<cudaStream_t>(stream)))
+  if (launch_failed(launch_absorb_uk(w->W_bKV, dst, cfg->kv_rank, cfg->n_kv_heads, cfg->d_nope, cfg->d_v,
+                       static_cast<cudaStream_t>(stream))))
     return GDLA_ERR_LAUNCH;
   out->w = *w;
   out->W_UKt = dst;
@@ -293,16 +321,17 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   RopeTable rope;
   fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
 
+  stage(0, st);
   GemmEpi ep{};
   ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = B; ep.pos_T = 1; ep.rope = rope;
   ep.C = D1; ep.N = cfg->q_rank;
-  if (launch_gemm(x_new, cfg->d_model, w->W_aQ, cfg->q_rank, false, B, ep.N, cfg->d_model, ep, ctl, st))
+  if (launch_failed(launch_gemm(x_new, cfg->d_model, w->W_aQ, cfg->q_rank, false, B, ep.N, cfg->d_model, ep, ctl, st)))
     return GDLA_ERR_LAUNCH;
   ep.C = D1 + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
-  if (launch_gemm(x_new, cfg->d_model, w->W_aKV, ep.N, false, B, ep.N, cfg->d_model, ep, ctl, st))
+  if (launch_failed(launch_gemm(x_new, cfg->d_model, w->W_aKV, ep.N, false, B, ep.N, cfg->d_model, ep, ctl, st)))
     return GDLA_ERR_LAUNCH;
   ep.C = D1 + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
-  if (launch_gemm(x_new, cfg->d_model, w->W_lambda, ep.N, false, B, ep.N, cfg->d_model, ep, ctl, st))
+  if (launch_failed(launch_gemm(x_new, cfg->d_model, w->W_lambda, ep.N, false, B, ep.N, cfg->d_model, ep, ctl, st)))
     return GDLA_ERR_LAUNCH;
 
   NormParams np{};
@@ -310,47 +339,63 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
   np.cQ = cQ; np.latent = nullptr; np.kR16 = nullptr; np.lam = lam; np.pos_T = 1;
   np.pos_ptr = cache_len; np.cache = kv_cache; np.cache_cap = cap; np.rope = rope; np.err = err;
-  if (launch_norm_rope(np, st)) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
 
   const int nqq = nH * (cfg->d_nope + cfg->d_rope);
   GemmEpi eq{};
   eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F32; eq.M = B; eq.N = nqq;
   eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = 1; eq.pos_ptr = cache_len;
   eq.rope = rope;
-  if (launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, B, nqq, cfg->q_rank, eq, ctl, st))
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, B, nqq, cfg->q_rank, eq, ctl, st)))
     return GDLA_ERR_LAUNCH;
   GemmEpi eg{};
   eg.C = G; eg.ldc = cfg->n_signal * cfg->d_v; eg.out_type = OUT_BF16; eg.M = B; eg.N = eg.ldc;
   eg.pos_T = 1;
-  if (launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, B, eg.N, cfg->q_rank, eg, ctl, st))
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, B, eg.N, cfg->q_rank, eg, ctl, st)))
     return GDLA_ERR_LAUNCH;
 
   DecQParams qp{};
   qp.B = B; qp.n_groups = cfg->n_noise; qp.n_signal = cfg->n_signal; qp.n_heads = nH;
   qp.QQ = QQ; qp.qq_ld = nqq; qp.rope_col0 = nH * cfg->d_nope; qp.W_UKt = ab->W_UKt; qp.qt = qt;
-  if (launch_qtilde(qp, st)) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_qtilde(qp, st))) return GDLA_ERR_LAUNCH;
 
+  stage(1, st);
   DecAttnParams dp{};
   dp.B = B; dp.cap = cap; dp.window = cfg->window; dp.n_split = nsplit; dp.cache_len = cache_len;
   dp.cache = kv_cache; dp.qt = qt;
   dp.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
   dp.part = part; dp.ml = ml; dp.err = err;
   if (nH != 80) return GDLA_ERR_UNSUPPORTED_SHAPE;
-  if (launch_dec_attn_simt(dp, st)) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_dec_attn_simt(dp, st))) return GDLA_ERR_LAUNCH;
 
+  stage(2, st);
   DecCombParams cp{};
   cp.B = B; cp.n_groups = cfg->n_noise; cp.n_signal = cfg->n_signal; cp.n_split = nsplit;
   cp.part = part; cp.ml = ml; cp.lam = lam; cp.G = G; cp.W_bKV = w->W_bKV; cp.Dg = Dg;
-  if (launch_dec_combine(cp, st)) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_dec_combine(cp, st))) return GDLA_ERR_LAUNCH;
 
+  stage(3, st);
   GemmEpi eo{};
   eo.C = y; eo.ldc = cfg->d_model; eo.out_type = OUT_BF16; eo.M = B; eo.N = cfg->d_model;
   eo.pos_T = 1;
-  if (launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, B, cfg->d_model,
-                  cfg->n_signal * cfg->d_v, eo, ctl, st))
+  if (launch_failed(launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, B, cfg->d_model,
+                  cfg->n_signal * cfg->d_v, eo, ctl, st)))
     return GDLA_ERR_LAUNCH;
+  stage(4, st);
   return GDLA_OK;
 }
+
+int gdla_set_stage_events(void* const* events, int n) {
+  if (n < 0 || n > 8 || (n > 0 && !events)) return GDLA_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    if (!events[i]) return GDLA_ERR_INVALID_ARG;
+    g_stage_ev[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_n_stage_ev = n;
+  return GDLA_OK;
+}
+
+unsigned long long gdla_kernel_launches(void) { return g_launches; }
 
 int gdla_device_error(void* stream, int* site, int clear) {
   if (!site) return GDLA_ERR_INVALID_ARG;
@@ -393,5 +438,6 @@ extern "C" int gdla_selftest_wait_timeout(unsigned long long limit_ns, void* str
   if (prev) return GDLA_ERR_DEVICE_TIMEOUT;  // an earlier failure is still unread
   selftest_wait_kernel<<<1, 32, 0, st>>>(kc);
   if (cudaPeekAtLastError() != cudaSuccess) return GDLA_ERR_LAUNCH;
+  ++g_launches;
   return gdla_device_error(stream, site, 1);
 }

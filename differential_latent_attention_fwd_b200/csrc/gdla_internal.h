@@ -46,6 +46,9 @@ int launch_gemm(const void* A, long long lda, const void* B, long long ldb, bool
 
 void fill_rope_table(RopeTable* t, int d_rope, double theta);
 
+// Device error word and current wait bound used by every launch of the library.
+int shared_kernel_ctl(KernelCtlHost* out);
+
 // Row-wise epilogue of the down-projection (norms, rotary key, lambda, latent-cache rows).
 struct NormParams {
   const float* D1;            // [M, ld1] fp32: x W_a^Q | x W_a^KV | x W^lambda

@@ -144,6 +144,44 @@ int gdla_workspace_offset(const gdla_config_t* cfg, int B, int T, int mode, int 
 
 const char* gdla_status_string(int status);
 
+/* Optional timing hook (process-wide, not thread-safe).  When n > 0, every subsequent call
+ * records the caller-created cudaEvent_t handles events[0..n-1] on its stream at stage
+ * boundaries:
+ *   gdla_prefill_fwd: [0] before the down-projection, [1] after it, [2] after the norm/RoPE
+ *     kernel, [3] after the up-projections, [4] after the fused attention, [5] after W^O;
+ *   gdla_decode_fwd:  [0] start, [1] after the query path (projections, norms, q~),
+ *     [2] after the latent attention, [3] after the split merge + combine, [4] after W^O.
+ * n = 0 disables it.  At most 8 events. */
+int gdla_set_stage_events(void* const* events, int n);
+
+/* Number of kernels this library has launched in this process (all devices). */
+unsigned long long gdla_kernel_launches(void);
+
+/* ---- Allocation-free attention stage.  The paper has no counterpart: this is a convenience
+ * for callers that cannot allocate device memory when they run (an engine plugin that is
+ * handed only its input and output buffers, a service that fixes its footprint at start-up).
+ *
+ * gdla_attn_prefill_noalloc runs the fused attention stage of gdla_prefill_fwd (softmax
+ * attention of every signal and noise head, lambda subtraction, sigmoid gate) on
+ * caller-provided inputs and output, and keeps its only scratch -- the noise-head outputs --
+ * in a fixed 32 MiB device array inside the library (present on every GPU that loads the
+ * library, until exit).  It calls no allocator.
+ *   qq   fp16 [B*T, n_H*(d_nope+d_rope)]: q^C of every head, then rotated q^R of every head
+ *   kv   fp16 [B*T, n_kv_heads*(d_nope+d_v)]: per KV head K^C then V
+ *   kr16 fp16 [B*T, d_rope]: rotated shared rope key
+ *   lam  fp32 [B*T, n_signal]; gate bf16 [B*T, n_signal*d_v] (logits G)
+ *   dg   bf16 [B*T, n_signal*d_v] (written): sigmoid(G) (.) (H_S - lambda H_N)
+ * (the same tensors gdla_prefill_fwd keeps in its workspace, slots 4, 6, 9, 3, 5 and 8 of
+ * gdla_workspace_offset).  B*T must not exceed GDLA_NOALLOC_MAX_TOKENS, else
+ * GDLA_ERR_WORKSPACE_TOO_SMALL.  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first call before any
+ * stream capture.  All calls share the one array: calls that overlap on the GPU (other
+ * streams, other threads) race and must be serialised by the caller. */
+#define GDLA_NOALLOC_MAX_TOKENS 4096
+int gdla_attn_prefill_noalloc(const gdla_config_t* cfg, const void* qq, const void* kv,
+                              const void* kr16, const float* lam, const void* gate, void* dg,
+                              int B, int T, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
