@@ -211,15 +211,16 @@ def run_gpu(args):
     y = torch.empty_like(x)
     ws = layer.workspace(B, T, gb.GDLA_MODE_PREFILL)
     windows = () if args.skip_decode else DECODE["windows"]
-    dinp = synth.make_decode_inputs(synth.GdlaShape(), DECODE["B"], 1 if args.skip_decode else DECODE["L"],
-                                    2 if args.skip_decode else DECODE["cap"], DECODE["seed"])
+    dec_L = 1 if args.skip_decode else args.decode_L
+    dinp = synth.make_decode_inputs(synth.GdlaShape(), DECODE["B"], dec_L, dec_L + 1, DECODE["seed"])
     cache = dinp.cache.to(dev)
     lens = dinp.cache_len.to(dev)
     x_new = dinp.x_new.to(dev)
     y_new = torch.empty_like(x_new)
     absorbed = layer.absorbed()
     dcfg = {w: gb.make_config(s.with_window(w)) for w in (0, 2048)}
-    dws = torch.empty(gb.gdla_workspace_size(dcfg[0], DECODE["B"], 1, gb.GDLA_MODE_DECODE),
+    dws = torch.empty(max(gb.gdla_workspace_size(dcfg[w], DECODE["B"], cache.shape[1],
+                                                 gb.GDLA_MODE_DECODE) for w in (0, 2048)),
                       dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
@@ -312,12 +313,12 @@ def run_gpu(args):
 
     decode = {}
     for w in windows:
-        keys_read = DECODE["L"] + 1 if w == 0 else min(w, DECODE["L"] + 1)
+        keys_read = dec_L + 1 if w == 0 else min(w, dec_L + 1)
         kv_bytes = DECODE["B"] * keys_read * s.latent_row * 2
         t_att = st[f"dec{w}_attn_ms"] * 1e-3
         t_all = st[f"dec{w}_ms"] * 1e-3
         decode["causal" if w == 0 else f"swa{w}"] = {
-            "B": DECODE["B"], "cache_len": DECODE["L"], "window": w,
+            "B": DECODE["B"], "cache_len": dec_L, "window": w,
             "tok_per_s": world * DECODE["B"] / t_all, "ms": st[f"dec{w}_ms"],
             "latent_attention_ms": st[f"dec{w}_attn_ms"], "query_path_ms": st[f"dec{w}_q_ms"],
             "combine_ms": st[f"dec{w}_comb_ms"],
@@ -393,13 +394,14 @@ def kernel_source_digest() -> str:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="gdla", choices=["gdla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=PREFILL["T"], help="prefill length (profiling runs)")
     ap.add_argument("--skip-decode", action="store_true", help="profiling runs: prefill only")
     ap.add_argument("--skip-e2e", action="store_true", help="profiling runs: no host-buffer pass")
+    ap.add_argument("--decode-L", type=int, default=DECODE["L"], help="cached positions (profiling runs)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

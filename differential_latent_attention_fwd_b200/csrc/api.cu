@@ -62,10 +62,6 @@ static int check_weights(const gdla_weights_t* w) {
 // ---------------------------------------------------------------- workspace layout
 enum { WS_D1, WS_CQ, WS_LATENT, WS_LAM, WS_QQ, WS_G, WS_KV, WS_ONOISE, WS_DG, WS_KR16, WS_N };
 
-static int decode_splits(int B) {
-  int s = (2 * 148 + B - 1) / B;
-  return s < 1 ? 1 : (s > 64 ? 64 : s);
-}
 
 static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS_N + 1]) {
   const long long M = mode == GDLA_MODE_PREFILL ? (long long)B * T : (long long)B;
@@ -85,7 +81,7 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
     sz[WS_ONOISE] = M * (long long)c->n_noise * c->d_v * 4;
     sz[WS_KR16] = M * c->d_rope * 2;
   } else {
-    const int ns = decode_splits(B);
+    const int ns = decode_split_count(B, T, c->window);   // T = cache capacity in decode mode
     sz[WS_LATENT] = 0;
     sz[WS_QQ] = M * qq * 4;                                          // fp32 q^C | q^R
     sz[WS_KV] = M * (long long)nH * (c->kv_rank + c->d_rope) * 2;    // q~ rows
@@ -299,7 +295,7 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   if (!aligned16(x_new) || !aligned16(kv_cache) || !aligned16(y) || !aligned16(workspace))
     return GDLA_ERR_INVALID_ARG;
   size_t off[WS_N + 1];
-  layout(cfg, B, 1, GDLA_MODE_DECODE, off);
+  layout(cfg, B, cap, GDLA_MODE_DECODE, off);
   if (ws_bytes < off[WS_N]) return GDLA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int* err;
@@ -317,7 +313,7 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   void* Dg = ws + off[WS_DG];
   const int nH = cfg->n_signal + cfg->n_noise;
   const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
-  const int nsplit = decode_splits(B);
+  const int nsplit = decode_split_count(B, cap, cfg->window);
   RopeTable rope;
   fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
 
@@ -366,7 +362,7 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   dp.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
   dp.part = part; dp.ml = ml; dp.err = err;
   if (nH != 80) return GDLA_ERR_UNSUPPORTED_SHAPE;
-  if (launch_failed(launch_dec_attn_simt(dp, st))) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_dec_attn_tc(dp, ctl, st))) return GDLA_ERR_LAUNCH;
 
   stage(2, st);
   DecCombParams cp{};

@@ -11,8 +11,9 @@
 //   Dg_s   = sigmoid(G_s) (.) D_s
 // so every cached byte (c_bar | k^R, 1152 bytes per position) is read once for all 80 heads.
 //
-// Kernels here: W_UK transpose (weight absorption), q~ formation, split-K latent attention
-// with per-split partial (max, sum, latent accumulator), and the split merge + combine + gate.
+// Kernels here: W_UK transpose (weight absorption), q~ formation, and the split merge +
+// latent differential combine + W_UV up-projection + gate.  The split-K latent attention
+// itself is the tensor-core kernel in decode_tc.cu.
 #include "gdla_common.cuh"
 #include "gdla_internal.h"
 #include "gdla_decode.h"
@@ -76,127 +77,6 @@ int launch_qtilde(const DecQParams& p, cudaStream_t st) {
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
-// ---------------------------------------------------------------- split-K latent attention
-// CUDA-core reference kernel: CTA (split, b) walks 64-position chunks of its key range.
-namespace dec {
-constexpr int CH = 64;            // positions per chunk
-constexpr int RW = 289;           // padded row stride in 32-bit words (576 bf16 = 288 words)
-constexpr int NH = 80;
-constexpr int SMEM = (NH * RW + CH * RW) * 4 + NH * CH * 4 + NH * 4 * 3;
-}  // namespace dec
-
-__global__ void __launch_bounds__(256, 1) dec_attn_simt_kernel(DecAttnParams p) {
-  using namespace dec;
-  extern __shared__ uint32_t sm[];
-  uint32_t* q_s = sm;                  // [80][RW] bf16x2
-  uint32_t* c_s = q_s + NH * RW;       // [64][RW]
-  float* sc = reinterpret_cast<float*>(c_s + CH * RW);   // [80][64]
-  float* m_s = sc + NH * CH;
-  float* l_s = m_s + NH;
-  float* a_s = l_s + NH;
-  const int sp = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  int L = p.cache_len[b];                        // keys 0..L (L cached + the new token)
-  if (L < 0 || L >= p.cap) {                     // reported; the sequence reads nothing
-    if (tid == 0) atomicCAS(p.err, 0, SITE_BAD_CACHE_LEN);
-    L = -1;
-  }
-  const int lo_all = p.window > 0 ? max(0, L - p.window + 1) : 0;
-  const int n_all = L - lo_all + 1;
-  const int per = (n_all + p.n_split - 1) / p.n_split;
-  const int lo = lo_all + sp * per;
-  const int hi = min(L, lo + per - 1);
-  const uint32_t* qsrc = reinterpret_cast<const uint32_t*>(p.qt) + (long long)b * NH * 288;
-  for (int i = tid; i < NH * 288; i += blockDim.x) q_s[(i / 288) * RW + i % 288] = qsrc[i];
-  if (tid < NH) {
-    m_s[tid] = -INFINITY;
-    l_s[tid] = 0.f;
-  }
-  float acc[NH][2];
-#pragma unroll
-  for (int h = 0; h < NH; ++h) acc[h][0] = acc[h][1] = 0.f;
-  const uint32_t* cache = reinterpret_cast<const uint32_t*>(p.cache) + (long long)b * p.cap * 288;
-  __syncthreads();
-  for (int p0 = lo; p0 <= hi; p0 += CH) {
-    const int np = min(CH, hi - p0 + 1);
-    for (int i = tid; i < CH * 72; i += blockDim.x) {   // 72 uint4 per row
-      const int r = i / 72, w4 = i % 72;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < np) v = reinterpret_cast<const uint4*>(cache + (long long)(p0 + r) * 288)[w4];
-      uint32_t* d = c_s + r * RW + w4 * 4;
-      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
-    }
-    __syncthreads();
-    for (int idx = tid; idx < NH * CH; idx += blockDim.x) {
-      const int h = idx / CH, r = idx % CH;
-      float s = -INFINITY;
-      if (r < np) {
-        const uint32_t* qa = q_s + h * RW;
-        const uint32_t* ca = c_s + r * RW;
-        float a0 = 0.f, a1 = 0.f;
-        for (int w = 0; w < 288; ++w) {
-          const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(qa + w);
-          const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(ca + w);
-          a0 = fmaf(__low2float(x), __low2float(y), a0);
-          a1 = fmaf(__high2float(x), __high2float(y), a1);
-        }
-        s = (a0 + a1) * p.scale_log2;
-      }
-      sc[h * CH + r] = s;
-    }
-    __syncthreads();
-    if (tid < NH) {
-      float mx = m_s[tid];
-      for (int r = 0; r < np; ++r) mx = fmaxf(mx, sc[tid * CH + r]);
-      const float alpha = ex2_approx(m_s[tid] - mx);  // m_s = -inf first: 0
-      float l = l_s[tid] * alpha;
-      for (int r = 0; r < CH; ++r) {
-        const float e = r < np ? ex2_approx(sc[tid * CH + r] - mx) : 0.f;
-        sc[tid * CH + r] = e;
-        l += e;
-      }
-      m_s[tid] = mx;
-      l_s[tid] = l;
-      a_s[tid] = alpha;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < NH; ++h) {
-      acc[h][0] *= a_s[h];
-      acc[h][1] *= a_s[h];
-    }
-    for (int r = 0; r < np; ++r) {
-      const __nv_bfloat162 cv = *reinterpret_cast<const __nv_bfloat162*>(c_s + r * RW + tid);
-      const float c0 = __low2float(cv), c1 = __high2float(cv);
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        const float pr = sc[h * CH + r];
-        acc[h][0] = fmaf(pr, c0, acc[h][0]);
-        acc[h][1] = fmaf(pr, c1, acc[h][1]);
-      }
-    }
-    __syncthreads();
-  }
-  // partial results: latent accumulator (relative to m), and (m, l) per head
-  float* part = p.part + ((long long)b * p.n_split + sp) * NH * 512;
-#pragma unroll
-  for (int h = 0; h < NH; ++h)
-    *reinterpret_cast<float2*>(part + h * 512 + 2 * tid) = make_float2(acc[h][0], acc[h][1]);
-  if (tid < NH) {
-    float* ml = p.ml + (((long long)b * p.n_split + sp) * NH + tid) * 2;
-    ml[0] = m_s[tid];
-    ml[1] = l_s[tid];
-  }
-}
-
-int launch_dec_attn_simt(const DecAttnParams& p, cudaStream_t st) {
-  if (cudaFuncSetAttribute(dec_attn_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dec::SMEM) != cudaSuccess)
-    return -4;
-  dim3 grid(p.n_split, p.B);
-  dec_attn_simt_kernel<<<grid, 256, dec::SMEM, st>>>(p);
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
-}
-
 // ---------------------------------------------------------------- split merge + combine + gate
 // CTA (b, j): merges the splits of the group's 5 heads, forms the latent differential
 // l_s - lambda_s l_noise for its 4 signal heads, up-projects with W_UV_j and applies the gate.
@@ -225,8 +105,11 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
   for (int i = tid; i < 5 * 512; i += blockDim.x) {
     const int hh = i / 512, l = i % 512;
     float a = 0.f;
-    for (int sp = 0; sp < p.n_split; ++sp)
-      a += wsp[sp][hh] * p.part[(((long long)b * p.n_split + sp) * NH + heads[hh]) * 512 + l];
+    for (int sp = 0; sp < p.n_split; ++sp) {
+      const float w = wsp[sp][hh];
+      if (w != 0.f)  // empty splits write no partial
+        a += w * p.part[(((long long)b * p.n_split + sp) * NH + heads[hh]) * 512 + l];
+    }
     lat[hh][l] = a * inv_L[hh];
   }
   __syncthreads();

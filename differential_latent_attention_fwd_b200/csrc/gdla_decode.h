@@ -3,6 +3,8 @@
 
 #include <cuda_runtime.h>
 
+#include "gdla_internal.h"
+
 namespace gdla {
 
 struct DecQParams {
@@ -37,7 +39,8 @@ struct DecCombParams {
 int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int d_nope, int d_v,
                      cudaStream_t st);
 int launch_qtilde(const DecQParams& p, cudaStream_t st);
-int launch_dec_attn_simt(const DecAttnParams& p, cudaStream_t st);
+int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t st);
+int decode_split_count(int B, int cap, int window);
 int launch_dec_combine(const DecCombParams& p, cudaStream_t st);
 
 }  // namespace gdla

@@ -53,6 +53,6 @@ class GdlaLayer:
         B, d = x_new.shape
         if y is None:
             y = torch.empty((B, d), dtype=torch.bfloat16, device=self.device)
-        ws = self.workspace(B, 1, gb.GDLA_MODE_DECODE)
+        ws = self.workspace(B, kv_cache.shape[1], gb.GDLA_MODE_DECODE)
         gb.gdla_decode_fwd(self.cfg, self.absorbed(stream), x_new, kv_cache, cache_len, y, ws, stream)
         return y

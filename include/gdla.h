@@ -90,7 +90,7 @@ typedef struct {
 enum { GDLA_MODE_PREFILL = 0, GDLA_MODE_DECODE = 1 };
 
 /* Bytes of workspace that gdla_prefill_fwd (mode 0: B sequences of T tokens) or
- * gdla_decode_fwd (mode 1: B sequences; T ignored) needs. */
+ * gdla_decode_fwd (mode 1: B sequences, T = the cache capacity `cap` of the call) needs. */
 int gdla_workspace_size(const gdla_config_t* cfg, int B, int T, int mode, size_t* bytes);
 
 /* Bytes of device memory gdla_absorb_weights writes. */
@@ -118,7 +118,10 @@ int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void*
  *   x_new [B, d_model] bf16.  kv_cache [B, cap, kv_rank + d_rope] bf16: rows 0..len[b]-1 hold
  *   the cached latent entries; the new token's entry is written at row len[b] (so
  *   len[b] < cap) and it attends to rows 0..len[b] (or the last `window` of them).
- *   cache_len [B] int32 (device).  y [B, d_model] bf16 (written). */
+ *   Rows after len[b] up to the end of its 128-row block are read (and multiplied by zero
+ *   weights), so they must hold finite values, e.g. a zero-initialised cache.
+ *   cache_len [B] int32 (device).  y [B, d_model] bf16 (written).
+ *   workspace: >= gdla_workspace_size(cfg, B, cap, GDLA_MODE_DECODE) bytes. */
 int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* absorbed, const void* x_new,
                     void* kv_cache, const int* cache_len, int cap, int B, void* y,
                     void* workspace, size_t ws_bytes, void* stream);
