@@ -231,31 +231,76 @@ def run_gpu(args):
         gb.gdla_set_stage_events(pev)
         gb.gdla_prefill_fwd(layer.cfg, layer.cw, x, y, ws, stream=stream)
 
-    def decode_once(w):
+    def decode_once(w, s=None):
         gb.gdla_set_stage_events(dev_ev[w])
-        gb.gdla_decode_fwd(dcfg[w], absorbed, x_new, cache, lens, y_new, dws, stream=stream)
+        gb.gdla_decode_fwd(dcfg[w], absorbed, x_new, cache, lens, y_new, dws,
+                           stream=stream if s is None else s)
+
+    # A decode step is ~20 short kernels: it is replayed as a CUDA graph (one capture per mask),
+    # as a serving loop would run it; the eager time is reported beside it.
+    graphs = {}
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     def step():
-        flush.fill_(1)
-        prefill_once()
-        torch.cuda.synchronize(dev)
-        rec = {"prefill_ms": pev[0].elapsed_time(pev[5]), "attn_ms": pev[3].elapsed_time(pev[4]),
-               "down_ms": pev[0].elapsed_time(pev[1]), "norm_ms": pev[1].elapsed_time(pev[2]),
-               "up_ms": pev[2].elapsed_time(pev[3]), "out_ms": pev[4].elapsed_time(pev[5])}
+        rec = {"prefill_ms": 0.0, "attn_ms": float("nan"), "down_ms": 0.0, "norm_ms": 0.0,
+               "up_ms": 0.0, "out_ms": 0.0}
+        if not args.skip_prefill:
+            flush.fill_(1)
+            prefill_once()
+            torch.cuda.synchronize(dev)
+            rec = {"prefill_ms": pev[0].elapsed_time(pev[5]), "attn_ms": pev[3].elapsed_time(pev[4]),
+                   "down_ms": pev[0].elapsed_time(pev[1]), "norm_ms": pev[1].elapsed_time(pev[2]),
+                   "up_ms": pev[2].elapsed_time(pev[3]), "out_ms": pev[4].elapsed_time(pev[5])}
         for w in windows:
             flush.fill_(1)
-            decode_once(w)
-            torch.cuda.synchronize(dev)
-            e = dev_ev[w]
-            rec[f"dec{w}_ms"] = e[0].elapsed_time(e[4])
-            rec[f"dec{w}_attn_ms"] = e[1].elapsed_time(e[2])
-            rec[f"dec{w}_q_ms"] = e[0].elapsed_time(e[1])
-            rec[f"dec{w}_comb_ms"] = e[2].elapsed_time(e[3])
+            if w in graphs:          # whole decode step as one graph: events around the replay
+                g0.record(stream)
+                graphs[w].replay()
+                g1.record(stream)
+                torch.cuda.synchronize(dev)
+                rec[f"dec{w}_ms"] = g0.elapsed_time(g1)
+            else:                    # eager call: per-stage events from inside the library
+                decode_once(w)
+                torch.cuda.synchronize(dev)
+                e = dev_ev[w]
+                rec[f"dec{w}_ms"] = e[0].elapsed_time(e[4])
+                rec[f"dec{w}_attn_ms"] = e[1].elapsed_time(e[2])
+                rec[f"dec{w}_q_ms"] = e[0].elapsed_time(e[1])
+                rec[f"dec{w}_comb_ms"] = e[2].elapsed_time(e[3])
         return rec
 
     for _ in range(max(3, args.warmup)):
         step()
     assert gb.gdla_device_error(stream) == 0, "device error during warm-up"
+    eager_dec = {w: [] for w in windows}
+    eager_stage = {w: {"attn": [], "q": [], "comb": []} for w in windows}
+    kernels_per_decode = {}
+    for _ in range(5):
+        for w in windows:
+            flush.fill_(1)
+            n0 = gb.gdla_kernel_launches()
+            decode_once(w)
+            kernels_per_decode[w] = gb.gdla_kernel_launches() - n0
+            torch.cuda.synchronize(dev)
+            e = dev_ev[w]
+            eager_dec[w].append(e[0].elapsed_time(e[4]))
+            eager_stage[w]["attn"].append(e[1].elapsed_time(e[2]))
+            eager_stage[w]["q"].append(e[0].elapsed_time(e[1]))
+            eager_stage[w]["comb"].append(e[2].elapsed_time(e[3]))
+    gb.gdla_set_stage_events([])     # no event nodes inside the captured graphs
+    for w in windows:
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(dev)
+        cs.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(cs):
+            with torch.cuda.graph(g, stream=cs):
+                gb.gdla_decode_fwd(dcfg[w], absorbed, x_new, cache, lens, y_new, dws, stream=cs)
+        torch.cuda.current_stream(dev).wait_stream(cs)
+        graphs[w] = g
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    assert gb.gdla_device_error(stream) == 0, "device error in graph warm-up"
 
     def barrier():
         if world > 1:
@@ -269,7 +314,8 @@ def run_gpu(args):
         for _ in range(args.steps):
             recs.append(step())
         barrier()
-    launches = gb.gdla_kernel_launches() - launches0
+    # graph replays launch the captured kernels without passing through the library's counter
+    launches = gb.gdla_kernel_launches() - launches0 + args.steps * sum(kernels_per_decode.values())
     gb.gdla_set_stage_events([])
     site = gb.gdla_device_error(stream)
     assert site == 0, f"device error site {site:#x} in the timed region"
@@ -287,7 +333,7 @@ def run_gpu(args):
     y_host = torch.empty_like(x_host).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_ms = []
-    for i in range(0 if args.skip_e2e else max(2, min(args.steps, 5)) + 1):
+    for i in range(0 if (args.skip_e2e or args.skip_prefill) else max(2, min(args.steps, 5)) + 1):
         flush.fill_(1)
         barrier()
         e0.record(stream)
@@ -307,21 +353,27 @@ def run_gpu(args):
     pairs = valid_pairs(T, 0)
     attn_flop = B * pairs * attn_flops_per_pair(s)
     layer_flop = attn_flop + B * T * proj_flops_per_token(s)
-    value = world * layer_flop / (st["prefill_ms"] * 1e-3) / 1e12
-    attn_tf = attn_flop / (st["attn_ms"] * 1e-3) / 1e12
-    e2e_val = world * layer_flop / (e2e_t.item() * 1e-3) / 1e12
+    def tflops(flop, ms):
+        return flop / (ms * 1e-3) / 1e12 if ms and ms == ms and ms > 0 else float("nan")
+
+    value = world * tflops(layer_flop, st["prefill_ms"])
+    attn_tf = tflops(attn_flop, st["attn_ms"])
+    e2e_val = world * tflops(layer_flop, e2e_t.item())
 
     decode = {}
     for w in windows:
         keys_read = dec_L + 1 if w == 0 else min(w, dec_L + 1)
         kv_bytes = DECODE["B"] * keys_read * s.latent_row * 2
-        t_att = st[f"dec{w}_attn_ms"] * 1e-3
+        t_att = statistics.median(eager_stage[w]["attn"]) * 1e-3
         t_all = st[f"dec{w}_ms"] * 1e-3
         decode["causal" if w == 0 else f"swa{w}"] = {
             "B": DECODE["B"], "cache_len": dec_L, "window": w,
             "tok_per_s": world * DECODE["B"] / t_all, "ms": st[f"dec{w}_ms"],
-            "latent_attention_ms": st[f"dec{w}_attn_ms"], "query_path_ms": st[f"dec{w}_q_ms"],
-            "combine_ms": st[f"dec{w}_comb_ms"],
+            "timing": "CUDA graph replay of one gdla_decode_fwd call",
+            "ms_eager": statistics.median(eager_dec[w]),
+            "latent_attention_ms": statistics.median(eager_stage[w]["attn"]),
+            "query_path_ms": statistics.median(eager_stage[w]["q"]),
+            "combine_ms": statistics.median(eager_stage[w]["comb"]),
             "kv_bytes": kv_bytes, "kv_gbs": kv_bytes / t_att / 1e9,
             "kv_frac_of_hbm": kv_bytes / t_att / 1e9 / peaks["hbm_gbs"],
         }
@@ -353,7 +405,7 @@ def run_gpu(args):
                     "down_proj_ms": st["down_ms"], "norm_rope_ms": st["norm_ms"],
                     "up_proj_ms": st["up_ms"], "out_proj_ms": st["out_ms"],
                     "layer_flop": layer_flop, "attention_flop": attn_flop,
-                    "attention_tflops": attn_tf, "tok_per_s": world * B * T / (st["prefill_ms"] * 1e-3),
+                    "attention_tflops": attn_tf, "tok_per_s": world * B * T / max(st["prefill_ms"] * 1e-3, 1e-12),
                     "layer_frac_of_bf16_peak": value / world / peaks["bf16_tflops_sustained"]},
         "decode": decode,
         "roofline": {"kernel": "attn_prefill_kernel", "bound": "tensor", "achieved": attn_tf,
@@ -368,7 +420,7 @@ def run_gpu(args):
         "clocks": clk.summary(),
     }
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.skip_prefill:
         dt, fl, rows = oracle_prefill_sample(inp, 8, seed=7)
         line["cpu_baseline"] = {
             "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads_used(), "kind": "oracle",
@@ -400,6 +452,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=PREFILL["T"], help="prefill length (profiling runs)")
     ap.add_argument("--skip-decode", action="store_true", help="profiling runs: prefill only")
+    ap.add_argument("--skip-prefill", action="store_true", help="profiling runs: decode only")
     ap.add_argument("--skip-e2e", action="store_true", help="profiling runs: no host-buffer pass")
     ap.add_argument("--decode-L", type=int, default=DECODE["L"], help="cached positions (profiling runs)")
     args = ap.parse_args()

@@ -26,6 +26,9 @@ static bool launch_failed(int rc) {
   if (rc == 0) ++g_launches;
   return rc != 0;
 }
+}  // namespace gdla
+namespace gdla {
+void count_extra_launch() { ++g_launches; }
 static const uint32_t kAbsorbedMagic = 0x47444C41u;  // "GDLA"
 
 static int error_word(int** out) {
@@ -60,7 +63,22 @@ static int check_weights(const gdla_weights_t* w) {
 }
 
 // ---------------------------------------------------------------- workspace layout
-enum { WS_D1, WS_CQ, WS_LATENT, WS_LAM, WS_QQ, WS_G, WS_KV, WS_ONOISE, WS_DG, WS_KR16, WS_N };
+enum { WS_D1, WS_CQ, WS_LATENT, WS_LAM, WS_QQ, WS_G, WS_KV, WS_ONOISE, WS_DG, WS_KR16, WS_SPLITK,
+       WS_N };
+
+// fp32 scratch of the split-K projections of a decode step (skinny M = B products).
+static long long decode_splitk_floats(const gdla_config_t* c, int B) {
+  const int nH = c->n_signal + c->n_noise;
+  const int shapes[6][2] = {{c->q_rank, c->d_model}, {c->kv_rank + c->d_rope, c->d_model},
+                            {c->n_signal, c->d_model}, {nH * (c->d_nope + c->d_rope), c->q_rank},
+                            {c->n_signal * c->d_v, c->q_rank}, {c->d_model, c->n_signal * c->d_v}};
+  long long m = 0;
+  for (auto& sh : shapes) {
+    const long long f = (long long)gemm_splitk_count(B, sh[0], sh[1]) * B * sh[0];
+    if (f > m) m = f;
+  }
+  return m;
+}
 
 
 static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS_N + 1]) {
@@ -80,13 +98,15 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
     sz[WS_KV] = M * (long long)c->n_kv_heads * (c->d_nope + c->d_v) * 2;
     sz[WS_ONOISE] = M * (long long)c->n_noise * c->d_v * 4;
     sz[WS_KR16] = M * c->d_rope * 2;
+    sz[WS_SPLITK] = 0;
   } else {
     const int ns = decode_split_count(B, T, c->window);   // T = cache capacity in decode mode
-    sz[WS_LATENT] = 0;
+    sz[WS_LATENT] = M * (long long)c->n_signal * c->kv_rank * 4;     // latent differentials
     sz[WS_QQ] = M * qq * 4;                                          // fp32 q^C | q^R
     sz[WS_KV] = M * (long long)nH * (c->kv_rank + c->d_rope) * 2;    // q~ rows
     sz[WS_ONOISE] = M * (long long)ns * nH * c->kv_rank * 4;         // split partials
     sz[WS_KR16] = M * (long long)ns * nH * 2 * 4;                    // split (max, sum)
+    sz[WS_SPLITK] = decode_splitk_floats(c, B) * 4;
   }
   size_t o = 0;
   for (int i = 0; i < WS_N; ++i) {
@@ -318,8 +338,11 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
 
   stage(0, st);
+  float* splitk = reinterpret_cast<float*>(ws + off[WS_SPLITK]);
+  const long long splitk_n = decode_splitk_floats(cfg, B);
   GemmEpi ep{};
   ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = B; ep.pos_T = 1; ep.rope = rope;
+  ep.splitk = splitk; ep.splitk_floats = splitk_n;
   ep.C = D1; ep.N = cfg->q_rank;
   if (launch_failed(launch_gemm(x_new, cfg->d_model, w->W_aQ, cfg->q_rank, false, B, ep.N, cfg->d_model, ep, ctl, st)))
     return GDLA_ERR_LAUNCH;
@@ -341,12 +364,12 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   GemmEpi eq{};
   eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F32; eq.M = B; eq.N = nqq;
   eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = 1; eq.pos_ptr = cache_len;
-  eq.rope = rope;
+  eq.rope = rope; eq.splitk = splitk; eq.splitk_floats = splitk_n;
   if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, B, nqq, cfg->q_rank, eq, ctl, st)))
     return GDLA_ERR_LAUNCH;
   GemmEpi eg{};
   eg.C = G; eg.ldc = cfg->n_signal * cfg->d_v; eg.out_type = OUT_BF16; eg.M = B; eg.N = eg.ldc;
-  eg.pos_T = 1;
+  eg.pos_T = 1; eg.splitk = splitk; eg.splitk_floats = splitk_n;
   if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, B, eg.N, cfg->q_rank, eg, ctl, st)))
     return GDLA_ERR_LAUNCH;
 
@@ -368,12 +391,13 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   DecCombParams cp{};
   cp.B = B; cp.n_groups = cfg->n_noise; cp.n_signal = cfg->n_signal; cp.n_split = nsplit;
   cp.part = part; cp.ml = ml; cp.lam = lam; cp.G = G; cp.W_bKV = w->W_bKV; cp.Dg = Dg;
+  cp.Dlat = reinterpret_cast<float*>(ws + off[WS_LATENT]);
   if (launch_failed(launch_dec_combine(cp, st))) return GDLA_ERR_LAUNCH;
 
   stage(3, st);
   GemmEpi eo{};
   eo.C = y; eo.ldc = cfg->d_model; eo.out_type = OUT_BF16; eo.M = B; eo.N = cfg->d_model;
-  eo.pos_T = 1;
+  eo.pos_T = 1; eo.splitk = splitk; eo.splitk_floats = splitk_n;
   if (launch_failed(launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, B, cfg->d_model,
                   cfg->n_signal * cfg->d_v, eo, ctl, st)))
     return GDLA_ERR_LAUNCH;

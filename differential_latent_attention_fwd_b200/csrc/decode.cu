@@ -78,12 +78,12 @@ int launch_qtilde(const DecQParams& p, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- split merge + combine + gate
-// CTA (b, j): merges the splits of the group's 5 heads, forms the latent differential
-// l_s - lambda_s l_noise for its 4 signal heads, up-projects with W_UV_j and applies the gate.
-__global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
+// Kernel 1, CTA (b, j): merges the splits of the group's 5 heads (rescaling each split's
+// partial by 2^(m_split - m)), normalises, and forms the latent differential
+// l_s - lambda_s l_noise for the group's 4 signal heads -> Dlat[j][b * 4 + s][512] (fp32).
+__global__ void __launch_bounds__(256) dec_merge_kernel(DecCombParams p) {
   const int b = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
   constexpr int NH = 80;
-  __shared__ float lat[5][512];
   __shared__ float wsp[64][5];
   __shared__ float inv_L[5];
   const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
@@ -102,42 +102,88 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
     inv_L[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
   }
   __syncthreads();
-  for (int i = tid; i < 5 * 512; i += blockDim.x) {
-    const int hh = i / 512, l = i % 512;
-    float a = 0.f;
-    for (int sp = 0; sp < p.n_split; ++sp) {
-      const float w = wsp[sp][hh];
-      if (w != 0.f)  // empty splits write no partial
-        a += w * p.part[(((long long)b * p.n_split + sp) * NH + heads[hh]) * 512 + l];
+  for (int l = tid; l < 512; l += blockDim.x) {
+    float lat[5];
+#pragma unroll
+    for (int hh = 0; hh < 5; ++hh) {
+      float a = 0.f;
+      for (int sp = 0; sp < p.n_split; ++sp) {
+        const float w = wsp[sp][hh];
+        if (w != 0.f)  // empty splits write no partial
+          a += w * p.part[(((long long)b * p.n_split + sp) * NH + heads[hh]) * 512 + l];
+      }
+      lat[hh] = a * inv_L[hh];
     }
-    lat[hh][l] = a * inv_L[hh];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const float lam = p.lam[(long long)b * p.n_signal + 4 * j + s];
+      p.Dlat[((long long)j * p.B + b) * 4 * 512 + s * 512 + l] = lat[1 + s] - lam * lat[0];
+    }
   }
-  __syncthreads();
-  // latent differential, in place for the 4 signal heads
-  for (int i = tid; i < 4 * 512; i += blockDim.x) {
-    const int s = i / 512, l = i % 512;
-    const float lam = p.lam[(long long)b * p.n_signal + 4 * j + s];
-    lat[1 + s][l] -= lam * lat[0][l];
+}
+
+// Kernel 2, CTA (j, 4 sequences): D = Dlat W_UV_j (16 rows x 128 columns, K = 512), then
+// Dg = sigmoid(G) (.) D.  W_UV_j is the V column block of W_b^KV for KV head j; it is staged
+// in shared memory (128 KB, coalesced 16-byte loads) before the product.
+__global__ void __launch_bounds__(256) dec_uv_gate_kernel(DecCombParams p) {
+  extern __shared__ uint8_t uv_smem[];
+  float (*dl)[512] = reinterpret_cast<float (*)[512]>(uv_smem);                      // [16][512]
+  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(uv_smem + 16 * 512 * 4);     // [512][128]
+  const int j = blockIdx.x, b0 = blockIdx.y * 4, tid = threadIdx.x;
+  const int nrows = min(4, p.B - b0) * 4;
+  const long long ldw = (long long)p.n_groups * 256;
+  const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_bKV) + j * 256 + 128;
+  for (int i = tid; i < 512 * 16; i += blockDim.x) {          // 16 uint4 per 128-column row
+    const int l = i >> 4, q = i & 15;
+    reinterpret_cast<uint4*>(wsm + l * 128)[q] = reinterpret_cast<const uint4*>(W + l * ldw)[q];
   }
+  const float* src = p.Dlat + ((long long)j * p.B + b0) * 4 * 512;
+  for (int i = tid; i < 16 * 512; i += blockDim.x)
+    dl[i / 512][i % 512] = (i / 512) < nrows ? src[i] : 0.f;
   __syncthreads();
-  const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_bKV);
-  const int ldw = p.n_groups * 256;
-  for (int o = tid; o < 4 * 128; o += blockDim.x) {
-    const int s = o / 128, c = o % 128;
-    float d = 0.f;
-    for (int l = 0; l < 512; ++l)
-      d = fmaf(lat[1 + s][l], __bfloat162float(W[(long long)l * ldw + j * 256 + 128 + c]), d);
-    const int sig = 4 * j + s;
-    const float g = __bfloat162float(static_cast<const __nv_bfloat16*>(p.G)[(long long)b * p.n_signal * 128 + sig * 128 + c]);
-    static_cast<__nv_bfloat16*>(p.Dg)[(long long)b * p.n_signal * 128 + sig * 128 + c] =
-        __float2bfloat16_rn(sigmoidf_fast(g) * d);
+  const int cq = tid & 31;          // columns 4 cq .. 4 cq + 3
+  const int rp = tid >> 5;          // rows 2 rp, 2 rp + 1
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
+  for (int l = 0; l < 512; ++l) {
+    const uint2 wv = *reinterpret_cast<const uint2*>(wsm + l * 128 + 4 * cq);
+    const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wv.x);
+    const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wv.y);
+    const float w[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
+    const float d0 = dl[2 * rp][l], d1 = dl[2 * rp + 1][l];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[0][e] = fmaf(d0, w[e], acc[0][e]);
+      acc[1][e] = fmaf(d1, w[e], acc[1][e]);
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int row = 2 * rp + rr;
+    if (row >= nrows) continue;
+    const int b = b0 + row / 4, s = row % 4, sig = 4 * j + s;
+    const long long o = (long long)b * p.n_signal * 128 + sig * 128 + 4 * cq;
+    const uint2 gv = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.G) + o);
+    const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&gv.x);
+    const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&gv.y);
+    uint2 out;
+    out.x = pack_bf162(sigmoidf_fast(__low2float(g01)) * acc[rr][0], sigmoidf_fast(__high2float(g01)) * acc[rr][1]);
+    out.y = pack_bf162(sigmoidf_fast(__low2float(g23)) * acc[rr][2], sigmoidf_fast(__high2float(g23)) * acc[rr][3]);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.Dg) + o) = out;
   }
 }
 
 int launch_dec_combine(const DecCombParams& p, cudaStream_t st) {
-  dim3 grid(p.B, p.n_groups);
-  dec_combine_kernel<<<grid, 256, 0, st>>>(p);
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
+  dec_merge_kernel<<<dim3(p.B, p.n_groups), 256, 0, st>>>(p);
+  if (cudaPeekAtLastError() != cudaSuccess) return -4;
+  const int uv_smem = 16 * 512 * 4 + 512 * 128 * 2;
+  if (cudaFuncSetAttribute(dec_uv_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, uv_smem) !=
+      cudaSuccess)
+    return -4;
+  dec_uv_gate_kernel<<<dim3(p.n_groups, (p.B + 3) / 4), 256, uv_smem, st>>>(p);
+  if (cudaPeekAtLastError() != cudaSuccess) return -4;
+  count_extra_launch();
+  return 0;
 }
 
 }  // namespace gdla

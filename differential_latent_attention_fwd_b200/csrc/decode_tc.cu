@@ -120,8 +120,11 @@ __global__ void __launch_bounds__(192, 1)
       for (int c = 0; c < 9; ++c)
         tma_load_2d(smem + QT_OFF + c * QBOX, &mapQ, &bars->q_full, c * 64, b * NH);
       uint32_t g = 0;
+      // The latent columns are read twice (scores, then PV): the first read asks L2 to keep
+      // them, the second (and the rope columns, read once) lets them go.
+      const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
       // unit order: S(0), S(1), P(0), S(2), P(1), ..., S(n-1), P(n-2), P(n-1)
-      auto load_unit = [&](int tile, int pair, bool rope) -> bool {
+      auto load_unit = [&](int tile, int pair, bool rope, bool second) -> bool {
         const int slot = g % NSLOT;
         const uint32_t ph = (g / NSLOT) & 1;
         if (g >= NSLOT && !mbar_wait(&bars->ring_empty[slot], ph ^ 1, ctl, SITE_DEC_PRODUCER))
@@ -130,11 +133,12 @@ __global__ void __launch_bounds__(192, 1)
         const int y = int(crow0 + (long long)(rg.t_begin + tile) * 128);
         if (rope) {
           mbar_expect_tx(&bars->ring_full[slot], 16384);
-          tma_load_2d(dst, &mapC, &bars->ring_full[slot], 512, y);
+          tma_load_2d_hint(dst, &mapC, &bars->ring_full[slot], 512, y, drop);
         } else {
+          const uint64_t pol = second ? drop : keep;
           mbar_expect_tx(&bars->ring_full[slot], 32768);
-          tma_load_2d(dst, &mapC, &bars->ring_full[slot], pair * 128, y);
-          tma_load_2d(dst + 16384, &mapC, &bars->ring_full[slot], pair * 128 + 64, y);
+          tma_load_2d_hint(dst, &mapC, &bars->ring_full[slot], pair * 128, y, pol);
+          tma_load_2d_hint(dst + 16384, &mapC, &bars->ring_full[slot], pair * 128 + 64, y, pol);
         }
         issued |= 1u << slot;
         par = (par & ~(1u << slot)) | (ph << slot);
@@ -143,9 +147,9 @@ __global__ void __launch_bounds__(192, 1)
       };
       for (int i = 0; i <= n_t && ok; ++i) {
         if (i < n_t)
-          for (int u = 0; u < 5 && ok; ++u) ok = load_unit(i, u, u == 4);
+          for (int u = 0; u < 5 && ok; ++u) ok = load_unit(i, u, u == 4, false);
         if (i >= 1)
-          for (int u = 0; u < 4 && ok; ++u) ok = load_unit(i - 1, u, false);
+          for (int u = 0; u < 4 && ok; ++u) ok = load_unit(i - 1, u, false, true);
       }
       for (int s = 0; s < NSLOT; ++s)
         if (issued & (1u << s)) mbar_drain(&bars->ring_full[s], (par >> s) & 1, ctl.err);

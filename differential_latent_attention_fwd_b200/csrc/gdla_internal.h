@@ -26,7 +26,19 @@ struct GemmEpi {
   int pos_T;             // row position = row % pos_T (used when pos_ptr is null)
   const int* pos_ptr;    // row position = pos_ptr[row]
   RopeTable rope;
+  // Optional split-K scratch for skinny products (M <= 128): fp32 [splits][M][N].  When set
+  // and worthwhile, K is split across CTAs and a reduce kernel applies this epilogue.
+  float* splitk;
+  long long splitk_floats;
+  // internal: set by launch_gemm for the split-K pass (raw fp32 partial tiles)
+  float* partial_out;
+  int kb_per_split;
 };
+
+// Number of K splits launch_gemm uses for an M x N x K product (1 = no split).
+int gemm_splitk_count(int M, int N, int K);
+// Counts a kernel launched by a helper beyond the one its caller counts.
+void count_extra_launch();
 
 struct KernelCtlHost {
   int* err;

@@ -37,7 +37,10 @@ __global__ void __launch_bounds__(128, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN;
-  const int nk = K / 64;
+  // K blocks of this CTA: all of them, or split blockIdx.z's share (split-K pass)
+  const int nk_all = K / 64;
+  const int kb0 = ep.kb_per_split > 0 ? int(blockIdx.z) * ep.kb_per_split : 0;
+  const int nk = ep.kb_per_split > 0 ? min(ep.kb_per_split, nk_all - kb0) : nk_all;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -67,13 +70,14 @@ __global__ void __launch_bounds__(128, 1)
       if (kb >= STAGES && !mbar_wait(&empty[s], ph ^ 1, ctl, SITE_GEMM_PRODUCER)) break;
       uint8_t* st = smem + s * STAGE;
       mbar_expect_tx(&full[s], STAGE);
-      tma_load_2d(st, &mapA, &full[s], kb * 64, m0);
+      const int kx = (kb0 + kb) * 64;
+      tma_load_2d(st, &mapA, &full[s], kx, m0);
       if (B_KMAJOR) {
-        tma_load_2d(st + A_BYTES, &mapB, &full[s], kb * 64, n0);
+        tma_load_2d(st + A_BYTES, &mapB, &full[s], kx, n0);
       } else {
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c)
-          tma_load_2d(st + A_BYTES + c * 8192, &mapB, &full[s], n0 + c * 64, kb * 64);
+          tma_load_2d(st + A_BYTES + c * 8192, &mapB, &full[s], n0 + c * 64, kx);
       }
       issued_mask |= 1u << s;
       last_par = (last_par & ~(1u << s)) | (ph << s);
@@ -123,6 +127,15 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
     const int col = n0 + c0;
+    if (ep.partial_out) {  // split-K pass: raw fp32 partial, epilogue applied by the reduce
+      if (row_ok) {
+        float* dst = ep.partial_out + ((long long)blockIdx.z * ep.M + row) * ep.N + col;
+#pragma unroll
+        for (int i = 0; i < 64; i += 4)
+          *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+      continue;
+    }
     if (col >= ep.rope_lo && col < ep.rope_hi) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -172,6 +185,43 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 1) tmem_dealloc(tmem, BN);
 }
 
+// Split-K reduce: out = epilogue(sum over splits).  Thread = column pair (i, i + 32) of a
+// 64-column block, so that rope pairs stay in one thread.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ GemmEpi ep, int splits) {
+  const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const int nblk = ep.N / 64;
+  if (idx >= (long long)ep.M * nblk * 32) return;
+  const int i = int(idx & 31);
+  const int blk = int((idx >> 5) % nblk);
+  const int row = int((idx >> 5) / nblk);
+  const int c1 = blk * 64 + i, c2 = c1 + 32;
+  float a = 0.f, b = 0.f;
+  for (int z = 0; z < splits; ++z) {
+    const float* pz = ep.splitk + ((long long)z * ep.M + row) * ep.N;
+    a += pz[c1];
+    b += pz[c2];
+  }
+  if (blk * 64 >= ep.rope_lo && blk * 64 < ep.rope_hi) {
+    const int pos = ep.pos_ptr ? ep.pos_ptr[row] : (row % ep.pos_T);
+    float cs, sn;
+    rope_cs(pos, ep.rope.inv_freq[i], &cs, &sn);
+    const float x1 = a, x2 = b;
+    a = x1 * cs - x2 * sn;
+    b = x2 * cs + x1 * sn;
+  }
+  const long long o = (long long)row * ep.ldc;
+  if (ep.out_type == OUT_F32) {
+    reinterpret_cast<float*>(ep.C)[o + c1] = a;
+    reinterpret_cast<float*>(ep.C)[o + c2] = b;
+  } else if (ep.out_type == OUT_BF16) {
+    reinterpret_cast<__nv_bfloat16*>(ep.C)[o + c1] = __float2bfloat16_rn(a);
+    reinterpret_cast<__nv_bfloat16*>(ep.C)[o + c2] = __float2bfloat16_rn(b);
+  } else {
+    reinterpret_cast<__half*>(ep.C)[o + c1] = __float2half_rn(a);
+    reinterpret_cast<__half*>(ep.C)[o + c2] = __float2half_rn(b);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -213,23 +263,59 @@ void fill_rope_table(RopeTable* t, int d_rope, double theta) {
 
 template <int BN, int STAGES, bool BK>
 static int run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K,
-                    const GemmEpi& ep, KernelCtlHost ctl, cudaStream_t st) {
+                    const GemmEpi& ep, KernelCtlHost ctl, cudaStream_t st, int splits) {
   constexpr int STAGE = 128 * 64 * 2 + BN * 64 * 2;
   const int smem = STAGES * STAGE + 1024 + 256;
   auto kfn = gemm_tc_kernel<BN, STAGES, BK>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return -4;
-  dim3 grid((M + 127) / 128, (N + BN - 1) / BN);
+  dim3 grid((M + 127) / 128, (N + BN - 1) / BN, splits);
   KernelCtl kc{ctl.err, ctl.limit_ns};
   kfn<<<grid, 128, smem, st>>>(ma, mb, K, ep, kc);
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
+  if (cudaPeekAtLastError() != cudaSuccess) return -4;
+  if (splits > 1) {
+    const long long threads = (long long)M * (N / 64) * 32;
+    splitk_reduce_kernel<<<unsigned((threads + 255) / 256), 256, 0, st>>>(ep, splits);
+    if (cudaPeekAtLastError() != cudaSuccess) return -4;
+    count_extra_launch();
+  }
+  return 0;
+}
+
+static int gemm_bn(int N) { return N >= 256 ? 256 : (N > 64 ? 128 : 64); }
+
+// Skinny products (one 128-row M tile) leave most SMs idle; split K so that about one wave of
+// CTAs streams the weights, each split keeping at least 4 K blocks of 64.
+int gemm_splitk_count(int M, int N, int K) {
+  if (M > 128 || N % 64 != 0 || K % 64 != 0) return 1;
+  const int BN = gemm_bn(N);
+  const int tiles = (N + BN - 1) / BN;
+  const int nk = K / 64;
+  int s = (148 + tiles - 1) / tiles;
+  s = s > nk / 4 ? nk / 4 : s;
+  if (s <= 1) return 1;
+  const int kps = (nk + s - 1) / s;
+  return (nk + kps - 1) / kps;
 }
 
 int launch_gemm(const void* A, long long lda, const void* B, long long ldb, bool b_kmajor, int M,
-                int N, int K, const GemmEpi& ep, KernelCtlHost ctl, cudaStream_t st) {
+                int N, int K, const GemmEpi& ep_in, KernelCtlHost ctl, cudaStream_t st) {
   if (M <= 0 || N <= 0) return 0;
   if (K <= 0 || K % 64 != 0) return -1;
-  const int BN = N >= 256 ? 256 : (N > 64 ? 128 : 64);
+  const int BN = gemm_bn(N);
+  GemmEpi ep = ep_in;
+  ep.partial_out = nullptr;
+  ep.kb_per_split = 0;
+  int splits = 1;
+  if (ep.splitk) {
+    splits = gemm_splitk_count(M, N, K);
+    if ((long long)splits * M * N > ep.splitk_floats) splits = 1;
+    if (splits > 1) {
+      const int nk = K / 64;
+      ep.kb_per_split = (nk + splits - 1) / splits;
+      ep.partial_out = ep.splitk;
+    }
+  }
   CUtensorMap ma, mb;
   if (make_tmap_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
@@ -243,13 +329,13 @@ int launch_gemm(const void* A, long long lda, const void* B, long long ldb, bool
                       CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return -3;
   if (b_kmajor) {
-    if (BN == 256) return run_gemm<256, 4, true>(ma, mb, M, N, K, ep, ctl, st);
-    if (BN == 128) return run_gemm<128, 6, true>(ma, mb, M, N, K, ep, ctl, st);
-    return run_gemm<64, 8, true>(ma, mb, M, N, K, ep, ctl, st);
+    if (BN == 256) return run_gemm<256, 4, true>(ma, mb, M, N, K, ep, ctl, st, splits);
+    if (BN == 128) return run_gemm<128, 6, true>(ma, mb, M, N, K, ep, ctl, st, splits);
+    return run_gemm<64, 8, true>(ma, mb, M, N, K, ep, ctl, st, splits);
   }
-  if (BN == 256) return run_gemm<256, 4, false>(ma, mb, M, N, K, ep, ctl, st);
-  if (BN == 128) return run_gemm<128, 6, false>(ma, mb, M, N, K, ep, ctl, st);
-  return run_gemm<64, 8, false>(ma, mb, M, N, K, ep, ctl, st);
+  if (BN == 256) return run_gemm<256, 4, false>(ma, mb, M, N, K, ep, ctl, st, splits);
+  if (BN == 128) return run_gemm<128, 6, false>(ma, mb, M, N, K, ep, ctl, st, splits);
+  return run_gemm<64, 8, false>(ma, mb, M, N, K, ep, ctl, st, splits);
 }
 
 }  // namespace gdla
