@@ -19,6 +19,7 @@ HEADER = os.path.join(HERE, "..", "include", "gdla.h")
 
 GDLA_MODE_PREFILL = 0
 GDLA_MODE_DECODE = 1
+GDLA_MODE_VARLEN = 2
 STATUS = {0: "GDLA_OK", -1: "GDLA_ERR_INVALID_ARG", -2: "GDLA_ERR_UNSUPPORTED_SHAPE",
           -3: "GDLA_ERR_WORKSPACE_TOO_SMALL", -4: "GDLA_ERR_LAUNCH",
           -5: "GDLA_ERR_DEVICE_TIMEOUT", -6: "GDLA_ERR_CUDA"}
@@ -74,6 +75,8 @@ def lib() -> ctypes.CDLL:
             "gdla_set_stage_events": [ctypes.POINTER(P), I],
             "gdla_kernel_launches": [],
             "gdla_attn_prefill_noalloc": [cfgp, P, P, P, P, P, P, I, I, P],
+            "gdla_prefill_varlen_fwd": [cfgp, wp, P, I, P, I, P, P, P, SZ, P],
+            "gdla_decode_multi_fwd": [cfgp, abp, P, I, P, P, I, I, P, P, SZ, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -162,6 +165,18 @@ def gdla_prefill_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, y: torch.Tensor,
         _stream(stream)))
 
 
+def gdla_prefill_varlen_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, cu_seqlens: torch.Tensor,
+                            y: torch.Tensor, workspace: torch.Tensor,
+                            kv_latent_out: torch.Tensor | None = None, stream=None) -> None:
+    total = x.shape[0]
+    _check("gdla_prefill_varlen_fwd", lib().gdla_prefill_varlen_fwd(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(x, torch.bfloat16, "x"), total,
+        _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cu_seqlens.numel() - 1,
+        _ptr(y, torch.bfloat16, "y"), _ptr(kv_latent_out, torch.bfloat16, "kv_latent_out"),
+        _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
 def gdla_absorb_weights(cfg, w: gdla_weights_t, dst: torch.Tensor, stream=None) -> gdla_absorbed_t:
     out = gdla_absorbed_t()
     _check("gdla_absorb_weights", lib().gdla_absorb_weights(
@@ -179,6 +194,18 @@ def gdla_decode_fwd(cfg, absorbed: gdla_absorbed_t, x_new: torch.Tensor, kv_cach
         ctypes.byref(cfg), ctypes.byref(absorbed), _ptr(x_new, torch.bfloat16, "x_new"),
         _ptr(kv_cache, torch.bfloat16, "kv_cache"), _ptr(cache_len, torch.int32, "cache_len"), cap, B,
         _ptr(y, torch.bfloat16, "y"), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gdla_decode_multi_fwd(cfg, absorbed: gdla_absorbed_t, x_new: torch.Tensor, kv_cache: torch.Tensor,
+                          cache_len: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor,
+                          stream=None) -> None:
+    """x_new [n_seq, q_len, d]: q_len new tokens per sequence (positions cache_len + i)."""
+    n_seq, q_len = x_new.shape[0], x_new.shape[1]
+    _check("gdla_decode_multi_fwd", lib().gdla_decode_multi_fwd(
+        ctypes.byref(cfg), ctypes.byref(absorbed), _ptr(x_new, torch.bfloat16, "x_new"), q_len,
+        _ptr(kv_cache, torch.bfloat16, "kv_cache"), _ptr(cache_len, torch.int32, "cache_len"),
+        kv_cache.shape[1], n_seq, _ptr(y, torch.bfloat16, "y"), _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

@@ -64,7 +64,12 @@ static int check_weights(const gdla_weights_t* w) {
 
 // ---------------------------------------------------------------- workspace layout
 enum { WS_D1, WS_CQ, WS_LATENT, WS_LAM, WS_QQ, WS_G, WS_KV, WS_ONOISE, WS_DG, WS_KR16, WS_SPLITK,
-       WS_N };
+       WS_VL_POS, WS_VL_UNITS, WS_VL_COUNT, WS_N };
+
+// Packed documents: bounds of the attention schedule for `total` tokens in up to `total`
+// non-empty documents (sum over documents of ceil(len / 256) <= total / 256 + documents).
+static int varlen_max_pairs(long long total) { return int((total + 255) / 256); }
+static int varlen_max_units(long long total) { return int(total + (total + 255) / 256); }
 
 // fp32 scratch of the split-K projections of a decode step (skinny M = B products).
 static long long decode_splitk_floats(const gdla_config_t* c, int B) {
@@ -82,7 +87,7 @@ static long long decode_splitk_floats(const gdla_config_t* c, int B) {
 
 
 static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS_N + 1]) {
-  const long long M = mode == GDLA_MODE_PREFILL ? (long long)B * T : (long long)B;
+  const long long M = mode == GDLA_MODE_DECODE ? (long long)B : (long long)B * T;
   const int nH = c->n_signal + c->n_noise;
   const long long qq = (long long)nH * (c->d_nope + c->d_rope);
   const long long d1 = c->q_rank + c->kv_rank + c->d_rope + c->n_signal;
@@ -92,7 +97,13 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
   sz[WS_LAM] = M * c->n_signal * 4;
   sz[WS_G] = M * (long long)c->n_signal * c->d_v * 2;
   sz[WS_DG] = M * (long long)c->n_signal * c->d_v * 2;
-  if (mode == GDLA_MODE_PREFILL) {
+  sz[WS_VL_POS] = sz[WS_VL_UNITS] = sz[WS_VL_COUNT] = 0;
+  if (mode == GDLA_MODE_VARLEN) {
+    sz[WS_VL_POS] = M * 4;
+    sz[WS_VL_UNITS] = (size_t)varlen_max_units(M) * 16;
+    sz[WS_VL_COUNT] = (size_t)(1 + 2 * varlen_max_pairs(M)) * 4;
+  }
+  if (mode == GDLA_MODE_PREFILL || mode == GDLA_MODE_VARLEN) {
     sz[WS_LATENT] = M * (c->kv_rank + c->d_rope) * 2;
     sz[WS_QQ] = M * qq * 2;
     sz[WS_KV] = M * (long long)c->n_kv_heads * (c->d_nope + c->d_v) * 2;
@@ -126,6 +137,126 @@ int shared_kernel_ctl(KernelCtlHost* out) {
   return GDLA_OK;
 }
 
+// Packed documents: cu_seqlens on the device; the latent rows go to latent_out (packed order).
+struct VarlenArgs {
+  const int* cu_seqlens;
+  int n_docs;
+  void* latent_out;
+};
+
+// Prefill body shared by equal-length batches (vl == nullptr) and packed documents (B = 1,
+// T = all tokens).  Arguments are already validated; off is the workspace layout.
+static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int B,
+                        int T, void* y, void* kv_cache_out, int cache_cap, uint8_t* ws,
+                        const size_t* off, cudaStream_t st, const VarlenArgs* vl) {
+  int rc;
+  int* err;
+  if ((rc = error_word(&err))) return rc;
+  KernelCtlHost ctl{err, g_wait_limit_ns};
+  float* D1 = reinterpret_cast<float*>(ws + off[WS_D1]);
+  void* cQ = ws + off[WS_CQ];
+  void* latent = ws + off[WS_LATENT];
+  float* lam = reinterpret_cast<float*>(ws + off[WS_LAM]);
+  void* QQ = ws + off[WS_QQ];
+  void* G = ws + off[WS_G];
+  void* KV = ws + off[WS_KV];
+  float* On = reinterpret_cast<float*>(ws + off[WS_ONOISE]);
+  void* Dg = ws + off[WS_DG];
+  void* kR16 = ws + off[WS_KR16];
+  const int M = B * T;
+  const int nH = cfg->n_signal + cfg->n_noise;
+  const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
+  RopeTable rope;
+  fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
+
+  stage(0, st);
+  // packed documents: per-token positions and the attention schedule
+  const int* positions = nullptr;
+  const int4* units = nullptr;
+  const int* n_units = nullptr;
+  int max_units = 0;
+  if (vl) {
+    int* pos = reinterpret_cast<int*>(ws + off[WS_VL_POS]);
+    int4* un = reinterpret_cast<int4*>(ws + off[WS_VL_UNITS]);
+    int* cnt = reinterpret_cast<int*>(ws + off[WS_VL_COUNT]);
+    max_units = varlen_max_units(M);
+    const int max_c = varlen_max_pairs(M);
+    if (launch_failed(launch_varlen_schedule(vl->cu_seqlens, vl->n_docs, M, pos, un, cnt, max_units,
+                                             cnt + 1, cnt + 1 + max_c, max_c, err, st)))
+      return GDLA_ERR_LAUNCH;
+    g_launches += 3;  // the schedule is four kernels
+    positions = pos;
+    units = un;
+    n_units = cnt;
+    if (vl->latent_out) latent = vl->latent_out;
+  }
+
+  // a1: [x W_aQ | x W_aKV | x W_lambda] in fp32
+  GemmEpi ep{};
+  ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = M; ep.rope_lo = ep.rope_hi = 0; ep.pos_T = T;
+  ep.rope = rope;
+  ep.C = D1; ep.N = cfg->q_rank;
+  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_aQ, cfg->q_rank, false, M, cfg->q_rank, cfg->d_model, ep, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  ep.C = D1 + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
+  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_aKV, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  ep.C = D1 + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
+  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_lambda, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+
+  stage(1, st);
+  // a2: norms, rotary key, lambda, latent rows
+  NormParams np{};
+  np.D1 = D1; np.ld1 = ld1; np.M = M; np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank;
+  np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
+  np.cQ = cQ; np.latent = latent; np.kR16 = kR16; np.lam = lam; np.pos_T = T; np.pos_ptr = positions;
+  np.cache = kv_cache_out; np.cache_cap = cache_cap; np.rope = rope; np.err = err;
+  if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
+
+  stage(2, st);
+  // a3: up-projections (q^C | rotated q^R), gate logits, K^C | V
+  const int nqq = nH * (cfg->d_nope + cfg->d_rope);
+  GemmEpi eq{};
+  eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F16; eq.M = M; eq.N = nqq;
+  eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = T; eq.pos_ptr = positions;
+  eq.rope = rope;
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, M, nqq, cfg->q_rank, eq, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  GemmEpi eg{};
+  eg.C = G; eg.ldc = cfg->n_signal * cfg->d_v; eg.out_type = OUT_BF16; eg.M = M; eg.N = eg.ldc;
+  eg.pos_T = T;
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, M, eg.N, cfg->q_rank, eg, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  GemmEpi ekv{};
+  const int nkv = cfg->n_kv_heads * (cfg->d_nope + cfg->d_v);
+  ekv.C = KV; ekv.ldc = nkv; ekv.out_type = OUT_F16; ekv.M = M; ekv.N = nkv; ekv.pos_T = T;
+  if (launch_failed(launch_gemm(latent, cfg->kv_rank + cfg->d_rope, w->W_bKV, nkv, false, M, nkv, cfg->kv_rank,
+                  ekv, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+
+  stage(3, st);
+  // a4: fused attention + differential combine + gate
+  AttnParams ap{};
+  ap.B = B; ap.T = T; ap.window = cfg->window; ap.n_groups = cfg->n_noise;
+  ap.n_signal = cfg->n_signal; ap.rope_col0 = nH * cfg->d_nope;
+  ap.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
+  ap.lam = lam; ap.G = G; ap.O_noise = On; ap.Dg = Dg;
+  ap.units = units; ap.n_units = n_units; ap.max_units = max_units;
+  if (launch_failed(launch_attn_prefill(QQ, nqq, KV, kR16, ap, ctl, st))) return GDLA_ERR_LAUNCH;
+
+  stage(4, st);
+  // a5: output projection
+  GemmEpi eo{};
+  eo.C = y; eo.ldc = cfg->d_model; eo.out_type = OUT_BF16; eo.M = M; eo.N = cfg->d_model;
+  eo.pos_T = T;
+  if (launch_failed(launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, M, cfg->d_model,
+                  cfg->n_signal * cfg->d_v, eo, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  stage(5, st);
+  return GDLA_OK;
+}
+
 }  // namespace gdla
 
 using namespace gdla;
@@ -153,8 +284,8 @@ int gdla_set_wait_limit_ns(unsigned long long ns) {
 int gdla_workspace_size(const gdla_config_t* cfg, int B, int T, int mode, size_t* bytes) {
   int rc = check_config(cfg);
   if (rc) return rc;
-  if (!bytes || B <= 0 || (mode == GDLA_MODE_PREFILL && T <= 0) ||
-      (mode != GDLA_MODE_PREFILL && mode != GDLA_MODE_DECODE))
+  if (!bytes || B <= 0 || (mode != GDLA_MODE_DECODE && T <= 0) ||
+      (mode != GDLA_MODE_PREFILL && mode != GDLA_MODE_DECODE && mode != GDLA_MODE_VARLEN))
     return GDLA_ERR_INVALID_ARG;
   size_t off[WS_N + 1];
   layout(cfg, B, T, mode, off);
@@ -195,90 +326,28 @@ int gdla_prefill_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const vo
   size_t off[WS_N + 1];
   layout(cfg, B, T, GDLA_MODE_PREFILL, off);
   if (ws_bytes < off[WS_N]) return GDLA_ERR_WORKSPACE_TOO_SMALL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int* err;
-  if ((rc = error_word(&err))) return rc;
-  KernelCtlHost ctl{err, g_wait_limit_ns};
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* D1 = reinterpret_cast<float*>(ws + off[WS_D1]);
-  void* cQ = ws + off[WS_CQ];
-  void* latent = ws + off[WS_LATENT];
-  float* lam = reinterpret_cast<float*>(ws + off[WS_LAM]);
-  void* QQ = ws + off[WS_QQ];
-  void* G = ws + off[WS_G];
-  void* KV = ws + off[WS_KV];
-  float* On = reinterpret_cast<float*>(ws + off[WS_ONOISE]);
-  void* Dg = ws + off[WS_DG];
-  void* kR16 = ws + off[WS_KR16];
-  const int M = B * T;
-  const int nH = cfg->n_signal + cfg->n_noise;
-  const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
-  RopeTable rope;
-  fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
+  return prefill_impl(cfg, w, x, B, T, y, kv_cache_out, cache_cap, static_cast<uint8_t*>(workspace),
+                      off, static_cast<cudaStream_t>(stream), nullptr);
+}
 
-  // a1: [x W_aQ | x W_aKV | x W_lambda] in fp32
-  stage(0, st);
-  GemmEpi ep{};
-  ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = M; ep.rope_lo = ep.rope_hi = 0; ep.pos_T = T;
-  ep.rope = rope;
-  ep.C = D1; ep.N = cfg->q_rank;
-  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_aQ, cfg->q_rank, false, M, cfg->q_rank, cfg->d_model, ep, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  ep.C = D1 + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
-  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_aKV, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  ep.C = D1 + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
-  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_lambda, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-
-  stage(1, st);
-  // a2: norms, rotary key, lambda, latent rows
-  NormParams np{};
-  np.D1 = D1; np.ld1 = ld1; np.M = M; np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank;
-  np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
-  np.cQ = cQ; np.latent = latent; np.kR16 = kR16; np.lam = lam; np.pos_T = T; np.pos_ptr = nullptr;
-  np.cache = kv_cache_out; np.cache_cap = cache_cap; np.rope = rope; np.err = err;
-  if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
-
-  stage(2, st);
-  // a3: up-projections (q^C | rotated q^R), gate logits, K^C | V
-  const int nqq = nH * (cfg->d_nope + cfg->d_rope);
-  GemmEpi eq{};
-  eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F16; eq.M = M; eq.N = nqq;
-  eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = T; eq.rope = rope;
-  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, M, nqq, cfg->q_rank, eq, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  GemmEpi eg{};
-  eg.C = G; eg.ldc = cfg->n_signal * cfg->d_v; eg.out_type = OUT_BF16; eg.M = M; eg.N = eg.ldc;
-  eg.pos_T = T;
-  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, M, eg.N, cfg->q_rank, eg, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  GemmEpi ekv{};
-  const int nkv = cfg->n_kv_heads * (cfg->d_nope + cfg->d_v);
-  ekv.C = KV; ekv.ldc = nkv; ekv.out_type = OUT_F16; ekv.M = M; ekv.N = nkv; ekv.pos_T = T;
-  if (launch_failed(launch_gemm(latent, cfg->kv_rank + cfg->d_rope, w->W_bKV, nkv, false, M, nkv, cfg->kv_rank,
-                  ekv, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-
-  stage(3, st);
-  // a4: fused attention + differential combine + gate
-  AttnParams ap{};
-  ap.B = B; ap.T = T; ap.window = cfg->window; ap.n_groups = cfg->n_noise;
-  ap.n_signal = cfg->n_signal; ap.rope_col0 = nH * cfg->d_nope;
-  ap.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
-  ap.lam = lam; ap.G = G; ap.O_noise = On; ap.Dg = Dg;
-  if (launch_failed(launch_attn_prefill(QQ, nqq, KV, kR16, ap, ctl, st))) return GDLA_ERR_LAUNCH;
-
-  stage(4, st);
-  // a5: output projection
-  GemmEpi eo{};
-  eo.C = y; eo.ldc = cfg->d_model; eo.out_type = OUT_BF16; eo.M = M; eo.N = cfg->d_model;
-  eo.pos_T = T;
-  if (launch_failed(launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, M, cfg->d_model,
-                  cfg->n_signal * cfg->d_v, eo, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  stage(5, st);
-  return GDLA_OK;
+int gdla_prefill_varlen_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x,
+                            int total, const int* cu_seqlens, int n_docs, void* y,
+                            void* kv_latent_out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_weights(w))) return rc;
+  if (!x || !y || !workspace || !cu_seqlens || total <= 0 || n_docs <= 0)
+    return GDLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(workspace) ||
+      (kv_latent_out && !aligned16(kv_latent_out)))
+    return GDLA_ERR_INVALID_ARG;
+  if ((long long)total > (1ll << 30) || n_docs > total) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  size_t off[WS_N + 1];
+  layout(cfg, 1, total, GDLA_MODE_VARLEN, off);
+  if (ws_bytes < off[WS_N]) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  VarlenArgs vl{cu_seqlens, n_docs, kv_latent_out};
+  return prefill_impl(cfg, w, x, 1, total, y, nullptr, 0, static_cast<uint8_t*>(workspace), off,
+                      static_cast<cudaStream_t>(stream), &vl);
 }
 
 int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void* dst,
@@ -303,6 +372,15 @@ int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void*
 int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const void* x_new,
                     void* kv_cache, const int* cache_len, int cap, int B, void* y, void* workspace,
                     size_t ws_bytes, void* stream) {
+  return gdla_decode_multi_fwd(cfg, ab, x_new, 1, kv_cache, cache_len, cap, B, y, workspace,
+                               ws_bytes, stream);
+}
+
+int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const void* x_new,
+                          int q_len, void* kv_cache, const int* cache_len, int cap, int n_seq,
+                          void* y, void* workspace, size_t ws_bytes, void* stream) {
+  if (q_len <= 0 || n_seq <= 0 || (long long)q_len * n_seq > (1 << 20)) return GDLA_ERR_INVALID_ARG;
+  const int B = q_len * n_seq;   // query rows: token r % q_len of sequence r / q_len
   int rc = check_config(cfg);
   if (rc) return rc;
   if (!ab || ab->magic != kAbsorbedMagic || !ab->W_UKt) return GDLA_ERR_INVALID_ARG;
@@ -357,13 +435,15 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   np.D1 = D1; np.ld1 = ld1; np.M = B; np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank;
   np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
   np.cQ = cQ; np.latent = nullptr; np.kR16 = nullptr; np.lam = lam; np.pos_T = 1;
-  np.pos_ptr = cache_len; np.cache = kv_cache; np.cache_cap = cap; np.rope = rope; np.err = err;
+  np.pos_ptr = cache_len; np.q_per_seq = q_len; np.cache = kv_cache; np.cache_cap = cap;
+  np.rope = rope; np.err = err;
   if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
 
   const int nqq = nH * (cfg->d_nope + cfg->d_rope);
   GemmEpi eq{};
   eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F32; eq.M = B; eq.N = nqq;
   eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = 1; eq.pos_ptr = cache_len;
+  eq.pos_div = q_len;
   eq.rope = rope; eq.splitk = splitk; eq.splitk_floats = splitk_n;
   if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, B, nqq, cfg->q_rank, eq, ctl, st)))
     return GDLA_ERR_LAUNCH;
@@ -381,6 +461,7 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
   stage(1, st);
   DecAttnParams dp{};
   dp.B = B; dp.cap = cap; dp.window = cfg->window; dp.n_split = nsplit; dp.cache_len = cache_len;
+  dp.q_len = q_len;
   dp.cache = kv_cache; dp.qt = qt;
   dp.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
   dp.part = part; dp.ml = ml; dp.err = err;

@@ -66,15 +66,29 @@ __global__ void __launch_bounds__(384, 1)
   AttnBars* bars = reinterpret_cast<AttnBars*>(smem + BAR_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work unit (heaviest causal units first)
-  const int n_pairs = (p.T + 255) / 256;
-  const int per_c = p.B * p.n_groups;
-  const int c = n_pairs - 1 - int(blockIdx.x) / per_c;
-  const int b = (int(blockIdx.x) % per_c) / p.n_groups;
-  const int j = int(blockIdx.x) % p.n_groups;
+  // ---- work unit: (sequence rows [rowbase, rowbase + T), KV head j, 256-row pair c), heaviest
+  // causal units first.  Equal-length batches derive it from blockIdx; packed documents read
+  // it from a schedule built on the device (surplus CTAs of the upper-bound grid exit here).
+  int c, rowbase, T, j;
+  if (p.units) {
+    const int u = int(blockIdx.x) / p.n_groups;
+    if (u >= *p.n_units) return;
+    const int4 un = p.units[u];
+    rowbase = un.x;
+    T = un.y;
+    c = un.z;
+    j = int(blockIdx.x) % p.n_groups;
+  } else {
+    const int n_pairs = (p.T + 255) / 256;
+    const int per_c = p.B * p.n_groups;
+    c = n_pairs - 1 - int(blockIdx.x) / per_c;
+    const int b = (int(blockIdx.x) % per_c) / p.n_groups;
+    j = int(blockIdx.x) % p.n_groups;
+    rowbase = b * p.T;
+    T = p.T;
+  }
   const int q0 = 256 * c;
-  const int rowbase = b * p.T;
-  const int t_hi = min(p.T - 1, q0 + 255) / 128;
+  const int t_hi = min(T - 1, q0 + 255) / 128;
   const int t_lo = p.window > 0 ? max(0, q0 - p.window + 1) / 128 : 0;
   const int n_kv = t_hi - t_lo + 1;
 
@@ -271,7 +285,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tmem + s * 128 + lane_off;
     const uint32_t tO = tmem + 256 + s * 128 + lane_off;
     const int qpos = q0 + 128 * s + r;
-    const bool row_valid = qpos < p.T;
+    const bool row_valid = qpos < T;
     const long long m_row = (long long)rowbase + qpos;
     const int W = p.window;
     uint32_t sf_par = 0;
@@ -362,7 +376,8 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(&bars->o_free[s]);
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-      if (!row_valid || *reinterpret_cast<volatile int*>(ctl.err) != 0) continue;
+      if (!row_valid || m_row >= (long long)p.B * p.T || *reinterpret_cast<volatile int*>(ctl.err) != 0)
+        continue;
       float* on_row = p.O_noise + (m_row * p.n_groups + j) * 128;
       if (pass == 0) {
 #pragma unroll
@@ -410,7 +425,7 @@ __global__ void __launch_bounds__(384, 1)
 int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* kR16,
                         const AttnParams& p, KernelCtlHost ctl, cudaStream_t st) {
   if (p.B <= 0 || p.T <= 0) return 0;
-  const long long M = (long long)p.B * p.T;
+  const long long M = (long long)p.B * p.T;   // rows of the (packed) token matrix
   CUtensorMap mq, mkv, mkr;
   if (make_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, QQ, qq_ld, M, (uint64_t)qq_ld * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -422,8 +437,7 @@ int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* k
   if (cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            attn::SMEM) != cudaSuccess)
     return -4;
-  const int n_pairs = (p.T + 255) / 256;
-  const int grid = n_pairs * p.B * p.n_groups;
+  const int grid = p.units ? p.max_units * p.n_groups : ((p.T + 255) / 256) * p.B * p.n_groups;
   KernelCtl kc{ctl.err, ctl.limit_ns};
   attn_prefill_kernel<<<grid, 384, attn::SMEM, st>>>(mq, mkv, mkr, p, kc);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;

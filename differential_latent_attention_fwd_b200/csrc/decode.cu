@@ -41,39 +41,59 @@ int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int 
 }
 
 // q~ rows: qt[b][h][0..511] = W_UK_j q^C_h, qt[b][h][512..575] = rotated q^R_h (bf16).
-// One CTA per (sequence b, KV head j) serves the group's g + 1 heads.
+// CTA (KV head j, 4 rows b): W_UK_j^T (128 x 512 bf16, 128 KB) is staged in shared memory with
+// asynchronous copies, then 20 query rows (4 rows x the group's 5 heads) are projected.
 __global__ void __launch_bounds__(256) qtilde_kernel(DecQParams p) {
-  const int b = blockIdx.x, j = blockIdx.y;
-  __shared__ float qc[5][128];
-  const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
-  for (int i = threadIdx.x; i < 5 * 128; i += blockDim.x) {
-    const int hh = i / 128, c = i % 128;
-    qc[hh][c] = p.QQ[(long long)b * p.qq_ld + heads[hh] * 128 + c];
-  }
-  __syncthreads();
+  extern __shared__ uint8_t qt_smem[];
+  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(qt_smem);            // [128][512]
+  float (*qc)[128] = reinterpret_cast<float (*)[128]>(qt_smem + 128 * 512 * 2);  // [20][128]
+  const int j = blockIdx.x, b0 = blockIdx.y * 4, tid = threadIdx.x;
+  const int nb = min(4, p.B - b0);
   const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_UKt) + (long long)j * 128 * 512;
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.qt);
-  for (int l = threadIdx.x; l < 512; l += blockDim.x) {
-    float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int c = 0; c < 128; ++c) {
-      const float w = __bfloat162float(W[c * 512 + l]);
-#pragma unroll
-      for (int hh = 0; hh < 5; ++hh) acc[hh] += w * qc[hh][c];
-    }
-#pragma unroll
-    for (int hh = 0; hh < 5; ++hh)
-      out[((long long)b * p.n_heads + heads[hh]) * 576 + l] = __float2bfloat16_rn(acc[hh]);
+  for (int i = tid; i < 128 * 512 / 8; i += blockDim.x) cp_async16(wsm + i * 8, W + i * 8);
+  const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
+  for (int i = tid; i < 20 * 128; i += blockDim.x) {
+    const int r = i / 128, c = i % 128, bb = r / 5, hh = r % 5;
+    qc[r][c] = bb < nb ? p.QQ[(long long)(b0 + bb) * p.qq_ld + heads[hh] * 128 + c] : 0.f;
   }
-  for (int i = threadIdx.x; i < 5 * 64; i += blockDim.x) {
-    const int hh = i / 64, r = i % 64;
-    out[((long long)b * p.n_heads + heads[hh]) * 576 + 512 + r] =
-        __float2bfloat16_rn(p.QQ[(long long)b * p.qq_ld + p.rope_col0 + heads[hh] * 64 + r]);
+  cp_async_wait_all();
+  __syncthreads();
+  // thread: latent columns 2 tid, 2 tid + 1 of all 20 rows
+  float acc[20][2];
+#pragma unroll
+  for (int r = 0; r < 20; ++r) acc[r][0] = acc[r][1] = 0.f;
+#pragma unroll 2
+  for (int c = 0; c < 128; ++c) {
+    const __nv_bfloat162 w2 = *reinterpret_cast<const __nv_bfloat162*>(wsm + c * 512 + 2 * tid);
+    const float w0 = __low2float(w2), w1 = __high2float(w2);
+#pragma unroll
+    for (int r = 0; r < 20; ++r) {
+      const float q = qc[r][c];
+      acc[r][0] = fmaf(q, w0, acc[r][0]);
+      acc[r][1] = fmaf(q, w1, acc[r][1]);
+    }
+  }
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.qt);
+#pragma unroll
+  for (int r = 0; r < 20; ++r) {
+    const int bb = r / 5, hh = r % 5;
+    if (bb >= nb) continue;
+    *reinterpret_cast<uint32_t*>(out + ((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 2 * tid) =
+        pack_bf162(acc[r][0], acc[r][1]);
+  }
+  for (int i = tid; i < 4 * 5 * 64; i += blockDim.x) {
+    const int r = i / 64, e = i % 64, bb = r / 5, hh = r % 5;
+    if (bb >= nb) continue;
+    out[((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 512 + e] =
+        __float2bfloat16_rn(p.QQ[(long long)(b0 + bb) * p.qq_ld + p.rope_col0 + heads[hh] * 64 + e]);
   }
 }
 
 int launch_qtilde(const DecQParams& p, cudaStream_t st) {
-  dim3 grid(p.B, p.n_groups);
-  qtilde_kernel<<<grid, 256, 0, st>>>(p);
+  const int smem = 128 * 512 * 2 + 20 * 128 * 4;
+  if (cudaFuncSetAttribute(qtilde_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return -4;
+  qtilde_kernel<<<dim3(p.n_groups, (p.B + 3) / 4), 256, smem, st>>>(p);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
@@ -133,13 +153,14 @@ __global__ void __launch_bounds__(256) dec_uv_gate_kernel(DecCombParams p) {
   const int nrows = min(4, p.B - b0) * 4;
   const long long ldw = (long long)p.n_groups * 256;
   const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_bKV) + j * 256 + 128;
-  for (int i = tid; i < 512 * 16; i += blockDim.x) {          // 16 uint4 per 128-column row
+  for (int i = tid; i < 512 * 16; i += blockDim.x) {          // 16 x 16 bytes per 128-column row
     const int l = i >> 4, q = i & 15;
-    reinterpret_cast<uint4*>(wsm + l * 128)[q] = reinterpret_cast<const uint4*>(W + l * ldw)[q];
+    cp_async16(wsm + l * 128 + q * 8, W + l * ldw + q * 8);
   }
   const float* src = p.Dlat + ((long long)j * p.B + b0) * 4 * 512;
   for (int i = tid; i < 16 * 512; i += blockDim.x)
     dl[i / 512][i % 512] = (i / 512) < nrows ? src[i] : 0.f;
+  cp_async_wait_all();
   __syncthreads();
   const int cq = tid & 31;          // columns 4 cq .. 4 cq + 3
   const int rp = tid >> 5;          // rows 2 rp, 2 rp + 1

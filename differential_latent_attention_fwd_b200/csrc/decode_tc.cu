@@ -58,8 +58,12 @@ struct DecRange {
 };
 __device__ __forceinline__ DecRange dec_range(const DecAttnParams& p, int b, int sp, int* err) {
   DecRange r;
-  int L = p.cache_len[b];
-  if (L < 0 || L >= p.cap) {
+  // row b is new token b % q_len of its sequence: it sees the cached keys and the new tokens
+  // up to itself, all held in the cache rows 0 .. cache_len + b % q_len
+  const int ql = p.q_len > 1 ? p.q_len : 1;
+  const int L0 = p.cache_len[b / ql];
+  int L = L0 + b % ql;
+  if (L0 < 0 || L0 + ql - 1 >= p.cap) {
     if (threadIdx.x == 0) atomicCAS(err, 0, SITE_BAD_CACHE_LEN);
     r.lo = 0; r.hi = -1; r.t_begin = 0; r.t_end = 0;
     return r;
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const long long crow0 = (long long)b * p.cap;
+  const long long crow0 = (long long)(b / (p.q_len > 1 ? p.q_len : 1)) * p.cap;
 
   if (warp == 0) {
     if (lane == 0 && n_t > 0) {

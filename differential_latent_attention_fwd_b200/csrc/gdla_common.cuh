@@ -32,6 +32,7 @@ enum : int {
   SITE_DRAIN = 0x301, SITE_SELFTEST = 0x401,
   SITE_DEC_PRODUCER = 0x501, SITE_DEC_MMA = 0x502, SITE_DEC_SOFTMAX = 0x503,
   SITE_BAD_CACHE_LEN = 0x601,  // a cache_len entry outside [0, cap): that sequence is skipped
+  SITE_BAD_CU_SEQLENS = 0x602, // document offsets not 0..total non-decreasing: bad documents skipped
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -238,6 +239,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
         "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),         \
         "r"(r[14]), "r"(r[15])                                                                   \
       : "memory")
+
+// 16-byte asynchronous global -> shared copy (all of a thread's copies stay in flight).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
 
 // Make generic-proxy writes to shared memory visible to the async proxy (TMA, tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -16,8 +16,9 @@ struct DecQParams {
 };
 
 struct DecAttnParams {
-  int B, cap, window, n_split;
-  const int* cache_len;   // [B] keys before the new token (its row sits at cache_len[b])
+  int B, cap, window, n_split;   // B = query rows = sequences x q_len
+  int q_len;              // new tokens per sequence: row r is token r % q_len of sequence r / q_len
+  const int* cache_len;   // [sequences] keys cached before the new tokens
   const void* cache;      // bf16 [B][cap][576]
   const void* qt;         // bf16 [B][80][576]
   float scale_log2;

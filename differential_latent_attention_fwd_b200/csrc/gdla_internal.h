@@ -24,7 +24,8 @@ struct GemmEpi {
   int M, N;
   int rope_lo, rope_hi;  // columns [rope_lo, rope_hi) (multiples of 64) hold 64-wide rope heads
   int pos_T;             // row position = row % pos_T (used when pos_ptr is null)
-  const int* pos_ptr;    // row position = pos_ptr[row]
+  const int* pos_ptr;    // row position = pos_ptr[row / pos_div] + row % pos_div
+  int pos_div;           // rows per pos_ptr entry (0 is read as 1)
   RopeTable rope;
   // Optional split-K scratch for skinny products (M <= 128): fp32 [splits][M][N].  When set
   // and worthwhile, K is split across CTAs and a reduce kernel applies this epilogue.
@@ -74,7 +75,8 @@ struct NormParams {
   void* kR16;                 // fp16 [M, 64] or null
   float* lam;                 // [M, n_signal]
   int pos_T;                  // prefill: pos = m % pos_T, sequence = m / pos_T
-  const int* pos_ptr;         // decode: pos = pos_ptr[m], sequence = m
+  const int* pos_ptr;         // decode: sequence = m / q_per_seq, pos = pos_ptr[sequence] + m % q_per_seq
+  int q_per_seq;              // new tokens per sequence (0 is read as 1)
   void* cache;                // optional bf16 [n_seq, cache_cap, kv_rank + 64]
   long long cache_cap;
   int* err;                   // device error word (bad cache_len is reported here)
@@ -93,7 +95,18 @@ struct AttnParams {
   const void* G;              // bf16 [B*T, n_signal*128] gate logits
   float* O_noise;             // [B*T, n_groups, 128] fp32 scratch
   void* Dg;                   // bf16 [B*T, n_signal*128]
+  // Packed documents (B = 1, T = all tokens): device schedule of work units
+  // {first row, document length, 256-row pair index, 0}; null for equal-length batches.
+  const int4* units;
+  const int* n_units;
+  int max_units;              // grid bound (units beyond *n_units exit at once)
 };
+
+// Device schedule of packed documents: per-token positions and the attention work units,
+// counting-sorted by pair index (heaviest causal units first).  Scratch: cnt/fill [max_c].
+int launch_varlen_schedule(const int* cu_seqlens, int n_docs, int total, int* positions,
+                           int4* units, int* n_units, int max_units, int* cnt, int* fill, int max_c,
+                           int* err, cudaStream_t st);
 int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* kR16,
                         const AttnParams& p, KernelCtlHost ctl, cudaStream_t st);
 

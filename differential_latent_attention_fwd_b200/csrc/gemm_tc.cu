@@ -114,7 +114,10 @@ __global__ void __launch_bounds__(128, 1)
   const int row = m0 + warp * 32 + lane;
   const bool row_ok = ok && row < ep.M && *reinterpret_cast<volatile int*>(ctl.err) == 0;
   int pos = 0;
-  if (ep.rope_hi > ep.rope_lo && row < ep.M) pos = ep.pos_ptr ? ep.pos_ptr[row] : (row % ep.pos_T);
+  if (ep.rope_hi > ep.rope_lo && row < ep.M) {
+    const int dv = ep.pos_div > 1 ? ep.pos_div : 1;
+    pos = ep.pos_ptr ? ep.pos_ptr[row / dv] + row % dv : (row % ep.pos_T);
+  }
   const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 64) {
@@ -202,7 +205,8 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
     b += pz[c2];
   }
   if (blk * 64 >= ep.rope_lo && blk * 64 < ep.rope_hi) {
-    const int pos = ep.pos_ptr ? ep.pos_ptr[row] : (row % ep.pos_T);
+    const int dv = ep.pos_div > 1 ? ep.pos_div : 1;
+    const int pos = ep.pos_ptr ? ep.pos_ptr[row / dv] + row % dv : (row % ep.pos_T);
     float cs, sn;
     rope_cs(pos, ep.rope.inv_freq[i], &cs, &sn);
     const float x1 = a, x2 = b;

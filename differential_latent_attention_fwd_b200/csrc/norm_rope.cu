@@ -72,8 +72,9 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(const __grid_constant__ 
   const float rkvn = rsqrtf(ss / float(p.kv_rank) + p.eps);
 
   // ---- k^R rotation: lane owns the pair (lane, lane + 32)
-  int pos = p.pos_ptr ? p.pos_ptr[m] : (m % p.pos_T);
-  const int seq = p.pos_ptr ? m : (m / p.pos_T);
+  const int qps = p.q_per_seq > 1 ? p.q_per_seq : 1;
+  int pos = p.pos_ptr ? p.pos_ptr[m / qps] + m % qps : (m % p.pos_T);
+  const int seq = p.pos_ptr ? m / qps : (m / p.pos_T);
   bool cache_ok = p.cache != nullptr;
   if (cache_ok && (pos < 0 || pos >= p.cache_cap)) {
     if (lane == 0 && p.err) atomicCAS(p.err, 0, SITE_BAD_CACHE_LEN);

@@ -41,6 +41,16 @@ class GdlaLayer:
         gb.gdla_prefill_fwd(self.cfg, self.cw, x, y, ws, kv_cache_out, cap, stream)
         return y
 
+    def prefill_packed(self, x: torch.Tensor, cu_seqlens: torch.Tensor, y: torch.Tensor | None = None,
+                       kv_latent_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """Independent documents packed row-wise in x [total, d]; cu_seqlens int32 [docs + 1]."""
+        total, d = x.shape
+        if y is None:
+            y = torch.empty((total, d), dtype=torch.bfloat16, device=self.device)
+        ws = self.workspace(1, total, gb.GDLA_MODE_VARLEN)
+        gb.gdla_prefill_varlen_fwd(self.cfg, self.cw, x, cu_seqlens, y, ws, kv_latent_out, stream)
+        return y
+
     def absorbed(self, stream=None) -> gb.gdla_absorbed_t:
         if self._absorbed is None:
             n = gb.gdla_absorbed_size(self.cfg)
@@ -55,4 +65,15 @@ class GdlaLayer:
             y = torch.empty((B, d), dtype=torch.bfloat16, device=self.device)
         ws = self.workspace(B, kv_cache.shape[1], gb.GDLA_MODE_DECODE)
         gb.gdla_decode_fwd(self.cfg, self.absorbed(stream), x_new, kv_cache, cache_len, y, ws, stream)
+        return y
+
+    def decode_multi(self, x_new: torch.Tensor, kv_cache: torch.Tensor, cache_len: torch.Tensor,
+                     y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """x_new [n_seq, q_len, d]: q_len consecutive new tokens per sequence in one call."""
+        n_seq, q_len, d = x_new.shape
+        if y is None:
+            y = torch.empty((n_seq, q_len, d), dtype=torch.bfloat16, device=self.device)
+        ws = self.workspace(n_seq * q_len, kv_cache.shape[1], gb.GDLA_MODE_DECODE)
+        gb.gdla_decode_multi_fwd(self.cfg, self.absorbed(stream), x_new, kv_cache, cache_len, y, ws,
+                                 stream)
         return y

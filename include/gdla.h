@@ -87,10 +87,11 @@ typedef struct {
   uint32_t magic;
 } gdla_absorbed_t;
 
-enum { GDLA_MODE_PREFILL = 0, GDLA_MODE_DECODE = 1 };
+enum { GDLA_MODE_PREFILL = 0, GDLA_MODE_DECODE = 1, GDLA_MODE_VARLEN = 2 };
 
-/* Bytes of workspace that gdla_prefill_fwd (mode 0: B sequences of T tokens) or
- * gdla_decode_fwd (mode 1: B sequences, T = the cache capacity `cap` of the call) needs. */
+/* Bytes of workspace that gdla_prefill_fwd (mode 0: B sequences of T tokens),
+ * gdla_decode_fwd (mode 1: B sequences, T = the cache capacity `cap` of the call) or
+ * gdla_prefill_varlen_fwd (mode 2: B = 1, T = total packed tokens) needs. */
 int gdla_workspace_size(const gdla_config_t* cfg, int B, int T, int mode, size_t* bytes);
 
 /* Bytes of device memory gdla_absorb_weights writes. */
@@ -105,6 +106,21 @@ int gdla_absorbed_size(const gdla_config_t* cfg, size_t* bytes);
 int gdla_prefill_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int B,
                      int T, void* y, void* kv_cache_out, int cache_cap, void* workspace,
                      size_t ws_bytes, void* stream);
+
+/* Prefill of packed documents.  The long-context workload of the report packs many documents
+ * into one sequence (paperglide.net summary, Figure 4a); here each document is an independent
+ * sequence: rotary positions restart at 0 and attention (causal or sliding window) never
+ * crosses a document boundary.
+ *   x [total, d_model] bf16; y [total, d_model] bf16 (written).
+ *   cu_seqlens: int32 [n_docs + 1] (device): document d is rows cu[d] .. cu[d+1]-1; cu[0] = 0,
+ *     non-decreasing, cu[n_docs] = total (violations are reported through the device error
+ *     word, and the offending documents are skipped).  n_docs <= total.
+ *   kv_latent_out: NULL, or bf16 [total, kv_rank + d_rope]: the latent-cache row of every token,
+ *     in packed order.
+ *   workspace: >= gdla_workspace_size(cfg, 1, total, GDLA_MODE_VARLEN) bytes. */
+int gdla_prefill_varlen_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x,
+                            int total, const int* cu_seqlens, int n_docs, void* y,
+                            void* kv_latent_out, void* workspace, size_t ws_bytes, void* stream);
 
 /* One-time weight preparation for the absorbed-form decode (MLA-style weight absorption:
  * attention runs in the latent space and K/V are never materialised; the pages note that
@@ -125,6 +141,20 @@ int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void*
 int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* absorbed, const void* x_new,
                     void* kv_cache, const int* cache_len, int cap, int B, void* y,
                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Decode of q_len new tokens per sequence at once (e.g. verifying tokens drafted by a
+ * multi-token-prediction head; the report ships such a head for self-speculative decoding,
+ * alphasignal.ai news page).  Token i of sequence b sits at position cache_len[b] + i, its
+ * latent-cache entry is written to row cache_len[b] + i (so cache_len[b] + q_len <= cap), and
+ * it attends to rows 0 .. cache_len[b] + i (or the last `window` of them): exactly what q_len
+ * consecutive single-token decode calls compute.
+ *   x_new [n_seq, q_len, d_model] bf16; y [n_seq, q_len, d_model] bf16 (written).
+ *   workspace: >= gdla_workspace_size(cfg, n_seq * q_len, cap, GDLA_MODE_DECODE) bytes.
+ * gdla_decode_fwd is the q_len = 1 case. */
+int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* absorbed,
+                          const void* x_new, int q_len, void* kv_cache, const int* cache_len,
+                          int cap, int n_seq, void* y, void* workspace, size_t ws_bytes,
+                          void* stream);
 
 /* Reads (and with clear != 0 resets) the device error word after synchronising `stream`:
  * *site = 0 when every kernel finished normally, else the site code of the first bounded wait

@@ -359,6 +359,19 @@ def gdla_prefill(x, weights: dict, cfg: OracleConfig, rows=None, g_q=None, g_kv=
     return (y, parts) if return_parts else y
 
 
+def gdla_prefill_packed(x_packed, cu_seqlens, weights: dict, cfg: OracleConfig, g_q=None, g_kv=None):
+    """Packed documents: document d = rows cu[d] .. cu[d+1]-1 of x_packed [total, d_model] is an
+    independent sequence (its own positions from 0, attention inside the document only).
+    Returns y [total, d_model] in packed order."""
+    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    out = np.empty((cu[-1], cfg.d_model))
+    for d in range(len(cu) - 1):
+        if cu[d + 1] > cu[d]:
+            out[cu[d]: cu[d + 1]] = gdla_prefill(x_packed[None, cu[d]: cu[d + 1]], weights, cfg,
+                                                  g_q=g_q, g_kv=g_kv)[0]
+    return out
+
+
 # --------------------------------------------------------------------------------------
 # full layer: decode (one new token per sequence, keys = cached latent rows + itself)
 # --------------------------------------------------------------------------------------
@@ -443,4 +456,28 @@ def gdla_decode_absorbed(x_new, weights: dict, cache, cache_len, cfg: OracleConf
         D = np.stack([Dlat[s_] @ W_UV[kvh[s_]] for s_ in range(cfg.n_signal)])
         Dg = sigmoid(G[b]) * D
         y[b] = Dg.reshape(-1) @ W["W_O"]
+    return y
+
+
+def gdla_decode_multi(x_new, weights: dict, cache, cache_len, cfg: OracleConfig, g_q=None, g_kv=None,
+                      route: str = "literal"):
+    """q_len new tokens per sequence: x_new [B, q_len, d].  Token i of sequence b is at position
+    cache_len[b] + i and sees the cached rows plus new tokens 0..i; this is q_len consecutive
+    single-token decodes, each over the cache extended by the earlier new tokens' latent rows
+    (computed here in float64).  route selects the literal or the weight-absorbed decode.
+    Returns y [B, q_len, d]."""
+    W = _weights64(weights)
+    gkv = None if g_kv is None else f64(g_kv)
+    one = gdla_decode if route == "literal" else gdla_decode_absorbed
+    xn = f64(x_new)
+    B, q = xn.shape[0], xn.shape[1]
+    lens = [int(v) for v in (cache_len.tolist() if hasattr(cache_len, "tolist") else cache_len)]
+    y = np.empty((B, q, cfg.d_model))
+    for b in range(B):
+        L = lens[b]
+        rows = f64(cache[b, :L]) if L else np.zeros((0, cfg.kv_rank + cfg.d_rope))
+        cbar, kR = kv_latent(xn[b], W["W_aKV"], gkv, L + np.arange(q), cfg)
+        ext = np.concatenate([rows, np.concatenate([cbar, kR], -1)], 0)[None]
+        for i in range(q):
+            y[b, i] = one(xn[b, i][None], weights, ext, [L + i], cfg, g_q=g_q, g_kv=g_kv)[0]
     return y

@@ -80,3 +80,49 @@ def test_bounded_wait_expires_and_context_survives(cuda_ok):
     torch.cuda.synchronize()
     assert gb.gdla_device_error() == 0
     check("prefill after the timeout self-test", to_np(y[0]), oracle_prefill(inp)[0])
+
+
+@pytest.mark.parametrize("window", [0, 64])
+def test_multi_token_decode(cuda_ok, window):
+    """Three new tokens per sequence in one call (multi-token verification) against the oracle,
+    including the three appended latent-cache rows."""
+    from differential_latent_attention_fwd_b200 import synth as S
+    shape = S.GdlaShape(window=window)
+    lens, q = [0, 50, 300], 3
+    inp = S.make_decode_inputs(shape, 3, lens, cap=320, seed=31)
+    xm = torch.randn((3, q, shape.d_model), generator=torch.Generator().manual_seed(5)).bfloat16()
+    layer = GdlaLayer(shape, inp.weights, inp.g_q, inp.g_kv, device="cuda")
+    cache = inp.cache.cuda()
+    y = layer.decode_multi(xm.cuda(), cache, inp.cache_len.cuda())
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
+    cfg = O.OracleConfig.from_shape(shape)
+    yo = O.gdla_decode_multi(xm, inp.weights, inp.cache, inp.cache_len, cfg, g_q=inp.g_q, g_kv=inp.g_kv)
+    errs = []
+    for b in range(3):
+        for i in range(q):
+            check(f"multi-token decode b={b} token {i} (len {lens[b]}, W={window})", to_np(y[b, i]),
+                  yo[b, i], errors=errs)
+    # appended rows: the q new latent rows sit at cache_len .. cache_len + q - 1
+    W64 = {k: O.f64(v) for k, v in inp.weights.items()}
+    for b in range(3):
+        cb, kr = O.kv_latent(O.f64(xm[b]), W64["W_aKV"], None, lens[b] + np.arange(q), cfg)
+        check(f"appended rows b={b}", to_np(cache[b, lens[b]:lens[b] + q]), np.concatenate([cb, kr], -1),
+              rel=4e-3, mabs=5e-2, errors=errs)
+    assert not errs, "\n".join(errs)
+
+
+def test_multi_token_decode_workload_size(cuda_ok):
+    """B=64 sequences x 2 new tokens over a 32768-position cache (absorbed oracle)."""
+    from differential_latent_attention_fwd_b200 import synth as S
+    shape = S.GdlaShape()
+    inp = S.make_decode_inputs(shape, 64, 32768, cap=32770, seed=4)
+    xm = torch.randn((64, 2, shape.d_model), generator=torch.Generator().manual_seed(6)).bfloat16()
+    layer = GdlaLayer(shape, inp.weights, inp.g_q, inp.g_kv, device="cuda")
+    y = layer.decode_multi(xm.cuda(), inp.cache.cuda(), inp.cache_len.cuda())
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
+    cfg = O.OracleConfig.from_shape(shape)
+    yo = O.gdla_decode_multi(xm, inp.weights, inp.cache, inp.cache_len, cfg, g_q=inp.g_q, g_kv=inp.g_kv,
+                             route="absorbed")
+    check("B64 x 2 tokens, L=32768", to_np(y).reshape(128, -1), yo.reshape(128, -1))

@@ -133,3 +133,45 @@ def test_workload_t262144_swa2048_sampled(cuda_ok):
 
 def test_workload_t262144_causal_sampled(cuda_ok):
     _sampled_workload("prefill_b1_t262144_causal")
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_packed_documents(cuda_ok, window):
+    """Packed documents (ragged lengths incl. 1, exact multiples of 128/256 and a tail) against
+    the oracle run per document, and the packed latent rows against the oracle's."""
+    from oracle import gdla_oracle as O
+    lens = [1, 100, 256, 513, 37, 300, 128]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total = int(cu[-1])
+    shape, inp, layer, x = prefill_case(1, total, window, seed=23)
+    xp = x[0].contiguous()
+    lat = torch.zeros((total, 576), dtype=torch.bfloat16, device="cuda")
+    y = layer.prefill_packed(xp, torch.from_numpy(cu).cuda(), kv_latent_out=lat)
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
+    cfg = O.OracleConfig.from_shape(shape)
+    yo = O.gdla_prefill_packed(inp.x[0], cu, inp.weights, cfg, g_q=inp.g_q, g_kv=inp.g_kv)
+    errs = []
+    for d in range(len(lens)):
+        a, b = int(cu[d]), int(cu[d + 1])
+        check(f"doc {d} (len {lens[d]}, W={window})", to_np(y[a:b]), yo[a:b], errors=errs)
+    assert not errs, "\n".join(errs)
+    # the same documents run one by one through the batch entry point give the same rows
+    for d in (2, 3):
+        a, b = int(cu[d]), int(cu[d + 1])
+        yd = layer.prefill(xp[a:b][None].contiguous())
+        torch.cuda.synchronize()
+        check(f"doc {d}: packed vs standalone GPU run", to_np(y[a:b]), to_np(yd[0]), rel=1e-6, mabs=1e-5)
+    # latent rows: positions restart inside every document
+    _, parts = O.gdla_prefill(inp.x[:, cu[3]:cu[4]], inp.weights, cfg, g_q=inp.g_q, g_kv=inp.g_kv,
+                              return_parts=True)
+    want = np.concatenate([parts[0]["cbar"], parts[0]["kR"]], -1)
+    check("packed latent rows of doc 3", to_np(lat[cu[3]:cu[4]]), want, rel=4e-3, mabs=5e-2)
+
+
+def test_packed_documents_reject_bad_offsets(cuda_ok):
+    shape, inp, layer, x = prefill_case(1, 64, 0, seed=2)
+    bad = torch.tensor([0, 40, 30, 64], dtype=torch.int32, device="cuda")   # decreasing offset
+    layer.prefill_packed(x[0].contiguous(), bad)
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0x602

@@ -399,3 +399,38 @@ def test_prefill_row_subsets_and_order_agree():
         rows = [39, 3, 17, 0, 25, 26, 8]
         sub = O.gdla_prefill(x, W, cfg, rows=rows)
         np.testing.assert_allclose(sub, full[:, rows], rtol=1e-12, atol=1e-13)
+
+
+def test_packed_documents_do_not_interact():
+    """Packed prefill: perturbing one document changes no other document's rows, and a
+    document's rows equal a standalone run of that document."""
+    cfg = tiny_cfg(window=3)
+    W = tiny_weights(cfg)
+    x = tiny_x(cfg, 1, 17)[0]
+    cu = [0, 5, 6, 13, 17]
+    y = O.gdla_prefill_packed(x, cu, W, cfg)
+    x2 = x.copy()
+    x2[6:13] += 1.0
+    y2 = O.gdla_prefill_packed(x2, cu, W, cfg)
+    np.testing.assert_array_equal(y2[:6], y[:6])
+    np.testing.assert_array_equal(y2[13:], y[13:])
+    assert np.abs(y2[6:13] - y[6:13]).min() > 0
+    np.testing.assert_allclose(y[13:17], O.gdla_prefill(x[None, 13:17], W, cfg)[0], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("window", [0, 3])
+def test_multi_token_decode_continues_prefill(window):
+    """q_len tokens decoded at once over prefill's latent rows of the earlier tokens equal the
+    prefill rows of those tokens (literal and absorbed routes)."""
+    cfg = tiny_cfg(window=window)
+    W = tiny_weights(cfg)
+    T = 11
+    x = tiny_x(cfg, 1, T)
+    y, parts = O.gdla_prefill(x, W, cfg, return_parts=True)
+    rows = np.concatenate([parts[0]["cbar"], parts[0]["kR"]], -1)
+    t0, q = 7, 4
+    cache = np.zeros((1, T, rows.shape[1]))
+    cache[0, :t0] = rows[:t0]
+    for route in ("literal", "absorbed"):
+        ym = O.gdla_decode_multi(x[:, t0:t0 + q], W, cache, [t0], cfg, route=route)
+        np.testing.assert_allclose(ym[0], y[0, t0:t0 + q], rtol=1e-10, atol=1e-11)
