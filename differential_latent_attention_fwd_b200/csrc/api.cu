@@ -66,10 +66,13 @@ static int check_weights(const gdla_weights_t* w) {
 enum { WS_D1, WS_CQ, WS_LATENT, WS_LAM, WS_QQ, WS_G, WS_KV, WS_ONOISE, WS_DG, WS_KR16, WS_SPLITK,
        WS_VL_POS, WS_VL_UNITS, WS_VL_COUNT, WS_N };
 
-// Packed documents: bounds of the attention schedule for `total` tokens in up to `total`
-// non-empty documents (sum over documents of ceil(len / 256) <= total / 256 + documents).
-static int varlen_max_pairs(long long total) { return int((total + 255) / 256); }
-static int varlen_max_units(long long total) { return int(total + (total + 255) / 256); }
+// Packed documents: bounds of the attention schedule for `total` tokens in `n_docs` documents
+// (sum over documents of ceil(len / R) <= ceil(total / R) + n_docs, R = ATTN_UNIT_ROWS).  The
+// workspace is sized for n_docs = total; the grid uses the actual document count.
+static int varlen_max_blocks(long long total) { return int((total + ATTN_UNIT_ROWS - 1) / ATTN_UNIT_ROWS); }
+static int varlen_max_units(long long total, long long n_docs) {
+  return int(varlen_max_blocks(total) + (n_docs < total ? n_docs : total));
+}
 
 // fp32 scratch of the split-K projections of a decode step (skinny M = B products).
 static long long decode_splitk_floats(const gdla_config_t* c, int B) {
@@ -100,14 +103,14 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
   sz[WS_VL_POS] = sz[WS_VL_UNITS] = sz[WS_VL_COUNT] = 0;
   if (mode == GDLA_MODE_VARLEN) {
     sz[WS_VL_POS] = M * 4;
-    sz[WS_VL_UNITS] = (size_t)varlen_max_units(M) * 16;
-    sz[WS_VL_COUNT] = (size_t)(1 + 2 * varlen_max_pairs(M)) * 4;
+    sz[WS_VL_UNITS] = (size_t)varlen_max_units(M, M) * 16;
+    sz[WS_VL_COUNT] = (size_t)(1 + 2 * varlen_max_blocks(M)) * 4;
   }
   if (mode == GDLA_MODE_PREFILL || mode == GDLA_MODE_VARLEN) {
     sz[WS_LATENT] = M * (c->kv_rank + c->d_rope) * 2;
     sz[WS_QQ] = M * qq * 2;
     sz[WS_KV] = M * (long long)c->n_kv_heads * (c->d_nope + c->d_v) * 2;
-    sz[WS_ONOISE] = M * (long long)c->n_noise * c->d_v * 4;
+    sz[WS_ONOISE] = ((M + 31) / 32 * 32) * (long long)c->n_noise * c->d_v * 4;   // 32-row blocks
     sz[WS_KR16] = M * c->d_rope * 2;
     sz[WS_SPLITK] = 0;
   } else {
@@ -179,8 +182,8 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
     int* pos = reinterpret_cast<int*>(ws + off[WS_VL_POS]);
     int4* un = reinterpret_cast<int4*>(ws + off[WS_VL_UNITS]);
     int* cnt = reinterpret_cast<int*>(ws + off[WS_VL_COUNT]);
-    max_units = varlen_max_units(M);
-    const int max_c = varlen_max_pairs(M);
+    max_units = varlen_max_units(M, vl->n_docs);
+    const int max_c = varlen_max_blocks(M);
     if (launch_failed(launch_varlen_schedule(vl->cu_seqlens, vl->n_docs, M, pos, un, cnt, max_units,
                                              cnt + 1, cnt + 1 + max_c, max_c, err, st)))
       return GDLA_ERR_LAUNCH;

@@ -8,87 +8,167 @@
 //   D_s = H_s - lambda_{t,s} H_noise(j)           Dg_s = sigmoid(G_{t,s}) (.) D_s
 // and writes Dg (bf16, head-major) for the output projection.
 //
-// Work unit (one CTA): sequence b, KV head j, and 256 consecutive query positions split into
-// two 128-row tiles ("slots").  The unit runs five passes, one per head of the group: first
-// the noise head (its normalised output is parked in an fp32 scratch row per token), then the
-// four signal heads, whose epilogue subtracts lambda times that row and applies the gate.
-// Every pass streams the group's K/V tiles (128 keys) through an 8-deep ring of 16 KB TMA
-// boxes (K^C low, K^C high, k^R; V low, V high) -- the tiles are shared by both slots, and the
-// 16 KB k^R box is the single rotary key shared by all KV heads.
+// Work unit (one pair of CTAs on one TPC, a cluster of 2): sequence b, KV head j and 512
+// consecutive query positions.  CTA rank r owns rows [256 r, 256 r + 256) of the block, split
+// into two 128-row tiles ("slots").  The unit runs five passes, one per head of the group:
+// first the noise head (its normalised output is parked in an fp32 scratch row per token),
+// then the four signal heads, whose epilogue subtracts lambda times that row and applies the
+// gate.  Every pass streams the group's keys in tiles of 128.
 //
-// Roles (384 threads):
-//   warp 0      TMA producer (Q tiles per pass; K/V ring)
-//   warp 1      TMEM owner; lane 0 issues tcgen05.mma:
-//                 S_slot = Q_slot K^T   (M 128, N 128 keys, K 192; fp16 operands, fp32 in TMEM)
-//                 O_slot += P_slot V    (P read from TMEM, two N = 64 halves of d_v)
+// The pair shares each tensor-core instruction (tcgen05 cta_group::2, M = 256): for
+//   S_slot = Q_slot K^T   (M 256 = 2 x 128 rows, N 128 keys, K 192; fp16, fp32 in TMEM)
+//   O_slot += P_slot V    (P read from TMEM, N = d_v 128)
+// the A operand (Q or P) and the accumulator rows live in the CTA that owns the rows, while
+// the B operand is split by columns: each CTA loads 64 of the tile's 128 keys of K^C / k^R
+// and 64 of the 128 value columns of V.  A CTA therefore moves 40 KB per key tile (half of
+// what a CTA computing the same 256 rows alone would load) and the freed shared memory holds
+// three tiles of K and three of V in flight.
+//
+// Roles (384 threads per CTA):
+//   warp 0      TMA producer, both CTAs (Q per pass; K and V rings).  Every load of the pair
+//               completes on the leader's barrier, which the leader arms with both CTAs' bytes.
+//   warp 1      TMEM owner in both CTAs; lane 0 of the leader (rank 0) issues the MMAs and
+//               commits each completion to the barriers of both CTAs.
 //   warps 4-7   softmax / epilogue of slot 0 (thread = query row = TMEM lane)
-//   warps 8-11  softmax / epilogue of slot 1
-// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P overwrites the first 64
-// columns of S as packed fp16 pairs.  The MMA order PV0(i), QK0(i+1), PV1(i), QK1(i+1) keeps the
-// tensor core busy with one slot while the other slot's softmax runs.  The running max is
-// only moved (and O rescaled) when it grows by more than 2^8, which is exact after the final
-// division by the row sum.
+//   warps 8-11  softmax / epilogue of slot 1; each warp reports "P written" and "O read" to
+//               the leader's barriers (8 warps per phase).
+// TMEM columns per CTA: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P overwrites the
+// first 64 columns of S as packed fp16 pairs.  The MMA order PV0(i), QK0(i+1), PV1(i),
+// QK1(i+1) keeps the tensor core busy with one slot while the other slot's softmax runs.  The
+// running max is only moved (and O rescaled) when it grows by more than 2^8, which is exact
+// after the final division by the row sum.
 #include "gdla_common.cuh"
 #include "gdla_internal.h"
 
 namespace gdla {
 
+
 namespace attn {
-constexpr int RING = 8;
-constexpr int SUB = 16384;                  // one 128 x 64 fp16 box
-constexpr int Q_BYTES = 2 * 3 * SUB;        // 2 slots x (q^C lo, q^C hi, q^R)
-constexpr int RING_OFF = Q_BYTES;
-constexpr int BAR_OFF = RING_OFF + RING * SUB;
-constexpr int SMEM = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
-constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
+constexpr int QSUB = 16384;                   // one 128-row x 64-column fp16 box
+constexpr int KBOX = 8192;                    // 64 keys x 64 columns
+constexpr int KSTAGE = 3 * KBOX;              // this CTA's K^C low, K^C high, k^R of one tile
+constexpr int VSTAGE = 16384;                 // 128 keys x this CTA's 64 value columns
+constexpr int KST = 3, VST = 3;               // tiles in flight
+constexpr int Q_BYTES = 2 * 3 * QSUB;         // 2 slots x (q^C lo, q^C hi, q^R)
+constexpr int K_OFF = Q_BYTES;
+constexpr int V_OFF = K_OFF + KST * KSTAGE;
+constexpr int BAR_OFF = V_OFF + VST * VSTAGE;
+constexpr int SMEM = BAR_OFF + 256 + 1024;    // + barriers + alignment slack
+constexpr float RESCALE_THRESHOLD = 8.0f;     // log2 units
+constexpr uint16_t BOTH = 3;                  // commit to the barriers of both CTAs
 }  // namespace attn
 
 struct AttnBars {
   uint64_t q_full[2], q_empty[2];
-  uint64_t ring_full[attn::RING], ring_empty[attn::RING];
+  uint64_t k_full[attn::KST], k_empty[attn::KST];
+  uint64_t v_full[attn::VST], v_empty[attn::VST];
   uint64_t s_full[2], p_ready[2], o_done[2], o_free[2];
   uint64_t mma_final;
   uint32_t tmem_base;
 };
+static_assert(sizeof(AttnBars) <= 256, "barrier block");
+
+
+// ---- softmax arithmetic.  Packed f32x2 instructions halve the issue slots of the scale,
+// subtract and sum steps; a quarter of the exponentials run on the FMA pipe instead of MUFU
+// (whose 16 results per clock per SM are the softmax's bottleneck).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// (d0, d1) = (a0, a1) + (b0, b1)
+__device__ __forceinline__ void fadd2v(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 d, a, b;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// (d0, d1) = (a0, a1) * (b0, b1) + (c, c)
+__device__ __forceinline__ void ffma2v(float& d0, float& d1, float a0, float a1, float b0, float b1, float c) {
+  asm("{\n\t.reg .b64 d, a, b, c;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %6};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c));
+}
+// (x0, x1) = (a0, a1) * b + c
+__device__ __forceinline__ void ffma2(float& x0, float& x1, float a0, float a1, float b, float c) {
+  ffma2v(x0, x1, a0, a1, b, b, c);
+}
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) {
+  fadd2v(s0, s1, s0, s1, a0, a1);
+}
+// sigmoid(z) = 1 / (1 + 2^(-z log2 e)) with the approximate reciprocal-divide (2 ulp): the
+// result is rounded to bf16.
+__device__ __forceinline__ float sigmoid_approx(float z) {
+  return __fdividef(1.0f, 1.0f + ex2_approx(-1.4426950408889634f * z));
+}
+// 2^x for a pair on the FMA pipe.  x = j + f with j = round(x) (adding and subtracting
+// 1.5 * 2^23 rounds to the nearest integer) and |f| <= 1/2; 2^f from a cubic fitted to 2^f
+// on [-1/2, 1/2] (iteratively reweighted least squares towards the minimax fit, max relative
+// error 7.5e-5, below the 2^-12 half-ulp of the fp16 P it feeds; exp2_poly_fit.py beside this
+// file reproduces the coefficients); j is added to the exponent field as an integer.  x is
+// clamped at -126, where the fp16 P is 0 either way.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& r0, float& r1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, j0, j1, f0, f1;
+  fadd2v(t0, t1, x0, x1, 12582912.f, 12582912.f);
+  fadd2v(j0, j1, t0, t1, -12582912.f, -12582912.f);
+  fadd2v(f0, f1, x0, x1, -j0, -j1);
+  float q0 = 0.05517144128680229f, q1 = 0.05517144128680229f;
+  ffma2v(q0, q1, q0, q1, f0, f1, 0.24261070787906647f);
+  ffma2v(q0, q1, q0, q1, f0, f1, 0.6932609677314758f);
+  ffma2v(q0, q1, q0, q1, f0, f1, 0.9999281167984009f);
+  // the low 9 bits of t's bit pattern hold j mod 512; * 2^23 moves them into the exponent field
+  r0 = __int_as_float(__float_as_int(t0) * 8388608 + __float_as_int(q0));
+  r1 = __int_as_float(__float_as_int(t1) * 8388608 + __float_as_int(q1));
+}
 
 __device__ __forceinline__ uint8_t* attn_align(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-__global__ void __launch_bounds__(384, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ,
-                        const __grid_constant__ CUtensorMap mapKV,
+                        const __grid_constant__ CUtensorMap mapK,
                         const __grid_constant__ CUtensorMap mapKR,
+                        const __grid_constant__ CUtensorMap mapV,
                         const __grid_constant__ AttnParams p, KernelCtl ctl) {
   using namespace attn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = attn_align(smem_raw);
   AttnBars* bars = reinterpret_cast<AttnBars*>(smem + BAR_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  // the leader's copy of one of this CTA's barriers
+  auto lead = [&](uint64_t* b) { return smem_map_rank(smem_u32(b), 0); };
 
-  // ---- work unit: (sequence rows [rowbase, rowbase + T), KV head j, 256-row pair c), heaviest
-  // causal units first.  Equal-length batches derive it from blockIdx; packed documents read
-  // it from a schedule built on the device (surplus CTAs of the upper-bound grid exit here).
+  // ---- work unit: (sequence rows [rowbase, rowbase + T), KV head j, 512-row block c), heaviest
+  // causal units first.  Equal-length batches derive it from the pair index; packed documents
+  // read it from a schedule built on the device (surplus pairs of the upper-bound grid exit
+  // here, both CTAs of a pair together, before any cluster-wide step).
+  const int pu = int(blockIdx.x) >> 1;
   int c, rowbase, T, j;
   if (p.units) {
-    const int u = int(blockIdx.x) / p.n_groups;
+    const int u = pu / p.n_groups;
     if (u >= *p.n_units) return;
     const int4 un = p.units[u];
     rowbase = un.x;
     T = un.y;
     c = un.z;
-    j = int(blockIdx.x) % p.n_groups;
+    j = pu % p.n_groups;
   } else {
-    const int n_pairs = (p.T + 255) / 256;
+    const int n_blk = (p.T + 511) / 512;
     const int per_c = p.B * p.n_groups;
-    c = n_pairs - 1 - int(blockIdx.x) / per_c;
-    const int b = (int(blockIdx.x) % per_c) / p.n_groups;
-    j = int(blockIdx.x) % p.n_groups;
+    c = n_blk - 1 - pu / per_c;
+    const int b = (pu % per_c) / p.n_groups;
+    j = pu % p.n_groups;
     rowbase = b * p.T;
     T = p.T;
   }
-  const int q0 = 256 * c;
-  const int t_hi = min(T - 1, q0 + 255) / 128;
+  const int q0 = 512 * c;
+  const int t_hi = min(T - 1, q0 + 511) / 128;
   const int t_lo = p.window > 0 ? max(0, q0 - p.window + 1) / 128 : 0;
   const int n_kv = t_hi - t_lo + 1;
 
@@ -97,34 +177,40 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_ready[s], 128);
+      mbar_init(&bars->p_ready[s], 8);
       mbar_init(&bars->o_done[s], 1);
-      mbar_init(&bars->o_free[s], 128);
+      mbar_init(&bars->o_free[s], 8);
     }
-    for (int s = 0; s < RING; ++s) {
-      mbar_init(&bars->ring_full[s], 1);
-      mbar_init(&bars->ring_empty[s], 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < VST; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->mma_final, 1);
     fence_mbar_init();
     tma_prefetch_desc(&mapQ);
-    tma_prefetch_desc(&mapKV);
+    tma_prefetch_desc(&mapK);
     tma_prefetch_desc(&mapKR);
+    tma_prefetch_desc(&mapV);
   }
   if (warp == 1) {
-    tmem_alloc(&bars->tmem_base, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(&bars->tmem_base, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();   // both CTAs' barriers exist before any cross-CTA arrive or copy
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
     if (lane == 0) {
       // ================================================================ TMA producer
-      uint32_t ring_issued = 0, ring_par = 0, q_issued = 0, q_par = 0;
-      uint32_t g = 0;
+      uint32_t kq = 0, vq = 0;
+      uint32_t k_armed = 0, k_par = 0, v_armed = 0, v_par = 0, q_armed = 0, q_par = 0;
       bool ok = true;
       for (int pass = 0; pass < 5 && ok; ++pass) {
         const int h = pass == 0 ? p.n_signal + j : 4 * j + pass - 1;
@@ -133,82 +219,104 @@ __global__ void __launch_bounds__(384, 1)
             ok = false;
             break;
           }
-          uint8_t* qd = smem + s * 3 * SUB;
-          const int y = rowbase + q0 + 128 * s;
-          mbar_expect_tx(&bars->q_full[s], 3 * SUB);
-          tma_load_2d(qd, &mapQ, &bars->q_full[s], h * 128, y);
-          tma_load_2d(qd + SUB, &mapQ, &bars->q_full[s], h * 128 + 64, y);
-          tma_load_2d(qd + 2 * SUB, &mapQ, &bars->q_full[s], p.rope_col0 + h * 64, y);
-          q_issued |= 1u << s;
-          q_par = (q_par & ~(1u << s)) | (uint32_t(pass & 1) << s);
+          uint8_t* qd = smem + s * 3 * QSUB;
+          const int y = rowbase + q0 + 256 * int(rank) + 128 * s;
+          if (leader) {
+            mbar_expect_tx(&bars->q_full[s], 2 * 3 * QSUB);
+            q_armed |= 1u << s;
+            q_par = (q_par & ~(1u << s)) | (uint32_t(pass & 1) << s);
+          }
+          const uint32_t bar = lead(&bars->q_full[s]);
+          tma_load_2d_pair(qd, &mapQ, bar, h * 128, y);
+          tma_load_2d_pair(qd + QSUB, &mapQ, bar, h * 128 + 64, y);
+          tma_load_2d_pair(qd + 2 * QSUB, &mapQ, bar, p.rope_col0 + h * 64, y);
         }
         for (int i = 0; i < n_kv && ok; ++i) {
-          const int y = rowbase + 128 * (t_lo + i);
-          for (int sub = 0; sub < 5; ++sub, ++g) {
-            const int slot = g % RING;
-            const uint32_t ph = (g / RING) & 1;
-            if (g >= RING && !mbar_wait(&bars->ring_empty[slot], ph ^ 1, ctl, SITE_ATTN_PRODUCER)) {
+          const int y0 = rowbase + 128 * (t_lo + i);
+          {  // this CTA's 64 keys of K^C and k^R
+            const int st = kq % KST;
+            const uint32_t ph = (kq / KST) & 1;
+            if (kq >= KST && !mbar_wait(&bars->k_empty[st], ph ^ 1, ctl, SITE_ATTN_PRODUCER)) {
               ok = false;
               break;
             }
-            uint8_t* dst = smem + RING_OFF + slot * SUB;
-            mbar_expect_tx(&bars->ring_full[slot], SUB);
-            if (sub == 2)
-              tma_load_2d(dst, &mapKR, &bars->ring_full[slot], 0, y);
-            else  // sub 0,1: K^C halves; 3,4: V halves
-              tma_load_2d(dst, &mapKV, &bars->ring_full[slot], j * 256 + (sub < 2 ? sub : sub - 1) * 64, y);
-            ring_issued |= 1u << slot;
-            ring_par = (ring_par & ~(1u << slot)) | (ph << slot);
+            if (leader) {
+              mbar_expect_tx(&bars->k_full[st], 2 * KSTAGE);
+              k_armed |= 1u << st;
+              k_par = (k_par & ~(1u << st)) | (ph << st);
+            }
+            uint8_t* dst = smem + K_OFF + st * KSTAGE;
+            const uint32_t bar = lead(&bars->k_full[st]);
+            const int yk = y0 + 64 * int(rank);
+            tma_load_2d_pair(dst, &mapK, bar, j * 256, yk);
+            tma_load_2d_pair(dst + KBOX, &mapK, bar, j * 256 + 64, yk);
+            tma_load_2d_pair(dst + 2 * KBOX, &mapKR, bar, 0, yk);
+            ++kq;
+          }
+          {  // all 128 keys of this CTA's 64 value columns
+            const int st = vq % VST;
+            const uint32_t ph = (vq / VST) & 1;
+            if (vq >= VST && !mbar_wait(&bars->v_empty[st], ph ^ 1, ctl, SITE_ATTN_PRODUCER)) {
+              ok = false;
+              break;
+            }
+            if (leader) {
+              mbar_expect_tx(&bars->v_full[st], 2 * VSTAGE);
+              v_armed |= 1u << st;
+              v_par = (v_par & ~(1u << st)) | (ph << st);
+            }
+            tma_load_2d_pair(smem + V_OFF + st * VSTAGE, &mapV, lead(&bars->v_full[st]),
+                             j * 256 + 128 + 64 * int(rank), y0);
+            ++vq;
           }
         }
       }
-      for (int s = 0; s < RING; ++s)
-        if (ring_issued & (1u << s)) mbar_drain(&bars->ring_full[s], (ring_par >> s) & 1, ctl.err);
+      // the leader's barriers count both CTAs' copies: let every armed phase land
+      for (int s = 0; s < KST; ++s)
+        if (k_armed & (1u << s)) mbar_drain(&bars->k_full[s], (k_par >> s) & 1, ctl.err);
+      for (int s = 0; s < VST; ++s)
+        if (v_armed & (1u << s)) mbar_drain(&bars->v_full[s], (v_par >> s) & 1, ctl.err);
       for (int s = 0; s < 2; ++s)
-        if (q_issued & (1u << s)) mbar_drain(&bars->q_full[s], (q_par >> s) & 1, ctl.err);
+        if (q_armed & (1u << s)) mbar_drain(&bars->q_full[s], (q_par >> s) & 1, ctl.err);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ================================================================ MMA issuer
-      constexpr uint32_t idesc_qk = make_idesc(128, 128, 0, 0, 0);
-      constexpr uint32_t idesc_pv = make_idesc(128, 64, 0, 0, 1);
+    if (lane == 0 && leader) {
+      // ================================================================ MMA issuer (leader)
+      constexpr uint32_t idesc_qk = make_idesc(256, 128, 0, 0, 0);
+      constexpr uint32_t idesc_pv = make_idesc(256, 128, 0, 0, 1);
       const uint32_t q_addr = smem_u32(smem);
-      const uint32_t ring_addr = smem_u32(smem + RING_OFF);
-      uint32_t g = 0, pr_par[2] = {0, 0};
+      const uint32_t k_addr = smem_u32(smem + K_OFF);
+      const uint32_t v_addr = smem_u32(smem + V_OFF);
+      uint32_t kq = 0, vq = 0, pr_par[2] = {0, 0};
       bool ok = true;
 
-      auto wait_ring = [&](uint32_t gg, int n) -> bool {
-        for (int k = 0; k < n; ++k) {
-          const uint32_t idx = gg + k;
-          if (!mbar_wait(&bars->ring_full[idx % RING], (idx / RING) & 1, ctl, SITE_ATTN_MMA))
-            return false;
-        }
-        return true;
-      };
-      auto issue_qk = [&](int s, uint32_t gk) {
+      // Descriptors are built once; an operand at byte offset o from a base adds o / 16 to the
+      // low word (start-address field, 14 bits: no carry for offsets inside shared memory).
+      const uint64_t dq = sdesc_sw128(q_addr, 16, 1024);
+      const uint64_t dk = sdesc_sw128(k_addr, 16, 1024);
+      const uint64_t dv = sdesc_sw128(v_addr, 8192, 1024);
+      const uint32_t q_lo = uint32_t(dq), q_hi = uint32_t(dq >> 32);
+      const uint32_t k_lo = uint32_t(dk), k_hi = uint32_t(dk >> 32);
+      const uint32_t v_lo = uint32_t(dv), v_hi = uint32_t(dv >> 32);
+      auto issue_qk = [&](int s, int kst) {
         const uint32_t d = tmem + s * 128;
+        const uint32_t a0 = q_lo + uint32_t(s * 3 * QSUB >> 4);
+        const uint32_t b0 = k_lo + uint32_t(kst * KSTAGE >> 4);
 #pragma unroll
         for (int kk = 0; kk < 12; ++kk) {
           const int sub = kk >> 2, k4 = kk & 3;
-          const uint64_t ad = sdesc_sw128(q_addr + (s * 3 + sub) * SUB + k4 * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(ring_addr + ((gk + sub) % RING) * SUB + k4 * 32, 16, 1024);
-          mma_ss(d, ad, bd, idesc_qk, kk > 0);
+          mma_ss_pair(d, a0 + uint32_t((sub * QSUB + k4 * 32) >> 4), q_hi,
+                      b0 + uint32_t((sub * KBOX + k4 * 32) >> 4), k_hi, idesc_qk, kk > 0);
         }
       };
-      auto issue_pv = [&](int s, uint32_t gv, bool acc) {
+      auto issue_pv = [&](int s, int vst, bool acc) {
         const uint32_t a = tmem + s * 128;
         const uint32_t d = tmem + 256 + s * 128;
+        const uint32_t b0 = v_lo + uint32_t(vst * VSTAGE >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const uint64_t bd = sdesc_sw128(ring_addr + ((gv + hf) % RING) * SUB + kk * 2048, 8192, 1024);
-            mma_ts(d + hf * 64, a + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-          }
-        }
-      };
-      auto release = [&](uint32_t gg, int n) {
-        for (int k = 0; k < n; ++k) mma_commit(&bars->ring_empty[(gg + k) % RING]);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts_pair(d, a + kk * 8, b0 + uint32_t(kk * 2048 >> 4), v_hi, idesc_pv,
+                      (acc || kk > 0) ? 1u : 0u);
       };
 
       for (int pass = 0; pass < 5 && ok; ++pass) {
@@ -217,63 +325,63 @@ __global__ void __launch_bounds__(384, 1)
           ok = false;
           break;
         }
-        tc_fence_after();
         // prologue: S = Q K(0)^T for both slots
-        uint32_t gk = g;
-        if (!wait_ring(gk, 3)) { ok = false; break; }
-        tc_fence_after();
-        issue_qk(0, gk);
-        mma_commit(&bars->s_full[0]);
-        issue_qk(1, gk);
-        mma_commit(&bars->s_full[1]);
-        release(gk, 3);
+        int kst = kq % KST;
+        if (!mbar_wait(&bars->k_full[kst], (kq / KST) & 1, ctl, SITE_ATTN_MMA)) { ok = false; break; }
+        issue_qk(0, kst);
+        mma_commit_pair(&bars->s_full[0], BOTH);
+        issue_qk(1, kst);
+        mma_commit_pair(&bars->s_full[1], BOTH);
+        mma_commit_pair(&bars->k_empty[kst], BOTH);
+        ++kq;
         if (n_kv == 1) {
-          mma_commit(&bars->q_empty[0]);
-          mma_commit(&bars->q_empty[1]);
+          mma_commit_pair(&bars->q_empty[0], BOTH);
+          mma_commit_pair(&bars->q_empty[1], BOTH);
         }
-        g += 3;
         for (int i = 0; i < n_kv; ++i) {
-          const uint32_t gv = g;
-          if (!wait_ring(gv, 2)) { ok = false; break; }
-          g += 2;
+          const int vst = vq % VST;
+          if (!mbar_wait(&bars->v_full[vst], (vq / VST) & 1, ctl, SITE_ATTN_MMA)) { ok = false; break; }
           // ---- slot 0: O0 += P0 V
-          if (i == 0 && pass > 0 && !mbar_wait(&bars->o_free[0], (pass - 1) & 1, ctl, SITE_ATTN_MMA)) { ok = false; break; }
+          if (i == 0 && pass > 0 &&
+              !mbar_wait(&bars->o_free[0], (pass - 1) & 1, ctl, SITE_ATTN_MMA)) { ok = false; break; }
           if (!mbar_wait(&bars->p_ready[0], pr_par[0], ctl, SITE_ATTN_MMA)) { ok = false; break; }
           pr_par[0] ^= 1;
           tc_fence_after();
-          issue_pv(0, gv, i > 0);
-          if (i == n_kv - 1) mma_commit(&bars->o_done[0]);
+          issue_pv(0, vst, i > 0);
+          if (i == n_kv - 1) mma_commit_pair(&bars->o_done[0], BOTH);
           // ---- slot 0: next S
           const bool more = i + 1 < n_kv;
           if (more) {
-            gk = g;
-            if (!wait_ring(gk, 3)) { ok = false; break; }
-            tc_fence_after();
-            issue_qk(0, gk);
-            mma_commit(&bars->s_full[0]);
+            kst = kq % KST;
+            if (!mbar_wait(&bars->k_full[kst], (kq / KST) & 1, ctl, SITE_ATTN_MMA)) { ok = false; break; }
+            issue_qk(0, kst);
+            mma_commit_pair(&bars->s_full[0], BOTH);
           }
           // ---- slot 1: O1 += P1 V
-          if (i == 0 && pass > 0 && !mbar_wait(&bars->o_free[1], (pass - 1) & 1, ctl, SITE_ATTN_MMA)) { ok = false; break; }
+          if (i == 0 && pass > 0 &&
+              !mbar_wait(&bars->o_free[1], (pass - 1) & 1, ctl, SITE_ATTN_MMA)) { ok = false; break; }
           if (!mbar_wait(&bars->p_ready[1], pr_par[1], ctl, SITE_ATTN_MMA)) { ok = false; break; }
           pr_par[1] ^= 1;
           tc_fence_after();
-          issue_pv(1, gv, i > 0);
-          if (i == n_kv - 1) mma_commit(&bars->o_done[1]);
-          release(gv, 2);
+          issue_pv(1, vst, i > 0);
+          if (i == n_kv - 1) mma_commit_pair(&bars->o_done[1], BOTH);
+          mma_commit_pair(&bars->v_empty[vst], BOTH);
+          ++vq;
           if (more) {
-            issue_qk(1, gk);
-            mma_commit(&bars->s_full[1]);
-            release(gk, 3);
+            issue_qk(1, kst);
+            mma_commit_pair(&bars->s_full[1], BOTH);
+            mma_commit_pair(&bars->k_empty[kst], BOTH);
+            ++kq;
             if (i + 1 == n_kv - 1) {
-              mma_commit(&bars->q_empty[0]);
-              mma_commit(&bars->q_empty[1]);
+              mma_commit_pair(&bars->q_empty[0], BOTH);
+              mma_commit_pair(&bars->q_empty[1], BOTH);
             }
-            g += 3;
           }
         }
       }
-      // every issued MMA must finish before TMEM is released
-      mma_commit(&bars->mma_final);
+      // every issued MMA (which reads the peer's shared memory and writes its TMEM) must
+      // finish before either CTA passes the closing cluster barrier
+      mma_commit_pair(&bars->mma_final, 1);
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
   } else if (warp >= 4) {
@@ -284,10 +392,12 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const uint32_t tS = tmem + s * 128 + lane_off;
     const uint32_t tO = tmem + 256 + s * 128 + lane_off;
-    const int qpos = q0 + 128 * s + r;
+    const int qpos = q0 + 256 * int(rank) + 128 * s + r;
     const bool row_valid = qpos < T;
     const long long m_row = (long long)rowbase + qpos;
     const int W = p.window;
+    const uint32_t p_ready_cl = lead(&bars->p_ready[s]);
+    const uint32_t o_free_cl = lead(&bars->o_free[s]);
     uint32_t sf_par = 0;
     bool ok = true;
 
@@ -317,9 +427,16 @@ __global__ void __launch_bounds__(384, 1)
             if (kp > qpos || (W > 0 && kp <= qpos - W)) sc[e] = -INFINITY;
           }
         }
-        float mx = sc[0];
+        // row max: eight independent chains of three-input maxima, then their maximum
+        float cm[8];
 #pragma unroll
-        for (int e = 1; e < 128; ++e) mx = fmaxf(mx, sc[e]);
+        for (int k = 0; k < 8; ++k) {
+          float m = fmax3f(sc[k], sc[k + 8], sc[k + 16]);
+#pragma unroll
+          for (int e = 24; e < 120; e += 16) m = fmax3f(m, sc[k + e], sc[k + e + 8]);
+          cm[k] = fmaxf(m, sc[k + 120]);
+        }
+        const float mx = fmax3f(fmax3f(cm[0], cm[1], cm[2]), fmax3f(cm[3], cm[4], cm[5]), fmaxf(cm[6], cm[7]));
         const float m_tile = mx * p.scale_log2;
         float alpha = 1.f;
         bool resc = false;
@@ -344,25 +461,40 @@ __global__ void __launch_bounds__(384, 1)
         }
         l_run *= alpha;
         const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-        uint32_t pk[64];
-        float lsum = 0.f;
+        // P = 2^(s * scale - m) as fp16 pairs over S's first 64 columns, written to TMEM in four
+        // 32-key chunks; every fourth pair takes the FMA-pipe exponential
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const float p0 = ex2_approx(fmaf(sc[2 * e], p.scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(sc[2 * e + 1], p.scale_log2, neg_m));
-          lsum += p0 + p1;
-          pk[e] = pack_half2(p0, p1);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int e = 16 * c + q;
+            float x0, x1, p0, p1;
+            ffma2(x0, x1, sc[2 * e], sc[2 * e + 1], p.scale_log2, neg_m);
+            if ((e & 3) == 3) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            fadd2(ls[2 * (e & 3)], ls[2 * (e & 3) + 1], p0, p1);
+            pk[q] = pack_half2(p0, p1);
+          }
+          GDLA_TMEM_ST16(tS + 16 * c, pk);
         }
+        const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         l_run += lsum;
-        GDLA_TMEM_ST32(tS + 0, pk);
-        GDLA_TMEM_ST32(tS + 32, (pk + 32));
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars->p_ready[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(p_ready_cl);
       }
       if (!ok) break;
 
-      // ---------------- epilogue of this pass
+      // ---------------- epilogue of this pass.  The parked noise rows are interleaved in
+      // blocks of 32 rows (the rows of one warp), so a warp's accesses to them are contiguous;
+      // the gate and noise operands are loaded a 32-column chunk at a time ahead of its math.
       bool w_ok = mbar_wait(&bars->o_done[s], pass & 1, ctl, SITE_ATTN_SOFTMAX);
       w_ok = __all_sync(0xffffffffu, w_ok);
       if (!w_ok) { ok = false; break; }
@@ -374,51 +506,63 @@ __global__ void __launch_bounds__(384, 1)
       GDLA_TMEM_LD32(tO + 96, (ou + 96));
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&bars->o_free[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(o_free_cl);
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       if (!row_valid || m_row >= (long long)p.B * p.T || *reinterpret_cast<volatile int*>(ctl.err) != 0)
         continue;
-      float* on_row = p.O_noise + (m_row * p.n_groups + j) * 128;
+      // column quad e/4 of row m: ((m/32 * n_groups + j) * 32 + e/4) * 128 + (m%32) * 4
+      float* on_q = p.O_noise + ((m_row >> 5) * p.n_groups + j) * 4096 + (m_row & 31) * 4;
       if (pass == 0) {
 #pragma unroll
         for (int e = 0; e < 128; e += 4)
-          *reinterpret_cast<float4*>(on_row + e) =
+          *reinterpret_cast<float4*>(on_q + (e / 4) * 128) =
               make_float4(__uint_as_float(ou[e]) * inv_l, __uint_as_float(ou[e + 1]) * inv_l,
                           __uint_as_float(ou[e + 2]) * inv_l, __uint_as_float(ou[e + 3]) * inv_l);
       } else {
         const int sig = 4 * j + pass - 1;
         const float lam = p.lam[m_row * p.n_signal + sig];
-        const __nv_bfloat16* g_row =
-            static_cast<const __nv_bfloat16*>(p.G) + (m_row * p.n_signal + sig) * 128;
-        __nv_bfloat16* d_row = static_cast<__nv_bfloat16*>(p.Dg) + (m_row * p.n_signal + sig) * 128;
+        const uint4* g_row = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.G) + (m_row * p.n_signal + sig) * 128);
+        uint4* d_row = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Dg) + (m_row * p.n_signal + sig) * 128);
 #pragma unroll
-        for (int e = 0; e < 128; e += 8) {
-          const uint4 gv = *reinterpret_cast<const uint4*>(g_row + e);
-          const float4 n0 = *reinterpret_cast<const float4*>(on_row + e);
-          const float4 n1 = *reinterpret_cast<const float4*>(on_row + e + 4);
-          const float nn[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-          uint32_t outw[4];
+        for (int c = 0; c < 4; ++c) {
+          uint4 gv[4];
+          float4 nv[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) gv[q] = __ldg(g_row + 4 * c + q);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) nv[q] = *reinterpret_cast<const float4*>(on_q + (8 * c + q) * 128);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(&gw[q]);
-            const float d0 = __uint_as_float(ou[e + 2 * q]) * inv_l - lam * nn[2 * q];
-            const float d1 = __uint_as_float(ou[e + 2 * q + 1]) * inv_l - lam * nn[2 * q + 1];
-            outw[q] = pack_bf162(sigmoidf_fast(__low2float(g2)) * d0,
-                                 sigmoidf_fast(__high2float(g2)) * d1);
+            const float nn[8] = {nv[2 * q].x, nv[2 * q].y, nv[2 * q].z, nv[2 * q].w,
+                                 nv[2 * q + 1].x, nv[2 * q + 1].y, nv[2 * q + 1].z, nv[2 * q + 1].w};
+            const uint32_t gw[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+            const int e = 32 * c + 8 * q;
+            uint32_t outw[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(&gw[h]);
+              const float d0 = __uint_as_float(ou[e + 2 * h]) * inv_l - lam * nn[2 * h];
+              const float d1 = __uint_as_float(ou[e + 2 * h + 1]) * inv_l - lam * nn[2 * h + 1];
+              outw[h] = pack_bf162(sigmoid_approx(__low2float(g2)) * d0,
+                                   sigmoid_approx(__high2float(g2)) * d1);
+            }
+            d_row[4 * c + q] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
           }
-          *reinterpret_cast<uint4*>(d_row + e) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
         }
       }
     }
   }
 
+  // Neither CTA leaves (or frees TMEM) while the other may still touch its shared memory or
+  // TMEM: the leader has waited for its last MMA, every role has returned from bounded waits.
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -426,20 +570,25 @@ int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* k
                         const AttnParams& p, KernelCtlHost ctl, cudaStream_t st) {
   if (p.B <= 0 || p.T <= 0) return 0;
   const long long M = (long long)p.B * p.T;   // rows of the (packed) token matrix
-  CUtensorMap mq, mkv, mkr;
+  const uint64_t kv_ld = (uint64_t)p.n_groups * 256;
+  CUtensorMap mq, mk, mkr, mv;
   if (make_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, QQ, qq_ld, M, (uint64_t)qq_ld * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      make_tmap_2d(&mkv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, KV, (uint64_t)p.n_groups * 256, M,
-                   (uint64_t)p.n_groups * 256 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      make_tmap_2d(&mkr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, kR16, 64, M, 128, 64, 128,
+      make_tmap_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, KV, kv_ld, M, kv_ld * 2, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      make_tmap_2d(&mkr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, kR16, 64, M, 128, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      make_tmap_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, KV, kv_ld, M, kv_ld * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return -3;
   if (cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            attn::SMEM) != cudaSuccess)
     return -4;
-  const int grid = p.units ? p.max_units * p.n_groups : ((p.T + 255) / 256) * p.B * p.n_groups;
+  const long long units = p.units ? (long long)p.max_units : (long long)((p.T + 511) / 512) * p.B;
+  const long long grid = 2 * units * p.n_groups;   // two CTAs (one cluster) per unit
+  if (grid > 0x7fffffffLL) return -2;
   KernelCtl kc{ctl.err, ctl.limit_ns};
-  attn_prefill_kernel<<<grid, 384, attn::SMEM, st>>>(mq, mkv, mkr, p, kc);
+  attn_prefill_kernel<<<unsigned(grid), 384, attn::SMEM, st>>>(mq, mk, mkr, mv, p, kc);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 

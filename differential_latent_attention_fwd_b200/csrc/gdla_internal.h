@@ -84,7 +84,9 @@ struct NormParams {
 };
 int launch_norm_rope(const NormParams& p, cudaStream_t st);
 
-// Fused prefill attention (QK^T, online softmax, PV, differential combine and gate).
+// Fused prefill attention (QK^T, online softmax, PV, differential combine and gate).  One
+// work unit = one KV head over ATTN_UNIT_ROWS consecutive query rows of one sequence.
+constexpr int ATTN_UNIT_ROWS = 512;
 struct AttnParams {
   int B, T, window;
   int n_groups;               // KV heads = noise heads
@@ -93,17 +95,20 @@ struct AttnParams {
   float scale_log2;           // log2(e) / sqrt(d_qk)
   const float* lam;           // [B*T, n_signal]
   const void* G;              // bf16 [B*T, n_signal*128] gate logits
-  float* O_noise;             // [B*T, n_groups, 128] fp32 scratch
+  float* O_noise;             // fp32 scratch, ceil(B*T / 32) * 32 * n_groups * 128 floats: for
+                              // row m, group j, column e at
+                              // ((m / 32 * n_groups + j) * 32 + e / 4) * 128 + (m % 32) * 4 + e % 4
   void* Dg;                   // bf16 [B*T, n_signal*128]
   // Packed documents (B = 1, T = all tokens): device schedule of work units
-  // {first row, document length, 256-row pair index, 0}; null for equal-length batches.
+  // {first row, document length, block index (rows [512 c, 512 c + 512)), 0}; null for
+  // equal-length batches.
   const int4* units;
   const int* n_units;
   int max_units;              // grid bound (units beyond *n_units exit at once)
 };
 
 // Device schedule of packed documents: per-token positions and the attention work units,
-// counting-sorted by pair index (heaviest causal units first).  Scratch: cnt/fill [max_c].
+// counting-sorted by block index (heaviest causal units first).  Scratch: cnt/fill [max_c].
 int launch_varlen_schedule(const int* cu_seqlens, int n_docs, int total, int* positions,
                            int4* units, int* n_units, int max_units, int* cnt, int* fill, int max_c,
                            int* err, cudaStream_t st);

@@ -4,8 +4,8 @@
 // 256K-token sequence of 473 documents) packs documents; each document is its own sequence
 // here: rotary positions restart at 0 and attention (causal or sliding window) stays inside
 // the document.  These kernels turn cu_seqlens (first row of every document, plus the total)
-// into per-token positions and the attention kernel's work units, sorted by pair index so the
-// longest causal units start first.
+// into per-token positions and the attention kernel's work units (blocks of ATTN_UNIT_ROWS
+// rows of one document), sorted by block index so the longest causal units start first.
 #include "gdla_common.cuh"
 #include "gdla_internal.h"
 
@@ -29,33 +29,33 @@ __global__ void varlen_positions_kernel(const int* __restrict__ cu, int n_docs, 
   pos[m] = m - cu[lo];
 }
 
-// pairs of 256 rows of document d; 0 for a document outside [0, total)
-__device__ __forceinline__ int doc_pairs(const int* cu, int d, int total, int max_c, int* start,
+// blocks of ATTN_UNIT_ROWS rows of document d; 0 for a document outside [0, total)
+__device__ __forceinline__ int doc_blocks(const int* cu, int d, int total, int max_c, int* start,
                                          int* len) {
   *start = cu[d];
   *len = cu[d + 1] - *start;
   if (*start < 0 || *len <= 0 || *start + *len > total) return 0;
-  return min((*len + 255) / 256, max_c);
+  return min((*len + ATTN_UNIT_ROWS - 1) / ATTN_UNIT_ROWS, max_c);
 }
 
-// cnt[c] = number of documents with more than c pairs of 256 rows
+// cnt[c] = number of documents with more than c blocks
 __global__ void varlen_count_kernel(const int* __restrict__ cu, int n_docs, int total, int* cnt,
                                     int max_c) {
   const int d = blockIdx.x * blockDim.x + threadIdx.x;
   if (d >= n_docs) return;
   int start, len;
-  const int np = doc_pairs(cu, d, total, max_c, &start, &len);
+  const int np = doc_blocks(cu, d, total, max_c, &start, &len);
   for (int c = 0; c < np; ++c) atomicAdd(&cnt[c], 1);
 }
 
-// offsets for pair index c in descending order; one CTA
+// offsets for block index c in descending order; one CTA
 __global__ void varlen_offsets_kernel(int* cnt, int* fill, int max_c, int* n_units, int max_units,
                                       int* err) {
   if (threadIdx.x == 0) {
     int acc = 0;
     for (int c = max_c - 1; c >= 0; --c) {
       const int k = cnt[c];
-      cnt[c] = acc;      // becomes the first slot of pair index c
+      cnt[c] = acc;      // becomes the first slot of block index c
       fill[c] = 0;
       acc += k;
     }
@@ -69,7 +69,7 @@ __global__ void varlen_fill_kernel(const int* __restrict__ cu, int n_docs, int t
   const int d = blockIdx.x * blockDim.x + threadIdx.x;
   if (d >= n_docs) return;
   int start, len;
-  const int np = doc_pairs(cu, d, total, max_c, &start, &len);
+  const int np = doc_blocks(cu, d, total, max_c, &start, &len);
   for (int c = 0; c < np; ++c) {
     const int slot = off[c] + atomicAdd(&fill[c], 1);
     if (slot < max_units) units[slot] = make_int4(start, len, c, 0);
