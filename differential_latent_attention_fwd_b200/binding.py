@@ -20,6 +20,7 @@ HEADER = os.path.join(HERE, "..", "include", "gdla.h")
 GDLA_MODE_PREFILL = 0
 GDLA_MODE_DECODE = 1
 GDLA_MODE_VARLEN = 2
+GDLA_MODE_CONTEXT = 3
 STATUS = {0: "GDLA_OK", -1: "GDLA_ERR_INVALID_ARG", -2: "GDLA_ERR_UNSUPPORTED_SHAPE",
           -3: "GDLA_ERR_WORKSPACE_TOO_SMALL", -4: "GDLA_ERR_LAUNCH",
           -5: "GDLA_ERR_DEVICE_TIMEOUT", -6: "GDLA_ERR_CUDA"}
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
             "gdla_attn_prefill_noalloc": [cfgp, P, P, P, P, P, P, I, I, P],
             "gdla_prefill_varlen_fwd": [cfgp, wp, P, I, P, I, P, P, P, SZ, P],
             "gdla_decode_multi_fwd": [cfgp, abp, P, I, P, P, I, I, P, P, SZ, P],
+            "gdla_latent_fwd": [cfgp, wp, P, I, I, P, P, SZ, P],
+            "gdla_prefill_context_fwd": [cfgp, wp, P, I, I, P, I, P, P, P, SZ, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -173,6 +176,29 @@ def gdla_prefill_varlen_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, cu_seqlens:
         ctypes.byref(cfg), ctypes.byref(w), _ptr(x, torch.bfloat16, "x"), total,
         _ptr(cu_seqlens, torch.int32, "cu_seqlens"), cu_seqlens.numel() - 1,
         _ptr(y, torch.bfloat16, "y"), _ptr(kv_latent_out, torch.bfloat16, "kv_latent_out"),
+        _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def gdla_latent_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, pos_offset: int, latent_out: torch.Tensor,
+                    workspace: torch.Tensor, stream=None) -> None:
+    T = x.shape[0]
+    _check("gdla_latent_fwd", lib().gdla_latent_fwd(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(x, torch.bfloat16, "x"), T, pos_offset,
+        _ptr(latent_out, torch.bfloat16, "latent_out"), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gdla_prefill_context_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, pos_offset: int,
+                             prefix_latent: torch.Tensor | None, y: torch.Tensor,
+                             workspace: torch.Tensor, latent_out: torch.Tensor | None = None,
+                             stream=None) -> None:
+    T = x.shape[0]
+    n_prefix = 0 if prefix_latent is None else prefix_latent.shape[0]
+    _check("gdla_prefill_context_fwd", lib().gdla_prefill_context_fwd(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(x, torch.bfloat16, "x"), T, pos_offset,
+        _ptr(prefix_latent, torch.bfloat16, "prefix_latent") if n_prefix else None, n_prefix,
+        _ptr(y, torch.bfloat16, "y"), _ptr(latent_out, torch.bfloat16, "latent_out"),
         _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream)))
 

@@ -106,7 +106,7 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
     sz[WS_VL_UNITS] = (size_t)varlen_max_units(M, M) * 16;
     sz[WS_VL_COUNT] = (size_t)(1 + 2 * varlen_max_blocks(M)) * 4;
   }
-  if (mode == GDLA_MODE_PREFILL || mode == GDLA_MODE_VARLEN) {
+  if (mode == GDLA_MODE_PREFILL || mode == GDLA_MODE_VARLEN || mode == GDLA_MODE_CONTEXT) {
     sz[WS_LATENT] = M * (c->kv_rank + c->d_rope) * 2;
     sz[WS_QQ] = M * qq * 2;
     sz[WS_KV] = M * (long long)c->n_kv_heads * (c->d_nope + c->d_v) * 2;
@@ -147,11 +147,22 @@ struct VarlenArgs {
   void* latent_out;
 };
 
-// Prefill body shared by equal-length batches (vl == nullptr) and packed documents (B = 1,
-// T = all tokens).  Arguments are already validated; off is the workspace layout.
+// A key prefix: the latent rows of the n_prefix tokens that precede x in its sequence.
+struct ContextArgs {
+  const void* prefix_latent;   // [n_prefix, kv_rank + d_rope] bf16
+  int n_prefix;
+  int pos_offset;              // position of the first local token (>= n_prefix)
+  void* latent_out;            // [T, kv_rank + d_rope] bf16 for the local tokens, or null
+};
+
+// Prefill body shared by equal-length batches (vl == ctx == nullptr), packed documents (vl; B =
+// 1, T = all tokens), and one sequence chunk after a key prefix (ctx; B = 1).  With latent_only
+// it stops after the latent rows (written to ctx->latent_out).  Arguments are already
+// validated; off is the workspace layout.
 static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int B,
                         int T, void* y, void* kv_cache_out, int cache_cap, uint8_t* ws,
-                        const size_t* off, cudaStream_t st, const VarlenArgs* vl) {
+                        const size_t* off, cudaStream_t st, const VarlenArgs* vl,
+                        const ContextArgs* ctx = nullptr, bool latent_only = false) {
   int rc;
   int* err;
   if ((rc = error_word(&err))) return rc;
@@ -169,6 +180,8 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
   const int M = B * T;
   const int nH = cfg->n_signal + cfg->n_noise;
   const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
+  const int row_w = cfg->kv_rank + cfg->d_rope;            // latent row: c_bar | rotated k^R
+  const int n_pre = ctx ? ctx->n_prefix : 0;               // key rows before the local tokens
   RopeTable rope;
   fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
 
@@ -215,7 +228,29 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
   np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
   np.cQ = cQ; np.latent = latent; np.kR16 = kR16; np.lam = lam; np.pos_T = T; np.pos_ptr = positions;
   np.cache = kv_cache_out; np.cache_cap = cache_cap; np.rope = rope; np.err = err;
+  if (ctx) {
+    // local rows follow the prefix rows in the key-side buffers; positions continue the prefix
+    np.pos_off = ctx->pos_offset;
+    np.latent = static_cast<__nv_bfloat16*>(latent) + (size_t)n_pre * row_w;
+    np.kR16 = static_cast<__half*>(kR16) + (size_t)n_pre * cfg->d_rope;
+    if (latent_only) { np.latent = ctx->latent_out; np.kR16 = nullptr; }
+    if (!latent_only && n_pre > 0) {
+      if (cudaMemcpyAsync(latent, ctx->prefix_latent, (size_t)n_pre * row_w * 2,
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return GDLA_ERR_CUDA;
+      if (launch_failed(launch_latent_to_kr16(ctx->prefix_latent, cfg->kv_rank, n_pre, kR16, st)))
+        return GDLA_ERR_LAUNCH;
+    }
+  }
   if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
+  if (latent_only) {
+    stage(5, st);
+    return GDLA_OK;
+  }
+  if (ctx && ctx->latent_out &&
+      cudaMemcpyAsync(ctx->latent_out, static_cast<const __nv_bfloat16*>(latent) + (size_t)n_pre * row_w,
+                      (size_t)M * row_w * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return GDLA_ERR_CUDA;
 
   stage(2, st);
   // a3: up-projections (q^C | rotated q^R), gate logits, K^C | V
@@ -223,7 +258,7 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
   GemmEpi eq{};
   eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F16; eq.M = M; eq.N = nqq;
   eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = T; eq.pos_ptr = positions;
-  eq.rope = rope;
+  eq.pos_off = ctx ? ctx->pos_offset : 0; eq.rope = rope;
   if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, M, nqq, cfg->q_rank, eq, ctl, st)))
     return GDLA_ERR_LAUNCH;
   GemmEpi eg{};
@@ -233,15 +268,16 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
     return GDLA_ERR_LAUNCH;
   GemmEpi ekv{};
   const int nkv = cfg->n_kv_heads * (cfg->d_nope + cfg->d_v);
-  ekv.C = KV; ekv.ldc = nkv; ekv.out_type = OUT_F16; ekv.M = M; ekv.N = nkv; ekv.pos_T = T;
-  if (launch_failed(launch_gemm(latent, cfg->kv_rank + cfg->d_rope, w->W_bKV, nkv, false, M, nkv, cfg->kv_rank,
-                  ekv, ctl, st)))
+  ekv.C = KV; ekv.ldc = nkv; ekv.out_type = OUT_F16; ekv.M = M + n_pre; ekv.N = nkv; ekv.pos_T = T;
+  if (launch_failed(launch_gemm(latent, cfg->kv_rank + cfg->d_rope, w->W_bKV, nkv, false, M + n_pre, nkv,
+                  cfg->kv_rank, ekv, ctl, st)))
     return GDLA_ERR_LAUNCH;
 
   stage(3, st);
   // a4: fused attention + differential combine + gate
   AttnParams ap{};
-  ap.B = B; ap.T = T; ap.window = cfg->window; ap.n_groups = cfg->n_noise;
+  ap.B = B; ap.T = T; ap.T_kv = T + n_pre; ap.q_off = n_pre; ap.window = cfg->window;
+  ap.n_groups = cfg->n_noise;
   ap.n_signal = cfg->n_signal; ap.rope_col0 = nH * cfg->d_nope;
   ap.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
   ap.lam = lam; ap.G = G; ap.O_noise = On; ap.Dg = Dg;
@@ -288,7 +324,8 @@ int gdla_workspace_size(const gdla_config_t* cfg, int B, int T, int mode, size_t
   int rc = check_config(cfg);
   if (rc) return rc;
   if (!bytes || B <= 0 || (mode != GDLA_MODE_DECODE && T <= 0) ||
-      (mode != GDLA_MODE_PREFILL && mode != GDLA_MODE_DECODE && mode != GDLA_MODE_VARLEN))
+      (mode != GDLA_MODE_PREFILL && mode != GDLA_MODE_DECODE && mode != GDLA_MODE_VARLEN &&
+       mode != GDLA_MODE_CONTEXT))
     return GDLA_ERR_INVALID_ARG;
   size_t off[WS_N + 1];
   layout(cfg, B, T, mode, off);
@@ -351,6 +388,43 @@ int gdla_prefill_varlen_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, c
   VarlenArgs vl{cu_seqlens, n_docs, kv_latent_out};
   return prefill_impl(cfg, w, x, 1, total, y, nullptr, 0, static_cast<uint8_t*>(workspace), off,
                       static_cast<cudaStream_t>(stream), &vl);
+}
+
+int gdla_latent_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int T,
+                    int pos_offset, void* latent_out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_weights(w))) return rc;
+  if (!x || !latent_out || !workspace || T <= 0 || pos_offset < 0) return GDLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(latent_out) || !aligned16(workspace)) return GDLA_ERR_INVALID_ARG;
+  if ((long long)T + pos_offset > (1ll << 30)) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  size_t off[WS_N + 1];
+  layout(cfg, 1, T, GDLA_MODE_PREFILL, off);
+  if (ws_bytes < off[WS_N]) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  ContextArgs ctx{nullptr, 0, pos_offset, latent_out};
+  return prefill_impl(cfg, w, x, 1, T, nullptr, nullptr, 0, static_cast<uint8_t*>(workspace), off,
+                      static_cast<cudaStream_t>(stream), nullptr, &ctx, true);
+}
+
+int gdla_prefill_context_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int T,
+                             int pos_offset, const void* prefix_latent, int n_prefix, void* y,
+                             void* latent_out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_weights(w))) return rc;
+  if (!x || !y || !workspace || T <= 0 || n_prefix < 0 || pos_offset < n_prefix ||
+      (n_prefix > 0 && !prefix_latent))
+    return GDLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(workspace) ||
+      (prefix_latent && !aligned16(prefix_latent)) || (latent_out && !aligned16(latent_out)))
+    return GDLA_ERR_INVALID_ARG;
+  if ((long long)T + pos_offset > (1ll << 30)) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  size_t off[WS_N + 1];
+  layout(cfg, 1, T + n_prefix, GDLA_MODE_CONTEXT, off);
+  if (ws_bytes < off[WS_N]) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  ContextArgs ctx{prefix_latent, n_prefix, pos_offset, latent_out};
+  return prefill_impl(cfg, w, x, 1, T, y, nullptr, 0, static_cast<uint8_t*>(workspace), off,
+                      static_cast<cudaStream_t>(stream), nullptr, &ctx, false);
 }
 
 int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void* dst,

@@ -144,18 +144,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   // the leader's copy of one of this CTA's barriers
   auto lead = [&](uint64_t* b) { return smem_map_rank(smem_u32(b), 0); };
 
-  // ---- work unit: (sequence rows [rowbase, rowbase + T), KV head j, 512-row block c), heaviest
-  // causal units first.  Equal-length batches derive it from the pair index; packed documents
-  // read it from a schedule built on the device (surplus pairs of the upper-bound grid exit
-  // here, both CTAs of a pair together, before any cluster-wide step).
+  // ---- work unit: (query rows [rowbase, rowbase + T) of a sequence whose keys are the rows
+  // [kvbase, kvbase + T_kv), KV head j, 512-row block c), heaviest causal units first.  Query
+  // row t sits at key position q_off + t (q_off > 0: a key prefix precedes the queries).
+  // Equal-length batches derive the unit from the pair index; packed documents read it from a
+  // schedule built on the device (surplus pairs of the upper-bound grid exit here, both CTAs
+  // of a pair together, before any cluster-wide step).
   const int pu = int(blockIdx.x) >> 1;
-  int c, rowbase, T, j;
+  int c, rowbase, kvbase, T, T_kv, q_off, j;
   if (p.units) {
     const int u = pu / p.n_groups;
     if (u >= *p.n_units) return;
     const int4 un = p.units[u];
-    rowbase = un.x;
-    T = un.y;
+    rowbase = kvbase = un.x;
+    T = T_kv = un.y;
+    q_off = 0;
     c = un.z;
     j = pu % p.n_groups;
   } else {
@@ -165,11 +168,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     const int b = (pu % per_c) / p.n_groups;
     j = pu % p.n_groups;
     rowbase = b * p.T;
+    kvbase = b * p.T_kv;
     T = p.T;
+    T_kv = p.T_kv;
+    q_off = p.q_off;
   }
   const int q0 = 512 * c;
-  const int t_hi = min(T - 1, q0 + 511) / 128;
-  const int t_lo = p.window > 0 ? max(0, q0 - p.window + 1) / 128 : 0;
+  const int t_hi = min(T_kv - 1, q_off + q0 + 511) / 128;
+  const int t_lo = p.window > 0 ? max(0, q_off + q0 - p.window + 1) / 128 : 0;
   const int n_kv = t_hi - t_lo + 1;
 
   if (threadIdx.x == 0) {
@@ -232,7 +238,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           tma_load_2d_pair(qd + 2 * QSUB, &mapQ, bar, p.rope_col0 + h * 64, y);
         }
         for (int i = 0; i < n_kv && ok; ++i) {
-          const int y0 = rowbase + 128 * (t_lo + i);
+          const int y0 = kvbase + 128 * (t_lo + i);
           {  // this CTA's 64 keys of K^C and k^R
             const int st = kq % KST;
             const uint32_t ph = (kq / KST) & 1;
@@ -392,9 +398,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const uint32_t tS = tmem + s * 128 + lane_off;
     const uint32_t tO = tmem + 256 + s * 128 + lane_off;
-    const int qpos = q0 + 256 * int(rank) + 128 * s + r;
-    const bool row_valid = qpos < T;
-    const long long m_row = (long long)rowbase + qpos;
+    const int qrow = q0 + 256 * int(rank) + 128 * s + r;   // query row within the sequence
+    const int qpos = q_off + qrow;                           // its key position
+    const bool row_valid = qrow < T;
+    const long long m_row = (long long)rowbase + qrow;
     const int W = p.window;
     const uint32_t p_ready_cl = lead(&bars->p_ready[s]);
     const uint32_t o_free_cl = lead(&bars->o_free[s]);
@@ -569,16 +576,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* kR16,
                         const AttnParams& p, KernelCtlHost ctl, cudaStream_t st) {
   if (p.B <= 0 || p.T <= 0) return 0;
-  const long long M = (long long)p.B * p.T;   // rows of the (packed) token matrix
+  if (p.T_kv < p.T + p.q_off || (p.units && (p.T_kv != p.T || p.q_off != 0))) return -2;
+  const long long M = (long long)p.B * p.T;      // query rows of the (packed) token matrix
+  const long long Mk = (long long)p.B * p.T_kv;  // key rows
   const uint64_t kv_ld = (uint64_t)p.n_groups * 256;
   CUtensorMap mq, mk, mkr, mv;
   if (make_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, QQ, qq_ld, M, (uint64_t)qq_ld * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      make_tmap_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, KV, kv_ld, M, kv_ld * 2, 64, 64,
+      make_tmap_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, KV, kv_ld, Mk, kv_ld * 2, 64, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      make_tmap_2d(&mkr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, kR16, 64, M, 128, 64, 64,
+      make_tmap_2d(&mkr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, kR16, 64, Mk, 128, 64, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      make_tmap_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, KV, kv_ld, M, kv_ld * 2, 64, 128,
+      make_tmap_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, KV, kv_ld, Mk, kv_ld * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return -3;
   if (cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

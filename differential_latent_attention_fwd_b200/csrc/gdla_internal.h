@@ -26,6 +26,7 @@ struct GemmEpi {
   int pos_T;             // row position = row % pos_T (used when pos_ptr is null)
   const int* pos_ptr;    // row position = pos_ptr[row / pos_div] + row % pos_div
   int pos_div;           // rows per pos_ptr entry (0 is read as 1)
+  int pos_off;           // added to the position (a key prefix of pos_off tokens precedes row 0)
   RopeTable rope;
   // Optional split-K scratch for skinny products (M <= 128): fp32 [splits][M][N].  When set
   // and worthwhile, K is split across CTAs and a reduce kernel applies this epilogue.
@@ -76,6 +77,7 @@ struct NormParams {
   float* lam;                 // [M, n_signal]
   int pos_T;                  // prefill: pos = m % pos_T, sequence = m / pos_T
   const int* pos_ptr;         // decode: sequence = m / q_per_seq, pos = pos_ptr[sequence] + m % q_per_seq
+  int pos_off;                // added to the position (a key prefix of pos_off tokens precedes row 0)
   int q_per_seq;              // new tokens per sequence (0 is read as 1)
   void* cache;                // optional bf16 [n_seq, cache_cap, kv_rank + 64]
   long long cache_cap;
@@ -88,7 +90,9 @@ int launch_norm_rope(const NormParams& p, cudaStream_t st);
 // work unit = one KV head over ATTN_UNIT_ROWS consecutive query rows of one sequence.
 constexpr int ATTN_UNIT_ROWS = 512;
 struct AttnParams {
-  int B, T, window;
+  int B, T, window;           // T = query rows per sequence
+  int T_kv;                   // key rows per sequence (= T, or T + q_off with a key prefix)
+  int q_off;                  // key position of query row 0 (the length of the key prefix)
   int n_groups;               // KV heads = noise heads
   int n_signal;               // 4 * n_groups
   int rope_col0;              // first q^R column of QQ (n_heads * 128)
@@ -112,6 +116,8 @@ struct AttnParams {
 int launch_varlen_schedule(const int* cu_seqlens, int n_docs, int total, int* positions,
                            int4* units, int* n_units, int max_units, int* cnt, int* fill, int max_c,
                            int* err, cudaStream_t st);
+// Rotated k^R of bf16 latent rows (columns kv_rank .. kv_rank + 63) -> fp16 rows of 64.
+int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void* kR16, cudaStream_t st);
 int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* kR16,
                         const AttnParams& p, KernelCtlHost ctl, cudaStream_t st);
 

@@ -70,7 +70,7 @@ extern "C" int gdla_attn_prefill_noalloc(const gdla_config_t* cfg, const void* q
   if ((rc = shared_kernel_ctl(&ctl))) return rc;
   const int nH = cfg->n_signal + cfg->n_noise;
   AttnParams ap{};
-  ap.B = B; ap.T = T; ap.window = cfg->window; ap.n_groups = cfg->n_noise;
+  ap.B = B; ap.T = T; ap.T_kv = T; ap.q_off = 0; ap.window = cfg->window; ap.n_groups = cfg->n_noise;
   ap.n_signal = cfg->n_signal; ap.rope_col0 = nH * cfg->d_nope;
   ap.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
   ap.lam = lam; ap.G = gate; ap.O_noise = scratch; ap.Dg = dg;

@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(const __grid_constant__ 
 
   // ---- k^R rotation: lane owns the pair (lane, lane + 32)
   const int qps = p.q_per_seq > 1 ? p.q_per_seq : 1;
-  int pos = p.pos_ptr ? p.pos_ptr[m / qps] + m % qps : (m % p.pos_T);
+  int pos = (p.pos_ptr ? p.pos_ptr[m / qps] + m % qps : (m % p.pos_T)) + p.pos_off;
   const int seq = p.pos_ptr ? m / qps : (m / p.pos_T);
   bool cache_ok = p.cache != nullptr;
   if (cache_ok && (pos < 0 || pos >= p.cache_cap)) {
@@ -118,6 +118,23 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(const __grid_constant__ 
   const float* rl = rkr + 64;
   for (int c = lane; c < p.n_signal; c += 32)
     p.lam[(long long)m * p.n_signal + c] = 1.0f / (1.0f + expf(-rl[c]));
+}
+
+// fp16 copy of the rotated k^R of bf16 latent rows (a key prefix handed in by the caller)
+__global__ void latent_to_kr16_kernel(const __nv_bfloat16* __restrict__ latent, int row_w,
+                                      int kv_rank, long long rows, __half* __restrict__ kR16) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows * 64) return;
+  const long long m = i >> 6;
+  kR16[i] = __float2half_rn(__bfloat162float(latent[m * row_w + kv_rank + (i & 63)]));
+}
+
+int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void* kR16, cudaStream_t st) {
+  if (rows <= 0) return 0;
+  const long long n = rows * 64;
+  latent_to_kr16_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(latent), kv_rank + 64, kv_rank, rows, static_cast<__half*>(kR16));
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
 int launch_norm_rope(const NormParams& p, cudaStream_t st) {

@@ -15,6 +15,7 @@ from .synth import GdlaShape, WEIGHT_NAMES
 class GdlaLayer:
     def __init__(self, shape: GdlaShape, weights: dict, g_q=None, g_kv=None, device="cuda"):
         self.shape = shape
+        self.window = shape.window        # 0 = full causal
         self.device = torch.device(device)
         self.w = {n: weights[n].to(self.device, torch.bfloat16).contiguous() for n in WEIGHT_NAMES}
         self.g_q = None if g_q is None else g_q.to(self.device, torch.bfloat16).contiguous()
@@ -49,6 +50,31 @@ class GdlaLayer:
             y = torch.empty((total, d), dtype=torch.bfloat16, device=self.device)
         ws = self.workspace(1, total, gb.GDLA_MODE_VARLEN)
         gb.gdla_prefill_varlen_fwd(self.cfg, self.cw, x, cu_seqlens, y, ws, kv_latent_out, stream)
+        return y
+
+    def latent(self, x: torch.Tensor, pos_offset: int = 0, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+        """Latent rows [T, kv_rank + d_rope] of tokens x [T, d] at positions pos_offset + t."""
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.cfg.kv_rank + self.cfg.d_rope), dtype=torch.bfloat16,
+                              device=self.device)
+        ws = self.workspace(1, T, gb.GDLA_MODE_PREFILL)
+        gb.gdla_latent_fwd(self.cfg, self.cw, x, pos_offset, out, ws, stream)
+        return out
+
+    def prefill_context(self, x: torch.Tensor, pos_offset: int, prefix_latent: torch.Tensor | None,
+                        y: torch.Tensor | None = None, latent_out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+        """Tokens x [T, d] at positions pos_offset + t, after the key prefix prefix_latent
+        [n_prefix, kv_rank + d_rope] (the latent rows of the n_prefix tokens just before)."""
+        T, d = x.shape
+        if y is None:
+            y = torch.empty((T, d), dtype=torch.bfloat16, device=self.device)
+        n_prefix = 0 if prefix_latent is None else prefix_latent.shape[0]
+        ws = self.workspace(1, T + n_prefix, gb.GDLA_MODE_CONTEXT)
+        gb.gdla_prefill_context_fwd(self.cfg, self.cw, x, pos_offset, prefix_latent, y, ws,
+                                    latent_out, stream)
         return y
 
     def absorbed(self, stream=None) -> gb.gdla_absorbed_t:

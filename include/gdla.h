@@ -87,11 +87,13 @@ typedef struct {
   uint32_t magic;
 } gdla_absorbed_t;
 
-enum { GDLA_MODE_PREFILL = 0, GDLA_MODE_DECODE = 1, GDLA_MODE_VARLEN = 2 };
+enum { GDLA_MODE_PREFILL = 0, GDLA_MODE_DECODE = 1, GDLA_MODE_VARLEN = 2, GDLA_MODE_CONTEXT = 3 };
 
 /* Bytes of workspace that gdla_prefill_fwd (mode 0: B sequences of T tokens),
- * gdla_decode_fwd (mode 1: B sequences, T = the cache capacity `cap` of the call) or
- * gdla_prefill_varlen_fwd (mode 2: B = 1, T = total packed tokens) needs. */
+ * gdla_decode_fwd (mode 1: B sequences, T = the cache capacity `cap` of the call),
+ * gdla_prefill_varlen_fwd (mode 2: B = 1, T = total packed tokens) or
+ * gdla_prefill_context_fwd (mode 3: B = 1, T = prefix rows + local tokens) needs.
+ * gdla_latent_fwd uses the mode-0 size for B = 1 and its T. */
 int gdla_workspace_size(const gdla_config_t* cfg, int B, int T, int mode, size_t* bytes);
 
 /* Bytes of device memory gdla_absorb_weights writes. */
@@ -121,6 +123,41 @@ int gdla_prefill_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const vo
 int gdla_prefill_varlen_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x,
                             int total, const int* cu_seqlens, int n_docs, void* y,
                             void* kv_latent_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Context parallelism.  The report trains 256K-token contexts by splitting the sequence over
+ * ranks, exchanging only key/value information: a sliding window needs the trailing W tokens of
+ * the preceding shard, full attention every preceding shard (paperglide.net summary,
+ * Figure 5 caption and the section on the hierarchical parallel layout).  Here the exchanged
+ * rows are the 576-value latent rows (RMSNorm'd c^KV | rotated k^R), from which every head's
+ * keys and values follow, instead of per-head K/V.  A rank first computes the latent rows of
+ * its own tokens (gdla_latent_fwd), the ranks exchange them, and each rank then runs its tokens
+ * with the rows of the tokens before them as a key prefix (gdla_prefill_context_fwd).  The two
+ * calls reproduce gdla_prefill_fwd on the whole sequence (the prefix keys' rotated k^R is read
+ * from the bf16 latent rows, as in decode).  No counterpart of this interface is printed in the
+ * pages.
+ *
+ * Latent rows of T tokens at positions pos_offset .. pos_offset + T - 1 of their sequence.
+ *   x [T, d_model] bf16 (device); latent_out [T, kv_rank + d_rope] bf16 (device, written).
+ *   workspace: >= gdla_workspace_size(cfg, 1, T, GDLA_MODE_PREFILL) bytes. */
+int gdla_latent_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int T,
+                    int pos_offset, void* latent_out, void* workspace, size_t ws_bytes,
+                    void* stream);
+
+/* Prefill of T tokens at positions pos_offset .. pos_offset + T - 1 of one sequence, after a
+ * key prefix given only by latent rows: the n_prefix tokens at positions
+ * pos_offset - n_prefix .. pos_offset - 1 (n_prefix <= pos_offset).  Full causal attention
+ * needs every preceding token (n_prefix = pos_offset); a sliding window W only the last
+ * min(W - 1, pos_offset) of them, and passing more changes nothing.
+ *   x [T, d_model] bf16; y [T, d_model] bf16 (written).
+ *   prefix_latent: bf16 [n_prefix, kv_rank + d_rope] (device), rows as gdla_latent_fwd or
+ *     gdla_prefill_fwd's kv_cache_out produce them (NULL when n_prefix = 0).
+ *   latent_out: NULL, or bf16 [T, kv_rank + d_rope]: the latent rows of the T local tokens.
+ *   workspace: >= gdla_workspace_size(cfg, 1, n_prefix + T, GDLA_MODE_CONTEXT) bytes.
+ * The key-side work for the prefix (its K^C | V) is recomputed from its latent rows. */
+int gdla_prefill_context_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x,
+                             int T, int pos_offset, const void* prefix_latent, int n_prefix,
+                             void* y, void* latent_out, void* workspace, size_t ws_bytes,
+                             void* stream);
 
 /* One-time weight preparation for the absorbed-form decode (MLA-style weight absorption:
  * attention runs in the latent space and K/V are never materialised; the pages note that

@@ -359,6 +359,41 @@ def gdla_prefill(x, weights: dict, cfg: OracleConfig, rows=None, g_q=None, g_kv=
     return (y, parts) if return_parts else y
 
 
+def gdla_prefill_after_prefix(x_local, prefix_latent, pos_offset: int, weights: dict,
+                              cfg: OracleConfig, g_q=None, g_kv=None):
+    """GDLA rows of the tokens x_local [T, d] at positions pos_offset .. pos_offset + T - 1 of
+    one sequence whose n_prefix preceding tokens (positions pos_offset - n_prefix ..
+    pos_offset - 1) are given only by their latent rows prefix_latent [n_prefix, kv_rank + d_rope]
+    (c_bar | rotated k^R, as a cache row).  The definition of section 2.2 of the picx.dev page
+    with the keys and values of those tokens expanded from the given rows; this is the unit a
+    context-parallel rank computes (paperglide.net summary, Figure 5 caption: ranks exchange
+    key/value information only).  Row by row, for small cases.  Returns y [T, d].
+    """
+    W = _weights64(weights)
+    gq = None if g_q is None else f64(g_q)
+    gkv = None if g_kv is None else f64(g_kv)
+    x = f64(x_local)
+    T = x.shape[0]
+    pre = np.zeros((0, cfg.kv_rank + cfg.d_rope)) if prefix_latent is None else f64(prefix_latent)
+    n_pre = pre.shape[0]
+    pos = pos_offset + np.arange(T)
+    cbar_l, kR_l = kv_latent(x, W["W_aKV"], gkv, pos, cfg)
+    cbar = np.concatenate([pre[:, : cfg.kv_rank], cbar_l], 0)
+    kR = np.concatenate([pre[:, cfg.kv_rank:], kR_l], 0)
+    KC, V = kv_heads(cbar, W["W_bKV"], cfg)
+    cQ, qC, qR = query_path(x, W["W_aQ"], W["W_bQ"], gq, pos, cfg)
+    lam = lambda_coeff(x, W["W_lambda"])
+    G = gate_logits(cQ, W["W_G"], cfg)
+    first = pos_offset - n_pre           # position of key row 0
+    y = np.empty((T, cfg.d_model))
+    for t in range(T):
+        lo, hi = key_range(int(pos[t]), cfg.window)
+        lo = max(lo, first)
+        H = attend_row(qC[t], qR[t], KC, kR, V, lo - first, hi - first, cfg)
+        _, y[t] = combine_row(H, lam[t], G[t], W["W_O"], cfg)
+    return y
+
+
 def gdla_prefill_packed(x_packed, cu_seqlens, weights: dict, cfg: OracleConfig, g_q=None, g_kv=None):
     """Packed documents: document d = rows cu[d] .. cu[d+1]-1 of x_packed [total, d_model] is an
     independent sequence (its own positions from 0, attention inside the document only).

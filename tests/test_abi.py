@@ -81,3 +81,30 @@ def test_misaligned_pointer_rejected(L):
     # workspace too small is reported before anything touches the device
     rc = L.gdla_prefill_fwd(ctypes.byref(cfg), ctypes.byref(w), fake, 1, 16, fake, None, 0, fake, 16, None)
     assert rc == -3
+
+
+def test_context_entry_points_validate_on_the_host(L):
+    cfg = gb.make_config(GdlaShape())
+    fake = ctypes.c_void_p(0x1000)
+    w = gb.gdla_weights_t(fake, fake, fake, fake, fake, fake, fake, None, None)
+    # context workspace covers prefix + local rows, like a prefill of that many tokens
+    assert gb.gdla_workspace_size(cfg, 1, 300, gb.GDLA_MODE_CONTEXT) == gb.gdla_workspace_size(cfg, 1, 300, 0)
+    big = 1 << 40
+    # a prefix longer than the position offset
+    rc = L.gdla_prefill_context_fwd(ctypes.byref(cfg), ctypes.byref(w), fake, 16, 8, fake, 16, fake, None,
+                                    fake, big, None)
+    assert rc == -1
+    # prefix rows announced but no pointer
+    rc = L.gdla_prefill_context_fwd(ctypes.byref(cfg), ctypes.byref(w), fake, 16, 16, None, 16, fake, None,
+                                    fake, big, None)
+    assert rc == -1
+    # workspace sized for the local tokens only
+    small = gb.gdla_workspace_size(cfg, 1, 16, 0)
+    rc = L.gdla_prefill_context_fwd(ctypes.byref(cfg), ctypes.byref(w), fake, 16, 512, fake, 512, fake, None,
+                                    fake, small, None)
+    assert rc == -3
+    # latent-only call: negative offset, null output
+    rc = L.gdla_latent_fwd(ctypes.byref(cfg), ctypes.byref(w), fake, 16, -1, fake, fake, big, None)
+    assert rc == -1
+    rc = L.gdla_latent_fwd(ctypes.byref(cfg), ctypes.byref(w), fake, 16, 0, None, fake, big, None)
+    assert rc == -1

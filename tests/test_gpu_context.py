@@ -1,0 +1,90 @@
+"""GPU context prefill (the per-rank unit of context parallelism) through the C ABI: a sequence
+run as consecutive chunks, each after the latent rows of the tokens before it, against the
+whole-sequence prefill on the GPU and against the fp64 oracle.  The chunks run one after the
+other on one device (no rank waits on another)."""
+import numpy as np
+import pytest
+import torch
+
+from differential_latent_attention_fwd_b200 import binding as gb
+from tests.gpu_helpers import check, oracle_prefill, prefill_case, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_chunks(layer, x, lengths, window, halo_only=True):
+    """y and latent rows of x [T, d] computed chunk by chunk; a window chunk gets only the last
+    W - 1 latent rows before it when halo_only."""
+    ys, lats, start = [], [], 0
+    for L in lengths:
+        xc = x[start: start + L].contiguous()
+        lat = layer.latent(xc, start)
+        if start == 0:
+            prefix = None
+        else:
+            allp = torch.cat(lats, 0)
+            n = start if (window == 0 or not halo_only) else min(window - 1, start)
+            prefix = allp[start - n:].contiguous()
+        lat_out = torch.empty_like(lat)
+        ys.append(layer.prefill_context(xc, start, prefix, latent_out=lat_out))
+        torch.cuda.synchronize()
+        assert gb.gdla_device_error() == 0
+        assert torch.equal(lat_out, lat), "latent rows of the context call differ from gdla_latent_fwd"
+        lats.append(lat)
+        start += L
+    return torch.cat(ys, 0), torch.cat(lats, 0)
+
+
+@pytest.mark.parametrize("window,lengths", [
+    (0, [300, 256, 444]),
+    (0, [1, 511, 512, 3]),
+    (128, [200, 129, 1, 370]),
+    (128, [100, 100, 100]),      # chunks shorter than W - 1: the prefix spans several chunks
+])
+def test_context_chunks_match_whole_sequence(cuda_ok, window, lengths):
+    T = sum(lengths)
+    shape, inp, layer, x = prefill_case(1, T, window, seed=13)
+    cache = torch.zeros((1, T, 576), dtype=torch.bfloat16, device="cuda")
+    y_full = layer.prefill(x, kv_cache_out=cache)
+    y_cp, lat_cp = _run_chunks(layer, x[0], lengths, window)
+    errs = []
+    # latent rows: same kernels on the same rows
+    check("latent rows, chunked vs whole", to_np(lat_cp), to_np(cache[0]), rel=4e-3, mabs=5e-2, errors=errs)
+    # outputs: the prefix keys' rotary part is read back from bf16 rows (as in decode)
+    check("y, chunked vs whole GPU prefill", to_np(y_cp), to_np(y_full[0]), rel=3e-3, mabs=1.5e-2, errors=errs)
+    rows = sorted(set([0, T - 1] + list(np.cumsum(lengths)[:-1]) + list(np.cumsum(lengths)[:-1] - 1)
+                      + list(np.linspace(0, T - 1, 24).astype(int))))
+    yo = oracle_prefill(inp, rows=rows)
+    check(f"y, chunked vs oracle ({len(rows)} rows)", to_np(y_cp[rows]), yo[0], errors=errs)
+    assert not errs, "\n".join(errs)
+
+
+def test_context_window_prefix_longer_than_halo_is_ignored(cuda_ok):
+    """Passing every earlier latent row instead of the last W - 1 gives the same result (up to
+    rounding: a longer prefix moves the 128-key tile boundaries the online softmax walks)."""
+    shape, inp, layer, x = prefill_case(1, 700, 128, seed=17)
+    a, _ = _run_chunks(layer, x[0], [300, 400], 128, halo_only=True)
+    b, _ = _run_chunks(layer, x[0], [300, 400], 128, halo_only=False)
+    check("window chunk: halo-only vs whole prefix", to_np(b), to_np(a), rel=1e-3, mabs=5e-3)
+
+
+def test_context_chunks_t8192(cuda_ok):
+    """Four 2048-token chunks of an 8192-token causal sequence (sampled oracle rows)."""
+    lengths = [2048] * 4
+    T = sum(lengths)
+    shape, inp, layer, x = prefill_case(1, T, 0, seed=19)
+    y_full = layer.prefill(x)
+    y_cp, _ = _run_chunks(layer, x[0], lengths, 0)
+    errs = []
+    check("T=8192 chunked vs whole GPU prefill", to_np(y_cp), to_np(y_full[0]), rel=3e-3, mabs=1.5e-2, errors=errs)
+    rows = sorted(set([0, 2047, 2048, 4095, 4096, 6143, 6144, T - 1] + list(np.linspace(0, T - 1, 40).astype(int))))
+    yo = oracle_prefill(inp, rows=rows)
+    check("T=8192 chunked vs oracle", to_np(y_cp[rows]), yo[0], errors=errs)
+    assert not errs, "\n".join(errs)
+
+
+def test_context_rejects_bad_offsets(cuda_ok):
+    shape, inp, layer, x = prefill_case(1, 64, 0, seed=2)
+    lat = layer.latent(x[0, :32].contiguous(), 0)
+    with pytest.raises(gb.GdlaError):
+        layer.prefill_context(x[0, 32:].contiguous(), 16, lat)     # 32 prefix rows before position 16
