@@ -349,6 +349,40 @@ def run_gpu(args):
     if world > 1:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
 
+    # ---- context parallelism: per-rank compute of an 8-way split of the same sequence (its
+    # latent pass + its tokens after the latent rows of every earlier token); the exchange of
+    # latent rows between ranks needs several GPUs and is reported as bytes only
+    cp = None
+    if not (args.skip_prefill or args.skip_cp) and world == 1:
+        P = 8
+        Tr = T // P
+        lat_all = layer.latent(x[0], 0)
+        lat_r = torch.empty((Tr, s.latent_row), dtype=torch.bfloat16, device=dev)
+        y_r = torch.empty((Tr, s.d_model), dtype=torch.bfloat16, device=dev)
+        cp_ms = {}
+        for r in (0, P - 1):
+            xr = x[0, r * Tr:(r + 1) * Tr]
+            prefix = lat_all[: r * Tr] if r else None
+            times = []
+            for i in range(4):
+                flush.fill_(1)
+                e0.record(stream)
+                layer.latent(xr, r * Tr, out=lat_r, stream=stream)
+                layer.prefill_context(xr, r * Tr, prefix, y=y_r, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                if i:
+                    times.append(e0.elapsed_time(e1))
+            cp_ms[r] = statistics.median(times)
+        last_pairs = Tr * (P - 1) * Tr + Tr * (Tr + 1) // 2
+        last_flop = (last_pairs * attn_flops_per_pair(s) + Tr * proj_flops_per_token(s)
+                     + (P - 1) * Tr * 2 * s.kv_rank * s.n_kv_heads * (s.d_nope + s.d_v))
+        cp = {"ranks": P, "tokens_per_rank": Tr, "first_rank_ms": cp_ms[0],
+              "last_rank_ms": cp_ms[P - 1], "last_rank_tflops": last_flop / (cp_ms[P - 1] * 1e-3) / 1e12,
+              "exchanged_bytes_per_token": s.latent_row * 2,
+              "last_rank_receives_bytes": (P - 1) * Tr * s.latent_row * 2,
+              "timing": "one GPU, each rank's two calls back to back (L2 flushed); no communication"}
+
     peaks, peak_src = load_peaks()
     pairs = valid_pairs(T, 0)
     attn_flop = B * pairs * attn_flops_per_pair(s)
@@ -408,6 +442,7 @@ def run_gpu(args):
                     "attention_tflops": attn_tf, "tok_per_s": world * B * T / max(st["prefill_ms"] * 1e-3, 1e-12),
                     "layer_frac_of_bf16_peak": value / world / peaks["bf16_tflops_sustained"]},
         "decode": decode,
+        "context_parallel": cp,
         "roofline": {"kernel": "attn_prefill_kernel", "bound": "tensor", "achieved": attn_tf,
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": attn_tf / peaks["bf16_tflops_sustained"],
@@ -455,6 +490,7 @@ def main():
     ap.add_argument("--skip-prefill", action="store_true", help="profiling runs: decode only")
     ap.add_argument("--skip-e2e", action="store_true", help="profiling runs: no host-buffer pass")
     ap.add_argument("--decode-L", type=int, default=DECODE["L"], help="cached positions (profiling runs)")
+    ap.add_argument("--skip-cp", action="store_true", help="profiling runs: no context-parallel split")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
