@@ -65,7 +65,7 @@ def test_context_window_prefix_longer_than_halo_is_ignored(cuda_ok):
     shape, inp, layer, x = prefill_case(1, 700, 128, seed=17)
     a, _ = _run_chunks(layer, x[0], [300, 400], 128, halo_only=True)
     b, _ = _run_chunks(layer, x[0], [300, 400], 128, halo_only=False)
-    check("window chunk: halo-only vs whole prefix", to_np(b), to_np(a), rel=1e-3, mabs=5e-3)
+    check("window chunk: halo-only vs whole prefix", to_np(b), to_np(a), rel=3e-3, mabs=1.5e-2)
 
 
 def test_context_chunks_t8192(cuda_ok):
