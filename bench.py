@@ -329,17 +329,18 @@ def run_gpu(args):
         dist.all_reduce(local_stats, op=dist.ReduceOp.MAX)
     st = dict(zip(keys, local_stats.tolist()))
 
-    # ---- end to end through the C ABI with host buffers (pinned H2D of x, D2H of y)
+    # ---- end to end through the C ABI with host buffers: gdla_prefill_host_fwd takes x from and
+    # writes y to pinned host memory, its copies overlapping the row-separable stages
     y_host = torch.empty_like(x_host).pin_memory()
+    ws_host = torch.empty(gb.gdla_workspace_size(layer.cfg, B, T, gb.GDLA_MODE_HOST) if not
+                          (args.skip_e2e or args.skip_prefill) else 1, dtype=torch.uint8, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_ms = []
     for i in range(0 if (args.skip_e2e or args.skip_prefill) else max(2, min(args.steps, 5)) + 1):
         flush.fill_(1)
         barrier()
         e0.record(stream)
-        x.copy_(x_host, non_blocking=True)
-        gb.gdla_prefill_fwd(layer.cfg, layer.cw, x, y, ws, stream=stream)
-        y_host.copy_(y, non_blocking=True)
+        gb.gdla_prefill_host_fwd(layer.cfg, layer.cw, x_host, y_host, ws_host, n_pieces=16, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         if i > 0:

@@ -21,6 +21,7 @@ GDLA_MODE_PREFILL = 0
 GDLA_MODE_DECODE = 1
 GDLA_MODE_VARLEN = 2
 GDLA_MODE_CONTEXT = 3
+GDLA_MODE_HOST = 4
 STATUS = {0: "GDLA_OK", -1: "GDLA_ERR_INVALID_ARG", -2: "GDLA_ERR_UNSUPPORTED_SHAPE",
           -3: "GDLA_ERR_WORKSPACE_TOO_SMALL", -4: "GDLA_ERR_LAUNCH",
           -5: "GDLA_ERR_DEVICE_TIMEOUT", -6: "GDLA_ERR_CUDA"}
@@ -80,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "gdla_decode_multi_fwd": [cfgp, abp, P, I, P, P, I, I, P, P, SZ, P],
             "gdla_latent_fwd": [cfgp, wp, P, I, I, P, P, SZ, P],
             "gdla_prefill_context_fwd": [cfgp, wp, P, I, I, P, I, P, P, P, SZ, P],
+            "gdla_prefill_host_fwd": [cfgp, wp, P, I, I, P, I, P, SZ, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -110,6 +112,16 @@ def _ptr(t, dtype=None, name="tensor"):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t, dtype, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host (CPU) tensor")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -178,6 +190,16 @@ def gdla_prefill_varlen_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, cu_seqlens:
         _ptr(y, torch.bfloat16, "y"), _ptr(kv_latent_out, torch.bfloat16, "kv_latent_out"),
         _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream)))
+
+
+def gdla_prefill_host_fwd(cfg, w: gdla_weights_t, x_host: torch.Tensor, y_host: torch.Tensor,
+                          workspace: torch.Tensor, n_pieces: int = 8, stream=None) -> None:
+    """x_host, y_host: [B, T, d] bf16 CPU tensors (pin them for overlapped copies)."""
+    B, T, _ = x_host.shape
+    _check("gdla_prefill_host_fwd", lib().gdla_prefill_host_fwd(
+        ctypes.byref(cfg), ctypes.byref(w), _host_ptr(x_host, torch.bfloat16, "x_host"), B, T,
+        _host_ptr(y_host, torch.bfloat16, "y_host"), n_pieces, _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def gdla_latent_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, pos_offset: int, latent_out: torch.Tensor,

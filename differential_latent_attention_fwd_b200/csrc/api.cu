@@ -8,6 +8,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 namespace gdla {
 
 // Device error word written by bounded waits (one instance per device that loads the library).
@@ -147,6 +149,100 @@ struct VarlenArgs {
   void* latent_out;
 };
 
+// a1 on token rows [r0, r1): [x W_aQ | x W_aKV | x W_lambda] in fp32 into D1 rows r0..r1-1.
+static int down_proj_rows(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x,
+                          float* D1, int pos_T, long long r0, long long r1, KernelCtlHost ctl,
+                          cudaStream_t st) {
+  const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
+  const int M = int(r1 - r0);
+  if (M <= 0) return GDLA_OK;
+  const void* xr = static_cast<const __nv_bfloat16*>(x) + r0 * cfg->d_model;
+  float* D = D1 + r0 * ld1;
+  GemmEpi ep{};
+  ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = M; ep.rope_lo = ep.rope_hi = 0; ep.pos_T = pos_T;
+  ep.C = D; ep.N = cfg->q_rank;
+  if (launch_failed(launch_gemm(xr, cfg->d_model, w->W_aQ, cfg->q_rank, false, M, cfg->q_rank, cfg->d_model, ep, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  ep.C = D + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
+  if (launch_failed(launch_gemm(xr, cfg->d_model, w->W_aKV, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  ep.C = D + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
+  if (launch_failed(launch_gemm(xr, cfg->d_model, w->W_lambda, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  return GDLA_OK;
+}
+
+// a5 on token rows [r0, r1): y = Dg W^O.
+static int out_proj_rows(const gdla_config_t* cfg, const gdla_weights_t* w, const void* Dg, void* y,
+                         int pos_T, long long r0, long long r1, KernelCtlHost ctl, cudaStream_t st) {
+  const int M = int(r1 - r0);
+  if (M <= 0) return GDLA_OK;
+  const int kdim = cfg->n_signal * cfg->d_v;
+  GemmEpi eo{};
+  eo.C = static_cast<__nv_bfloat16*>(y) + r0 * cfg->d_model; eo.ldc = cfg->d_model;
+  eo.out_type = OUT_BF16; eo.M = M; eo.N = cfg->d_model; eo.pos_T = pos_T;
+  if (launch_failed(launch_gemm(static_cast<const __nv_bfloat16*>(Dg) + r0 * kdim, kdim, w->W_O,
+                                cfg->d_model, false, M, cfg->d_model, kdim, eo, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  return GDLA_OK;
+}
+
+// a2 + a3 on token rows [r0, r1) of B sequences of T tokens (no key prefix, no packed
+// documents): norms, rotary key, lambda and latent rows, then q^C | rotated q^R, gate logits and
+// K^C | V of those rows.
+static int norm_up_rows(const gdla_config_t* cfg, const gdla_weights_t* w, uint8_t* ws,
+                        const size_t* off, int T, long long r0, long long r1, const RopeTable& rope,
+                        int* err, KernelCtlHost ctl, cudaStream_t st) {
+  const int M = int(r1 - r0);
+  if (M <= 0) return GDLA_OK;
+  const int nH = cfg->n_signal + cfg->n_noise;
+  const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
+  const int row_w = cfg->kv_rank + cfg->d_rope;
+  const int nqq = nH * (cfg->d_nope + cfg->d_rope);
+  const int ldg = cfg->n_signal * cfg->d_v;
+  const int nkv = cfg->n_kv_heads * (cfg->d_nope + cfg->d_v);
+  __nv_bfloat16* cQ = reinterpret_cast<__nv_bfloat16*>(ws + off[WS_CQ]) + r0 * cfg->q_rank;
+  __nv_bfloat16* latent = reinterpret_cast<__nv_bfloat16*>(ws + off[WS_LATENT]) + r0 * row_w;
+  NormParams np{};
+  np.D1 = reinterpret_cast<float*>(ws + off[WS_D1]) + r0 * ld1; np.ld1 = ld1; np.M = M;
+  np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank; np.n_signal = cfg->n_signal;
+  np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
+  np.cQ = cQ; np.latent = latent;
+  np.kR16 = reinterpret_cast<__half*>(ws + off[WS_KR16]) + r0 * cfg->d_rope;
+  np.lam = reinterpret_cast<float*>(ws + off[WS_LAM]) + r0 * cfg->n_signal;
+  np.pos_T = T; np.row_off = int(r0); np.rope = rope; np.err = err;
+  if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
+  GemmEpi eq{};
+  eq.C = reinterpret_cast<__half*>(ws + off[WS_QQ]) + r0 * nqq; eq.ldc = nqq; eq.out_type = OUT_F16;
+  eq.M = M; eq.N = nqq; eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = T;
+  eq.row_off = int(r0); eq.rope = rope;
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, M, nqq, cfg->q_rank, eq, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  GemmEpi eg{};
+  eg.C = reinterpret_cast<__nv_bfloat16*>(ws + off[WS_G]) + r0 * ldg; eg.ldc = ldg; eg.out_type = OUT_BF16;
+  eg.M = M; eg.N = ldg; eg.pos_T = T;
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_G, ldg, false, M, ldg, cfg->q_rank, eg, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  GemmEpi ekv{};
+  ekv.C = reinterpret_cast<__half*>(ws + off[WS_KV]) + r0 * nkv; ekv.ldc = nkv; ekv.out_type = OUT_F16;
+  ekv.M = M; ekv.N = nkv; ekv.pos_T = T;
+  if (launch_failed(launch_gemm(latent, row_w, w->W_bKV, nkv, false, M, nkv, cfg->kv_rank, ekv, ctl, st)))
+    return GDLA_ERR_LAUNCH;
+  return GDLA_OK;
+}
+
+// Host-buffer prefill: x arrives and y leaves in row pieces on two copy streams; the
+// row-separable stages before the attention (a1 - a3) of a piece start as soon as it has
+// landed, and each piece of y leaves as soon as its output projection is done.  Null = the
+// whole-buffer device path.
+struct HostPipeArgs {
+  const void* x_host;
+  void* y_host;
+  int n_pieces;
+  cudaStream_t h2d, d2h;
+  cudaEvent_t* ev;            // >= 2 * n_pieces + 2 events
+};
+
 // A key prefix: the latent rows of the n_prefix tokens that precede x in its sequence.
 struct ContextArgs {
   const void* prefix_latent;   // [n_prefix, kv_rank + d_rope] bf16
@@ -162,7 +258,8 @@ struct ContextArgs {
 static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int B,
                         int T, void* y, void* kv_cache_out, int cache_cap, uint8_t* ws,
                         const size_t* off, cudaStream_t st, const VarlenArgs* vl,
-                        const ContextArgs* ctx = nullptr, bool latent_only = false) {
+                        const ContextArgs* ctx = nullptr, bool latent_only = false,
+                        const HostPipeArgs* hp = nullptr) {
   int rc;
   int* err;
   if ((rc = error_word(&err))) return rc;
@@ -207,21 +304,36 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
     if (vl->latent_out) latent = vl->latent_out;
   }
 
-  // a1: [x W_aQ | x W_aKV | x W_lambda] in fp32
-  GemmEpi ep{};
-  ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = M; ep.rope_lo = ep.rope_hi = 0; ep.pos_T = T;
-  ep.rope = rope;
-  ep.C = D1; ep.N = cfg->q_rank;
-  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_aQ, cfg->q_rank, false, M, cfg->q_rank, cfg->d_model, ep, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  ep.C = D1 + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
-  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_aKV, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  ep.C = D1 + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
-  if (launch_failed(launch_gemm(x, cfg->d_model, w->W_lambda, ep.N, false, M, ep.N, cfg->d_model, ep, ctl, st)))
-    return GDLA_ERR_LAUNCH;
+  // a1: [x W_aQ | x W_aKV | x W_lambda] in fp32 (with host buffers: piece by piece as x lands)
+  if (hp) {
+    const long long piece = (M + hp->n_pieces - 1) / hp->n_pieces;
+    // the copies must not overtake earlier work on the caller's stream (the workspace may be busy)
+    if (cudaEventRecord(hp->ev[0], st) != cudaSuccess || cudaStreamWaitEvent(hp->h2d, hp->ev[0], 0) != cudaSuccess)
+      return GDLA_ERR_CUDA;
+    for (int k = 0; k < hp->n_pieces; ++k) {
+      const long long r0 = k * piece, r1 = r0 + piece < M ? r0 + piece : M;
+      if (r0 >= r1) break;
+      const size_t bytes = size_t(r1 - r0) * cfg->d_model * 2, off_b = size_t(r0) * cfg->d_model * 2;
+      if (cudaMemcpyAsync(static_cast<uint8_t*>(const_cast<void*>(x)) + off_b,
+                          static_cast<const uint8_t*>(hp->x_host) + off_b, bytes, cudaMemcpyHostToDevice,
+                          hp->h2d) != cudaSuccess ||
+          cudaEventRecord(hp->ev[2 + k], hp->h2d) != cudaSuccess)
+        return GDLA_ERR_CUDA;
+    }
+    for (int k = 0; k < hp->n_pieces; ++k) {
+      const long long r0 = k * piece, r1 = r0 + piece < M ? r0 + piece : M;
+      if (r0 >= r1) break;
+      if (cudaStreamWaitEvent(st, hp->ev[2 + k], 0) != cudaSuccess) return GDLA_ERR_CUDA;
+      if ((rc = down_proj_rows(cfg, w, x, D1, T, r0, r1, ctl, st))) return rc;
+      if ((rc = norm_up_rows(cfg, w, ws, off, T, r0, r1, rope, err, ctl, st))) return rc;
+    }
+  } else {
+    if ((rc = down_proj_rows(cfg, w, x, D1, T, 0, M, ctl, st))) return rc;
+  }
 
+  const int nqq = nH * (cfg->d_nope + cfg->d_rope);
   stage(1, st);
+  if (!hp) {
   // a2: norms, rotary key, lambda, latent rows
   NormParams np{};
   np.D1 = D1; np.ld1 = ld1; np.M = M; np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank;
@@ -254,7 +366,6 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
 
   stage(2, st);
   // a3: up-projections (q^C | rotated q^R), gate logits, K^C | V
-  const int nqq = nH * (cfg->d_nope + cfg->d_rope);
   GemmEpi eq{};
   eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F16; eq.M = M; eq.N = nqq;
   eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = T; eq.pos_ptr = positions;
@@ -272,6 +383,7 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
   if (launch_failed(launch_gemm(latent, cfg->kv_rank + cfg->d_rope, w->W_bKV, nkv, false, M + n_pre, nkv,
                   cfg->kv_rank, ekv, ctl, st)))
     return GDLA_ERR_LAUNCH;
+  }  // !hp (the host-buffer path ran a2 and a3 piece by piece above)
 
   stage(3, st);
   // a4: fused attention + differential combine + gate
@@ -285,13 +397,26 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
   if (launch_failed(launch_attn_prefill(QQ, nqq, KV, kR16, ap, ctl, st))) return GDLA_ERR_LAUNCH;
 
   stage(4, st);
-  // a5: output projection
-  GemmEpi eo{};
-  eo.C = y; eo.ldc = cfg->d_model; eo.out_type = OUT_BF16; eo.M = M; eo.N = cfg->d_model;
-  eo.pos_T = T;
-  if (launch_failed(launch_gemm(Dg, cfg->n_signal * cfg->d_v, w->W_O, cfg->d_model, false, M, cfg->d_model,
-                  cfg->n_signal * cfg->d_v, eo, ctl, st)))
-    return GDLA_ERR_LAUNCH;
+  // a5: output projection (with host buffers: piece by piece, each piece of y leaving at once)
+  if (hp) {
+    const long long piece = (M + hp->n_pieces - 1) / hp->n_pieces;
+    for (int k = 0; k < hp->n_pieces; ++k) {
+      const long long r0 = k * piece, r1 = r0 + piece < M ? r0 + piece : M;
+      if (r0 >= r1) break;
+      if ((rc = out_proj_rows(cfg, w, Dg, y, T, r0, r1, ctl, st))) return rc;
+      const size_t bytes = size_t(r1 - r0) * cfg->d_model * 2, off_b = size_t(r0) * cfg->d_model * 2;
+      if (cudaEventRecord(hp->ev[2 + hp->n_pieces + k], st) != cudaSuccess ||
+          cudaStreamWaitEvent(hp->d2h, hp->ev[2 + hp->n_pieces + k], 0) != cudaSuccess ||
+          cudaMemcpyAsync(static_cast<uint8_t*>(hp->y_host) + off_b, static_cast<const uint8_t*>(y) + off_b,
+                          bytes, cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
+        return GDLA_ERR_CUDA;
+    }
+    // the caller's stream completes only after the last piece of y has reached the host
+    if (cudaEventRecord(hp->ev[1], hp->d2h) != cudaSuccess || cudaStreamWaitEvent(st, hp->ev[1], 0) != cudaSuccess)
+      return GDLA_ERR_CUDA;
+  } else {
+    if ((rc = out_proj_rows(cfg, w, Dg, y, T, 0, M, ctl, st))) return rc;
+  }
   stage(5, st);
   return GDLA_OK;
 }
@@ -320,13 +445,28 @@ int gdla_set_wait_limit_ns(unsigned long long ns) {
   return GDLA_OK;
 }
 
+// Host-buffer prefill: the prefill layout, then device copies of x and y.
+static size_t host_extra_offset(const gdla_config_t* c, int B, int T, size_t* y_off, size_t* total) {
+  size_t off[WS_N + 1];
+  layout(c, B, T, GDLA_MODE_PREFILL, off);
+  const size_t xy = ((size_t)B * T * c->d_model * 2 + 255) & ~size_t(255);
+  *y_off = off[WS_N] + xy;
+  *total = off[WS_N] + 2 * xy;
+  return off[WS_N];
+}
+
 int gdla_workspace_size(const gdla_config_t* cfg, int B, int T, int mode, size_t* bytes) {
   int rc = check_config(cfg);
   if (rc) return rc;
   if (!bytes || B <= 0 || (mode != GDLA_MODE_DECODE && T <= 0) ||
       (mode != GDLA_MODE_PREFILL && mode != GDLA_MODE_DECODE && mode != GDLA_MODE_VARLEN &&
-       mode != GDLA_MODE_CONTEXT))
+       mode != GDLA_MODE_CONTEXT && mode != GDLA_MODE_HOST))
     return GDLA_ERR_INVALID_ARG;
+  if (mode == GDLA_MODE_HOST) {
+    size_t y_off;
+    host_extra_offset(cfg, B, T, &y_off, bytes);
+    return GDLA_OK;
+  }
   size_t off[WS_N + 1];
   layout(cfg, B, T, mode, off);
   *bytes = off[WS_N];
@@ -425,6 +565,60 @@ int gdla_prefill_context_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, 
   ContextArgs ctx{prefix_latent, n_prefix, pos_offset, latent_out};
   return prefill_impl(cfg, w, x, 1, T, y, nullptr, 0, static_cast<uint8_t*>(workspace), off,
                       static_cast<cudaStream_t>(stream), nullptr, &ctx, false);
+}
+
+// Copy streams and events of the host-buffer prefill, one set per device, created on first use
+// and kept for the life of the process (like the device error word).
+namespace {
+constexpr int kMaxPieces = 64;
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev[2 * kMaxPieces + 2];
+};
+constexpr int kMaxDevices = 64;
+HostPipe g_pipes[kMaxDevices];
+std::mutex g_pipe_mu;
+}  // namespace
+
+static int host_pipe(HostPipe** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe& p = g_pipes[dev];
+  if (!p.ready) {
+    if (cudaStreamCreateWithFlags(&p.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&p.d2h, cudaStreamNonBlocking) != cudaSuccess)
+      return GDLA_ERR_CUDA;
+    for (auto& e : p.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return GDLA_ERR_CUDA;
+    p.ready = true;
+  }
+  *out = &p;
+  return GDLA_OK;
+}
+
+int gdla_prefill_host_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x_host, int B,
+                          int T, void* y_host, int n_pieces, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if ((rc = check_weights(w))) return rc;
+  if (!x_host || !y_host || !workspace || B <= 0 || T <= 0 || n_pieces < 1 || n_pieces > kMaxPieces)
+    return GDLA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return GDLA_ERR_INVALID_ARG;
+  if ((long long)B * T > (1ll << 30)) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  size_t y_off, total;
+  const size_t x_off = host_extra_offset(cfg, B, T, &y_off, &total);
+  if (ws_bytes < total) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  HostPipe* pipe;
+  if ((rc = host_pipe(&pipe))) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  size_t off[WS_N + 1];
+  layout(cfg, B, T, GDLA_MODE_PREFILL, off);
+  HostPipeArgs hp{x_host, y_host, n_pieces, pipe->h2d, pipe->d2h, pipe->ev};
+  return prefill_impl(cfg, w, ws + x_off, B, T, ws + y_off, nullptr, 0, ws, off,
+                      static_cast<cudaStream_t>(stream), nullptr, nullptr, false, &hp);
 }
 
 int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void* dst,

@@ -27,6 +27,7 @@ struct GemmEpi {
   const int* pos_ptr;    // row position = pos_ptr[row / pos_div] + row % pos_div
   int pos_div;           // rows per pos_ptr entry (0 is read as 1)
   int pos_off;           // added to the position (a key prefix of pos_off tokens precedes row 0)
+  int row_off;           // row index of output row 0 in the full token matrix (row pieces)
   RopeTable rope;
   // Optional split-K scratch for skinny products (M <= 128): fp32 [splits][M][N].  When set
   // and worthwhile, K is split across CTAs and a reduce kernel applies this epilogue.
@@ -78,6 +79,7 @@ struct NormParams {
   int pos_T;                  // prefill: pos = m % pos_T, sequence = m / pos_T
   const int* pos_ptr;         // decode: sequence = m / q_per_seq, pos = pos_ptr[sequence] + m % q_per_seq
   int pos_off;                // added to the position (a key prefix of pos_off tokens precedes row 0)
+  int row_off;                // token index of row 0 in the full token matrix (row pieces)
   int q_per_seq;              // new tokens per sequence (0 is read as 1)
   void* cache;                // optional bf16 [n_seq, cache_cap, kv_rank + 64]
   long long cache_cap;

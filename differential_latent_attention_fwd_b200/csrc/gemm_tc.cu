@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(128, 1)
   int pos = 0;
   if (ep.rope_hi > ep.rope_lo && row < ep.M) {
     const int dv = ep.pos_div > 1 ? ep.pos_div : 1;
-    pos = (ep.pos_ptr ? ep.pos_ptr[row / dv] + row % dv : (row % ep.pos_T)) + ep.pos_off;
+    pos = (ep.pos_ptr ? ep.pos_ptr[row / dv] + row % dv : ((row + ep.row_off) % ep.pos_T)) + ep.pos_off;
   }
   const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
 #pragma unroll 1
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
   }
   if (blk * 64 >= ep.rope_lo && blk * 64 < ep.rope_hi) {
     const int dv = ep.pos_div > 1 ? ep.pos_div : 1;
-    const int pos = (ep.pos_ptr ? ep.pos_ptr[row / dv] + row % dv : (row % ep.pos_T)) + ep.pos_off;
+    const int pos = (ep.pos_ptr ? ep.pos_ptr[row / dv] + row % dv : ((row + ep.row_off) % ep.pos_T)) + ep.pos_off;
     float cs, sn;
     rope_cs(pos, ep.rope.inv_freq[i], &cs, &sn);
     const float x1 = a, x2 = b;

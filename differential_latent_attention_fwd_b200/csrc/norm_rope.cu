@@ -73,8 +73,8 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(const __grid_constant__ 
 
   // ---- k^R rotation: lane owns the pair (lane, lane + 32)
   const int qps = p.q_per_seq > 1 ? p.q_per_seq : 1;
-  int pos = (p.pos_ptr ? p.pos_ptr[m / qps] + m % qps : (m % p.pos_T)) + p.pos_off;
-  const int seq = p.pos_ptr ? m / qps : (m / p.pos_T);
+  int pos = (p.pos_ptr ? p.pos_ptr[m / qps] + m % qps : ((m + p.row_off) % p.pos_T)) + p.pos_off;
+  const int seq = p.pos_ptr ? m / qps : ((m + p.row_off) / p.pos_T);
   bool cache_ok = p.cache != nullptr;
   if (cache_ok && (pos < 0 || pos >= p.cache_cap)) {
     if (lane == 0 && p.err) atomicCAS(p.err, 0, SITE_BAD_CACHE_LEN);

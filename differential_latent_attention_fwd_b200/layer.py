@@ -52,6 +52,17 @@ class GdlaLayer:
         gb.gdla_prefill_varlen_fwd(self.cfg, self.cw, x, cu_seqlens, y, ws, kv_latent_out, stream)
         return y
 
+    def prefill_host(self, x_host: torch.Tensor, y_host: torch.Tensor | None = None, n_pieces: int = 8,
+                     stream=None) -> torch.Tensor:
+        """x_host [B, T, d] bf16 on the host (pinned for overlapped copies) -> y_host [B, T, d];
+        returns once the work is enqueued: synchronise `stream` before reading y_host."""
+        B, T, d = x_host.shape
+        if y_host is None:
+            y_host = torch.empty((B, T, d), dtype=torch.bfloat16, pin_memory=True)
+        ws = self.workspace(B, T, gb.GDLA_MODE_HOST)
+        gb.gdla_prefill_host_fwd(self.cfg, self.cw, x_host, y_host, ws, n_pieces, stream)
+        return y_host
+
     def latent(self, x: torch.Tensor, pos_offset: int = 0, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
         """Latent rows [T, kv_rank + d_rope] of tokens x [T, d] at positions pos_offset + t."""

@@ -87,7 +87,8 @@ typedef struct {
   uint32_t magic;
 } gdla_absorbed_t;
 
-enum { GDLA_MODE_PREFILL = 0, GDLA_MODE_DECODE = 1, GDLA_MODE_VARLEN = 2, GDLA_MODE_CONTEXT = 3 };
+enum { GDLA_MODE_PREFILL = 0, GDLA_MODE_DECODE = 1, GDLA_MODE_VARLEN = 2, GDLA_MODE_CONTEXT = 3,
+       GDLA_MODE_HOST = 4 };
 
 /* Bytes of workspace that gdla_prefill_fwd (mode 0: B sequences of T tokens),
  * gdla_decode_fwd (mode 1: B sequences, T = the cache capacity `cap` of the call),
@@ -108,6 +109,25 @@ int gdla_absorbed_size(const gdla_config_t* cfg, size_t* bytes);
 int gdla_prefill_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int B,
                      int T, void* y, void* kv_cache_out, int cache_cap, void* workspace,
                      size_t ws_bytes, void* stream);
+
+/* Prefill with x and y in host memory (no counterpart in the pages: an I/O convenience).
+ * Same result as copying x to the device, gdla_prefill_fwd, and copying y back, but the copies
+ * overlap the work: x goes up in n_pieces row pieces on a copy stream, each piece's
+ * down-projection starting as soon as it has landed, and each piece of y goes back on a second
+ * copy stream as soon as its output projection is done (the attention in between needs every
+ * row).  The copies run asynchronously only if x_host and y_host are page-locked.
+ *   x_host [B, T, d_model] bf16, y_host [B, T, d_model] bf16 (host; y written).
+ *   n_pieces: 1 .. 64.
+ *   workspace: >= gdla_workspace_size(cfg, B, T, GDLA_MODE_HOST) bytes (device): the prefill
+ *     workspace plus device copies of x and y.
+ * The two copy streams and their events belong to the library (one set per device, created on
+ * the first call and kept); everything the call enqueues is ordered before the completion of
+ * `stream`, and nothing starts before work already enqueued on `stream`.  Calls enqueued one
+ * after another are ordered; host threads that call it for the same device at the same time
+ * must serialise their calls (they share the copy streams' events). */
+int gdla_prefill_host_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x_host,
+                          int B, int T, void* y_host, int n_pieces, void* workspace,
+                          size_t ws_bytes, void* stream);
 
 /* Prefill of packed documents.  The long-context workload of the report packs many documents
  * into one sequence (paperglide.net summary, Figure 4a); here each document is an independent
