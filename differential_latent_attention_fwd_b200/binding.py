@@ -82,6 +82,9 @@ def lib() -> ctypes.CDLL:
             "gdla_latent_fwd": [cfgp, wp, P, I, I, P, P, SZ, P],
             "gdla_prefill_context_fwd": [cfgp, wp, P, I, I, P, I, P, P, P, SZ, P],
             "gdla_prefill_host_fwd": [cfgp, wp, P, I, I, P, I, P, SZ, P],
+            "gdla_attn_train_workspace_size": [cfgp, I, I, ctypes.POINTER(SZ), ctypes.POINTER(SZ)],
+            "gdla_attn_train_fwd": [cfgp, P, P, P, P, P, I, I, P, P, P, P, SZ, P],
+            "gdla_attn_bwd": [cfgp, P, P, P, P, P, P, P, P, I, I, P, P, P, P, P, P, SZ, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -199,6 +202,35 @@ def gdla_prefill_host_fwd(cfg, w: gdla_weights_t, x_host: torch.Tensor, y_host: 
     _check("gdla_prefill_host_fwd", lib().gdla_prefill_host_fwd(
         ctypes.byref(cfg), ctypes.byref(w), _host_ptr(x_host, torch.bfloat16, "x_host"), B, T,
         _host_ptr(y_host, torch.bfloat16, "y_host"), n_pieces, _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gdla_attn_train_workspace_size(cfg, B: int, T: int) -> tuple:
+    f, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check("gdla_attn_train_workspace_size",
+           lib().gdla_attn_train_workspace_size(ctypes.byref(cfg), B, T, ctypes.byref(f), ctypes.byref(b)))
+    return f.value, b.value
+
+
+def gdla_attn_train_fwd(cfg, qq, kv, kr16, lam, gate, B: int, T: int, dg_out, h_out, lse_out,
+                        workspace, stream=None) -> None:
+    _check("gdla_attn_train_fwd", lib().gdla_attn_train_fwd(
+        ctypes.byref(cfg), _ptr(qq, torch.float16, "qq"), _ptr(kv, torch.float16, "kv"),
+        _ptr(kr16, torch.float16, "kr16"), _ptr(lam, torch.float32, "lam"), _ptr(gate, torch.bfloat16, "gate"),
+        B, T, _ptr(dg_out, torch.bfloat16, "dg_out"), _ptr(h_out, torch.bfloat16, "h_out"),
+        _ptr(lse_out, torch.float32, "lse_out"), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gdla_attn_bwd(cfg, qq, kv, kr16, lam, gate, h, lse, d_dg, B: int, T: int, d_qq, d_kv, d_kr,
+                  d_lam, d_gate, workspace, stream=None) -> None:
+    _check("gdla_attn_bwd", lib().gdla_attn_bwd(
+        ctypes.byref(cfg), _ptr(qq, torch.float16, "qq"), _ptr(kv, torch.float16, "kv"),
+        _ptr(kr16, torch.float16, "kr16"), _ptr(lam, torch.float32, "lam"), _ptr(gate, torch.bfloat16, "gate"),
+        _ptr(h, torch.bfloat16, "h"), _ptr(lse, torch.float32, "lse"), _ptr(d_dg, torch.bfloat16, "d_dg"),
+        B, T, _ptr(d_qq, torch.float32, "d_qq"), _ptr(d_kv, torch.float32, "d_kv"),
+        _ptr(d_kr, torch.float32, "d_kr"), _ptr(d_lam, torch.float32, "d_lam"),
+        _ptr(d_gate, torch.float32, "d_gate"), _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

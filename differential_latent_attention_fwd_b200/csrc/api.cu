@@ -621,6 +621,74 @@ int gdla_prefill_host_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, con
                       static_cast<cudaStream_t>(stream), nullptr, nullptr, false, &hp);
 }
 
+// ---------------------------------------------------------------- attention stage for training
+int gdla_attn_train_workspace_size(const gdla_config_t* cfg, int B, int T, size_t* fwd_bytes,
+                                   size_t* bwd_bytes) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!fwd_bytes || !bwd_bytes || B <= 0 || T <= 0) return GDLA_ERR_INVALID_ARG;
+  const long long M = (long long)B * T;
+  *fwd_bytes = (size_t)((M + 31) / 32 * 32) * cfg->n_noise * cfg->d_v * 4;
+  *bwd_bytes = attn_bwd_workspace_bytes(M, T, cfg->n_signal + cfg->n_noise, cfg->n_noise);
+  return GDLA_OK;
+}
+
+int gdla_attn_train_fwd(const gdla_config_t* cfg, const void* qq, const void* kv, const void* kr16,
+                        const float* lam, const void* gate, int B, int T, void* dg_out, void* h_out,
+                        float* lse_out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!qq || !kv || !kr16 || !lam || !gate || !dg_out || !h_out || !lse_out || !workspace || B <= 0 || T <= 0)
+    return GDLA_ERR_INVALID_ARG;
+  for (const void* ptr : {qq, kv, kr16, (const void*)lam, gate, (const void*)dg_out, (const void*)h_out,
+                          (const void*)lse_out, (const void*)workspace})
+    if (!aligned16(ptr)) return GDLA_ERR_INVALID_ARG;
+  if ((long long)B * T > (1ll << 30)) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  size_t fb, bb;
+  gdla_attn_train_workspace_size(cfg, B, T, &fb, &bb);
+  if (ws_bytes < fb) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  int* err;
+  if ((rc = error_word(&err))) return rc;
+  KernelCtlHost ctl{err, g_wait_limit_ns};
+  const int nH = cfg->n_signal + cfg->n_noise;
+  AttnParams ap{};
+  ap.B = B; ap.T = T; ap.T_kv = T; ap.q_off = 0; ap.window = cfg->window; ap.n_groups = cfg->n_noise;
+  ap.n_signal = cfg->n_signal; ap.rope_col0 = nH * cfg->d_nope;
+  ap.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
+  ap.lam = lam; ap.G = gate; ap.O_noise = static_cast<float*>(workspace); ap.Dg = dg_out;
+  ap.H_out = h_out; ap.lse_out = lse_out;
+  if (launch_failed(launch_attn_prefill(qq, nH * (cfg->d_nope + cfg->d_rope), kv, kr16, ap, ctl,
+                                        static_cast<cudaStream_t>(stream))))
+    return GDLA_ERR_LAUNCH;
+  return GDLA_OK;
+}
+
+int gdla_attn_bwd(const gdla_config_t* cfg, const void* qq, const void* kv, const void* kr16,
+                  const float* lam, const void* gate, const void* h, const float* lse, const void* d_dg,
+                  int B, int T, float* d_qq, float* d_kv, float* d_kr, float* d_lam, float* d_gate,
+                  void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  for (const void* ptr : {qq, kv, kr16, (const void*)lam, gate, h, (const void*)lse, d_dg, (const void*)d_qq,
+                          (const void*)d_kv, (const void*)d_kr, (const void*)d_lam, (const void*)d_gate,
+                          (const void*)workspace})
+    if (!ptr || !aligned16(ptr)) return GDLA_ERR_INVALID_ARG;
+  if (B <= 0 || T <= 0) return GDLA_ERR_INVALID_ARG;
+  if ((long long)B * T > (1ll << 30)) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  size_t fb, bb;
+  gdla_attn_train_workspace_size(cfg, B, T, &fb, &bb);
+  if (ws_bytes < bb) return GDLA_ERR_WORKSPACE_TOO_SMALL;
+  AttnBwdParams a{};
+  a.B = B; a.T = T; a.window = cfg->window; a.n_signal = cfg->n_signal; a.n_groups = cfg->n_noise;
+  a.scale = float(1.0 / sqrt(double(cfg->d_nope + cfg->d_rope)));
+  a.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
+  a.QQ = qq; a.KV = kv; a.kR16 = kr16; a.lam = lam; a.G = gate; a.H = h; a.lse = lse; a.d_dg = d_dg;
+  a.d_qq = d_qq; a.d_kv = d_kv; a.d_kr = d_kr; a.d_lam = d_lam; a.d_G = d_gate; a.ws = workspace;
+  rc = launch_attn_bwd(a, static_cast<cudaStream_t>(stream));
+  if (rc == 0) return GDLA_OK;
+  return rc == -6 ? GDLA_ERR_CUDA : GDLA_ERR_LAUNCH;
+}
+
 int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void* dst,
                         size_t dst_bytes, gdla_absorbed_t* out, void* stream) {
   int rc = check_config(cfg);

@@ -128,6 +128,10 @@ __device__ __forceinline__ uint8_t* attn_align(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// SAVE: also write every head's normalised output and log-sum-exp (for the backward).
+// PREFIX: keys and queries are different row ranges (a key prefix before the queries); without
+// it the key rows are the query rows and the offsets fold away at compile time.
+template <bool SAVE, bool PREFIX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap mapQ,
                         const __grid_constant__ CUtensorMap mapK,
@@ -168,10 +172,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     const int b = (pu % per_c) / p.n_groups;
     j = pu % p.n_groups;
     rowbase = b * p.T;
-    kvbase = b * p.T_kv;
     T = p.T;
-    T_kv = p.T_kv;
-    q_off = p.q_off;
+    kvbase = PREFIX ? b * p.T_kv : rowbase;
+    T_kv = PREFIX ? p.T_kv : T;
+    q_off = PREFIX ? p.q_off : 0;
   }
   const int q0 = 512 * c;
   const int t_hi = min(T_kv - 1, q_off + q0 + 511) / 128;
@@ -518,6 +522,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       if (!row_valid || m_row >= (long long)p.B * p.T || *reinterpret_cast<volatile int*>(ctl.err) != 0)
         continue;
+      if (SAVE) {
+        // for the backward: this head's normalised output and log2-sum-exp2 of its scores
+        const int head = pass == 0 ? p.n_signal + j : 4 * j + pass - 1;
+        const long long hrow = m_row * (p.n_signal + p.n_groups) + head;
+        uint4* hd = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.H_out) + hrow * 128);
+#pragma unroll
+        for (int e = 0; e < 128; e += 8)
+          hd[e / 8] = make_uint4(
+              pack_bf162(__uint_as_float(ou[e]) * inv_l, __uint_as_float(ou[e + 1]) * inv_l),
+              pack_bf162(__uint_as_float(ou[e + 2]) * inv_l, __uint_as_float(ou[e + 3]) * inv_l),
+              pack_bf162(__uint_as_float(ou[e + 4]) * inv_l, __uint_as_float(ou[e + 5]) * inv_l),
+              pack_bf162(__uint_as_float(ou[e + 6]) * inv_l, __uint_as_float(ou[e + 7]) * inv_l));
+        p.lse_out[hrow] = m_run + __log2f(l_run);
+      }
       // column quad e/4 of row m: ((m/32 * n_groups + j) * 32 + e/4) * 128 + (m%32) * 4
       float* on_q = p.O_noise + ((m_row >> 5) * p.n_groups + j) * 4096 + (m_row & 31) * 4;
       if (pass == 0) {
@@ -590,14 +608,17 @@ int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* k
       make_tmap_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, KV, kv_ld, Mk, kv_ld * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return -3;
-  if (cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           attn::SMEM) != cudaSuccess)
+  const bool prefix = p.q_off != 0 || p.T_kv != p.T;
+  if (p.H_out && (!p.lse_out || prefix)) return -2;
+  auto kern = p.H_out ? attn_prefill_kernel<true, false>
+                      : (prefix ? attn_prefill_kernel<false, true> : attn_prefill_kernel<false, false>);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn::SMEM) != cudaSuccess)
     return -4;
   const long long units = p.units ? (long long)p.max_units : (long long)((p.T + 511) / 512) * p.B;
   const long long grid = 2 * units * p.n_groups;   // two CTAs (one cluster) per unit
   if (grid > 0x7fffffffLL) return -2;
   KernelCtl kc{ctl.err, ctl.limit_ns};
-  attn_prefill_kernel<<<unsigned(grid), 384, attn::SMEM, st>>>(mq, mk, mkr, mv, p, kc);
+  kern<<<unsigned(grid), 384, attn::SMEM, st>>>(mq, mk, mkr, mv, p, kc);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 

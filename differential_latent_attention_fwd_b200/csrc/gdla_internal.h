@@ -111,6 +111,10 @@ struct AttnParams {
   const int4* units;
   const int* n_units;
   int max_units;              // grid bound (units beyond *n_units exit at once)
+  // Saved for the backward (null = not written): every head's normalised output H (bf16
+  // [B*T, n_heads, d_v]) and log-sum-exp of its scaled scores in log2 units ([B*T, n_heads]).
+  void* H_out;
+  float* lse_out;
 };
 
 // Device schedule of packed documents: per-token positions and the attention work units,
@@ -118,6 +122,29 @@ struct AttnParams {
 int launch_varlen_schedule(const int* cu_seqlens, int n_docs, int total, int* positions,
                            int4* units, int* n_units, int max_units, int* cnt, int* fill, int max_c,
                            int* err, cudaStream_t st);
+// Backward of the attention stage (attn_backward.cu): query rows per block.
+constexpr int ATTN_BWD_BQ = 256;
+struct AttnBwdParams {
+  int B, T, window, n_signal, n_groups;
+  float scale_log2, scale;    // log2(e) / sqrt(d_qk), 1 / sqrt(d_qk)
+  const void* QQ;             // fp16 [B*T, n_heads * 192]: q^C of all heads, then rotated q^R
+  const void* KV;             // fp16 [B*T, n_groups * 256]: K^C | V per KV head
+  const void* kR16;           // fp16 [B*T, 64]: rotated k^R
+  const float* lam;           // [B*T, n_signal]
+  const void* G;              // bf16 [B*T, n_signal * 128]: gate logits
+  const void* H;              // bf16 [B*T, n_heads, 128]: saved per-head outputs
+  const float* lse;           // [B*T, n_heads]: saved log2-sum-exp2 of the scaled scores
+  const void* d_dg;           // bf16 [B*T, n_signal * 128]: gradient of Dg
+  float* d_qq;                // [B*T, n_heads * 192]
+  float* d_kv;                // [B*T, n_groups * 256]
+  float* d_kr;                // [B*T, 64]
+  float* d_lam;               // [B*T, n_signal]
+  float* d_G;                 // [B*T, n_signal * 128]
+  void* ws;                   // attn_bwd_workspace_bytes(...)
+};
+size_t attn_bwd_workspace_bytes(long long M, int T, int n_heads, int n_groups);
+int launch_attn_bwd(const AttnBwdParams& a, cudaStream_t st);
+
 // Rotated k^R of bf16 latent rows (columns kv_rank .. kv_rank + 63) -> fp16 rows of 64.
 int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void* kR16, cudaStream_t st);
 int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* kR16,

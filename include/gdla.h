@@ -179,6 +179,38 @@ int gdla_prefill_context_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, 
                              void* y, void* latent_out, void* workspace, size_t ws_bytes,
                              void* stream);
 
+/* Training: the attention stage forward with saved tensors, and its backward (the projections
+ * around it are plain GEMMs).  The report trains 256K-token contexts with full activation
+ * recomputation (paperglide.net summary, the question on the memory demands of 256K-token
+ * contexts); these two calls are the attention stage of such a step.  Layouts are those of the prefill's intermediates:
+ *   qq   fp16 [B*T, n_heads * 192]: q^C of every head (n_heads * 128), then rotated q^R (n_heads * 64)
+ *   kv   fp16 [B*T, n_kv_heads * 256]: K^C (128) | V (128) of every KV head
+ *   kr16 fp16 [B*T, 64]: rotated k^R;  lam fp32 [B*T, n_signal] (after the sigmoid);
+ *   gate bf16 [B*T, n_signal * 128]: gate logits G (before the sigmoid).
+ * Workspace sizes of both calls (device bytes). */
+int gdla_attn_train_workspace_size(const gdla_config_t* cfg, int B, int T, size_t* fwd_bytes,
+                                   size_t* bwd_bytes);
+
+/* Attention stage forward (the prefill's fused kernel) that also saves, for the backward,
+ *   h_out bf16 [B*T, n_heads, 128]: every head's normalised output H (signal heads first), and
+ *   lse_out fp32 [B*T, n_heads]: log2 of the sum over visible keys of 2^(score log2(e)/sqrt(192)).
+ *   dg_out bf16 [B*T, n_signal * 128]: the stage output Dg = sigmoid(G) (.) (H_S - lambda H_N). */
+int gdla_attn_train_fwd(const gdla_config_t* cfg, const void* qq, const void* kv, const void* kr16,
+                        const float* lam, const void* gate, int B, int T, void* dg_out, void* h_out,
+                        float* lse_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of the attention stage: from d_dg = dL/dDg (bf16 [B*T, n_signal * 128]) and the
+ * tensors saved by gdla_attn_train_fwd, the fp32 gradients dL/d of qq (d_qq, same layout),
+ * kv (d_kv), kr16 (d_kr), lam (d_lam, with respect to lambda itself) and gate (d_gate, with
+ * respect to the logits).  The softmax probabilities are recomputed from the scores and the
+ * saved log-sum-exp; the contractions are strided-batched cuBLAS GEMMs (fp16 operands, fp32
+ * accumulation) over blocks of 256 query rows; the library's cuBLAS handle is created once per
+ * device and uses only the caller's workspace as its GEMM workspace. */
+int gdla_attn_bwd(const gdla_config_t* cfg, const void* qq, const void* kv, const void* kr16,
+                  const float* lam, const void* gate, const void* h, const float* lse,
+                  const void* d_dg, int B, int T, float* d_qq, float* d_kv, float* d_kr,
+                  float* d_lam, float* d_gate, void* workspace, size_t ws_bytes, void* stream);
+
 /* One-time weight preparation for the absorbed-form decode (MLA-style weight absorption:
  * attention runs in the latent space and K/V are never materialised; the pages note that
  * MLA rebuilds the keys/values only inside the attention computation).

@@ -394,6 +394,74 @@ def gdla_prefill_after_prefix(x_local, prefix_latent, pos_offset: int, weights: 
     return y
 
 
+def attention_stage(qC, qR, KC, V, kR, lam, G, cfg: OracleConfig):
+    """The attention stage of one sequence on its projected inputs (section 2.2 of the picx.dev
+    page: attention per head, D = H_S - lambda Repeat_g(H_N), sigmoid(G) gate).
+
+    qC [T, n_H, d_nope], qR [T, n_H, d_rope] (rotated), KC [T, n_KV, d_nope], V [T, n_KV, d_v],
+    kR [T, d_rope] (rotated), lam [T, n_S] (already sigmoided), G [T, n_S, d_v] (logits).
+    Returns (Dg [T, n_S, d_v], H [T, n_H, d_v]).
+    """
+    T = qC.shape[0]
+    H = np.empty((T, cfg.n_heads, cfg.d_v))
+    for t in range(T):
+        lo, hi = key_range(t, cfg.window)
+        H[t] = attend_row(qC[t], qR[t], KC, kR, V, lo, hi, cfg)
+    nmap = noise_of_signal(cfg)
+    Dg = np.empty((T, cfg.n_signal, cfg.d_v))
+    for t in range(T):
+        _, Dg[t] = differential_combine(H[t, : cfg.n_signal], H[t, cfg.n_signal:], lam[t], G[t], nmap)
+    return Dg, H
+
+
+def attention_stage_backward(qC, qR, KC, V, kR, lam, G, dDg, cfg: OracleConfig):
+    """Gradient of sum(dDg * Dg) with respect to every input of attention_stage.
+
+    Written out from the definition by the chain rule: with g = sigmoid(G), D = H_S - lambda H_N,
+      dG = dDg g (1 - g) D,  dH_S = dDg g,  dlambda_s = -sum_c dH_S[c] H_N(s)[c],
+      dH_N(n) = -sum_{s -> n} lambda_s dH_S,
+    and for each head's softmax attention H = P V, P = softmax(s), s = scale q.k:
+      dV += P^T dH,  dP = dH V^T,  ds = P (dP - sum_k P dP) = P (dP - dH.H),
+      dq = scale ds K,  dK += scale ds^T q  (K = [K^C ; k^R], q = [q^C ; q^R]).
+    Returns a dict of dqC, dqR, dKC, dV, dkR, dlam, dG (same shapes as the inputs).
+    """
+    T = qC.shape[0]
+    scale = 1.0 / np.sqrt(cfg.d_nope + cfg.d_rope)
+    _, H = attention_stage(qC, qR, KC, V, kR, lam, G, cfg)
+    nmap = noise_of_signal(cfg)
+    kvh = kv_head_of(cfg)
+    g = sigmoid(G)
+    HS, HN = H[:, : cfg.n_signal], H[:, cfg.n_signal:]
+    D = HS - lam[..., None] * HN[:, nmap]
+    out = {k: np.zeros_like(v) for k, v in dict(dqC=qC, dqR=qR, dKC=KC, dV=V, dkR=kR).items()}
+    out["dG"] = dDg * g * (1.0 - g) * D
+    dHS = dDg * g
+    out["dlam"] = -np.einsum("tsc,tsc->ts", dHS, HN[:, nmap])
+    dH = np.zeros_like(H)
+    dH[:, : cfg.n_signal] = dHS
+    for s_ in range(cfg.n_signal):
+        dH[:, cfg.n_signal + nmap[s_]] -= lam[:, s_, None] * dHS[:, s_]
+    for t in range(T):
+        lo, hi = key_range(t, cfg.window)
+        for h in range(cfg.n_heads):
+            j = kvh[h]
+            k = np.concatenate([KC[lo: hi + 1, j], kR[lo: hi + 1]], -1)
+            q = np.concatenate([qC[t, h], qR[t, h]])
+            sc = (k @ q) * scale
+            p = np.exp(sc - sc.max())
+            p /= p.sum()
+            dP = V[lo: hi + 1, j] @ dH[t, h]
+            ds = p * (dP - dH[t, h] @ H[t, h])
+            out["dV"][lo: hi + 1, j] += np.outer(p, dH[t, h])
+            dq = scale * (ds @ k)
+            out["dqC"][t, h] += dq[: cfg.d_nope]
+            out["dqR"][t, h] += dq[cfg.d_nope:]
+            dk = scale * np.outer(ds, q)
+            out["dKC"][lo: hi + 1, j] += dk[:, : cfg.d_nope]
+            out["dkR"][lo: hi + 1] += dk[:, cfg.d_nope:]
+    return out
+
+
 def gdla_prefill_packed(x_packed, cu_seqlens, weights: dict, cfg: OracleConfig, g_q=None, g_kv=None):
     """Packed documents: document d = rows cu[d] .. cu[d+1]-1 of x_packed [total, d_model] is an
     independent sequence (its own positions from 0, attention inside the document only).

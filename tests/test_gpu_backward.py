@@ -1,0 +1,82 @@
+"""Attention-stage backward on the GPU (saving forward + gdla_attn_bwd through the C ABI)
+against the fp64 oracle's gradient, on seeded inputs of the stage itself (q, K, V, k^R,
+lambda, gate logits and dL/dDg drawn directly)."""
+import numpy as np
+import pytest
+import torch
+
+from differential_latent_attention_fwd_b200 import binding as gb
+from differential_latent_attention_fwd_b200 import synth
+from oracle import gdla_oracle as O
+from tests.gpu_helpers import check, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _stage_inputs(B, T, seed):
+    g = torch.Generator().manual_seed(seed)
+    nH, nS, nK = 80, 64, 16
+    qq = torch.randn((B * T, nH * 192), generator=g).half()
+    kv = torch.randn((B * T, nK * 256), generator=g).half()
+    kr = torch.randn((B * T, 64), generator=g).half()
+    lam = torch.rand((B * T, nS), generator=g) * 0.9 + 0.05
+    gate = torch.randn((B * T, nS * 128), generator=g).bfloat16()
+    d_dg = torch.randn((B * T, nS * 128), generator=g).bfloat16()
+    return qq, kv, kr, lam, gate, d_dg
+
+
+def _run_gpu(shape, B, T, qq, kv, kr, lam, gate, d_dg):
+    cfg = gb.make_config(shape)
+    dev = "cuda"
+    t = [v.to(dev) for v in (qq, kv, kr, lam, gate, d_dg)]
+    fwd_b, bwd_b = gb.gdla_attn_train_workspace_size(cfg, B, T)
+    M = B * T
+    dg = torch.empty((M, 64 * 128), dtype=torch.bfloat16, device=dev)
+    h = torch.empty((M, 80, 128), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((M, 80), dtype=torch.float32, device=dev)
+    gb.gdla_attn_train_fwd(cfg, t[0], t[1], t[2], t[3], t[4], B, T, dg, h, lse,
+                           torch.empty(fwd_b, dtype=torch.uint8, device=dev))
+    outs = [torch.empty((M, 80 * 192), device=dev), torch.empty((M, 16 * 256), device=dev),
+            torch.empty((M, 64), device=dev), torch.empty((M, 64), device=dev),
+            torch.empty((M, 64 * 128), device=dev)]
+    gb.gdla_attn_bwd(cfg, t[0], t[1], t[2], t[3], t[4], h, lse, t[5], B, T, *outs,
+                     torch.empty(bwd_b, dtype=torch.uint8, device=dev))
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
+    return dg, h, outs
+
+
+@pytest.mark.parametrize("B,T,window", [(1, 300, 0), (2, 260, 64)])
+def test_attention_backward_matches_oracle(cuda_ok, B, T, window):
+    shape = synth.GdlaShape(window=window)
+    cfg = O.OracleConfig.from_shape(shape)
+    qq, kv, kr, lam, gate, d_dg = _stage_inputs(B, T, seed=41 + T)
+    dg, h, (d_qq, d_kv, d_kr, d_lam, d_gate) = _run_gpu(shape, B, T, qq, kv, kr, lam, gate, d_dg)
+    errs = []
+    for b in range(B):
+        r = slice(b * T, (b + 1) * T)
+        qC = O.f64(qq[r, : 80 * 128]).reshape(T, 80, 128)
+        qR = O.f64(qq[r, 80 * 128:]).reshape(T, 80, 64)
+        kvb = O.f64(kv[r]).reshape(T, 16, 256)
+        KC, V = kvb[..., :128], kvb[..., 128:]
+        kR = O.f64(kr[r])
+        lam_b = O.f64(lam[r])
+        G = O.f64(gate[r]).reshape(T, 64, 128)
+        dDg = O.f64(d_dg[r]).reshape(T, 64, 128)
+        Dg_o, H_o = O.attention_stage(qC, qR, KC, V, kR, lam_b, G, cfg)
+        check(f"b={b} forward Dg", to_np(dg[r]).reshape(T, 64, 128), Dg_o, errors=errs)
+        check(f"b={b} saved H", to_np(h[r]), H_o, rel=6e-3, mabs=5e-2, errors=errs)
+        gr = O.attention_stage_backward(qC, qR, KC, V, kR, lam_b, G, dDg, cfg)
+        dqq = to_np(d_qq[r])
+        dkv = to_np(d_kv[r]).reshape(T, 16, 256)
+        for name, got, want in [
+            ("dq^C", dqq[:, : 80 * 128].reshape(T, 80, 128), gr["dqC"]),
+            ("dq^R", dqq[:, 80 * 128:].reshape(T, 80, 64), gr["dqR"]),
+            ("dK^C", dkv[..., :128], gr["dKC"]),
+            ("dV", dkv[..., 128:], gr["dV"]),
+            ("dk^R", to_np(d_kr[r]), gr["dkR"]),
+            ("dlambda", to_np(d_lam[r]), gr["dlam"]),
+            ("dG", to_np(d_gate[r]).reshape(T, 64, 128), gr["dG"]),
+        ]:
+            check(f"b={b} {name}", got, want, rel=1e-2, mabs=np.abs(want).max() * 2e-2 + 1e-3, errors=errs)
+    assert not errs, "\n".join(errs)
