@@ -15,6 +15,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -384,6 +385,51 @@ def run_gpu(args):
               "last_rank_receives_bytes": (P - 1) * Tr * s.latent_row * 2,
               "timing": "one GPU, each rank's two calls back to back (L2 flushed); no communication"}
 
+    # ---- training: the attention stage's saving forward and its backward on the projected
+    # inputs the prefill left in its workspace (dL/dDg synthetic, seeded)
+    bwd = None
+    if not (args.skip_prefill or args.skip_bwd) and world == 1 and B == 1:
+        def slot(which, dtype, shape):
+            o = gb.gdla_workspace_offset(layer.cfg, B, T, gb.GDLA_MODE_PREFILL, which)
+            n = int(math.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+            return ws[o: o + n].view(dtype).view(*shape)
+        M = B * T
+        nH = s.n_signal + s.n_noise
+        qq = slot(4, torch.float16, (M, nH * 192)); kvs = slot(6, torch.float16, (M, s.n_kv_heads * 256))
+        kr = slot(9, torch.float16, (M, 64)); lam_t = slot(3, torch.float32, (M, s.n_signal))
+        gate = slot(5, torch.bfloat16, (M, s.n_signal * 128))
+        fb, bb = gb.gdla_attn_train_workspace_size(layer.cfg, B, T)
+        wsf = torch.empty(fb, dtype=torch.uint8, device=dev)
+        wsb = torch.empty(bb, dtype=torch.uint8, device=dev)
+        dg_t = torch.empty((M, s.n_signal * 128), dtype=torch.bfloat16, device=dev)
+        h_t = torch.empty((M, nH, 128), dtype=torch.bfloat16, device=dev)
+        lse_t = torch.empty((M, nH), dtype=torch.float32, device=dev)
+        ddg = torch.randn((M, s.n_signal * 128), generator=torch.Generator(device=dev).manual_seed(9),
+                          device=dev).bfloat16()
+        grads = [torch.empty((M, nH * 192), device=dev), torch.empty((M, s.n_kv_heads * 256), device=dev),
+                 torch.empty((M, 64), device=dev), torch.empty((M, s.n_signal), device=dev),
+                 torch.empty((M, s.n_signal * 128), device=dev)]
+        e2 = torch.cuda.Event(enable_timing=True)
+        tf_ms, tb_ms = [], []
+        for i in range(3):
+            e0.record(stream)
+            gb.gdla_attn_train_fwd(layer.cfg, qq, kvs, kr, lam_t, gate, B, T, dg_t, h_t, lse_t, wsf, stream=stream)
+            e1.record(stream)
+            gb.gdla_attn_bwd(layer.cfg, qq, kvs, kr, lam_t, gate, h_t, lse_t, ddg, B, T, *grads, wsb, stream=stream)
+            e2.record(stream)
+            torch.cuda.synchronize(dev)
+            if i:
+                tf_ms.append(e0.elapsed_time(e1))
+                tb_ms.append(e1.elapsed_time(e2))
+        bwd_flop = B * valid_pairs(T, 0) * nH * 2 * (192 + 128 + 192 + 192 + 128)
+        bwd = {"seq_len": T, "train_fwd_ms": statistics.median(tf_ms), "bwd_ms": statistics.median(tb_ms),
+               "bwd_flop": bwd_flop, "bwd_tflops": bwd_flop / (statistics.median(tb_ms) * 1e-3) / 1e12,
+               "bwd_frac_of_bf16_peak": bwd_flop / (statistics.median(tb_ms) * 1e-3) / 1e12
+               / load_peaks()[0]["bf16_tflops_sustained"],
+               "method": "per 256-query block: strided-batched cuBLAS GEMMs (fp16, fp32 accumulate) for S, dP, "
+                         "dq, dK, dV; own kernels for P, dS, dH/Delta/dlambda/dG"}
+        del wsb, grads, h_t
+
     peaks, peak_src = load_peaks()
     pairs = valid_pairs(T, 0)
     attn_flop = B * pairs * attn_flops_per_pair(s)
@@ -444,6 +490,7 @@ def run_gpu(args):
                     "layer_frac_of_bf16_peak": value / world / peaks["bf16_tflops_sustained"]},
         "decode": decode,
         "context_parallel": cp,
+        "backward": bwd,
         "roofline": {"kernel": "attn_prefill_kernel", "bound": "tensor", "achieved": attn_tf,
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": attn_tf / peaks["bf16_tflops_sustained"],
@@ -492,6 +539,7 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true", help="profiling runs: no host-buffer pass")
     ap.add_argument("--decode-L", type=int, default=DECODE["L"], help="cached positions (profiling runs)")
     ap.add_argument("--skip-cp", action="store_true", help="profiling runs: no context-parallel split")
+    ap.add_argument("--skip-bwd", action="store_true", help="profiling runs: no backward pass")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
