@@ -426,8 +426,9 @@ def run_gpu(args):
                "bwd_flop": bwd_flop, "bwd_tflops": bwd_flop / (statistics.median(tb_ms) * 1e-3) / 1e12,
                "bwd_frac_of_bf16_peak": bwd_flop / (statistics.median(tb_ms) * 1e-3) / 1e12
                / load_peaks()[0]["bf16_tflops_sustained"],
-               "method": "per 256-query block: strided-batched cuBLAS GEMMs (fp16, fp32 accumulate) for S, dP, "
-                         "dq, dK, dV; own kernels for P, dS, dH/Delta/dlambda/dG"}
+               "method": "per 512-query block: strided-batched cuBLAS GEMMs (fp16, fp32 accumulate) for S, dP, "
+                         "dq, dK, dV on gathered 192-wide q and k rows; own kernels for P and dS' (one pass), "
+                         "dH/Delta/dlambda/dG, gathers and scatters"}
         del wsb, grads, h_t
 
     peaks, peak_src = load_peaks()

@@ -123,7 +123,7 @@ int launch_varlen_schedule(const int* cu_seqlens, int n_docs, int total, int* po
                            int4* units, int* n_units, int max_units, int* cnt, int* fill, int max_c,
                            int* err, cudaStream_t st);
 // Backward of the attention stage (attn_backward.cu): query rows per block.
-constexpr int ATTN_BWD_BQ = 256;
+constexpr int ATTN_BWD_BQ = 512;
 struct AttnBwdParams {
   int B, T, window, n_signal, n_groups;
   float scale_log2, scale;    // log2(e) / sqrt(d_qk), 1 / sqrt(d_qk)

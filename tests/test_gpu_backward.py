@@ -46,7 +46,9 @@ def _run_gpu(shape, B, T, qq, kv, kr, lam, gate, d_dg):
     return dg, h, outs
 
 
-@pytest.mark.parametrize("B,T,window", [(1, 300, 0), (2, 260, 64)])
+# T > 512 spans several 512-row query blocks (the window case with a key range that starts
+# after row 0 in the later blocks)
+@pytest.mark.parametrize("B,T,window", [(1, 300, 0), (2, 260, 64), (1, 700, 0), (1, 600, 100)])
 def test_attention_backward_matches_oracle(cuda_ok, B, T, window):
     shape = synth.GdlaShape(window=window)
     cfg = O.OracleConfig.from_shape(shape)
