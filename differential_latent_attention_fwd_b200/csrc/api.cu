@@ -117,7 +117,7 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
     sz[WS_SPLITK] = 0;
   } else {
     const int ns = decode_split_count(B, T, c->window);   // T = cache capacity in decode mode
-    sz[WS_LATENT] = M * (long long)c->n_signal * c->kv_rank * 4;     // latent differentials
+    sz[WS_LATENT] = 0;
     sz[WS_QQ] = M * qq * 4;                                          // fp32 q^C | q^R
     sz[WS_KV] = M * (long long)nH * (c->kv_rank + c->d_rope) * 2;    // q~ rows
     sz[WS_ONOISE] = M * (long long)ns * nH * c->kv_rank * 4;         // split partials
@@ -811,7 +811,6 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   DecCombParams cp{};
   cp.B = B; cp.n_groups = cfg->n_noise; cp.n_signal = cfg->n_signal; cp.n_split = nsplit;
   cp.part = part; cp.ml = ml; cp.lam = lam; cp.G = G; cp.W_bKV = w->W_bKV; cp.Dg = Dg;
-  cp.Dlat = reinterpret_cast<float*>(ws + off[WS_LATENT]);
   if (launch_failed(launch_dec_combine(cp, st))) return GDLA_ERR_LAUNCH;
 
   stage(3, st);

@@ -12,7 +12,7 @@
 // so every cached byte (c_bar | k^R, 1152 bytes per position) is read once for all 80 heads.
 //
 // Kernels here: W_UK transpose (weight absorption), q~ formation, and the split merge +
-// latent differential combine + W_UV up-projection + gate.  The split-K latent attention
+// latent differential combine + W_UV up-projection + gate (one kernel).  The split-K latent attention
 // itself is the tensor-core kernel in decode_tc.cu.
 #include "gdla_common.cuh"
 #include "gdla_internal.h"
@@ -41,47 +41,60 @@ int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int 
 }
 
 // q~ rows: qt[b][h][0..511] = W_UK_j q^C_h, qt[b][h][512..575] = rotated q^R_h (bf16).
-// CTA (KV head j, 4 rows b): W_UK_j^T (128 x 512 bf16, 128 KB) is staged in shared memory with
-// asynchronous copies, then 20 query rows (4 rows x the group's 5 heads) are projected.
+// CTA (KV head j, QT_RB rows b): W_UK_j^T (128 x 512 bf16, 128 KB) is staged in shared memory
+// with asynchronous copies, then the 5 QT_RB query rows of the group's heads are projected in
+// fp32.  Thread: latent columns 4 cq .. 4 cq + 3 of half of those rows.
+constexpr int QT_RB = 8;
 __global__ void __launch_bounds__(256) qtilde_kernel(DecQParams p) {
+  constexpr int NR = 5 * QT_RB;                // query rows of a CTA
+  constexpr int HR = NR / 2;                   // rows per thread
   extern __shared__ uint8_t qt_smem[];
-  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(qt_smem);            // [128][512]
-  float (*qc)[128] = reinterpret_cast<float (*)[128]>(qt_smem + 128 * 512 * 2);  // [20][128]
-  const int j = blockIdx.x, b0 = blockIdx.y * 4, tid = threadIdx.x;
-  const int nb = min(4, p.B - b0);
+  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(qt_smem);              // [128][512]
+  float (*qc)[128] = reinterpret_cast<float (*)[128]>(qt_smem + 128 * 512 * 2);  // [NR][128]
+  const int j = blockIdx.x, b0 = blockIdx.y * QT_RB, tid = threadIdx.x;
+  const int nb = min(QT_RB, p.B - b0);
   const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_UKt) + (long long)j * 128 * 512;
   for (int i = tid; i < 128 * 512 / 8; i += blockDim.x) cp_async16(wsm + i * 8, W + i * 8);
   const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
-  for (int i = tid; i < 20 * 128; i += blockDim.x) {
+  for (int i = tid; i < NR * 128; i += blockDim.x) {
     const int r = i / 128, c = i % 128, bb = r / 5, hh = r % 5;
     qc[r][c] = bb < nb ? p.QQ[(long long)(b0 + bb) * p.qq_ld + heads[hh] * 128 + c] : 0.f;
   }
   cp_async_wait_all();
   __syncthreads();
-  // thread: latent columns 2 tid, 2 tid + 1 of all 20 rows
-  float acc[20][2];
+  const int cq = tid & 127, r0 = (tid >> 7) * HR;
+  float acc[HR][4];
 #pragma unroll
-  for (int r = 0; r < 20; ++r) acc[r][0] = acc[r][1] = 0.f;
-#pragma unroll 2
-  for (int c = 0; c < 128; ++c) {
-    const __nv_bfloat162 w2 = *reinterpret_cast<const __nv_bfloat162*>(wsm + c * 512 + 2 * tid);
-    const float w0 = __low2float(w2), w1 = __high2float(w2);
+  for (int r = 0; r < HR; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < 128; c += 4) {
+    float w[4][4];
 #pragma unroll
-    for (int r = 0; r < 20; ++r) {
-      const float q = qc[r][c];
-      acc[r][0] = fmaf(q, w0, acc[r][0]);
-      acc[r][1] = fmaf(q, w1, acc[r][1]);
+    for (int k = 0; k < 4; ++k) {
+      const uint2 wv = *reinterpret_cast<const uint2*>(wsm + (c + k) * 512 + 4 * cq);
+      const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.x));
+      const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.y));
+      w[k][0] = w01.x; w[k][1] = w01.y; w[k][2] = w23.x; w[k][3] = w23.y;
+    }
+#pragma unroll
+    for (int r = 0; r < HR; ++r) {
+      const float4 q4 = *reinterpret_cast<const float4*>(&qc[r0 + r][c]);
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(qv[k], w[k][e], acc[r][e]);
     }
   }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.qt);
 #pragma unroll
-  for (int r = 0; r < 20; ++r) {
-    const int bb = r / 5, hh = r % 5;
+  for (int r = 0; r < HR; ++r) {
+    const int bb = (r0 + r) / 5, hh = (r0 + r) % 5;
     if (bb >= nb) continue;
-    *reinterpret_cast<uint32_t*>(out + ((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 2 * tid) =
-        pack_bf162(acc[r][0], acc[r][1]);
+    *reinterpret_cast<uint2*>(out + ((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 4 * cq) =
+        make_uint2(pack_bf162(acc[r][0], acc[r][1]), pack_bf162(acc[r][2], acc[r][3]));
   }
-  for (int i = tid; i < 4 * 5 * 64; i += blockDim.x) {
+  for (int i = tid; i < NR * 64; i += blockDim.x) {
     const int r = i / 64, e = i % 64, bb = r / 5, hh = r % 5;
     if (bb >= nb) continue;
     out[((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 512 + e] =
@@ -90,121 +103,158 @@ __global__ void __launch_bounds__(256) qtilde_kernel(DecQParams p) {
 }
 
 int launch_qtilde(const DecQParams& p, cudaStream_t st) {
-  const int smem = 128 * 512 * 2 + 20 * 128 * 4;
+  const int smem = 128 * 512 * 2 + 5 * QT_RB * 128 * 4;
   if (cudaFuncSetAttribute(qtilde_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return -4;
-  qtilde_kernel<<<dim3(p.n_groups, (p.B + 3) / 4), 256, smem, st>>>(p);
+  qtilde_kernel<<<dim3(p.n_groups, (p.B + QT_RB - 1) / QT_RB), 256, smem, st>>>(p);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
 // ---------------------------------------------------------------- split merge + combine + gate
-// Kernel 1, CTA (b, j): merges the splits of the group's 5 heads (rescaling each split's
-// partial by 2^(m_split - m)), normalises, and forms the latent differential
-// l_s - lambda_s l_noise for the group's 4 signal heads -> Dlat[j][b * 4 + s][512] (fp32).
-__global__ void __launch_bounds__(256) dec_merge_kernel(DecCombParams p) {
-  const int b = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+// CTA (KV group j, CB query rows b): while W_UV_j (the V column block of W_b^KV for KV head j,
+// 512 x 128 bf16) streams into shared memory, the key-range splits of the group's 5 heads are
+// merged (each split's partial rescaled by 2^(m_split - m), then normalised) and the latent
+// differentials l_s - lambda_s l_noise of its 4 signal heads formed in shared memory (fp32);
+// then D = Dlat W_UV_j (4 CB rows x 128 columns, K = 512) and Dg = sigmoid(G) (.) D.
+constexpr int CB = 8;
+__global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
   constexpr int NH = 80;
-  __shared__ float wsp[64][5];
-  __shared__ float inv_L[5];
-  const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
-  if (tid < 5) {
-    const int h = heads[tid];
-    float M = -INFINITY;
-    for (int sp = 0; sp < p.n_split; ++sp)
-      M = fmaxf(M, p.ml[(((long long)b * p.n_split + sp) * NH + h) * 2]);
-    float Ls = 0.f;
-    for (int sp = 0; sp < p.n_split; ++sp) {
-      const float* ml = p.ml + (((long long)b * p.n_split + sp) * NH + h) * 2;
-      const float w = ml[1] > 0.f ? ex2_approx(ml[0] - M) : 0.f;
-      wsp[sp][tid] = w;
-      Ls += w * ml[1];
-    }
-    inv_L[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
-  }
-  __syncthreads();
-  for (int l = tid; l < 512; l += blockDim.x) {
-    float lat[5];
-#pragma unroll
-    for (int hh = 0; hh < 5; ++hh) {
-      float a = 0.f;
-      for (int sp = 0; sp < p.n_split; ++sp) {
-        const float w = wsp[sp][hh];
-        if (w != 0.f)  // empty splits write no partial
-          a += w * p.part[(((long long)b * p.n_split + sp) * NH + heads[hh]) * 512 + l];
-      }
-      lat[hh] = a * inv_L[hh];
-    }
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const float lam = p.lam[(long long)b * p.n_signal + 4 * j + s];
-      p.Dlat[((long long)j * p.B + b) * 4 * 512 + s * 512 + l] = lat[1 + s] - lam * lat[0];
-    }
-  }
-}
-
-// Kernel 2, CTA (j, 4 sequences): D = Dlat W_UV_j (16 rows x 128 columns, K = 512), then
-// Dg = sigmoid(G) (.) D.  W_UV_j is the V column block of W_b^KV for KV head j; it is staged
-// in shared memory (128 KB, coalesced 16-byte loads) before the product.
-__global__ void __launch_bounds__(256) dec_uv_gate_kernel(DecCombParams p) {
-  extern __shared__ uint8_t uv_smem[];
-  float (*dl)[512] = reinterpret_cast<float (*)[512]>(uv_smem);                      // [16][512]
-  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(uv_smem + 16 * 512 * 4);     // [512][128]
-  const int j = blockIdx.x, b0 = blockIdx.y * 4, tid = threadIdx.x;
-  const int nrows = min(4, p.B - b0) * 4;
+  extern __shared__ uint8_t cb_smem[];
+  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(cb_smem);                  // [512][128]
+  float (*dl)[512] = reinterpret_cast<float (*)[512]>(cb_smem + 512 * 128 * 2);     // [4 CB][512]
+  float (*wsp)[64] = reinterpret_cast<float (*)[64]>(cb_smem + 512 * 128 * 2 + 4 * CB * 512 * 4);  // [5 CB][64]
+  float* inv_L = reinterpret_cast<float*>(cb_smem + 512 * 128 * 2 + 4 * CB * 512 * 4 + 5 * CB * 64 * 4);
+  const int j = blockIdx.x, b0 = blockIdx.y * CB, tid = threadIdx.x;
+  const int nb = min(CB, p.B - b0);
   const long long ldw = (long long)p.n_groups * 256;
   const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_bKV) + j * 256 + 128;
   for (int i = tid; i < 512 * 16; i += blockDim.x) {          // 16 x 16 bytes per 128-column row
     const int l = i >> 4, q = i & 15;
     cp_async16(wsm + l * 128 + q * 8, W + l * ldw + q * 8);
   }
-  const float* src = p.Dlat + ((long long)j * p.B + b0) * 4 * 512;
-  for (int i = tid; i < 16 * 512; i += blockDim.x)
-    dl[i / 512][i % 512] = (i / 512) < nrows ? src[i] : 0.f;
+  const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
+  if (tid < 5 * CB) {
+    const int bb = tid / 5, h = heads[tid % 5];
+    float Ls = 0.f;
+    if (bb < nb) {
+      const int b = b0 + bb;
+      float M = -INFINITY;
+      for (int sp = 0; sp < p.n_split; ++sp) M = fmaxf(M, p.ml[(((long long)b * p.n_split + sp) * NH + h) * 2]);
+      for (int sp = 0; sp < p.n_split; ++sp) {
+        const float* ml = p.ml + (((long long)b * p.n_split + sp) * NH + h) * 2;
+        const float w = ml[1] > 0.f ? ex2_approx(ml[0] - M) : 0.f;
+        wsp[tid][sp] = w;
+        Ls += w * ml[1];
+      }
+    } else {
+      for (int sp = 0; sp < p.n_split; ++sp) wsp[tid][sp] = 0.f;
+    }
+    inv_L[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
+  }
+  __syncthreads();
+  {
+    // thread: latent columns 4 cq .. 4 cq + 3 of rows rb .. rb + CB / 2 - 1; splits outermost so
+    // that a split's 5 CB / 2 float4 loads are independent (a partial an empty split never
+    // wrote is dropped by a select, never multiplied)
+    constexpr int RB = CB / 2;
+    const int cq = tid & 127, rb = (tid >> 7) * RB;
+    float4 m4[RB][5];
+#pragma unroll
+    for (int k = 0; k < RB; ++k)
+#pragma unroll
+      for (int hh = 0; hh < 5; ++hh) m4[k][hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < p.n_split; ++sp) {
+      float4 v4[RB][5];
+#pragma unroll
+      for (int k = 0; k < RB; ++k) {
+        const int bb = rb + k;
+        const float* src = p.part + ((long long)(b0 + (bb < nb ? bb : 0)) * p.n_split + sp) * NH * 512 + 4 * cq;
+#pragma unroll
+        for (int hh = 0; hh < 5; ++hh)
+          v4[k][hh] = bb < nb ? *reinterpret_cast<const float4*>(src + (long long)heads[hh] * 512)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < RB; ++k)
+#pragma unroll
+        for (int hh = 0; hh < 5; ++hh) {
+          const float w = wsp[5 * (rb + k) + hh][sp];
+          if (w != 0.f) {
+            m4[k][hh].x = fmaf(w, v4[k][hh].x, m4[k][hh].x);
+            m4[k][hh].y = fmaf(w, v4[k][hh].y, m4[k][hh].y);
+            m4[k][hh].z = fmaf(w, v4[k][hh].z, m4[k][hh].z);
+            m4[k][hh].w = fmaf(w, v4[k][hh].w, m4[k][hh].w);
+          }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+      const int bb = rb + k;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (bb < nb) {
+          const float lam = p.lam[(long long)(b0 + bb) * p.n_signal + 4 * j + s];
+          const float iS = inv_L[5 * bb + 1 + s], iN = inv_L[5 * bb];
+          o.x = m4[k][1 + s].x * iS - lam * (m4[k][0].x * iN);
+          o.y = m4[k][1 + s].y * iS - lam * (m4[k][0].y * iN);
+          o.z = m4[k][1 + s].z * iS - lam * (m4[k][0].z * iN);
+          o.w = m4[k][1 + s].w * iS - lam * (m4[k][0].w * iN);
+        }
+        *reinterpret_cast<float4*>(&dl[4 * bb + s][4 * cq]) = o;
+      }
+    }
+  }
   cp_async_wait_all();
   __syncthreads();
   const int cq = tid & 31;          // columns 4 cq .. 4 cq + 3
-  const int rp = tid >> 5;          // rows 2 rp, 2 rp + 1
-  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 8
-  for (int l = 0; l < 512; ++l) {
-    const uint2 wv = *reinterpret_cast<const uint2*>(wsm + l * 128 + 4 * cq);
-    const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wv.x);
-    const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wv.y);
-    const float w[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
-    const float d0 = dl[2 * rp][l], d1 = dl[2 * rp + 1][l];
+  const int r0 = (tid >> 5) * 4;    // rows r0 .. r0 + 3 of the 4 CB latent differentials
+  float acc[4][4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      acc[0][e] = fmaf(d0, w[e], acc[0][e]);
-      acc[1][e] = fmaf(d1, w[e], acc[1][e]);
+  for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+#pragma unroll 1
+  for (int l = 0; l < 512; l += 4) {
+    float w[4][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint2 wv = *reinterpret_cast<const uint2*>(wsm + (l + k) * 128 + 4 * cq);
+      const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.x));
+      const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.y));
+      w[k][0] = w01.x; w[k][1] = w01.y; w[k][2] = w23.x; w[k][3] = w23.y;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 d4 = *reinterpret_cast<const float4*>(&dl[r0 + r][l]);
+      const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(dv[k], w[k][e], acc[r][e]);
     }
   }
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int row = 2 * rp + rr;
-    if (row >= nrows) continue;
+  for (int r = 0; r < 4; ++r) {
+    const int row = r0 + r;
+    if (row >= 4 * nb) continue;
     const int b = b0 + row / 4, s = row % 4, sig = 4 * j + s;
     const long long o = (long long)b * p.n_signal * 128 + sig * 128 + 4 * cq;
     const uint2 gv = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.G) + o);
     const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&gv.x);
     const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&gv.y);
     uint2 out;
-    out.x = pack_bf162(sigmoidf_fast(__low2float(g01)) * acc[rr][0], sigmoidf_fast(__high2float(g01)) * acc[rr][1]);
-    out.y = pack_bf162(sigmoidf_fast(__low2float(g23)) * acc[rr][2], sigmoidf_fast(__high2float(g23)) * acc[rr][3]);
+    out.x = pack_bf162(sigmoidf_fast(__low2float(g01)) * acc[r][0], sigmoidf_fast(__high2float(g01)) * acc[r][1]);
+    out.y = pack_bf162(sigmoidf_fast(__low2float(g23)) * acc[r][2], sigmoidf_fast(__high2float(g23)) * acc[r][3]);
     *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.Dg) + o) = out;
   }
 }
 
 int launch_dec_combine(const DecCombParams& p, cudaStream_t st) {
-  dec_merge_kernel<<<dim3(p.B, p.n_groups), 256, 0, st>>>(p);
-  if (cudaPeekAtLastError() != cudaSuccess) return -4;
-  const int uv_smem = 16 * 512 * 4 + 512 * 128 * 2;
-  if (cudaFuncSetAttribute(dec_uv_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, uv_smem) !=
-      cudaSuccess)
+  if (p.n_split > 64) return -1;
+  const int smem = 512 * 128 * 2 + 4 * CB * 512 * 4 + 5 * CB * 64 * 4 + 5 * CB * 4;
+  if (cudaFuncSetAttribute(dec_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return -4;
-  dec_uv_gate_kernel<<<dim3(p.n_groups, (p.B + 3) / 4), 256, uv_smem, st>>>(p);
-  if (cudaPeekAtLastError() != cudaSuccess) return -4;
-  count_extra_launch();
-  return 0;
+  dec_combine_kernel<<<dim3(p.n_groups, (p.B + CB - 1) / CB), 256, smem, st>>>(p);
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
 }  // namespace gdla

@@ -34,7 +34,6 @@ struct DecCombParams {
   const float* lam;       // [B][n_signal]
   const void* G;          // bf16 [B][n_signal * 128]
   const void* W_bKV;      // bf16 [kv_rank][n_groups * 256]
-  float* Dlat;            // [n_groups][B][4][512] latent differentials (scratch)
   void* Dg;               // bf16 [B][n_signal * 128]
 };
 

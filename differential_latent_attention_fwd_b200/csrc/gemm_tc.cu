@@ -464,14 +464,14 @@ static int run_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, 
 
 static int gemm_bn(int N) { return N >= 256 ? 256 : (N > 64 ? 128 : 64); }
 
-// Skinny products (one 128-row M tile) leave most SMs idle; split K so that about one wave of
-// CTAs streams the weights, each split keeping at least 4 K blocks of 64.
+// Skinny products (one 128-row M tile) leave most SMs idle; split K so that the CTAs streaming
+// the weights fill at most one wave, each split keeping at least 4 K blocks of 64.
 int gemm_splitk_count(int M, int N, int K) {
   if (M > 128 || N % 64 != 0 || K % 64 != 0) return 1;
   const int BN = gemm_bn(N);
   const int tiles = (N + BN - 1) / BN;
   const int nk = K / 64;
-  int s = (148 + tiles - 1) / tiles;
+  int s = g_num_sms() / tiles;
   s = s > nk / 4 ? nk / 4 : s;
   if (s <= 1) return 1;
   const int kps = (nk + s - 1) / s;
