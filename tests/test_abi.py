@@ -108,3 +108,33 @@ def test_context_entry_points_validate_on_the_host(L):
     assert rc == -1
     rc = L.gdla_latent_fwd(ctypes.byref(cfg), ctypes.byref(w), fake, 16, 0, None, fake, big, None)
     assert rc == -1
+
+
+def test_training_entry_points_validate_on_the_host(L):
+    cfg = gb.make_config(GdlaShape())
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1002)
+    f, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert L.gdla_attn_train_workspace_size(ctypes.byref(cfg), 0, 16, ctypes.byref(f), ctypes.byref(b)) == -1
+    assert L.gdla_attn_train_workspace_size(ctypes.byref(cfg), 1, 16, None, ctypes.byref(b)) == -1
+    sizes = []
+    for T in (16, 600, 1200):
+        assert L.gdla_attn_train_workspace_size(ctypes.byref(cfg), 1, T, ctypes.byref(f), ctypes.byref(b)) == 0
+        assert f.value > 0 and b.value > 0
+        sizes.append(b.value)
+    assert sizes[0] < sizes[1] < sizes[2]   # the backward's score buffers grow with T
+    big = 1 << 40
+    fwd = lambda *a: L.gdla_attn_train_fwd(ctypes.byref(cfg), *a)
+    # qq, kv, kr16, lam, gate, B, T, dg_out, h_out, lse_out, ws, ws_bytes, stream
+    assert fwd(None, fake, fake, fake, fake, 1, 16, fake, fake, fake, fake, big, None) == -1
+    assert fwd(fake, fake, odd, fake, fake, 1, 16, fake, fake, fake, fake, big, None) == -1
+    assert fwd(fake, fake, fake, fake, fake, 1, 0, fake, fake, fake, fake, big, None) == -1
+    assert fwd(fake, fake, fake, fake, fake, 1, 16, fake, fake, fake, fake, 16, None) == -3
+    bwd = lambda *a: L.gdla_attn_bwd(ctypes.byref(cfg), *a)
+    # qq, kv, kr16, lam, gate, h, lse, d_dg, B, T, d_qq, d_kv, d_kr, d_lam, d_gate, ws, ws_bytes, stream
+    ok8 = [fake] * 8
+    outs = [fake] * 5
+    assert bwd(*([None] + ok8[1:]), 1, 16, *outs, fake, big, None) == -1
+    assert bwd(*ok8, 1, 16, *(outs[:4] + [odd]), fake, big, None) == -1
+    assert bwd(*ok8, -1, 16, *outs, fake, big, None) == -1
+    assert bwd(*ok8, 1, 16, *outs, fake, 16, None) == -3
