@@ -35,6 +35,11 @@ Readings where the pages are silent (each also listed in the design notes):
 
 Parity: every function here is pinned by tests/test_oracle_pins.py (worked example, closed
 forms, library routines, invariants, brute force) except where a docstring says otherwise.
+Parity unpinned by the pages: the constants taken where the pages are silent (the softmax
+scale 1/sqrt(192), the rotate-half RoPE pairing with theta 10000, the RMSNorm eps) are
+readings, not printed values; the pins fix the forms these steps take (a rotation, a norm, a
+softmax), and the kernels share the constants by construction, not by a check against the
+pages.
 """
 from __future__ import annotations
 
