@@ -117,7 +117,7 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
     sz[WS_SPLITK] = 0;
   } else {
     const int ns = decode_split_count(B, T, c->window);   // T = cache capacity in decode mode
-    sz[WS_LATENT] = 0;
+    sz[WS_LATENT] = 0;                                               // unused by decode
     sz[WS_QQ] = M * qq * 4;                                          // fp32 q^C | q^R
     sz[WS_KV] = M * (long long)nH * (c->kv_rank + c->d_rope) * 2;    // q~ rows
     sz[WS_ONOISE] = M * (long long)ns * nH * c->kv_rank * 4;         // split partials
