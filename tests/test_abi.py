@@ -138,3 +138,25 @@ def test_training_entry_points_validate_on_the_host(L):
     assert bwd(*ok8, 1, 16, *(outs[:4] + [odd]), fake, big, None) == -1
     assert bwd(*ok8, -1, 16, *outs, fake, big, None) == -1
     assert bwd(*ok8, 1, 16, *outs, fake, 16, None) == -3
+
+
+def test_binding_rejects_wrong_tensors_before_the_library():
+    """Argument marshalling refuses host tensors where device memory is expected (and the
+    reverse), wrong dtypes and non-contiguous views; nothing reaches the C ABI."""
+    import pytest
+    import torch
+    cfg = gb.make_config(GdlaShape())
+    dev_like = torch.zeros(16, dtype=torch.float16)          # a host tensor: refused as device memory
+    with pytest.raises(ValueError):
+        gb.gdla_attn_train_fwd(cfg, dev_like, dev_like, dev_like, torch.zeros(4), torch.zeros(4).bfloat16(),
+                               1, 16, None, None, None, torch.zeros(16, dtype=torch.uint8))
+    with pytest.raises(TypeError):
+        gb.gdla_attn_train_fwd(cfg, torch.zeros(16), dev_like, dev_like, torch.zeros(4),
+                               torch.zeros(4).bfloat16(), 1, 16, None, None, None, torch.zeros(16, dtype=torch.uint8))
+    with pytest.raises(TypeError):
+        gb._ptr([1, 2, 3], None, "x")
+    with pytest.raises(ValueError):
+        gb._host_ptr(torch.zeros(8, 8).t(), torch.float32, "x")   # non-contiguous
+    with pytest.raises(TypeError):
+        gb._host_ptr(torch.zeros(8), torch.bfloat16, "x")
+    assert gb._host_ptr(torch.zeros(8, dtype=torch.bfloat16), torch.bfloat16, "x").value is not None
