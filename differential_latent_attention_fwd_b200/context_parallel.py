@@ -54,14 +54,17 @@ def exchange_prefix(latent: torch.Tensor, lengths: list, rank: int, window: int,
     need = min(window - 1, start)
     halo = window - 1
     if all(t >= halo for t in lengths[:-1]):
-        # every shard but the last can serve the next one alone: one point-to-point halo
+        # every shard but the last can serve the next one alone: one point-to-point halo.
+        # P2POp takes the peer as a global rank, so the group's neighbours are mapped.
+        def peer(r):
+            return r if group is None else dist.get_global_rank(group, r)
         ops = []
         recv = None
         if rank + 1 < world and halo > 0:
-            ops.append(dist.P2POp(dist.isend, latent[latent.shape[0] - halo:].contiguous(), rank + 1, group))
+            ops.append(dist.P2POp(dist.isend, latent[latent.shape[0] - halo:].contiguous(), peer(rank + 1), group))
         if rank > 0 and halo > 0:
             recv = torch.empty((halo, latent.shape[1]), dtype=latent.dtype, device=latent.device)
-            ops.append(dist.P2POp(dist.irecv, recv, rank - 1, group))
+            ops.append(dist.P2POp(dist.irecv, recv, peer(rank - 1), group))
         if ops:
             for req in dist.batch_isend_irecv(ops):
                 req.wait()

@@ -80,3 +80,48 @@ def test_cp_prefill_matches_whole_sequence(window, lengths):
     y = O.gdla_prefill(inp.x, inp.weights, O.OracleConfig.from_shape(shape))[0]
     full = np.concatenate([got[r] for r in range(world)], 0)
     np.testing.assert_allclose(full, y, rtol=0, atol=1e-10)
+
+
+def _worker_subgroup(rank, world, port, window, lengths, seed, q):
+    """Ranks 1..world-1 of a world_size `world` job form the context-parallel group; rank 0 is
+    outside it (it only takes part in creating the group)."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        grp = dist.new_group(list(range(1, world)))
+        if rank == 0:
+            q.put((rank, None))
+            return
+        shape = synth.GdlaShape(window=window, **SMALL)
+        inp = synth.make_prefill_inputs(shape, 1, sum(lengths), seed)
+        gr = rank - 1
+        start = sum(lengths[:gr])
+        x = inp.x[0, start: start + lengths[gr]]
+        y = cp_prefill(OracleLayer(shape, inp.weights), x, group=grp)
+        q.put((rank, y.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("window,lengths", [(6, [9, 8, 12]), (0, [7, 13, 10])])
+def test_cp_prefill_on_a_subgroup(window, lengths):
+    """The sequence is split over ranks 1..3 of 4: the halo's point-to-point peers are the
+    group's neighbours, addressed by their global ranks."""
+    world = len(lengths) + 1
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_subgroup, args=(r, world, port, window, lengths, 3, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=240) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    shape = synth.GdlaShape(window=window, **SMALL)
+    inp = synth.make_prefill_inputs(shape, 1, sum(lengths), 3)
+    y = O.gdla_prefill(inp.x, inp.weights, O.OracleConfig.from_shape(shape))[0]
+    full = np.concatenate([got[r] for r in range(1, world)], 0)
+    np.testing.assert_allclose(full, y, rtol=0, atol=1e-10)
