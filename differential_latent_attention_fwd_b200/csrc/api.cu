@@ -66,7 +66,7 @@ static int check_weights(const gdla_weights_t* w) {
 
 // ---------------------------------------------------------------- workspace layout
 enum { WS_D1, WS_CQ, WS_LATENT, WS_LAM, WS_QQ, WS_G, WS_KV, WS_ONOISE, WS_DG, WS_KR16, WS_SPLITK,
-       WS_VL_POS, WS_VL_UNITS, WS_VL_COUNT, WS_N };
+       WS_VL_POS, WS_VL_UNITS, WS_VL_COUNT, WS_DSCHED, WS_N };
 
 // Packed documents: bounds of the attention schedule for `total` tokens in `n_docs` documents
 // (sum over documents of ceil(len / R) <= ceil(total / R) + n_docs, R = ATTN_UNIT_ROWS).  The
@@ -102,7 +102,7 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
   sz[WS_LAM] = M * c->n_signal * 4;
   sz[WS_G] = M * (long long)c->n_signal * c->d_v * 2;
   sz[WS_DG] = M * (long long)c->n_signal * c->d_v * 2;
-  sz[WS_VL_POS] = sz[WS_VL_UNITS] = sz[WS_VL_COUNT] = 0;
+  sz[WS_VL_POS] = sz[WS_VL_UNITS] = sz[WS_VL_COUNT] = sz[WS_DSCHED] = 0;
   if (mode == GDLA_MODE_VARLEN) {
     sz[WS_VL_POS] = M * 4;
     sz[WS_VL_UNITS] = (size_t)varlen_max_units(M, M) * 16;
@@ -116,13 +116,15 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
     sz[WS_KR16] = M * c->d_rope * 2;
     sz[WS_SPLITK] = 0;
   } else {
-    const int ns = decode_split_count(B, T, c->window);   // T = cache capacity in decode mode
+    // the attention's segments: one partial slot per (CTA, row) pair that can meet
+    const long long slots = (long long)decode_cta_count() + M;
     sz[WS_LATENT] = 0;                                               // unused by decode
     sz[WS_QQ] = M * qq * 4;                                          // fp32 q^C | q^R
     sz[WS_KV] = M * (long long)nH * (c->kv_rank + c->d_rope) * 2;    // q~ rows
-    sz[WS_ONOISE] = M * (long long)ns * nH * c->kv_rank * 4;         // split partials
-    sz[WS_KR16] = M * (long long)ns * nH * 2 * 4;                    // split (max, sum)
+    sz[WS_ONOISE] = slots * nH * c->kv_rank * 4;                     // segment partials
+    sz[WS_KR16] = slots * nH * 2 * 4;                                // segment (max, sum)
     sz[WS_SPLITK] = decode_splitk_floats(c, B) * 4;
+    sz[WS_DSCHED] = (M + 1) * 4;                                     // tile prefix over the rows
   }
   size_t o = 0;
   for (int i = 0; i < WS_N; ++i) {
@@ -350,7 +352,7 @@ static int prefill_impl(const gdla_config_t* cfg, const gdla_weights_t* w, const
       if (cudaMemcpyAsync(latent, ctx->prefix_latent, (size_t)n_pre * row_w * 2,
                           cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return GDLA_ERR_CUDA;
-      if (launch_failed(launch_latent_to_kr16(ctx->prefix_latent, cfg->kv_rank, n_pre, kR16, st)))
+      if (launch_failed(launch_latent_to_kr16(ctx->prefix_latent, cfg->kv_rank, n_pre, kR16, err, st)))
         return GDLA_ERR_LAUNCH;
     }
   }
@@ -436,6 +438,7 @@ const char* gdla_status_string(int s) {
     case GDLA_ERR_LAUNCH: return "kernel launch failed";
     case GDLA_ERR_DEVICE_TIMEOUT: return "bounded in-kernel wait expired";
     case GDLA_ERR_CUDA: return "CUDA runtime error";
+    case GDLA_ERR_DEVICE_DATA: return "a kernel met bad input data (see gdla_device_error)";
     default: return "unknown status";
   }
 }
@@ -750,7 +753,6 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   void* Dg = ws + off[WS_DG];
   const int nH = cfg->n_signal + cfg->n_noise;
   const int ld1 = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
-  const int nsplit = decode_split_count(B, cap, cfg->window);
   RopeTable rope;
   fill_rope_table(&rope, cfg->d_rope, cfg->rope_theta);
 
@@ -797,19 +799,24 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   qp.QQ = QQ; qp.qq_ld = nqq; qp.rope_col0 = nH * cfg->d_nope; qp.W_UKt = ab->W_UKt; qp.qt = qt;
   if (launch_failed(launch_qtilde(qp, st))) return GDLA_ERR_LAUNCH;
 
-  stage(1, st);
   DecAttnParams dp{};
-  dp.B = B; dp.cap = cap; dp.window = cfg->window; dp.n_split = nsplit; dp.cache_len = cache_len;
+  dp.R = B; dp.n_seq = n_seq; dp.cap = cap; dp.window = cfg->window; dp.cache_len = cache_len;
   dp.q_len = q_len;
   dp.cache = kv_cache; dp.qt = qt;
   dp.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
+  dp.tstart = reinterpret_cast<int*>(ws + off[WS_DSCHED]);
+  dp.n_ctas = decode_cta_count();
   dp.part = part; dp.ml = ml; dp.err = err;
   if (nH != 80) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  if (launch_failed(launch_dec_sched(dp, st))) return GDLA_ERR_LAUNCH;
+
+  stage(1, st);
   if (launch_failed(launch_dec_attn_tc(dp, ctl, st))) return GDLA_ERR_LAUNCH;
 
   stage(2, st);
   DecCombParams cp{};
-  cp.B = B; cp.n_groups = cfg->n_noise; cp.n_signal = cfg->n_signal; cp.n_split = nsplit;
+  cp.B = B; cp.n_groups = cfg->n_noise; cp.n_signal = cfg->n_signal; cp.n_ctas = dp.n_ctas;
+  cp.tstart = dp.tstart;
   cp.part = part; cp.ml = ml; cp.lam = lam; cp.G = G; cp.W_bKV = w->W_bKV; cp.Dg = Dg;
   if (launch_failed(launch_dec_combine(cp, st))) return GDLA_ERR_LAUNCH;
 
@@ -846,7 +853,9 @@ int gdla_device_error(void* stream, int* site, int clear) {
     if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return GDLA_ERR_CUDA;
   }
   *site = v;
-  return v ? GDLA_ERR_DEVICE_TIMEOUT : GDLA_OK;
+  if (!v) return GDLA_OK;
+  // 0x6xx / 0x7xx: a kernel met bad input data; the other sites are expired waits
+  return (v >= 0x600 && v < 0x800) ? GDLA_ERR_DEVICE_DATA : GDLA_ERR_DEVICE_TIMEOUT;
 }
 
 }  // extern "C"

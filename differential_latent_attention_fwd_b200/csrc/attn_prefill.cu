@@ -69,61 +69,11 @@ struct AttnBars {
 static_assert(sizeof(AttnBars) <= 256, "barrier block");
 
 
-// ---- softmax arithmetic.  Packed f32x2 instructions halve the issue slots of the scale,
-// subtract and sum steps; a quarter of the exponentials run on the FMA pipe instead of MUFU
-// (whose 16 results per clock per SM are the softmax's bottleneck).
-__device__ __forceinline__ float fmax3f(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-// (d0, d1) = (a0, a1) + (b0, b1)
-__device__ __forceinline__ void fadd2v(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 d, a, b;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-      "add.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-// (d0, d1) = (a0, a1) * (b0, b1) + (c, c)
-__device__ __forceinline__ void ffma2v(float& d0, float& d1, float a0, float a1, float b0, float b1, float c) {
-  asm("{\n\t.reg .b64 d, a, b, c;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %6};\n\t"
-      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
-      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c));
-}
-// (x0, x1) = (a0, a1) * b + c
-__device__ __forceinline__ void ffma2(float& x0, float& x1, float a0, float a1, float b, float c) {
-  ffma2v(x0, x1, a0, a1, b, b, c);
-}
-// (s0, s1) += (a0, a1)
-__device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) {
-  fadd2v(s0, s1, s0, s1, a0, a1);
-}
 // sigmoid(z) = 1 / (1 + 2^(-z log2 e)) with the approximate reciprocal-divide (2 ulp): the
 // result is rounded to bf16.
 __device__ __forceinline__ float sigmoid_approx(float z) {
   return __fdividef(1.0f, 1.0f + ex2_approx(-1.4426950408889634f * z));
 }
-// 2^x for a pair on the FMA pipe.  x = j + f with j = round(x) (adding and subtracting
-// 1.5 * 2^23 rounds to the nearest integer) and |f| <= 1/2; 2^f from a cubic fitted to 2^f
-// on [-1/2, 1/2] (iteratively reweighted least squares towards the minimax fit, max relative
-// error 7.5e-5, below the 2^-12 half-ulp of the fp16 P it feeds; exp2_poly_fit.py beside this
-// file reproduces the coefficients); j is added to the exponent field as an integer.  x is
-// clamped at -126, where the fp16 P is 0 either way.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& r0, float& r1) {
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  float t0, t1, j0, j1, f0, f1;
-  fadd2v(t0, t1, x0, x1, 12582912.f, 12582912.f);
-  fadd2v(j0, j1, t0, t1, -12582912.f, -12582912.f);
-  fadd2v(f0, f1, x0, x1, -j0, -j1);
-  float q0 = 0.05517144128680229f, q1 = 0.05517144128680229f;
-  ffma2v(q0, q1, q0, q1, f0, f1, 0.24261070787906647f);
-  ffma2v(q0, q1, q0, q1, f0, f1, 0.6932609677314758f);
-  ffma2v(q0, q1, q0, q1, f0, f1, 0.9999281167984009f);
-  // the low 9 bits of t's bit pattern hold j mod 512; * 2^23 moves them into the exponent field
-  r0 = __int_as_float(__float_as_int(t0) * 8388608 + __float_as_int(q0));
-  r1 = __int_as_float(__float_as_int(t1) * 8388608 + __float_as_int(q1));
-}
-
 __device__ __forceinline__ uint8_t* attn_align(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }

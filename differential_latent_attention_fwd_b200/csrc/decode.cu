@@ -11,9 +11,10 @@
 //   Dg_s   = sigmoid(G_s) (.) D_s
 // so every cached byte (c_bar | k^R, 1152 bytes per position) is read once for all 80 heads.
 //
-// Kernels here: W_UK transpose (weight absorption), q~ formation, and the split merge +
-// latent differential combine + W_UV up-projection + gate (one kernel).  The split-K latent attention
-// itself is the tensor-core kernel in decode_tc.cu.
+// Kernels here: W_UK transpose (weight absorption), q~ formation, and the segment merge +
+// latent differential combine + W_UV up-projection + gate (one kernel).  The latent attention
+// itself (one wave of CTAs over the key tiles of all rows) is the tensor-core kernel in
+// decode_tc.cu.
 #include "gdla_common.cuh"
 #include "gdla_internal.h"
 #include "gdla_decode.h"
@@ -110,20 +111,25 @@ int launch_qtilde(const DecQParams& p, cudaStream_t st) {
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
-// ---------------------------------------------------------------- split merge + combine + gate
+// ---------------------------------------------------------------- segment merge + combine + gate
 // CTA (KV group j, CB query rows b): while W_UV_j (the V column block of W_b^KV for KV head j,
-// 512 x 128 bf16) streams into shared memory, the key-range splits of the group's 5 heads are
-// merged (each split's partial rescaled by 2^(m_split - m), then normalised) and the latent
+// 512 x 128 bf16) streams into shared memory, the key-range segments of the group's 5 heads are
+// merged (each segment's partial rescaled by 2^(m_seg - m), then normalised) and the latent
 // differentials l_s - lambda_s l_noise of its 4 signal heads formed in shared memory (fp32);
 // then D = Dlat W_UV_j (4 CB rows x 128 columns, K = 512) and Dg = sigmoid(G) (.) D.
+// Row b's segments are the attention CTAs c_lo .. c_hi whose tile ranges meet the row's tiles
+// [tstart[b], tstart[b + 1]); CTA c wrote its piece to slot c + b.
 constexpr int CB = 8;
+constexpr int MAXSEG = DEC_MAX_CTAS;
 __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
   constexpr int NH = 80;
   extern __shared__ uint8_t cb_smem[];
   __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(cb_smem);                  // [512][128]
   float (*dl)[512] = reinterpret_cast<float (*)[512]>(cb_smem + 512 * 128 * 2);     // [4 CB][512]
-  float (*wsp)[64] = reinterpret_cast<float (*)[64]>(cb_smem + 512 * 128 * 2 + 4 * CB * 512 * 4);  // [5 CB][64]
-  float* inv_L = reinterpret_cast<float*>(cb_smem + 512 * 128 * 2 + 4 * CB * 512 * 4 + 5 * CB * 64 * 4);
+  float (*wsp)[MAXSEG] = reinterpret_cast<float (*)[MAXSEG]>(cb_smem + 512 * 128 * 2 + 4 * CB * 512 * 4);
+  float* inv_L = reinterpret_cast<float*>(cb_smem + 512 * 128 * 2 + 4 * CB * 512 * 4 + 5 * CB * MAXSEG * 4);
+  int* seg_lo = reinterpret_cast<int*>(inv_L + 5 * CB);
+  int* seg_n = seg_lo + CB;
   const int j = blockIdx.x, b0 = blockIdx.y * CB, tid = threadIdx.x;
   const int nb = min(CB, p.B - b0);
   const long long ldw = (long long)p.n_groups * 256;
@@ -132,53 +138,70 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
     const int l = i >> 4, q = i & 15;
     cp_async16(wsm + l * 128 + q * 8, W + l * ldw + q * 8);
   }
+  if (tid < CB) {
+    int lo = 0, n = 0;
+    if (tid < nb) {
+      const int b = b0 + tid;
+      const long long N = p.tstart[p.B], G = N < p.n_ctas ? N : p.n_ctas;
+      const long long t0 = p.tstart[b], t1 = p.tstart[b + 1];
+      if (t1 > t0) {
+        // CTA c < G = min(grid, N) covers tiles [c N / G, (c + 1) N / G) (never empty): tile t
+        // lies in CTA ((t + 1) G - 1) / N
+        const int c_lo = int(((t0 + 1) * G - 1) / N), c_hi = int((t1 * G - 1) / N);
+        lo = c_lo + b;
+        n = c_hi - c_lo + 1;
+      }
+    }
+    seg_lo[tid] = lo;
+    seg_n[tid] = n;
+  }
+  __syncthreads();
   const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
   if (tid < 5 * CB) {
     const int bb = tid / 5, h = heads[tid % 5];
-    float Ls = 0.f;
-    if (bb < nb) {
-      const int b = b0 + bb;
-      float M = -INFINITY;
-      for (int sp = 0; sp < p.n_split; ++sp) M = fmaxf(M, p.ml[(((long long)b * p.n_split + sp) * NH + h) * 2]);
-      for (int sp = 0; sp < p.n_split; ++sp) {
-        const float* ml = p.ml + (((long long)b * p.n_split + sp) * NH + h) * 2;
-        const float w = ml[1] > 0.f ? ex2_approx(ml[0] - M) : 0.f;
-        wsp[tid][sp] = w;
-        Ls += w * ml[1];
-      }
-    } else {
-      for (int sp = 0; sp < p.n_split; ++sp) wsp[tid][sp] = 0.f;
+    const int n = seg_n[bb], lo = seg_lo[bb];
+    float M = -INFINITY, Ls = 0.f;
+    for (int k = 0; k < n; ++k) M = fmaxf(M, p.ml[((long long)(lo + k) * NH + h) * 2]);
+    for (int k = 0; k < n; ++k) {
+      const float* ml = p.ml + ((long long)(lo + k) * NH + h) * 2;
+      const float w = ml[1] > 0.f ? ex2_approx(ml[0] - M) : 0.f;
+      wsp[tid][k] = w;
+      Ls += w * ml[1];
     }
     inv_L[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
   }
   __syncthreads();
   {
-    // thread: latent columns 4 cq .. 4 cq + 3 of rows rb .. rb + CB / 2 - 1; splits outermost so
-    // that a split's 5 CB / 2 float4 loads are independent (a partial an empty split never
-    // wrote is dropped by a select, never multiplied)
+    // thread: latent columns 4 cq .. 4 cq + 3 of rows rb .. rb + CB / 2 - 1; segments outermost
+    // so that a segment's 5 CB / 2 float4 loads are independent (rows with fewer segments load
+    // nothing for the rest)
     constexpr int RB = CB / 2;
     const int cq = tid & 127, rb = (tid >> 7) * RB;
+    int max_n = 0;
+#pragma unroll
+    for (int k = 0; k < RB; ++k) max_n = max(max_n, seg_n[rb + k]);
     float4 m4[RB][5];
 #pragma unroll
     for (int k = 0; k < RB; ++k)
 #pragma unroll
       for (int hh = 0; hh < 5; ++hh) m4[k][hh] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp = 0; sp < p.n_split; ++sp) {
+    for (int sg = 0; sg < max_n; ++sg) {
       float4 v4[RB][5];
 #pragma unroll
       for (int k = 0; k < RB; ++k) {
         const int bb = rb + k;
-        const float* src = p.part + ((long long)(b0 + (bb < nb ? bb : 0)) * p.n_split + sp) * NH * 512 + 4 * cq;
+        const bool has = sg < seg_n[bb];
+        const float* src = p.part + (long long)(has ? seg_lo[bb] + sg : 0) * NH * 512 + 4 * cq;
 #pragma unroll
         for (int hh = 0; hh < 5; ++hh)
-          v4[k][hh] = bb < nb ? *reinterpret_cast<const float4*>(src + (long long)heads[hh] * 512)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          v4[k][hh] = has ? *reinterpret_cast<const float4*>(src + (long long)heads[hh] * 512)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int k = 0; k < RB; ++k)
 #pragma unroll
         for (int hh = 0; hh < 5; ++hh) {
-          const float w = wsp[5 * (rb + k) + hh][sp];
+          const float w = sg < seg_n[rb + k] ? wsp[5 * (rb + k) + hh][sg] : 0.f;
           if (w != 0.f) {
             m4[k][hh].x = fmaf(w, v4[k][hh].x, m4[k][hh].x);
             m4[k][hh].y = fmaf(w, v4[k][hh].y, m4[k][hh].y);
@@ -249,8 +272,8 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
 }
 
 int launch_dec_combine(const DecCombParams& p, cudaStream_t st) {
-  if (p.n_split > 64) return -1;
-  const int smem = 512 * 128 * 2 + 4 * CB * 512 * 4 + 5 * CB * 64 * 4 + 5 * CB * 4;
+  if (p.n_ctas > MAXSEG) return -1;
+  const int smem = 512 * 128 * 2 + 4 * CB * 512 * 4 + 5 * CB * MAXSEG * 4 + 5 * CB * 4 + 2 * CB * 4;
   if (cudaFuncSetAttribute(dec_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return -4;
   dec_combine_kernel<<<dim3(p.n_groups, (p.B + CB - 1) / CB), 256, smem, st>>>(p);

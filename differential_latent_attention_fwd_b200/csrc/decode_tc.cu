@@ -1,111 +1,166 @@
-// Absorbed-form GDLA decode attention on the tensor cores (sm_100a).
+// Absorbed-form GDLA decode attention on the tensor cores (sm_100a), reading every cached byte
+// into the SM once.
 //
-// For one sequence b the 80 query heads all attend over the same latent-cache rows
-// c_p = [c_bar_p (512) | rotated k^R_p (64)] (the MLA weight absorption: q~_h = [W_UK q^C_h ; q^R_h],
-// score_{h,p} = q~_h . c_p / sqrt(192); picx.dev Motif 3 summary, section 2.2, with K and V
-// regrouped into the latent space).  A CTA owns one (sequence, split of the key range) and
-// computes, per 128-position tile and with positions on the 128 TMEM lanes ("swap AB"):
-//   S^T[p, h]   = C[p, :] . q~[h, :]            tcgen05.mma M 128 (positions), N 80, K 576
-//   P[p, h]     = 2^(S^T log2e/sqrt(192) - m_h)  (softmax numerators, bf16, in shared memory)
-//   O^T[l, h]  += C[:, l]^T P[:, h]              4 x tcgen05.mma M 128 (latent rows), N 80, K 128
-// and finally writes the split's partial (O^T, m_h, sum_p P) for the merge kernel.
+// For one query row r (one new token of one sequence) the 80 heads attend over the latent-cache
+// rows c_p = [c_bar_p (512) | rotated k^R_p (64)] (the MLA weight absorption: q~_h =
+// [W_UK q^C_h ; q^R_h], score_{h,p} = q~_h . c_p / sqrt(192); picx.dev Motif 3 summary, section
+// 2.2, with K and V regrouped into the latent space).  Per 64-position tile:
+//   S[h, p]    = q~[h, :] . C[p, :]        tcgen05.mma M 128 (heads, 80 used), N 64, K 576
+//   P[h, p]    = 2^(S log2e / sqrt(192) - m_h)   (bf16, one thread per head, into shared memory)
+//   O^T[l, h] += C[:, l]^T P[h, :]^T        4 x tcgen05.mma M 128 (latent rows), N 80, K 64
+// The tile stays in shared memory from the score MMAs to the PV MMAs, so nothing is re-read.
+// That needs room: q~ of 80 heads is 90 KB, so its first 256 latent dims live in TMEM as the
+// A operand of the score MMA (128 columns), and only dims 256..575 (50 KB) in shared memory.
+// TMEM: q~ part 128 columns | S 64 | O^T 4 x 80 = 512.  Shared memory: q~ part 50 KB, P 10 KB,
+// a ring of nine 16 KB latent slots (two [64 positions][64 dims] boxes each) and two 8 KB
+// rotary slots (a tile takes four latent slots and one rotary slot): about 2.2 tiles.
 //
-// Shared memory cannot hold q~ (80 x 576 bf16 = 90 KB) together with a whole 128-position tile
-// (144 KB), so the tile's latent columns are fetched twice: once with the rope columns for the
-// scores, and again for the PV product right after (an L2 hit).  The TMA ring has three 32 KB
-// slots, each holding a pair of 64-column boxes (the two halves of one 128-row M block of C^T).
-// The running maximum m_h moves only when a score exceeds it by more than 2^8 (then O^T and the
-// per-position partial sums are rescaled), which is exact after the final division.
+// Work split ("stream-K"): the key tiles of all rows form one list, rows in order; CTA c of
+// G = min(grid, N) takes tiles [c N / G, (c + 1) N / G), i.e. one wave with equal work per SM
+// whatever the cache lengths.  The piece of a row inside one CTA's range is a segment: it gets its own online
+// softmax and writes a partial (m_h, l_h, O^T) to slot c + r; the merge kernel in decode.cu
+// combines a row's segments.  The rows of one sequence's q_len new tokens are consecutive, so
+// CTAs c and c + N_r G / N read the same cache tiles at about the same time (one DRAM read).
 //
-// Roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5 softmax
-// (thread = position = TMEM lane; later thread = latent row for the O^T read-out).
+// Roles (192 threads): warps 0-3 softmax and O^T epilogue (warp w reads TMEM lanes 32 w ..
+// 32 w + 31: thread = head h = 32 w + lane for h < 80, thread = latent row for O^T), warp 4 TMA
+// producer, warp 5 TMEM owner + MMA issuer.  The tensor core runs S(J), PV(J - 1), S(J + 1),
+// PV(J), ...: the softmax of tile J (read S, maximum, exponentials, P) overlaps PV(J - 1) and
+// S(J + 1), so the tensor core does not wait for it.  The single S buffer is released as soon
+// as the softmax has read it into registers; the single P buffer is written once PV(J - 1) is
+// done; the ring holds tiles J - 1 and J plus one slot of J + 1.  The issuer steps through
+// precomputed descriptor words: at these shapes an MMA costs ~50-75 cycles, and rebuilding
+// 64-bit descriptors per MMA had made the issue loop, not the tensor core, the bound.  The
+// producer also prefetches the tile three ahead into L2, so that the ring only has to cover L2
+// latency.
+// The running maximum m_h moves only when a score exceeds it by more than 2^8 (O^T and l_h are
+// then rescaled), which is exact after the final division.  Rows of the last tile beyond the
+// row's last key are zeroed in shared memory before the PV, so that a cache tail the caller
+// never wrote (NaN, Inf) cannot reach the output through 0 * NaN.
 #include "gdla_common.cuh"
 #include "gdla_decode.h"
 #include "gdla_internal.h"
 
 namespace gdla {
 
-namespace dtc {
+namespace dsk {
 constexpr int NH = 80;
-constexpr int SLOT = 32768;
-constexpr int NSLOT = 3;
-constexpr int QBOX = NH * 128;                 // one [80 rows][64 bf16] box of q~
-constexpr int RING_OFF = 0;
-constexpr int QT_OFF = NSLOT * SLOT;           // 9 boxes of q~
-constexpr int P_OFF = QT_OFF + 9 * QBOX;       // P^T: [80 heads][128 positions] as 2 K-chunks
-constexpr int BAR_OFF = P_OFF + 2 * QBOX;
-constexpr int SMEM = BAR_OFF + 2048 + 1024;
-constexpr int S_COL0 = 0, S_COL1 = 96, O_COL = 192;   // TMEM columns
+constexpr int TP = 64;                          // positions per tile
+constexpr int QS_BOX = NH * 128;                // [80 rows][64 bf16] box of q~ (10 KB)
+constexpr int QS_OFF = 0;                       // q~ dims 256..575: 5 boxes
+constexpr int P_OFF = QS_OFF + 5 * QS_BOX;      // P [80 heads][64 positions] bf16
+constexpr int LAT_SLOT = 16384;                 // [64 pos][64 dims] x 2 (128 latent dims)
+constexpr int NLAT = 9;
+constexpr int ROPE_SLOT = 8192;                 // [64 pos][64 rope dims]
+constexpr int NROPE = 2;
+constexpr int LAT_OFF = P_OFF + NH * 128;
+constexpr int ROPE_OFF = LAT_OFF + NLAT * LAT_SLOT;
+constexpr int BAR_OFF = ROPE_OFF + NROPE * ROPE_SLOT;
+constexpr int SMEM = BAR_OFF + 1024 + 1024;    // barriers + alignment slack
+constexpr int QT_COL = 0, S_COL = 128, O_COL = 192;   // TMEM columns
 constexpr float RESCALE_THRESHOLD = 8.0f;
-}  // namespace dtc
+constexpr int PREFETCH_AHEAD = 3;               // tiles of L2 prefetch ahead of the TMA loads
+static_assert(SMEM <= 232448, "shared memory");
+// The M = 128 score MMA reads 128 rows of each 80-row q~ box: the 48 rows past a box are the
+// next box, or (for the last box) the first 6 KB of P.  They only feed unused score rows.
+static_assert(P_OFF + 48 * 128 <= LAT_OFF, "q~ box over-read stays in the P buffer");
+}  // namespace dsk
 
-struct DecBars {
-  float m_ref[dtc::NH];        // reference maxima (log2 units), 16-byte aligned for float4 reads
-  float red[4][dtc::NH];       // cross-warp reduction scratch
-  uint64_t q_full;
-  uint64_t ring_full[dtc::NSLOT], ring_empty[dtc::NSLOT];
-  uint64_t s_full[2], p_ready, pv_done, mma_final;
+struct SkBars {
+  float scale[dsk::NH];
+  uint64_t q_ready;                               // q~ (TMA part + TMEM part) of a segment
+  uint64_t lat_full[dsk::NLAT], lat_empty[dsk::NLAT];
+  uint64_t rope_full[dsk::NROPE], rope_empty[dsk::NROPE];
+  uint64_t s_full, s_free, p_ready, pv_done, seg_done, mma_final;
   uint32_t tmem_base;
 };
 
-__device__ __forceinline__ uint8_t* dtc_align(uint8_t* p) {
+__device__ __forceinline__ uint8_t* dsk_align(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Key tiles [t_begin, t_end) of this split and the sequence's valid key range [lo, hi].
-struct DecRange {
-  int lo, hi, t_begin, t_end;
-};
-__device__ __forceinline__ DecRange dec_range(const DecAttnParams& p, int b, int sp, int* err) {
-  DecRange r;
-  // row b is new token b % q_len of its sequence: it sees the cached keys and the new tokens
-  // up to itself, all held in the cache rows 0 .. cache_len + b % q_len
+// Key range of query row r: it is new token r % q_len of sequence r / q_len and sees the cache
+// rows 0 .. cache_len + r % q_len (the window keeps the last W of them).
+__device__ __forceinline__ void dsk_row_range(const DecAttnParams& p, int r, int* lo, int* hi) {
   const int ql = p.q_len > 1 ? p.q_len : 1;
-  const int L0 = p.cache_len[b / ql];
-  int L = L0 + b % ql;
-  if (L0 < 0 || L0 + ql - 1 >= p.cap) {
-    if (threadIdx.x == 0) atomicCAS(err, 0, SITE_BAD_CACHE_LEN);
-    r.lo = 0; r.hi = -1; r.t_begin = 0; r.t_end = 0;
-    return r;
-  }
-  r.hi = L;
-  r.lo = p.window > 0 ? max(0, L - p.window + 1) : 0;
-  const int t0 = r.lo / 128, t1 = r.hi / 128 + 1;
-  const int per = (t1 - t0 + p.n_split - 1) / p.n_split;
-  r.t_begin = min(t1, t0 + sp * per);
-  r.t_end = min(t1, r.t_begin + per);
-  return r;
+  const int L = p.cache_len[r / ql] + r % ql;
+  *hi = L;
+  *lo = p.window > 0 ? max(0, L - p.window + 1) : 0;
 }
 
+// One segment: the tiles [g0, g1) of the global list, all in row r.
+struct DskSeg {
+  int r, g0, g1;        // row; global tile range
+  int tile0;            // tile index (of TP positions) within the row of global tile g0
+  int lo, hi;           // row's key range
+};
+
+// Walks the segments of this CTA's range in order; every role walks the same sequence.
+struct DskWalk {
+  int t, t_end, r;
+  __device__ void init(const DecAttnParams& p) {
+    // G = min(grid, N) CTAs share the N tiles, so that no CTA range is empty (the merge kernel
+    // relies on it); the CTAs beyond G have nothing to do
+    const long long N = p.tstart[p.R];
+    const long long G = N < (long long)gridDim.x ? N : (long long)gridDim.x;
+    if ((long long)blockIdx.x >= G) {
+      t = t_end = r = 0;
+      return;
+    }
+    t = int(N * blockIdx.x / G);
+    t_end = int(N * (blockIdx.x + 1) / G);
+    // the row holding tile t: the largest r with tstart[r] <= t
+    int a = 0, b = p.R - 1;
+    while (a < b) {
+      const int m = (a + b + 1) >> 1;
+      if (p.tstart[m] <= t) a = m; else b = m - 1;
+    }
+    r = a;
+  }
+  __device__ bool next(const DecAttnParams& p, DskSeg* s) {
+    if (t >= t_end) return false;
+    while (p.tstart[r + 1] <= t) ++r;
+    s->r = r;
+    s->g0 = t;
+    s->g1 = min(t_end, p.tstart[r + 1]);
+    dsk_row_range(p, r, &s->lo, &s->hi);
+    s->tile0 = s->lo / dsk::TP + (t - p.tstart[r]);
+    t = s->g1;
+    return true;
+  }
+};
+
 __global__ void __launch_bounds__(192, 1)
-    dec_attn_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapC,
+    dec_attn_sk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapC,
                        const __grid_constant__ DecAttnParams p, KernelCtl ctl) {
-  using namespace dtc;
+  using namespace dsk;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = dtc_align(smem_raw);
-  DecBars* bars = reinterpret_cast<DecBars*>(smem + BAR_OFF);
+  uint8_t* smem = dsk_align(smem_raw);
+  SkBars* bars = reinterpret_cast<SkBars*>(smem + BAR_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sp = blockIdx.x, b = blockIdx.y;
-  const DecRange rg = dec_range(p, b, sp, ctl.err);
-  const int n_t = rg.t_end - rg.t_begin;
+  const int ql = p.q_len > 1 ? p.q_len : 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < NSLOT; ++s) {
-      mbar_init(&bars->ring_full[s], 1);
-      mbar_init(&bars->ring_empty[s], 1);
+    mbar_init(&bars->q_ready, 5);          // producer's expect_tx + the four softmax warps
+    for (int s = 0; s < NLAT; ++s) {
+      mbar_init(&bars->lat_full[s], 1);
+      mbar_init(&bars->lat_empty[s], 1);
     }
-    mbar_init(&bars->s_full[0], 1);
-    mbar_init(&bars->s_full[1], 1);
-    mbar_init(&bars->p_ready, 128);
+    for (int s = 0; s < NROPE; ++s) {
+      mbar_init(&bars->rope_full[s], 1);
+      mbar_init(&bars->rope_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 4);           // one arrival per softmax warp: S read out of TMEM
+    mbar_init(&bars->p_ready, 4);          // one arrival per softmax warp: P written
     mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->seg_done, 1);
     mbar_init(&bars->mma_final, 1);
     fence_mbar_init();
     tma_prefetch_desc(&mapQ);
     tma_prefetch_desc(&mapC);
   }
-  if (threadIdx.x < NH) bars->m_ref[threadIdx.x] = -INFINITY;
-  if (warp == 1) {
+  if (warp == 5) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -113,259 +168,333 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const long long crow0 = (long long)(b / (p.q_len > 1 ? p.q_len : 1)) * p.cap;
 
-  if (warp == 0) {
-    if (lane == 0 && n_t > 0) {
+  DskWalk walk;
+  walk.init(p);
+  DskSeg sg;
+
+  if (warp == 4) {
+    if (lane == 0) {
       // ============================================================ TMA producer
-      uint32_t issued = 0, par = 0;
+      uint32_t lat_issued = 0, lat_par = 0, rope_issued = 0, rope_par = 0;
+      bool q_issued = false;
       bool ok = true;
-      mbar_expect_tx(&bars->q_full, 9 * QBOX);
-      for (int c = 0; c < 9; ++c)
-        tma_load_2d(smem + QT_OFF + c * QBOX, &mapQ, &bars->q_full, c * 64, b * NH);
-      uint32_t g = 0;
-      // The latent columns are read twice (scores, then PV): the first read asks L2 to keep
-      // them, the second (and the rope columns, read once) lets them go.
-      const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
-      // unit order: S(0), S(1), P(0), S(2), P(1), ..., S(n-1), P(n-2), P(n-1)
-      auto load_unit = [&](int tile, int pair, bool rope, bool second) -> bool {
-        const int slot = g % NSLOT;
-        const uint32_t ph = (g / NSLOT) & 1;
-        if (g >= NSLOT && !mbar_wait(&bars->ring_empty[slot], ph ^ 1, ctl, SITE_DEC_PRODUCER))
-          return false;
-        uint8_t* dst = smem + RING_OFF + slot * SLOT;
-        const int y = int(crow0 + (long long)(rg.t_begin + tile) * 128);
-        if (rope) {
-          mbar_expect_tx(&bars->ring_full[slot], 16384);
-          tma_load_2d_hint(dst, &mapC, &bars->ring_full[slot], 512, y, drop);
-        } else {
-          const uint64_t pol = second ? drop : keep;
-          mbar_expect_tx(&bars->ring_full[slot], 32768);
-          tma_load_2d_hint(dst, &mapC, &bars->ring_full[slot], pair * 128, y, pol);
-          tma_load_2d_hint(dst + 16384, &mapC, &bars->ring_full[slot], pair * 128 + 64, y, pol);
-        }
-        issued |= 1u << slot;
-        par = (par & ~(1u << slot)) | (ph << slot);
-        ++g;
-        return true;
-      };
-      for (int i = 0; i <= n_t && ok; ++i) {
-        if (i < n_t)
-          for (int u = 0; u < 5 && ok; ++u) ok = load_unit(i, u, u == 4, false);
-        if (i >= 1)
-          for (int u = 0; u < 4 && ok; ++u) ok = load_unit(i - 1, u, false, true);
-      }
-      for (int s = 0; s < NSLOT; ++s)
-        if (issued & (1u << s)) mbar_drain(&bars->ring_full[s], (par >> s) & 1, ctl.err);
-      mbar_drain(&bars->q_full, 0, ctl.err);
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && n_t > 0) {
-      // ============================================================ MMA issuer
-      constexpr uint32_t idesc_s = make_idesc(128, NH, 1, 0, 0);
-      constexpr uint32_t idesc_o = make_idesc(128, NH, 1, 1, 0);
-      const uint32_t ring = smem_u32(smem + RING_OFF);
-      const uint32_t qt = smem_u32(smem + QT_OFF);
-      const uint32_t pt = smem_u32(smem + P_OFF);
-      uint32_t g = 0, pr_par = 0;
-      bool ok = mbar_wait(&bars->q_full, 0, ctl, SITE_DEC_MMA);
-      // ring units are consumed strictly in load order, one at a time: wait, issue, release
-      auto wait_unit = [&]() -> bool {
-        if (!mbar_wait(&bars->ring_full[g % NSLOT], (g / NSLOT) & 1, ctl, SITE_DEC_MMA)) return false;
-        tc_fence_after();
-        return true;
-      };
-      auto release_unit = [&]() {
-        mma_commit(&bars->ring_empty[g % NSLOT]);
-        ++g;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(&bars->p_ready, pr_par, ctl, SITE_DEC_MMA)) return false;
-        pr_par ^= 1;
-        tc_fence_after();
-#pragma unroll 1
-        for (int mb = 0; mb < 4; ++mb) {
-          if (!wait_unit()) return false;
-          const uint32_t a0 = ring + (g % NSLOT) * SLOT;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = sdesc_sw128(a0 + kk * 2048, 16384, 1024);
-            const uint64_t bd = sdesc_sw128(pt + (kk >> 2) * QBOX + (kk & 3) * 32, 16, 1024);
-            mma_ss(tmem + O_COL + NH * mb, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+      int J = 0;            // CTA-local tile counter (over all segments)
+      int seg = 0;
+      while (ok && walk.next(p, &sg)) {
+        const long long crow0 = (long long)(sg.r / ql) * p.cap;
+        bool q_done = false;
+        auto load_q = [&]() -> bool {
+          // the previous segment's score MMAs read the shared q~ boxes until it is done
+          if (seg > 0 && !mbar_wait(&bars->seg_done, (seg - 1) & 1, ctl, SITE_DEC_PRODUCER)) return false;
+          mbar_expect_tx(&bars->q_ready, 5 * QS_BOX);
+          for (int c = 0; c < 5; ++c)
+            tma_load_2d(smem + QS_OFF + c * QS_BOX, &mapQ, &bars->q_ready, 256 + 64 * c, sg.r * NH);
+          q_issued = true;
+          return true;
+        };
+        const int n_tiles = sg.g1 - sg.g0;
+        // the segment's key rows lie in one sequence: [crow0 + lo', crow0 + hi], contiguous
+        auto prefetch = [&](int jj) {
+          const int pos = (sg.tile0 + jj) * TP;
+          const int first = max(pos, sg.lo), last = min(pos + TP - 1, sg.hi);
+          if (first <= last)
+            l2_prefetch_bulk(static_cast<const uint8_t*>(p.cache) + (crow0 + first) * 1152,
+                             uint32_t(last - first + 1) * 1152u);
+        };
+        for (int jj = 0; jj < PREFETCH_AHEAD && jj < n_tiles; ++jj) prefetch(jj);
+        for (int j = 0; j < n_tiles && ok; ++j, ++J) {
+          if (j + PREFETCH_AHEAD < n_tiles) prefetch(j + PREFETCH_AHEAD);
+          const int y = int(crow0 + (long long)(sg.tile0 + j) * TP);
+          for (int u = 0; u < 4 && ok; ++u) {
+            const int gl = 4 * J + u, s = gl % NLAT;
+            const uint32_t ph = (gl / NLAT) & 1;
+            if (gl >= NLAT && !mbar_wait(&bars->lat_empty[s], ph ^ 1, ctl, SITE_DEC_PRODUCER)) { ok = false; break; }
+            uint8_t* dst = smem + LAT_OFF + s * LAT_SLOT;
+            mbar_expect_tx(&bars->lat_full[s], LAT_SLOT);
+            tma_load_2d(dst, &mapC, &bars->lat_full[s], 128 * u, y);
+            tma_load_2d(dst + LAT_SLOT / 2, &mapC, &bars->lat_full[s], 128 * u + 64, y);
+            lat_issued |= 1u << s;
+            lat_par = (lat_par & ~(1u << s)) | (ph << s);
           }
-          release_unit();
+          if (!ok) break;
+          {
+            const int s = J % NROPE;
+            const uint32_t ph = (J / NROPE) & 1;
+            if (J >= NROPE && !mbar_wait(&bars->rope_empty[s], ph ^ 1, ctl, SITE_DEC_PRODUCER)) { ok = false; break; }
+            mbar_expect_tx(&bars->rope_full[s], ROPE_SLOT);
+            tma_load_2d(smem + ROPE_OFF + s * ROPE_SLOT, &mapC, &bars->rope_full[s], 512, y);
+            rope_issued |= 1u << s;
+            rope_par = (rope_par & ~(1u << s)) | (ph << s);
+          }
+          // q~ of this segment goes after its first tile: that tile's loads overlap the wait
+          // for the previous segment to finish with the shared q~ boxes
+          if (!q_done) {
+            if (!load_q()) { ok = false; break; }
+            q_done = true;
+          }
+        }
+        ++seg;
+      }
+      for (int s = 0; s < NLAT; ++s)
+        if (lat_issued & (1u << s)) mbar_drain(&bars->lat_full[s], (lat_par >> s) & 1, ctl.err);
+      for (int s = 0; s < NROPE; ++s)
+        if (rope_issued & (1u << s)) mbar_drain(&bars->rope_full[s], (rope_par >> s) & 1, ctl.err);
+      if (q_issued) mbar_drain(&bars->q_ready, (seg - 1) & 1, ctl.err);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ============================================================ MMA issuer
+      // Descriptors as (low, high) words; offsets below are in 16-byte units of the low word.
+      constexpr uint32_t idesc_s = make_idesc(128, TP, 1, 0, 0);
+      constexpr uint32_t idesc_o = make_idesc(128, NH, 1, 1, 0);
+      const uint32_t hi = uint32_t(sdesc_sw128(smem_u32(smem), 16, 1024) >> 32);
+      const uint32_t qs_lo = uint32_t(sdesc_sw128(smem_u32(smem + QS_OFF), 16, 1024));
+      const uint32_t p_lo = uint32_t(sdesc_sw128(smem_u32(smem + P_OFF), 16, 1024));
+      const uint32_t lat_lo = uint32_t(sdesc_sw128(smem_u32(smem + LAT_OFF), 16, 1024));        // K-major
+      const uint32_t latv_lo = uint32_t(sdesc_sw128(smem_u32(smem + LAT_OFF), LAT_SLOT / 2, 1024));  // MN-major
+      const uint32_t rope_lo = uint32_t(sdesc_sw128(smem_u32(smem + ROPE_OFF), 16, 1024));
+      const uint32_t tS = tmem + S_COL;
+      bool ok = true;
+      int J = 0, seg = 0;
+      int ls = 0, rs = 0;                      // ring slot of the tile's first latent unit / its rope unit
+      uint32_t lph = 0, rph = 0;               // parity of the next full-wait, per slot
+      // PV of the tile before: O^T += C(J)^T P^T once the softmax has written P (slots of the
+      // tile are released block by block)
+      auto issue_pv = [&](int Jp, bool first) -> bool {
+        if (!mbar_wait(&bars->p_ready, Jp & 1, ctl, SITE_DEC_MMA)) return false;
+        tc_fence_after();
+        int s0 = (4 * Jp) % NLAT;
+#pragma unroll
+        for (int mb = 0; mb < 4; ++mb) {
+          int s = s0 + mb;
+          if (s >= NLAT) s -= NLAT;
+          const uint32_t a = latv_lo + uint32_t(s) * (LAT_SLOT / 16);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss_w(tmem + O_COL + NH * mb, a + uint32_t(kk * 128), hi, p_lo + uint32_t(kk * 2), hi,
+                     idesc_o, (!first || kk > 0) ? 1u : 0u);
+          mma_commit(&bars->lat_empty[s]);
         }
         mma_commit(&bars->pv_done);
         return true;
       };
-      for (int i = 0; i < n_t && ok; ++i) {
-        // ---- S^T(i) = C(i) q~^T into S buffer i & 1, one ring unit (64-col box pair) at a time
-        const uint32_t d = tmem + ((i & 1) ? S_COL1 : S_COL0);
-#pragma unroll 1
-        for (int u = 0; u < 5 && ok; ++u) {
-          if (!wait_unit()) { ok = false; break; }
-          const uint32_t slot = ring + (g % NSLOT) * SLOT;
-          const int nbox = u < 4 ? 2 : 1;
-          for (int bx = 0; bx < nbox; ++bx) {
-            const int c = u < 4 ? 2 * u + bx : 8;    // K chunk: latent 0..7, rope 8
-            const uint32_t a0 = slot + bx * 16384;
-            const uint32_t b0 = qt + c * QBOX;
+      while (ok && walk.next(p, &sg)) {
+        if (!mbar_wait(&bars->q_ready, seg & 1, ctl, SITE_DEC_MMA)) { ok = false; break; }
+        tc_fence_after();
+        for (int j = 0; j < sg.g1 - sg.g0; ++j, ++J) {
+          // ---- S(J) = q~ C(J)^T, once the softmax has read S(J - 1) out of TMEM: latent dims
+          // 0..255 with A in TMEM, 256..511 and rope with A in smem
+          if (j > 0 && !mbar_wait(&bars->s_free, (J - 1) & 1, ctl, SITE_DEC_MMA)) { ok = false; break; }
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ss(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
-                     idesc_s, (c | kk) != 0);
+          for (int u = 0; u < 4; ++u) {
+            int s = ls + u;
+            if (s >= NLAT) s -= NLAT;
+            if (!mbar_wait(&bars->lat_full[s], (lph >> s) & 1, ctl, SITE_DEC_MMA)) { ok = false; break; }
+            lph ^= 1u << s;
+            tc_fence_after();
+            const uint32_t b = lat_lo + uint32_t(s) * (LAT_SLOT / 16);
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx) {
+              const int c = 2 * u + bx;             // 64-dim chunk of the latent
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t bd = b + uint32_t(bx * (LAT_SLOT / 32) + kk * 2);
+                if (c < 4)
+                  mma_ts_w(tS, tmem + QT_COL + (4 * c + kk) * 8, bd, hi, idesc_s, (c | kk) != 0);
+                else
+                  mma_ss_w(tS, qs_lo + uint32_t((c - 4) * (QS_BOX / 16) + kk * 2), hi, bd, hi, idesc_s, 1u);
+              }
+            }
           }
-          release_unit();
+          if (!ok) break;
+          if (!mbar_wait(&bars->rope_full[rs], (rph >> rs) & 1, ctl, SITE_DEC_MMA)) { ok = false; break; }
+          rph ^= 1u << rs;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss_w(tS, qs_lo + uint32_t(4 * (QS_BOX / 16) + kk * 2), hi,
+                     rope_lo + uint32_t(rs * (ROPE_SLOT / 16) + kk * 2), hi, idesc_s, 1u);
+          mma_commit(&bars->s_full);
+          mma_commit(&bars->rope_empty[rs]);
+          rs = rs + 1 == NROPE ? 0 : rs + 1;
+          ls += 4;
+          if (ls >= NLAT) ls -= NLAT;
+          // ---- PV(J - 1) behind S(J): the softmax of tile J overlaps it
+          if (j > 0 && !issue_pv(J - 1, j == 1)) { ok = false; break; }
         }
         if (!ok) break;
-        mma_commit(&bars->s_full[i & 1]);
-        // ---- O^T += C(i-1)^T P(i-1)
-        if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+        if (!issue_pv(J - 1, sg.g1 - sg.g0 == 1)) { ok = false; break; }
+        mma_commit(&bars->seg_done);
+        ++seg;
       }
-      if (ok) issue_pv(n_t - 1);
       mma_commit(&bars->mma_final);
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
   } else {
-    // ============================================================ softmax (warps 2..5)
-    const int q = warp & 3;                 // TMEM lane quarter of this warp
-    const int r = q * 32 + lane;            // position within the tile / latent row
-    const int tw = threadIdx.x - 64;        // 0..127 inside the softmax group
+    // ============================================================ softmax / epilogue (warps 0-3)
+    const int q = warp;                      // TMEM lane quarter
+    const int h = 32 * q + lane;             // head of this thread (h < 80), latent row in O^T
+    const bool hv = h < NH;
     const uint32_t lane_off = uint32_t(q * 32) << 16;
-    float l_part[NH];
-#pragma unroll
-    for (int h = 0; h < NH; ++h) l_part[h] = 0.f;
-    uint32_t s_par[2] = {0, 0};
-    int pv_seen = 0;                        // PVs known complete
-    bool ok = true;
-    auto wait_pv = [&](int k) -> bool {     // wait until PV(k) has completed
-      if (pv_seen > k) return true;
-      bool w = mbar_wait(&bars->pv_done, k & 1, ctl, SITE_DEC_SOFTMAX);
-      w = __all_sync(0xffffffffu, w);
-      if (w) pv_seen = k + 1;
-      return w;
-    };
     uint8_t* P = smem + P_OFF;
-    // Every outcome of a bounded wait is made uniform over the 128 softmax threads before it
-    // steers control flow, so that no thread is left alone at a named barrier.
+    bool ok = true;
+    int J = 0, seg = 0;
     auto group_ok = [&](bool w) { return !named_bar_or(1, 128, !w); };
-    for (int i = 0; i < n_t && ok; ++i) {
-      const int buf = i & 1;
-      const bool w = mbar_wait(&bars->s_full[buf], s_par[buf], ctl, SITE_DEC_SOFTMAX);
-      if (!group_ok(w)) { ok = false; break; }
-      s_par[buf] ^= 1;
-      tc_fence_after();
-      const uint32_t tS = tmem + (buf ? S_COL1 : S_COL0) + lane_off;
-      const int pos = (rg.t_begin + i) * 128 + r;
-      const bool valid = pos >= rg.lo && pos <= rg.hi;
-      // scores are re-read from TMEM in 16-head chunks: (log2-scaled) score of head 16c + e
-      auto load_chunk = [&](int c, float* v) {
-        uint32_t u[16];
-        GDLA_TMEM_LD16(tS + 16 * c, u);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = valid ? __uint_as_float(u[e]) * p.scale_log2 : -INFINITY;
-      };
-      bool above = false;
+    while (ok && walk.next(p, &sg)) {
+      // ---- q~ dims 0..255 of this row into TMEM (lane = head, two dims per column)
+      // (from the second segment on, the previous segment's MMAs are complete and its partial
+      // was read out at the end of the loop below)
+      if (q < 3) {
+        uint32_t v[32];
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.qt) +
+                                                          ((long long)sg.r * NH + (hv ? h : 0)) * 576);
 #pragma unroll 1
-      for (int c = 0; c < 5; ++c) {
-        float v[16];
-        load_chunk(c, v);
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) above |= v[e] > bars->m_ref[16 * c + e] + RESCALE_THRESHOLD;
-      }
-      if (named_bar_or(1, 128, above)) {
-        // exact per-head maximum of this tile, then move the reference maxima
-#pragma unroll 1
-        for (int c = 0; c < 5; ++c) {
-          float v[16];
-          load_chunk(c, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float x = v[e];
-#pragma unroll
-            for (int o = 16; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-            if (lane == ((16 * c + e) & 31)) bars->red[q][16 * c + e] = x;
+          for (int k = 0; k < 8; ++k) {
+            const uint4 w = hv ? src[8 * c + k] : make_uint4(0u, 0u, 0u, 0u);
+            v[4 * k] = w.x; v[4 * k + 1] = w.y; v[4 * k + 2] = w.z; v[4 * k + 3] = w.w;
           }
+          GDLA_TMEM_ST32(tmem + QT_COL + 32 * c + lane_off, v);
         }
-        named_bar_sync(1, 128);
-        if (tw < NH) {
-          const float tmax = fmaxf(fmaxf(bars->red[0][tw], bars->red[1][tw]),
-                                   fmaxf(bars->red[2][tw], bars->red[3][tw]));
-          const float mo = bars->m_ref[tw];
-          const float mn = fmaxf(mo, tmax);
-          bars->red[0][tw] = mn == -INFINITY ? 1.f : ex2_approx(mo - mn);   // scale of old terms
-          bars->red[1][tw] = mn;
-        }
-        named_bar_sync(1, 128);
-#pragma unroll
-        for (int h = 0; h < NH; ++h) l_part[h] *= bars->red[0][h];
-        if (i > 0) {
-          // O^T must hold PV(0..i-1) before it is rescaled
-          if (!group_ok(wait_pv(i - 1))) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < 4 * 5; ++c) {          // 4 M blocks x 5 chunks of 16 heads
-            const uint32_t tO = tmem + O_COL + NH * (c / 5) + 16 * (c % 5) + lane_off;
-            uint32_t o[16];
-            GDLA_TMEM_LD16(tO, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              o[e] = __float_as_uint(__uint_as_float(o[e]) * bars->red[0][16 * (c % 5) + e]);
-            GDLA_TMEM_ST16(tO, o);
-          }
-          tmem_st_wait();
-        }
-        named_bar_sync(1, 128);
-        if (tw < NH) bars->m_ref[tw] = bars->red[1][tw];
-        named_bar_sync(1, 128);
+        tmem_st_wait();
       }
-      // the single P buffer is free once PV(i-1) has completed
-      if (i > 0 && !group_ok(wait_pv(i - 1))) { ok = false; break; }
-      {
-        // numerators of this tile, rounded to bf16 (the row sums use the rounded values)
-        const int chunk = r >> 6, pc = r & 63;
-        uint8_t* base = P + chunk * QBOX + ((pc & 7) << 1);
-#pragma unroll
-        for (int c = 0; c < 5; ++c) {
-          float v[16];
-          load_chunk(c, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int hh = 16 * c + e;
-            const float mr = bars->m_ref[hh];
-            const float mu = mr == -INFINITY ? 0.f : mr;
-            const __nv_bfloat16 pbv = __float2bfloat16_rn(ex2_approx(v[e] - mu));
-            l_part[hh] += __bfloat162float(pbv);
-            *reinterpret_cast<__nv_bfloat16*>(base + hh * 128 + ((((pc >> 3) ^ (hh & 7))) << 4)) = pbv;
-          }
-        }
-      }
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->p_ready);
-    }
-    // ---------------- split partials
-    if (ok && n_t > 0 && !group_ok(wait_pv(n_t - 1))) ok = false;
-    tc_fence_after();
-    // row sums: per head, over the 128 positions
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q_ready);
+
+      float m_ref = -INFINITY;
+      float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;   // row sum, in four partials
+      bool carried_fail = false;                          // a wait of the last tile expired
+      for (int j = 0; j < sg.g1 - sg.g0; ++j, ++J) {
+        // (warp-uniform: the TMEM load below is a warp-collective instruction)
+        const bool w = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, J & 1, ctl, SITE_DEC_SOFTMAX));
+        tc_fence_after();
+        const int pos0 = (sg.tile0 + j) * TP;
+        const int a = sg.lo - pos0, bnd = sg.hi - pos0;   // valid columns a .. bnd
+        const bool edge = a > 0 || bnd < TP - 1;           // uniform: a boundary tile of the row
+        float v[TP];
+        float mt = -INFINITY;
+        if (q < 3 && w) {
+          uint32_t u[TP];
+          GDLA_TMEM_LD32(tmem + S_COL + lane_off, u);
+          GDLA_TMEM_LD32(tmem + S_COL + 32 + lane_off, (u + 32));
+          tmem_ld_wait();
 #pragma unroll
-    for (int h = 0; h < NH; ++h) {
-      float v = l_part[h];
+          for (int c = 0; c < TP; ++c) v[c] = __uint_as_float(u[c]);
+        }
+        // S is in registers: the MMA issuer may overwrite it with the next tile's scores
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
+        if (q < 3) {
+          if (edge) {
 #pragma unroll
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == (h & 31)) bars->red[q][h] = v;
-    }
-    named_bar_sync(1, 128);
-    const long long pbase = ((long long)b * p.n_split + sp) * NH;
-    if (tw < NH) {
-      float* ml = p.ml + (pbase + tw) * 2;
-      const float lsum = bars->red[0][tw] + bars->red[1][tw] + bars->red[2][tw] + bars->red[3][tw];
-      ml[0] = bars->m_ref[tw];
-      ml[1] = (ok && n_t > 0) ? lsum : 0.f;
-    }
-    if (ok && n_t > 0) {
+            for (int c = 0; c < TP; ++c) v[c] = (c >= a && c <= bnd) ? v[c] : -INFINITY;
+          }
+          float m8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            m8[k] = fmax3f(fmax3f(v[8 * k], v[8 * k + 1], v[8 * k + 2]), fmax3f(v[8 * k + 3], v[8 * k + 4], v[8 * k + 5]),
+                           fmaxf(v[8 * k + 6], v[8 * k + 7]));
+          mt = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * p.scale_log2;
+        }
+        // the one barrier of the common path: does any head need its reference maximum moved
+        // (or did any wait expire)?
+        const bool need = hv && mt > m_ref + RESCALE_THRESHOLD;
+        if (named_bar_or(1, 128, need || !w || carried_fail)) {
+          if (named_bar_or(1, 128, !w || carried_fail)) { ok = false; break; }
+          // O^T must hold PV(J - 1) before it is rescaled (PV(J) comes after this tile's P)
+          bool w2 = j == 0 || mbar_wait(&bars->pv_done, (J - 1) & 1, ctl, SITE_DEC_SOFTMAX);
+          if (named_bar_or(1, 128, !w2)) { ok = false; break; }
+          tc_fence_after();
+          if (hv) {
+            const float mn = need ? mt : m_ref;
+            const float sc = need ? ex2_approx(m_ref - mn) : 1.f;   // 2^-inf = 0 on the first tile
+            ls0 *= sc; ls1 *= sc; ls2 *= sc; ls3 *= sc;
+            m_ref = mn;
+            bars->scale[h] = sc;
+          }
+          named_bar_sync(1, 128);
+          if (j > 0) {
+#pragma unroll 1
+            for (int c = 0; c < 4 * 5; ++c) {
+              const uint32_t tO = tmem + O_COL + NH * (c / 5) + 16 * (c % 5) + lane_off;
+              uint32_t o[16];
+              GDLA_TMEM_LD16(tO, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                o[e] = __float_as_uint(__uint_as_float(o[e]) * bars->scale[16 * (c % 5) + e]);
+              GDLA_TMEM_ST16(tO, o);
+            }
+            tmem_st_wait();
+          }
+          named_bar_sync(1, 128);
+        }
+        // P has one buffer: PV(J - 1) must have read it (earlier segments' PVs are complete)
+        const bool w3 = j == 0 || mbar_wait(&bars->pv_done, (J - 1) & 1, ctl, SITE_DEC_SOFTMAX);
+        carried_fail = !w3;
+        if (edge && bnd < TP - 1) {
+          // rows past the row's last key: zero them in the four latent slots before the PV
+          const int r0 = bnd + 1;
+          const int nbytes = (TP - r0) * 128;
+#pragma unroll 1
+          for (int bx = 0; bx < 8; ++bx) {
+            uint8_t* box = smem + LAT_OFF + ((4 * J + bx / 2) % NLAT) * LAT_SLOT + (bx & 1) * (LAT_SLOT / 2);
+            for (int o = (q * 32 + lane) * 16; o < nbytes; o += 128 * 16)
+              *reinterpret_cast<uint4*>(box + r0 * 128 + o) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        // numerators 2^(s scale - m) (every fourth pair on the FMA pipe), rounded to bf16, one
+        // 128-byte row of P per head in the 128-byte-swizzled K-major layout of the PV's B operand
+        const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
+        uint8_t* row = P + h * 128;
+        if (hv && w3) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 8 * k + 2 * e;
+              float x0, x1, p0, p1;
+              ffma2(x0, x1, v[c], v[c + 1], p.scale_log2, neg_m);
+              if (e == 3) {
+                exp2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              if (edge) {
+                p0 = (c >= a && c <= bnd) ? p0 : 0.f;
+                p1 = (c + 1 >= a && c + 1 <= bnd) ? p1 : 0.f;
+              }
+              pk[e] = pack_bf162(p0, p1);
+              // the row sum adds the rounded values the PV multiplies (weights summing to 1)
+              const float r0 = __uint_as_float(pk[e] << 16), r1 = __uint_as_float(pk[e] & 0xFFFF0000u);
+              if (e & 1) fadd2(ls2, ls3, r0, r1); else fadd2(ls0, ls1, r0, r1);
+            }
+            *reinterpret_cast<uint4*>(row + ((k ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_ready);
+      }
+      const float l_sum = (ls0 + ls1) + (ls2 + ls3);
+      if (!ok) break;
+      // ---- segment partial: (m_h, l_h) and O^T, to slot blockIdx.x + r
+      const bool w = mbar_wait(&bars->seg_done, seg & 1, ctl, SITE_DEC_SOFTMAX);
+      if (!group_ok(w && !carried_fail)) { ok = false; break; }
+      tc_fence_after();
+      const long long slot = (long long)blockIdx.x + sg.r;
+      if (hv) {
+        float* ml = p.ml + (slot * NH + h) * 2;
+        ml[0] = m_ref;
+        ml[1] = l_sum;
+      }
 #pragma unroll 1
       for (int mb = 0; mb < 4; ++mb) {
         const uint32_t tO = tmem + O_COL + NH * mb + lane_off;
@@ -374,54 +503,103 @@ __global__ void __launch_bounds__(192, 1)
         GDLA_TMEM_LD32(tO + 32, (o + 32));
         GDLA_TMEM_LD16(tO + 64, (o + 64));
         tmem_ld_wait();
-        float* dst = p.part + pbase * 512 + 128 * mb + r;
+        float* dst = p.part + slot * NH * 512 + 128 * mb + h;
 #pragma unroll
-        for (int h = 0; h < NH; ++h) dst[(long long)h * 512] = __uint_as_float(o[h]);
+        for (int hh = 0; hh < NH; ++hh) dst[(long long)hh * 512] = __uint_as_float(o[hh]);
       }
+      tc_fence_before();
+      ++seg;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 5) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t st) {
-  CUtensorMap mq, mc;
-  if (make_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.qt, 576, (uint64_t)p.B * dtc::NH, 576 * 2,
-                   64, dtc::NH, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      make_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.cache, 576, (uint64_t)p.B * p.cap, 576 * 2,
-                   64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
-    return -3;
-  if (cudaFuncSetAttribute(dec_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dtc::SMEM) != cudaSuccess)
-    return -4;
-  dim3 grid(p.n_split, p.B);
-  KernelCtl kc{ctl.err, ctl.limit_ns};
-  dec_attn_tc_kernel<<<grid, 192, dtc::SMEM, st>>>(mq, mc, p, kc);
+// Tile prefix over the query rows: tstart[r] = tiles of rows < r, tstart[R] = all tiles.  A row
+// whose cache_len entry is outside [0, cap - q_len] gets no tiles (its output is zero) and the
+// error word records SITE_BAD_CACHE_LEN.  One CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) dec_sched_kernel(const int* __restrict__ cache_len, int R, int q_len,
+                                                         int cap, int window, int* __restrict__ tstart,
+                                                         int* err) {
+  __shared__ int wsum[32];
+  __shared__ int carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ql = q_len > 1 ? q_len : 1;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < R; base += blockDim.x) {
+    const int r = base + threadIdx.x;
+    int n = 0;
+    if (r < R) {
+      const int L0 = cache_len[r / ql];
+      if (L0 < 0 || L0 > cap - ql) {
+        if (r % ql == 0) atomicCAS(err, 0, SITE_BAD_CACHE_LEN);
+      } else {
+        const int L = L0 + r % ql;
+        const int lo = window > 0 ? max(0, L - window + 1) : 0;
+        n = L / dsk::TP - lo / dsk::TP + 1;
+      }
+    }
+    int x = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int s = lane < int(blockDim.x >> 5) ? wsum[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      wsum[lane] = s;
+    }
+    __syncthreads();
+    const int incl = x + (warp > 0 ? wsum[warp - 1] : 0) + carry;
+    if (r < R) tstart[r] = incl - n;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) tstart[R] = carry;
+}
+
+int launch_dec_sched(const DecAttnParams& p, cudaStream_t st) {
+  dec_sched_kernel<<<1, 1024, 0, st>>>(p.cache_len, p.R, p.q_len, p.cap, p.window, p.tstart, p.err);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
-// Number of key-range splits per sequence: minimises (waves of 148 CTAs) x (tiles per split + 2),
-// the +2 standing for the per-CTA set-up and drain.
-int decode_split_count(int B, int cap, int window) {
-  const int keys = window > 0 ? (window < cap ? window : cap) : cap;
-  const int tiles = (keys + 127) / 128 + 1;
-  int best = 1;
-  long long best_cost = -1;
-  for (int s = 1; s <= 64; ++s) {
-    const long long waves = ((long long)B * s + 147) / 148;
-    const long long cost = waves * ((tiles + s - 1) / s + 2);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = s;
-    }
-  }
-  return best;
+int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t st) {
+  CUtensorMap mq, mc;
+  if (make_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.qt, 576, (uint64_t)p.R * dsk::NH, 576 * 2,
+                   64, dsk::NH, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      make_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.cache, 576, (uint64_t)p.n_seq * p.cap, 576 * 2,
+                   64, dsk::TP, CU_TENSOR_MAP_SWIZZLE_128B))
+    return -3;
+  if (cudaFuncSetAttribute(dec_attn_sk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dsk::SMEM) != cudaSuccess)
+    return -4;
+  KernelCtl kc{ctl.err, ctl.limit_ns};
+  dec_attn_sk_kernel<<<p.n_ctas, 192, dsk::SMEM, st>>>(mq, mc, p, kc);
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
+}
+
+// CTAs of the decode attention: one per SM (its shared memory and 512 TMEM columns fill one).
+int decode_cta_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  return n < DEC_MAX_CTAS ? n : DEC_MAX_CTAS;
 }
 
 }  // namespace gdla

@@ -33,6 +33,7 @@ enum : int {
   SITE_DEC_PRODUCER = 0x501, SITE_DEC_MMA = 0x502, SITE_DEC_SOFTMAX = 0x503,
   SITE_BAD_CACHE_LEN = 0x601,  // a cache_len entry outside [0, cap): that sequence is skipped
   SITE_BAD_CU_SEQLENS = 0x602, // document offsets not 0..total non-decreasing: bad documents skipped
+  SITE_FP16_RANGE = 0x701,     // an fp16 attention operand was outside +-65504 (saturated) or NaN
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -117,6 +118,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y) : "memory");
 }
 
+// Bulk prefetch of [addr, addr + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void l2_prefetch_bulk(const void* addr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(addr), "r"(bytes) : "memory");
+}
+
 // L2 cache policies for TMA loads: keep a line for an upcoming re-read, or let it go first.
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
@@ -170,6 +176,25 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// The same two with shared-memory descriptors given as (low, high) 32-bit words: the low word
+// holds the start address (and the leading offset), so an issuer steps through a buffer with
+// one 32-bit add per operand instead of rebuilding 64-bit descriptors.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                        uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate) : "memory");
 }
 // Arrive once on `bar` when every previously issued tcgen05.mma of this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -365,6 +390,56 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// ---- softmax arithmetic.  Packed f32x2 instructions halve the issue slots of the scale,
+// subtract and sum steps; the attention kernels run part of their exponentials on the FMA pipe
+// (exp2_poly2) instead of MUFU, whose 16 results per clock per SM bound a softmax.
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// (d0, d1) = (a0, a1) + (b0, b1)
+__device__ __forceinline__ void fadd2v(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 d, a, b;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// (d0, d1) = (a0, a1) * (b0, b1) + (c, c)
+__device__ __forceinline__ void ffma2v(float& d0, float& d1, float a0, float a1, float b0, float b1, float c) {
+  asm("{\n\t.reg .b64 d, a, b, c;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %6};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c));
+}
+// (x0, x1) = (a0, a1) * b + c
+__device__ __forceinline__ void ffma2(float& x0, float& x1, float a0, float a1, float b, float c) {
+  ffma2v(x0, x1, a0, a1, b, b, c);
+}
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) {
+  fadd2v(s0, s1, s0, s1, a0, a1);
+}
+// 2^x for a pair on the FMA pipe.  x = j + f with j = round(x) (adding and subtracting
+// 1.5 * 2^23 rounds to the nearest integer) and |f| <= 1/2; 2^f from a cubic fitted to 2^f
+// on [-1/2, 1/2] (iteratively reweighted least squares towards the minimax fit, max relative
+// error 7.5e-5, below the 2^-12 half-ulp of the fp16 or bf16 P it feeds; exp2_poly_fit.py beside this
+// file reproduces the coefficients); j is added to the exponent field as an integer.  x is
+// clamped at -126, where P is 0 either way in fp16 and ~2^-126 in bf16.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& r0, float& r1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, j0, j1, f0, f1;
+  fadd2v(t0, t1, x0, x1, 12582912.f, 12582912.f);
+  fadd2v(j0, j1, t0, t1, -12582912.f, -12582912.f);
+  fadd2v(f0, f1, x0, x1, -j0, -j1);
+  float q0 = 0.05517144128680229f, q1 = 0.05517144128680229f;
+  ffma2v(q0, q1, q0, q1, f0, f1, 0.24261070787906647f);
+  ffma2v(q0, q1, q0, q1, f0, f1, 0.6932609677314758f);
+  ffma2v(q0, q1, q0, q1, f0, f1, 0.9999281167984009f);
+  // the low 9 bits of t's bit pattern hold j mod 512; * 2^23 moves them into the exponent field
+  r0 = __int_as_float(__float_as_int(t0) * 8388608 + __float_as_int(q0));
+  r1 = __int_as_float(__float_as_int(t1) * 8388608 + __float_as_int(q1));
+}
+
 __device__ __forceinline__ float sigmoidf_fast(float z) {
   // 1 / (1 + 2^(-z log2 e)); the hardware exp2 has ~2 ulp relative error.
   return 1.0f / (1.0f + ex2_approx(-z * 1.4426950408889634f));
@@ -372,6 +447,21 @@ __device__ __forceinline__ float sigmoidf_fast(float z) {
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+// fp16 pair for the attention operands (q, K^C, V, k^R): a finite value beyond the fp16 range
+// saturates to +-65504 instead of becoming Inf, and `bad` is set for it and for NaN, so that
+// the caller can record SITE_FP16_RANGE.
+__device__ __forceinline__ uint32_t pack_half2_sat(float lo, float hi, bool& bad) {
+  constexpr float kMax = 65504.f;
+  bad |= !(fabsf(lo) <= kMax) || !(fabsf(hi) <= kMax);
+  lo = fabsf(lo) > kMax ? copysignf(kMax, lo) : lo;
+  hi = fabsf(hi) > kMax ? copysignf(kMax, hi) : hi;
+  return pack_half2(lo, hi);
+}
+__device__ __forceinline__ __half half_sat(float v, bool& bad) {
+  constexpr float kMax = 65504.f;
+  bad |= !(fabsf(v) <= kMax);
+  return __float2half_rn(fabsf(v) > kMax ? copysignf(kMax, v) : v);
 }
 __device__ __forceinline__ uint32_t pack_bf162(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

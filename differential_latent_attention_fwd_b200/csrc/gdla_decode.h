@@ -15,21 +15,30 @@ struct DecQParams {
   void* qt;               // bf16 [B][n_heads][576]
 };
 
+// Upper bound of the decode attention grid (the merge kernel keeps one weight per segment of a
+// row in shared memory, and a row has at most one segment per CTA).
+constexpr int DEC_MAX_CTAS = 160;
+
 struct DecAttnParams {
-  int B, cap, window, n_split;   // B = query rows = sequences x q_len
-  int q_len;              // new tokens per sequence: row r is token r % q_len of sequence r / q_len
-  const int* cache_len;   // [sequences] keys cached before the new tokens
-  const void* cache;      // bf16 [B][cap][576]
-  const void* qt;         // bf16 [B][80][576]
+  int R;                  // query rows = n_seq x q_len: row r is token r % q_len of sequence r / q_len
+  int n_seq, cap, window;
+  int q_len;              // new tokens per sequence
+  const int* cache_len;   // [n_seq] keys cached before the new tokens
+  const void* cache;      // bf16 [n_seq][cap][576]
+  const void* qt;         // bf16 [R][80][576]
   float scale_log2;
-  float* part;            // [B][n_split][80][512] latent accumulators
-  float* ml;              // [B][n_split][80][2]  (running max in log2 units, row sum)
+  int* tstart;            // [R + 1] tile prefix over the rows (dec_sched_kernel)
+  int n_ctas;             // grid of the attention kernel (G): slots = G + R - 1
+  float* part;            // [slots][80][512] latent accumulators of each segment
+  float* ml;              // [slots][80][2]  (running max in log2 units, row sum)
   int* err;               // device error word
 };
 
 struct DecCombParams {
-  int B, n_groups, n_signal, n_split;
-  const float* part;
+  int B, n_groups, n_signal;   // B = query rows
+  int n_ctas;                  // G of the attention launch
+  const int* tstart;           // [B + 1] tile prefix over the rows
+  const float* part;           // segment partials, slot c + r for CTA c and row r
   const float* ml;
   const float* lam;       // [B][n_signal]
   const void* G;          // bf16 [B][n_signal * 128]
@@ -40,8 +49,9 @@ struct DecCombParams {
 int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int d_nope, int d_v,
                      cudaStream_t st);
 int launch_qtilde(const DecQParams& p, cudaStream_t st);
+int launch_dec_sched(const DecAttnParams& p, cudaStream_t st);
 int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t st);
-int decode_split_count(int B, int cap, int window);
+int decode_cta_count();
 int launch_dec_combine(const DecCombParams& p, cudaStream_t st);
 
 }  // namespace gdla

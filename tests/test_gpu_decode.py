@@ -56,6 +56,41 @@ def test_decode_workload(cuda_ok, name):
     check(f"{name}: all 64 sequences", to_np(y), yo)
 
 
+@pytest.mark.parametrize("window", [0, 64])
+def test_decode_ignores_unwritten_cache_tail(cuda_ok, window):
+    """Cache rows past each sequence's new token were never written by the caller: here they
+    hold NaN and Inf.  The output must equal the oracle's, which never reads those rows."""
+    shape = synth.GdlaShape(window=window)
+    lens = [0, 63, 64, 200, 317]
+    inp = synth.make_decode_inputs(shape, len(lens), lens, cap=320, seed=23)
+    cache = inp.cache.clone()
+    for b, L in enumerate(lens):
+        cache[b, L + 1:, ::2] = float("nan")       # row L is the appended one
+        cache[b, L + 1:, 1::2] = float("inf")
+    layer = GdlaLayer(shape, inp.weights, inp.g_q, inp.g_kv, device="cuda")
+    y = layer.decode(inp.x_new.cuda(), cache.cuda(), inp.cache_len.cuda())
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
+    cfg = O.OracleConfig.from_shape(shape)
+    yo = O.gdla_decode(inp.x_new, inp.weights, inp.cache, inp.cache_len, cfg, g_q=inp.g_q, g_kv=inp.g_kv)
+    errs = []
+    for b in range(len(lens)):
+        check(f"decode with a NaN/Inf tail b={b} len={lens[b]} W={window}", to_np(y[b]), yo[b], errors=errs)
+    assert not errs, "\n".join(errs)
+
+
+def test_decode_single_sequence_long_cache(cuda_ok):
+    """One sequence over a long cache: its key tiles are spread over every SM (many segments of
+    one row), then merged."""
+    shape = synth.GdlaShape()
+    inp = synth.make_decode_inputs(shape, 1, [20000], cap=20001, seed=25)
+    y, _ = _decode(inp)
+    cfg = O.OracleConfig.from_shape(shape)
+    yo = O.gdla_decode_absorbed(inp.x_new, inp.weights, inp.cache, inp.cache_len, cfg,
+                                g_q=inp.g_q, g_kv=inp.g_kv)
+    check("B=1, L=20000", to_np(y), yo)
+
+
 def test_prefill_then_decode_continues_sequence(cuda_ok):
     """Prefill T tokens into a cache, decode token T: equals row T of a (T+1)-token prefill."""
     T, cap = 200, 256
