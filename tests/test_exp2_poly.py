@@ -1,6 +1,6 @@
-"""The FMA-pipe exponential of the prefill attention softmax, checked on the CPU.
+"""The FMA-pipe exponential of the attention softmaxes (prefill and decode), checked on the CPU.
 
-The kernel evaluates 2^x for a quarter of the attention probabilities as round-to-nearest
+The kernels evaluate 2^x for a quarter of the attention probabilities as round-to-nearest
 range reduction (add / subtract 1.5 * 2^23), a cubic in the remainder, and an integer add into
 the exponent field.  This test re-derives the cubic with the fitting script that sits beside
 the kernel, checks that the kernel source carries exactly those coefficients, and emulates the
@@ -23,7 +23,7 @@ def _fit_module():
 
 
 def _kernel_coefficients():
-    src = (CSRC / "attn_prefill.cu").read_text()
+    src = (CSRC / "gdla_common.cuh").read_text()
     body = src[src.index("void exp2_poly2("):]
     body = body[: body.index("\n}\n")]
     nums = [float(v) for v in re.findall(r"(\d\.\d+)f", body)]

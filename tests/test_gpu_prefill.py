@@ -67,6 +67,8 @@ def test_stagewise_intermediates_t256(cuda_ok):
 @pytest.mark.parametrize("B,T,window", [
     (1, 1, 0), (1, 100, 0), (1, 129, 0), (1, 300, 0), (2, 200, 64), (1, 700, 128),
     (1, 384, 1), (1, 257, 256), (3, 130, 0),
+    # a window at least as long as the sequence: every row sees its whole causal prefix
+    (1, 100, 2048), (2, 300, 512), (1, 256, 256), (1, 513, 600),
 ])
 def test_prefill_edge_shapes(cuda_ok, B, T, window):
     shape, inp, layer, x = prefill_case(B, T, window, seed=11)
@@ -175,3 +177,65 @@ def test_packed_documents_reject_bad_offsets(cuda_ok):
     layer.prefill_packed(x[0].contiguous(), bad)
     torch.cuda.synchronize()
     assert gb.gdla_device_error() == 0x602
+
+
+def _stage_oracle_on_gpu_operands(ws, cfg, shape, T, window):
+    """The oracle's attention stage evaluated on the fp16/fp32 operands the GPU left in its
+    workspace (q, K^C, V, k^R, lambda, gate logits): isolates the attention kernel's arithmetic
+    from the rounding of its inputs."""
+    from oracle import gdla_oracle as O
+    nH = shape.n_heads
+    qq = to_np(ws_view(ws, cfg, 1, T, 0, WS_QQ, torch.float16, (T, nH * shape.d_qk)))
+    kv = to_np(ws_view(ws, cfg, 1, T, 0, WS_KV, torch.float16, (T, shape.n_kv_heads, 256)))
+    kr = to_np(ws_view(ws, cfg, 1, T, 0, 9, torch.float16, (T, shape.d_rope)))
+    lam = to_np(ws_view(ws, cfg, 1, T, 0, WS_LAM, torch.float32, (T, shape.n_signal)))
+    gate = to_np(ws_view(ws, cfg, 1, T, 0, WS_G, torch.bfloat16, (T, shape.n_signal, shape.d_v)))
+    ocfg = O.OracleConfig.from_shape(synth.GdlaShape(window=window))
+    Dg, _ = O.attention_stage(qq[:, : nH * 128].reshape(T, nH, 128), qq[:, nH * 128:].reshape(T, nH, 64),
+                              kv[..., :128], kv[..., 128:], kr, lam, gate, ocfg)
+    return Dg, max(np.abs(qq).max(), np.abs(kv).max(), np.abs(kr).max())
+
+
+def test_large_norm_gains_keep_fp16_operands_finite(cuda_ok):
+    """RMSNorm gains of 50 (q and KV latents): the fp16 attention operands grow 50x and stay
+    finite; no range error is reported, and the attention kernel matches the oracle's
+    attention stage on those operands."""
+    T, window = 200, 0
+    shape = synth.GdlaShape(window=window)
+    inp = synth.make_prefill_inputs(shape, 1, T, seed=13)
+    from differential_latent_attention_fwd_b200.layer import GdlaLayer
+    g50q = (torch.ones(shape.q_rank) * 50).bfloat16()
+    g50kv = (torch.ones(shape.kv_rank) * 50).bfloat16()
+    layer = GdlaLayer(shape, inp.weights, g50q, g50kv, device="cuda")
+    y = layer.prefill(inp.x.cuda())
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
+    assert bool(torch.isfinite(y).all())
+    Dg_o, amax = _stage_oracle_on_gpu_operands(layer._ws, layer.cfg, shape, T, window)
+    assert 10.0 < amax < 65504.0, amax
+    dg = to_np(ws_view(layer._ws, layer.cfg, 1, T, 0, WS_DG, torch.bfloat16, (T, 64, 128)))
+    # the gains scale V (hence D and Dg) by 50: the absolute bound scales with it, the relative
+    # one does not
+    check("Dg with gains x50 vs the oracle's stage on the same operands", dg, Dg_o, mabs=MAX_ABS * 50)
+
+
+def test_fp16_operand_overflow_is_reported(cuda_ok):
+    """A query-latent gain of 1e5 pushes q^C past the fp16 range: the values saturate at
+    +-65504, the output stays finite, and the device error word reports site 0x701."""
+    T = 64
+    shape = synth.GdlaShape()
+    inp = synth.make_prefill_inputs(shape, 1, T, seed=14)
+    from differential_latent_attention_fwd_b200.layer import GdlaLayer
+    gq = (torch.ones(shape.q_rank) * 1e5).bfloat16()
+    layer = GdlaLayer(shape, inp.weights, gq, inp.g_kv, device="cuda")
+    y = layer.prefill(inp.x.cuda())
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0x701
+    assert bool(torch.isfinite(y).all())
+    qq = ws_view(layer._ws, layer.cfg, 1, T, 0, WS_QQ, torch.float16, (T, shape.n_heads * shape.d_qk))
+    assert float(qq.float().abs().max()) == 65504.0
+    # the next call with ordinary gains reports nothing
+    layer2 = GdlaLayer(shape, inp.weights, inp.g_q, inp.g_kv, device="cuda")
+    layer2.prefill(inp.x.cuda())
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
