@@ -24,7 +24,8 @@ GDLA_MODE_CONTEXT = 3
 GDLA_MODE_HOST = 4
 STATUS = {0: "GDLA_OK", -1: "GDLA_ERR_INVALID_ARG", -2: "GDLA_ERR_UNSUPPORTED_SHAPE",
           -3: "GDLA_ERR_WORKSPACE_TOO_SMALL", -4: "GDLA_ERR_LAUNCH",
-          -5: "GDLA_ERR_DEVICE_TIMEOUT", -6: "GDLA_ERR_CUDA"}
+          -5: "GDLA_ERR_DEVICE_TIMEOUT", -6: "GDLA_ERR_CUDA",
+          -7: "GDLA_ERR_DEVICE_DATA"}
 
 
 class GdlaError(RuntimeError):
@@ -292,7 +293,7 @@ def gdla_decode_multi_fwd(cfg, absorbed: gdla_absorbed_t, x_new: torch.Tensor, k
 def gdla_device_error(stream=None, clear: bool = True) -> int:
     site = ctypes.c_int(0)
     rc = lib().gdla_device_error(_stream(stream), ctypes.byref(site), int(clear))
-    if rc not in (0, -5):
+    if rc not in (0, -5, -7):
         _check("gdla_device_error", rc)
     return site.value
 
@@ -304,7 +305,7 @@ def gdla_set_wait_limit_ns(ns: int) -> None:
 def gdla_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     site = ctypes.c_int(0)
     rc = lib().gdla_selftest_wait_timeout(int(limit_ns), _stream(stream), ctypes.byref(site))
-    if rc not in (0, -5):
+    if rc not in (0, -5, -7):
         _check("gdla_selftest_wait_timeout", rc)
     return site.value
 
@@ -322,7 +323,15 @@ def gdla_kernel_launches() -> int:
     return int(lib().gdla_kernel_launches())
 
 
-GDLA_NOALLOC_MAX_TOKENS = 4096
+def _header_define(name: str) -> int:
+    m = re.search(r"#define\s+" + name + r"\s+(\d+)", open(HEADER).read())
+    if not m:
+        raise RuntimeError(f"{name} is not defined in {HEADER}")
+    return int(m.group(1))
+
+
+# token limit of gdla_attn_prefill_noalloc's fixed scratch, as the header defines it
+GDLA_NOALLOC_MAX_TOKENS = _header_define("GDLA_NOALLOC_MAX_TOKENS")
 
 
 def gdla_attn_prefill_noalloc(cfg, qq: torch.Tensor, kv: torch.Tensor, kr16: torch.Tensor,

@@ -44,11 +44,12 @@ int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int 
 // q~ rows: qt[b][h][0..511] = W_UK_j q^C_h, qt[b][h][512..575] = rotated q^R_h (bf16).
 // CTA (KV head j, QT_RB rows b): W_UK_j^T (128 x 512 bf16, 128 KB) is staged in shared memory
 // with asynchronous copies, then the 5 QT_RB query rows of the group's heads are projected in
-// fp32.  Thread: latent columns 4 cq .. 4 cq + 3 of half of those rows.
+// fp32.  Thread tile: 10 query rows x 8 latent columns, so that one 16-byte load of weights and
+// one broadcast 16-byte load of q^C feed 40 FMAs (the kernel is FMA-bound, not load-bound).
 constexpr int QT_RB = 8;
 __global__ void __launch_bounds__(256) qtilde_kernel(DecQParams p) {
   constexpr int NR = 5 * QT_RB;                // query rows of a CTA
-  constexpr int HR = NR / 2;                   // rows per thread
+  constexpr int TR = NR / 4;                   // rows per thread (4 row groups)
   extern __shared__ uint8_t qt_smem[];
   __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(qt_smem);              // [128][512]
   float (*qc)[128] = reinterpret_cast<float (*)[128]>(qt_smem + 128 * 512 * 2);  // [NR][128]
@@ -57,43 +58,51 @@ __global__ void __launch_bounds__(256) qtilde_kernel(DecQParams p) {
   const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_UKt) + (long long)j * 128 * 512;
   for (int i = tid; i < 128 * 512 / 8; i += blockDim.x) cp_async16(wsm + i * 8, W + i * 8);
   const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
-  for (int i = tid; i < NR * 128; i += blockDim.x) {
-    const int r = i / 128, c = i % 128, bb = r / 5, hh = r % 5;
-    qc[r][c] = bb < nb ? p.QQ[(long long)(b0 + bb) * p.qq_ld + heads[hh] * 128 + c] : 0.f;
+  for (int i = tid; i < NR * 32; i += blockDim.x) {
+    const int r = i / 32, c4 = i % 32, bb = r / 5, hh = r % 5;
+    *reinterpret_cast<float4*>(&qc[r][4 * c4]) =
+        bb < nb ? *reinterpret_cast<const float4*>(p.QQ + (long long)(b0 + bb) * p.qq_ld + heads[hh] * 128 + 4 * c4)
+                : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   cp_async_wait_all();
   __syncthreads();
-  const int cq = tid & 127, r0 = (tid >> 7) * HR;
-  float acc[HR][4];
+  const int cg = tid & 63, rg = tid >> 6;      // latent columns 8 cg .. 8 cg + 7; rows rg, rg + 4, ...
+  float acc[TR][8];
 #pragma unroll
-  for (int r = 0; r < HR; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+  for (int r = 0; r < TR; ++r)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
 #pragma unroll 1
   for (int c = 0; c < 128; c += 4) {
-    float w[4][4];
+    float w[4][8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const uint2 wv = *reinterpret_cast<const uint2*>(wsm + (c + k) * 512 + 4 * cq);
-      const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.x));
-      const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.y));
-      w[k][0] = w01.x; w[k][1] = w01.y; w[k][2] = w23.x; w[k][3] = w23.y;
+      const uint4 wv = *reinterpret_cast<const uint4*>(wsm + (c + k) * 512 + 8 * cg);
+      const uint32_t u[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w[k][2 * e] = __uint_as_float(u[e] << 16);
+        w[k][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      }
     }
 #pragma unroll
-    for (int r = 0; r < HR; ++r) {
-      const float4 q4 = *reinterpret_cast<const float4*>(&qc[r0 + r][c]);
+    for (int r = 0; r < TR; ++r) {
+      const float4 q4 = *reinterpret_cast<const float4*>(&qc[rg + 4 * r][c]);
       const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(qv[k], w[k][e], acc[r][e]);
+        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(qv[k], w[k][e], acc[r][e]);
     }
   }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.qt);
 #pragma unroll
-  for (int r = 0; r < HR; ++r) {
-    const int bb = (r0 + r) / 5, hh = (r0 + r) % 5;
+  for (int r = 0; r < TR; ++r) {
+    const int row = rg + 4 * r, bb = row / 5, hh = row % 5;
     if (bb >= nb) continue;
-    *reinterpret_cast<uint2*>(out + ((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 4 * cq) =
-        make_uint2(pack_bf162(acc[r][0], acc[r][1]), pack_bf162(acc[r][2], acc[r][3]));
+    *reinterpret_cast<uint4*>(out + ((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 8 * cg) =
+        make_uint4(pack_bf162(acc[r][0], acc[r][1]), pack_bf162(acc[r][2], acc[r][3]),
+                   pack_bf162(acc[r][4], acc[r][5]), pack_bf162(acc[r][6], acc[r][7]));
   }
   for (int i = tid; i < NR * 64; i += blockDim.x) {
     const int r = i / 64, e = i % 64, bb = r / 5, hh = r % 5;
@@ -230,44 +239,52 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
   }
   cp_async_wait_all();
   __syncthreads();
-  const int cq = tid & 31;          // columns 4 cq .. 4 cq + 3
-  const int r0 = (tid >> 5) * 4;    // rows r0 .. r0 + 3 of the 4 CB latent differentials
-  float acc[4][4];
+  // D = Dlat W_UV_j: thread tile 2 rows x 8 columns (one 16-byte weight load and one broadcast
+  // 16-byte row load per 4 x 8 FMAs)
+  const int cg = tid & 15;          // columns 8 cg .. 8 cg + 7
+  const int r0 = (tid >> 4) * 2;    // rows r0, r0 + 1 of the 4 CB latent differentials
+  float acc[2][8];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
 #pragma unroll 1
   for (int l = 0; l < 512; l += 4) {
-    float w[4][4];
+    float w[4][8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const uint2 wv = *reinterpret_cast<const uint2*>(wsm + (l + k) * 128 + 4 * cq);
-      const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.x));
-      const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.y));
-      w[k][0] = w01.x; w[k][1] = w01.y; w[k][2] = w23.x; w[k][3] = w23.y;
+      const uint4 wv = *reinterpret_cast<const uint4*>(wsm + (l + k) * 128 + 8 * cg);
+      const uint32_t u[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w[k][2 * e] = __uint_as_float(u[e] << 16);
+        w[k][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      }
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < 2; ++r) {
       const float4 d4 = *reinterpret_cast<const float4*>(&dl[r0 + r][l]);
       const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(dv[k], w[k][e], acc[r][e]);
+        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(dv[k], w[k][e], acc[r][e]);
     }
   }
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
+  for (int r = 0; r < 2; ++r) {
     const int row = r0 + r;
     if (row >= 4 * nb) continue;
     const int b = b0 + row / 4, s = row % 4, sig = 4 * j + s;
-    const long long o = (long long)b * p.n_signal * 128 + sig * 128 + 4 * cq;
-    const uint2 gv = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.G) + o);
-    const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&gv.x);
-    const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&gv.y);
-    uint2 out;
-    out.x = pack_bf162(sigmoidf_fast(__low2float(g01)) * acc[r][0], sigmoidf_fast(__high2float(g01)) * acc[r][1]);
-    out.y = pack_bf162(sigmoidf_fast(__low2float(g23)) * acc[r][2], sigmoidf_fast(__high2float(g23)) * acc[r][3]);
-    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.Dg) + o) = out;
+    const long long o = (long long)b * p.n_signal * 128 + sig * 128 + 8 * cg;
+    const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.G) + o);
+    const uint32_t gu[4] = {gv.x, gv.y, gv.z, gv.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      out[e] = pack_bf162(sigmoidf_fast(__uint_as_float(gu[e] << 16)) * acc[r][2 * e],
+                          sigmoidf_fast(__uint_as_float(gu[e] & 0xFFFF0000u)) * acc[r][2 * e + 1]);
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Dg) + o) = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 

@@ -26,13 +26,14 @@
 // 32 w + 31: thread = head h = 32 w + lane for h < 80, thread = latent row for O^T), warp 4 TMA
 // producer, warp 5 TMEM owner + MMA issuer.  The tensor core runs S(J), PV(J - 1), S(J + 1),
 // PV(J), ...: the softmax of tile J (read S, maximum, exponentials, P) overlaps PV(J - 1) and
-// S(J + 1), so the tensor core does not wait for it.  The single S buffer is released as soon
-// as the softmax has read it into registers; the single P buffer is written once PV(J - 1) is
-// done; the ring holds tiles J - 1 and J plus one slot of J + 1.  The issuer steps through
-// precomputed descriptor words: at these shapes an MMA costs ~50-75 cycles, and rebuilding
-// 64-bit descriptors per MMA had made the issue loop, not the tensor core, the bound.  The
-// producer also prefetches the tile three ahead into L2, so that the ring only has to cover L2
-// latency.
+// S(J + 1), so the tensor core never waits for it.  The single S buffer is released as soon as
+// the softmax has read it into registers; the single P buffer is written once PV(J - 1) is done;
+// the ring holds tiles J - 1 and J plus one slot of J + 1.  The issuer steps through
+// precomputed descriptor words (rebuilding 64-bit descriptors per MMA had made the issue loop,
+// not the tensor core, the bound).  What bounds the kernel now: a tile's slots are held from its
+// S to its PV, about two tile periods in this order, so the ring's 2.25 tiles leave the loads of
+// tile J + 2 (issued as PV(J) frees tile J's slots) about one PV of lead against a load latency
+// of ~2300 cycles; the S MMAs of tile J + 2 wait for its last units.
 // The running maximum m_h moves only when a score exceeds it by more than 2^8 (O^T and l_h are
 // then rescaled), which is exact after the final division.  Rows of the last tile beyond the
 // row's last key are zeroed in shared memory before the PV, so that a cache tail the caller
@@ -59,7 +60,8 @@ constexpr int BAR_OFF = ROPE_OFF + NROPE * ROPE_SLOT;
 constexpr int SMEM = BAR_OFF + 1024 + 1024;    // barriers + alignment slack
 constexpr int QT_COL = 0, S_COL = 128, O_COL = 192;   // TMEM columns
 constexpr float RESCALE_THRESHOLD = 8.0f;
-constexpr int PREFETCH_AHEAD = 3;               // tiles of L2 prefetch ahead of the TMA loads
+constexpr int PREFETCH_AHEAD = 0;               // tiles of L2 prefetch ahead of the TMA loads (0: none;
+                                                // measured no faster at 3, slower at 6 and 12)
 static_assert(SMEM <= 232448, "shared memory");
 // The M = 128 score MMA reads 128 rows of each 80-row q~ box: the 48 rows past a box are the
 // next box, or (for the last box) the first 6 KB of P.  They only feed unused score rows.
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(192, 1)
         };
         for (int jj = 0; jj < PREFETCH_AHEAD && jj < n_tiles; ++jj) prefetch(jj);
         for (int j = 0; j < n_tiles && ok; ++j, ++J) {
-          if (j + PREFETCH_AHEAD < n_tiles) prefetch(j + PREFETCH_AHEAD);
+          if (PREFETCH_AHEAD > 0 && j + PREFETCH_AHEAD < n_tiles) prefetch(j + PREFETCH_AHEAD);
           const int y = int(crow0 + (long long)(sg.tile0 + j) * TP);
           for (int u = 0; u < 4 && ok; ++u) {
             const int gl = 4 * J + u, s = gl % NLAT;

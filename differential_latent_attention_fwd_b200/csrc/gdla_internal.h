@@ -36,6 +36,7 @@ struct GemmEpi {
   // internal: set by launch_gemm for the split-K pass (raw fp32 partial tiles)
   float* partial_out;
   int kb_per_split;
+  int* err;              // internal: device error word (fp16 outputs out of range are reported)
 };
 
 // Number of K splits launch_gemm uses for an M x N x K product (1 = no split).
@@ -146,7 +147,8 @@ size_t attn_bwd_workspace_bytes(long long M, int T, int n_heads, int n_groups);
 int launch_attn_bwd(const AttnBwdParams& a, cudaStream_t st);
 
 // Rotated k^R of bf16 latent rows (columns kv_rank .. kv_rank + 63) -> fp16 rows of 64.
-int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void* kR16, cudaStream_t st);
+int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void* kR16, int* err,
+                          cudaStream_t st);
 int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* kR16,
                         const AttnParams& p, KernelCtlHost ctl, cudaStream_t st);
 

@@ -87,8 +87,10 @@ __device__ __forceinline__ void gemm_epilogue_row(uint32_t t_row, int row, int n
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = pack_bf162(v[2 * i], v[2 * i + 1]);
       } else {
+        bool bad = false;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_half2(v[2 * i], v[2 * i + 1]);
+        for (int i = 0; i < 32; ++i) pk[i] = pack_half2_sat(v[2 * i], v[2 * i + 1], bad);
+        if (bad && ep.err) atomicCAS(ep.err, 0, SITE_FP16_RANGE);
       }
       uint16_t* dst = reinterpret_cast<uint16_t*>(ep.C) + (long long)row * ep.ldc + col;
       if (ncols == 64) {
@@ -374,8 +376,10 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
     reinterpret_cast<__nv_bfloat16*>(ep.C)[o + c1] = __float2bfloat16_rn(a);
     reinterpret_cast<__nv_bfloat16*>(ep.C)[o + c2] = __float2bfloat16_rn(b);
   } else {
-    reinterpret_cast<__half*>(ep.C)[o + c1] = __float2half_rn(a);
-    reinterpret_cast<__half*>(ep.C)[o + c2] = __float2half_rn(b);
+    bool bad = false;
+    reinterpret_cast<__half*>(ep.C)[o + c1] = half_sat(a, bad);
+    reinterpret_cast<__half*>(ep.C)[o + c2] = half_sat(b, bad);
+    if (bad && ep.err) atomicCAS(ep.err, 0, SITE_FP16_RANGE);
   }
 }
 
@@ -484,6 +488,7 @@ int launch_gemm(const void* A, long long lda, const void* B, long long ldb, bool
   if (K <= 0 || K % 64 != 0) return -1;
   const int BN = gemm_bn(N);
   GemmEpi ep = ep_in;
+  ep.err = ctl.err;
   ep.partial_out = nullptr;
   ep.kb_per_split = 0;
   int splits = 1;

@@ -27,18 +27,52 @@ static __device__ __align__(256) float g_noalloc_scratch[kScratchFloats];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
+// Per device: the context the address was looked up in, and the address.  A device reset (or
+// any teardown of the primary context) gives the device a new context with a new ID, and the
+// next call looks the address up again instead of using a pointer into the old context.
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 float* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once per device.
-// In host code g_noalloc_scratch names a host-side shadow, never the device memory itself.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique ID (for the process's life) of the calling thread's current context; 0 if unknown.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device.  It is looked up once per device
+// (and again after the device's context was recreated), with that device current.  In host code
+// g_noalloc_scratch names a host-side shadow, never the device memory itself.
 int scratch_on_current_device(float** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDLA_ERR_CUDA;
+  // (no current context yet: ID 0, and the lookup below creates the device's primary context)
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || ctx == 0 || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDLA_ERR_CUDA;
     g_scratch_ptr[dev] = static_cast<float*>(p);
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return GDLA_OK;

@@ -110,8 +110,10 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(const __grid_constant__ 
     dst[p.kv_rank + lane + 32] = __float2bfloat16_rn(k2);
   }
   if (kR16) {
-    kR16[(long long)m * 64 + lane] = __float2half_rn(k1);
-    kR16[(long long)m * 64 + lane + 32] = __float2half_rn(k2);
+    bool bad = false;
+    kR16[(long long)m * 64 + lane] = half_sat(k1, bad);
+    kR16[(long long)m * 64 + lane + 32] = half_sat(k2, bad);
+    if (bad && p.err) atomicCAS(p.err, 0, SITE_FP16_RANGE);
   }
 
   // ---- lambda
@@ -122,18 +124,21 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(const __grid_constant__ 
 
 // fp16 copy of the rotated k^R of bf16 latent rows (a key prefix handed in by the caller)
 __global__ void latent_to_kr16_kernel(const __nv_bfloat16* __restrict__ latent, int row_w,
-                                      int kv_rank, long long rows, __half* __restrict__ kR16) {
+                                      int kv_rank, long long rows, __half* __restrict__ kR16, int* err) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= rows * 64) return;
   const long long m = i >> 6;
-  kR16[i] = __float2half_rn(__bfloat162float(latent[m * row_w + kv_rank + (i & 63)]));
+  bool bad = false;
+  kR16[i] = half_sat(__bfloat162float(latent[m * row_w + kv_rank + (i & 63)]), bad);
+  if (bad && err) atomicCAS(err, 0, SITE_FP16_RANGE);
 }
 
-int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void* kR16, cudaStream_t st) {
+int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void* kR16, int* err,
+                          cudaStream_t st) {
   if (rows <= 0) return 0;
   const long long n = rows * 64;
   latent_to_kr16_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(latent), kv_rank + 64, kv_rank, rows, static_cast<__half*>(kR16));
+      static_cast<const __nv_bfloat16*>(latent), kv_rank + 64, kv_rank, rows, static_cast<__half*>(kR16), err);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 

@@ -57,7 +57,8 @@ typedef enum {
   GDLA_ERR_WORKSPACE_TOO_SMALL = -3,
   GDLA_ERR_LAUNCH = -4,             /* a kernel launch or tensor-map encode failed */
   GDLA_ERR_DEVICE_TIMEOUT = -5,     /* a bounded in-kernel wait expired (see gdla_device_error) */
-  GDLA_ERR_CUDA = -6                /* a CUDA runtime call failed */
+  GDLA_ERR_CUDA = -6,               /* a CUDA runtime call failed */
+  GDLA_ERR_DEVICE_DATA = -7         /* a kernel met bad input data (see gdla_device_error) */
 } gdla_status_t;
 
 /* Layer shape.  window: 0 = full causal attention, W > 0 = sliding window of W keys. */
@@ -248,8 +249,13 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* absor
                           void* stream);
 
 /* Reads (and with clear != 0 resets) the device error word after synchronising `stream`:
- * *site = 0 when every kernel finished normally, else the site code of the first bounded wait
- * that expired.  Returns GDLA_OK, or GDLA_ERR_DEVICE_TIMEOUT when *site != 0. */
+ * *site = 0 when every kernel finished normally, else the site code of the first problem:
+ *   0x1xx-0x5xx  a bounded wait expired (GDLA_ERR_DEVICE_TIMEOUT);
+ *   0x601        a cache_len entry outside [0, cap - q_len]: that sequence read and wrote nothing;
+ *   0x602        cu_seqlens not 0 .. total and non-decreasing: the bad documents were skipped;
+ *   0x701        an fp16 attention operand (q, K^C, V, k^R) was beyond +-65504 and was saturated
+ *                there, or was NaN (0x6xx and 0x7xx return GDLA_ERR_DEVICE_DATA).
+ * Returns GDLA_OK when *site == 0. */
 int gdla_device_error(void* stream, int* site, int clear);
 
 /* Bound of one in-kernel wait, in nanoseconds (default 2e9).  Values < 1000 are clamped. */
@@ -298,8 +304,9 @@ unsigned long long gdla_kernel_launches(void);
  * (the same tensors gdla_prefill_fwd keeps in its workspace, slots 4, 6, 9, 3, 5 and 8 of
  * gdla_workspace_offset).  B*T must not exceed GDLA_NOALLOC_MAX_TOKENS, else
  * GDLA_ERR_WORKSPACE_TOO_SMALL.  The first call on each device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first call before any
- * stream capture.  All calls share the one array: calls that overlap on the GPU (other
+ * address (cudaGetSymbolAddress) with that device current, and so does the first call after
+ * the device's context was recreated (cudaDeviceReset); make those calls before any stream
+ * capture.  All calls share the one array: calls that overlap on the GPU (other
  * streams, other threads) race and must be serialised by the caller. */
 #define GDLA_NOALLOC_MAX_TOKENS 4096
 int gdla_attn_prefill_noalloc(const gdla_config_t* cfg, const void* qq, const void* kv,
