@@ -426,9 +426,10 @@ def run_gpu(args):
                "bwd_flop": bwd_flop, "bwd_tflops": bwd_flop / (statistics.median(tb_ms) * 1e-3) / 1e12,
                "bwd_frac_of_bf16_peak": bwd_flop / (statistics.median(tb_ms) * 1e-3) / 1e12
                / load_peaks()[0]["bf16_tflops_sustained"],
-               "method": "per 512-query block: strided-batched cuBLAS GEMMs (fp16, fp32 accumulate) for S, dP, "
-                         "dq, dK, dV on gathered 192-wide q and k rows; own kernels for P and dS' (one pass), "
-                         "dH/Delta/dlambda/dG, gathers and scatters"}
+               "method": "tcgen05 kernels (fp16 operands, fp32 accumulators in TMEM): keys-stationary dK/dV "
+                         "per (KV group, 128 keys) over 64-query tiles x 5 heads, queries-stationary dq per "
+                         "(head, 128 queries) over 64-key tiles; P recomputed from the saved log-sum-exp; "
+                         "plus dH/Delta/dlambda/dG, gathers and the dk^R sum"}
         del wsb, grads, h_t
 
     peaks, peak_src = load_peaks()

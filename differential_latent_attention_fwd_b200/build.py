@@ -6,7 +6,6 @@ from __future__ import annotations
 
 import glob
 import os
-import shutil
 import subprocess
 import sys
 
@@ -35,10 +34,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + ".tmp"
-    # cuBLAS serves the plain GEMMs of the attention backward (found next to nvcc at run time too)
-    cuda_lib = os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(shutil.which(nvcc) or nvcc))), "lib64")
-    cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(HERE, "..", "include"), "-o", tmp, *sources(),
-           "-lcublas", "-Xlinker", "-rpath", "-Xlinker", cuda_lib]
+    cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(HERE, "..", "include"), "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)

@@ -687,9 +687,15 @@ int gdla_attn_bwd(const gdla_config_t* cfg, const void* qq, const void* kv, cons
   a.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
   a.QQ = qq; a.KV = kv; a.kR16 = kr16; a.lam = lam; a.G = gate; a.H = h; a.lse = lse; a.d_dg = d_dg;
   a.d_qq = d_qq; a.d_kv = d_kv; a.d_kr = d_kr; a.d_lam = d_lam; a.d_G = d_gate; a.ws = workspace;
-  rc = launch_attn_bwd(a, static_cast<cudaStream_t>(stream));
-  if (rc == 0) return GDLA_OK;
-  return rc == -6 ? GDLA_ERR_CUDA : GDLA_ERR_LAUNCH;
+  int* err;
+  if ((rc = error_word(&err))) return rc;
+  KernelCtlHost ctl{err, g_wait_limit_ns};
+  rc = launch_attn_bwd(a, ctl, static_cast<cudaStream_t>(stream));
+  if (rc == 0) {
+    g_launches += 6;   // pre-pass, two gathers, dK/dV, dq, dk^R reduce
+    return GDLA_OK;
+  }
+  return GDLA_ERR_LAUNCH;
 }
 
 int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void* dst,

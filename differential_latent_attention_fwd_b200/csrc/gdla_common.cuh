@@ -31,6 +31,7 @@ enum : int {
   SITE_ATTN_PRODUCER = 0x201, SITE_ATTN_MMA = 0x202, SITE_ATTN_SOFTMAX = 0x203,
   SITE_DRAIN = 0x301, SITE_SELFTEST = 0x401,
   SITE_DEC_PRODUCER = 0x501, SITE_DEC_MMA = 0x502, SITE_DEC_SOFTMAX = 0x503,
+  SITE_BWD_PRODUCER = 0x511, SITE_BWD_MMA = 0x512, SITE_BWD_SOFTMAX = 0x513,
   SITE_BAD_CACHE_LEN = 0x601,  // a cache_len entry outside [0, cap): that sequence is skipped
   SITE_BAD_CU_SEQLENS = 0x602, // document offsets not 0..total non-decreasing: bad documents skipped
   SITE_FP16_RANGE = 0x701,     // an fp16 attention operand was outside +-65504 (saturated) or NaN
@@ -420,6 +421,19 @@ __device__ __forceinline__ void ffma2v(float& d0, float& d1, float a0, float a1,
   asm("{\n\t.reg .b64 d, a, b, c;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %6};\n\t"
       "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
       : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c));
+}
+// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1)
+__device__ __forceinline__ void ffma2vv(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                        float c1) {
+  asm("{\n\t.reg .b64 d, a, b, c;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+// (d0, d1) = (a0, a1) * (b0, b1)
+__device__ __forceinline__ void fmul2v(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 d, a, b;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 // (x0, x1) = (a0, a1) * b + c
 __device__ __forceinline__ void ffma2(float& x0, float& x1, float a0, float a1, float b, float c) {

@@ -123,8 +123,7 @@ struct AttnParams {
 int launch_varlen_schedule(const int* cu_seqlens, int n_docs, int total, int* positions,
                            int4* units, int* n_units, int max_units, int* cnt, int* fill, int max_c,
                            int* err, cudaStream_t st);
-// Backward of the attention stage (attn_backward.cu): query rows per block.
-constexpr int ATTN_BWD_BQ = 512;
+// Backward of the attention stage (attn_backward.cu).
 struct AttnBwdParams {
   int B, T, window, n_signal, n_groups;
   float scale_log2, scale;    // log2(e) / sqrt(d_qk), 1 / sqrt(d_qk)
@@ -144,7 +143,7 @@ struct AttnBwdParams {
   void* ws;                   // attn_bwd_workspace_bytes(...)
 };
 size_t attn_bwd_workspace_bytes(long long M, int T, int n_heads, int n_groups);
-int launch_attn_bwd(const AttnBwdParams& a, cudaStream_t st);
+int launch_attn_bwd(const AttnBwdParams& a, const KernelCtlHost& ctl, cudaStream_t st);
 
 // Rotated k^R of bf16 latent rows (columns kv_rank .. kv_rank + 63) -> fp16 rows of 64.
 int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void* kR16, int* err,

@@ -204,11 +204,12 @@ int gdla_attn_train_fwd(const gdla_config_t* cfg, const void* qq, const void* kv
  * tensors saved by gdla_attn_train_fwd, the fp32 gradients dL/d of qq (d_qq, same layout),
  * kv (d_kv), kr16 (d_kr), lam (d_lam, with respect to lambda itself) and gate (d_gate, with
  * respect to the logits).  The softmax probabilities are recomputed from the scores and the
- * saved log-sum-exp; the contractions are strided-batched cuBLAS GEMMs (fp16 operands, fp32
- * accumulation) over blocks of 512 query rows, with queries and keys gathered into 192-wide
- * [nope | rope] rows so that the scores, dq and dk are one contraction each; the library's
- * cuBLAS handle is created once per device and uses only the caller's workspace as its GEMM
- * workspace. */
+ * saved log-sum-exp.  Every contraction runs in the library's tensor-core kernels (fp16
+ * operands, fp32 accumulation in tensor memory): one keys-stationary kernel forms dK and dV
+ * per (sequence, KV group, 128 keys), one queries-stationary kernel forms dq per (sequence,
+ * head, 128 queries); queries and keys are first gathered into 192-wide [nope | rope] rows.
+ * Nothing is allocated; the workspace holds the gathered rows, dH, Delta and the per-group dk.
+ * A bounded wait that expires is reported by gdla_device_error (sites 0x511-0x513). */
 int gdla_attn_bwd(const gdla_config_t* cfg, const void* qq, const void* kv, const void* kr16,
                   const float* lam, const void* gate, const void* h, const float* lse,
                   const void* d_dg, int B, int T, float* d_qq, float* d_kv, float* d_kr,

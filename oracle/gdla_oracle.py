@@ -467,6 +467,84 @@ def attention_stage_backward(qC, qR, KC, V, kR, lam, G, dDg, cfg: OracleConfig):
     return out
 
 
+def attention_stage_backward_group(qC, qR, KC, V, kR, lam, G, dDg, cfg: OracleConfig, j: int,
+                                   q_rows, k_rows, block: int = 512):
+    """The part of attention_stage_backward that belongs to KV group j, at chosen rows.
+
+    Returns dq^C, dq^R of the group's heads (its noise head and the signal heads that subtract
+    it) at query rows q_rows; dK^C_j and dV_j at key rows k_rows; dlambda and dG of those signal
+    heads at q_rows.  Same chain rule as attention_stage_backward; every query row's softmax
+    statistics (the normaliser and H) are formed exactly, one block of rows at a time, so that
+    long sequences need O(T^2) work for one group only.  Keys: dict with arrays "dqC" [len(q_rows),
+    heads, d_nope], "dqR", "dKC" [len(k_rows), d_nope], "dV", "dlam" [len(q_rows), signals], "dG",
+    and the head order "heads" (noise head first) and "signals".
+    """
+    T = qC.shape[0]
+    scale = 1.0 / np.sqrt(cfg.d_nope + cfg.d_rope)
+    nmap = noise_of_signal(cfg)
+    signals = [s for s in range(cfg.n_signal) if nmap[s] == j]
+    heads = [cfg.n_signal + j] + signals
+    k = np.concatenate([KC[:, j], kR], -1)              # [T, 192]
+    v = V[:, j]                                          # [T, d_v]
+    # dH of every row needs only that row's inputs
+    g = sigmoid(G[:, signals])
+    dHS = dDg[:, signals] * g
+    dH = {cfg.n_signal + j: -np.einsum("ts,tsc->tc", lam[:, signals], dHS)}
+    for i, s_ in enumerate(signals):
+        dH[s_] = dHS[:, i]
+    # forward statistics of the group's heads over all query rows
+    logZ = {h: np.empty(T) for h in heads}
+    Hh = {h: np.empty((T, cfg.d_v)) for h in heads}
+    tt = np.arange(T)
+    for r0 in range(0, T, block):
+        r1 = min(T, r0 + block)
+        rows = tt[r0:r1]
+        lo = np.array([key_range(int(t), cfg.window)[0] for t in rows])
+        allowed = (tt[None, :] <= rows[:, None]) & (tt[None, :] >= lo[:, None])
+        for h in heads:
+            q = np.concatenate([qC[r0:r1, h], qR[r0:r1, h]], -1)
+            sc = np.where(allowed, (q @ k.T) * scale, -np.inf)
+            m = sc.max(-1, keepdims=True)
+            e = np.exp(sc - m)
+            z = e.sum(-1, keepdims=True)
+            logZ[h][r0:r1] = (m + np.log(z))[:, 0]
+            Hh[h][r0:r1] = (e / z) @ v
+    delta = {h: np.einsum("tc,tc->t", dH[h], Hh[h]) for h in heads}
+    out = {"heads": heads, "signals": signals}
+    # key rows: dV_j[s] = sum_h sum_t P_h[t, s] dH_h[t];  dK_j[s] = scale sum_h sum_t dS_h[t, s] q_h[t]
+    dKC = np.zeros((len(k_rows), cfg.d_nope))
+    dVk = np.zeros((len(k_rows), cfg.d_v))
+    for i, s in enumerate(k_rows):
+        vis = np.array([key_range(int(t), cfg.window)[0] <= s <= t for t in range(T)])
+        for h in heads:
+            q = np.concatenate([qC[:, h], qR[:, h]], -1)
+            p = np.where(vis, np.exp((q @ k[s]) * scale - logZ[h]), 0.0)
+            dVk[i] += p @ dH[h]
+            ds = p * (dH[h] @ v[s] - delta[h])
+            dKC[i] += scale * (ds @ q)[: cfg.d_nope]
+    out["dKC"], out["dV"] = dKC, dVk
+    # query rows: dq_h[t] = scale sum_s dS_h[t, s] k[s]; dlambda, dG from H_S, H_N of row t
+    dqC = np.zeros((len(q_rows), len(heads), cfg.d_nope))
+    dqR = np.zeros((len(q_rows), len(heads), cfg.d_rope))
+    dlam = np.zeros((len(q_rows), len(signals)))
+    dG = np.zeros((len(q_rows), len(signals), cfg.d_v))
+    for i, t in enumerate(q_rows):
+        lo, hi = key_range(int(t), cfg.window)
+        for a, h in enumerate(heads):
+            q = np.concatenate([qC[t, h], qR[t, h]])
+            p = np.exp((k[lo: hi + 1] @ q) * scale - logZ[h][t])
+            ds = p * (v[lo: hi + 1] @ dH[h][t] - delta[h][t])
+            dq = scale * (ds @ k[lo: hi + 1])
+            dqC[i, a], dqR[i, a] = dq[: cfg.d_nope], dq[cfg.d_nope:]
+        HN = Hh[cfg.n_signal + j][t]
+        for b_, s_ in enumerate(signals):
+            dlam[i, b_] = -dHS[t, b_] @ HN
+            gs = sigmoid(G[t, s_])
+            dG[i, b_] = dDg[t, s_] * gs * (1.0 - gs) * (Hh[s_][t] - lam[t, s_] * HN)
+    out.update(dqC=dqC, dqR=dqR, dlam=dlam, dG=dG)
+    return out
+
+
 def gdla_prefill_packed(x_packed, cu_seqlens, weights: dict, cfg: OracleConfig, g_q=None, g_kv=None):
     """Packed documents: document d = rows cu[d] .. cu[d+1]-1 of x_packed [total, d_model] is an
     independent sequence (its own positions from 0, attention inside the document only).

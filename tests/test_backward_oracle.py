@@ -53,3 +53,22 @@ def test_backward_of_first_row_only_touches_key_zero():
     assert np.abs(g["dqC"][1:]).max() == 0
     # a single key: softmax is constant, so no gradient flows to q or K
     assert np.abs(g["dqC"][0]).max() < 1e-12 and np.abs(g["dKC"][0]).max() < 1e-12
+
+
+@pytest.mark.parametrize("window", [0, 5])
+def test_group_backward_equals_full_backward(window):
+    """The group-restricted gradient at chosen rows (used at long lengths) equals the full
+    oracle gradient's rows of that group, which the finite-difference test above pins."""
+    cfg, x, dDg = _inputs(window, T=23, seed=8)
+    full = O.attention_stage_backward(x["qC"], x["qR"], x["KC"], x["V"], x["kR"], x["lam"], x["G"], dDg, cfg)
+    q_rows, k_rows = [0, 4, 11, 22], [0, 3, 17, 22]
+    for j in range(cfg.n_kv_heads):
+        part = O.attention_stage_backward_group(x["qC"], x["qR"], x["KC"], x["V"], x["kR"], x["lam"], x["G"],
+                                                dDg, cfg, j, q_rows, k_rows, block=5)
+        heads, sig = part["heads"], part["signals"]
+        np.testing.assert_allclose(part["dqC"], full["dqC"][q_rows][:, heads], rtol=0, atol=1e-11)
+        np.testing.assert_allclose(part["dqR"], full["dqR"][q_rows][:, heads], rtol=0, atol=1e-11)
+        np.testing.assert_allclose(part["dKC"], full["dKC"][k_rows, j], rtol=0, atol=1e-11)
+        np.testing.assert_allclose(part["dV"], full["dV"][k_rows, j], rtol=0, atol=1e-11)
+        np.testing.assert_allclose(part["dlam"], full["dlam"][q_rows][:, sig], rtol=0, atol=1e-11)
+        np.testing.assert_allclose(part["dG"], full["dG"][q_rows][:, sig], rtol=0, atol=1e-11)

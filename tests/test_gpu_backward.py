@@ -82,3 +82,38 @@ def test_attention_backward_matches_oracle(cuda_ok, B, T, window):
         ]:
             check(f"b={b} {name}", got, want, rel=1e-2, mabs=np.abs(want).max() * 2e-2 + 1e-3, errors=errs)
     assert not errs, "\n".join(errs)
+
+
+@pytest.mark.parametrize("window", [0, 2048])
+def test_attention_backward_sampled_rows_t8192(cuda_ok, window):
+    """T = 8192 (128 key blocks of the dK/dV kernel, 64 query blocks of the dq kernel): the
+    gradients of KV group 5 (its noise head and four signal heads) at 48 sampled query rows and
+    48 sampled key rows against the oracle, which forms the group's softmax statistics over the
+    whole sequence."""
+    B, T, j = 1, 8192, 5
+    shape = synth.GdlaShape(window=window)
+    cfg = O.OracleConfig.from_shape(shape)
+    qq, kv, kr, lam, gate, d_dg = _stage_inputs(B, T, seed=77 + window)
+    dg, h, (d_qq, d_kv, d_kr, d_lam, d_gate) = _run_gpu(shape, B, T, qq, kv, kr, lam, gate, d_dg)
+    q_rows = synth.sample_rows(T, window, 48, seed=3)
+    k_rows = synth.sample_rows(T, window, 48, seed=4)
+    kvb = O.f64(kv).reshape(T, 16, 256)
+    part = O.attention_stage_backward_group(
+        O.f64(qq[:, : 80 * 128]).reshape(T, 80, 128), O.f64(qq[:, 80 * 128:]).reshape(T, 80, 64),
+        kvb[..., :128], kvb[..., 128:], O.f64(kr), O.f64(lam), O.f64(gate).reshape(T, 64, 128),
+        O.f64(d_dg).reshape(T, 64, 128), cfg, j, q_rows, k_rows)
+    heads, sig = part["heads"], part["signals"]
+    dqq = to_np(d_qq[q_rows]).reshape(len(q_rows), -1)
+    got_qC = dqq[:, : 80 * 128].reshape(-1, 80, 128)[:, heads]
+    got_qR = dqq[:, 80 * 128:].reshape(-1, 80, 64)[:, heads]
+    dkv = to_np(d_kv[k_rows]).reshape(len(k_rows), 16, 256)[:, j]
+    errs = []
+    for name, got, want in [
+        ("dq^C", got_qC, part["dqC"]), ("dq^R", got_qR, part["dqR"]),
+        ("dK^C", dkv[:, :128], part["dKC"]), ("dV", dkv[:, 128:], part["dV"]),
+        ("dlambda", to_np(d_lam[q_rows])[:, sig], part["dlam"]),
+        ("dG", to_np(d_gate[q_rows]).reshape(-1, 64, 128)[:, sig], part["dG"]),
+    ]:
+        check(f"T={T} W={window} group {j} {name}", got, want, rel=1e-2, mabs=np.abs(want).max() * 2e-2 + 1e-3,
+              errors=errs)
+    assert not errs, "\n".join(errs)
