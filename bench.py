@@ -28,7 +28,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "GDLA prefill TFLOP/s (% BF16 peak) at 32K; decode tok/s & KV GB/s vs HBM"
 PREFILL = dict(name="prefill_b1_t32768_causal", B=1, T=32768, window=0, seed=2)
-DECODE = dict(B=64, L=32768, cap=32769, seed=4, windows=(0, 2048))
+DECODE = dict(B=64, L=32768, seed=4, windows=(0, 2048), multi=(2, 3))
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -213,93 +213,99 @@ def run_gpu(args):
     ws = layer.workspace(B, T, gb.GDLA_MODE_PREFILL)
     windows = () if args.skip_decode else DECODE["windows"]
     dec_L = 1 if args.skip_decode else args.decode_L
-    dinp = synth.make_decode_inputs(synth.GdlaShape(), DECODE["B"], dec_L, dec_L + 1, DECODE["seed"])
+    qmax = max(DECODE["multi"])
+    # cache capacity: the cached positions plus room for up to qmax new tokens per sequence
+    dinp = synth.make_decode_inputs(synth.GdlaShape(), DECODE["B"], dec_L, dec_L + qmax, DECODE["seed"])
     cache = dinp.cache.to(dev)
     lens = dinp.cache_len.to(dev)
     x_new = dinp.x_new.to(dev)
     y_new = torch.empty_like(x_new)
+    multis = () if args.skip_decode else DECODE["multi"]
+    x_multi = {q: torch.randn((DECODE["B"], q, s.d_model), generator=torch.Generator().manual_seed(6 + q))
+               .bfloat16().to(dev) for q in multis}
+    y_multi = {q: torch.empty_like(x_multi[q]) for q in multis}
     absorbed = layer.absorbed()
     dcfg = {w: gb.make_config(s.with_window(w)) for w in (0, 2048)}
-    dws = torch.empty(max(gb.gdla_workspace_size(dcfg[w], DECODE["B"], cache.shape[1],
+    dws = torch.empty(max(gb.gdla_workspace_size(dcfg[w], DECODE["B"] * qmax, cache.shape[1],
                                                  gb.GDLA_MODE_DECODE) for w in (0, 2048)),
                       dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
     pev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-    dev_ev = {w: [torch.cuda.Event(enable_timing=True) for _ in range(5)] for w in windows}
+    dev_ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+              for k in ["c", "w2048", "c_q2", "c_q3"]}
 
     def prefill_once():
         gb.gdla_set_stage_events(pev)
         gb.gdla_prefill_fwd(layer.cfg, layer.cw, x, y, ws, stream=stream)
 
-    def decode_once(w, s=None):
-        gb.gdla_set_stage_events(dev_ev[w])
-        gb.gdla_decode_fwd(dcfg[w], absorbed, x_new, cache, lens, y_new, dws,
-                           stream=stream if s is None else s)
+    # A decode step is ~20 short kernels: it is replayed as a CUDA graph (one capture per
+    # configuration), as a serving loop runs it; the eager time is reported beside it.  Decode
+    # is timed as its own run of back-to-back replays (continuous decoding), not right after a
+    # prefill, whose power draw would leave the decode at the prefill's reduced clocks; the
+    # caches (2.4 GB causal, 151 MB for the 2048 window) exceed the 126 MB L2, so no flush.
+    dec_keys = [("c" if w == 0 else f"w{w}", w, 1) for w in windows] + [(f"c_q{q}", 0, q) for q in multis]
 
-    # A decode step is ~20 short kernels: it is replayed as a CUDA graph (one capture per mask),
-    # as a serving loop would run it; the eager time is reported beside it.
+    def decode_call(key, st):
+        _, w, q = next(d for d in dec_keys if d[0] == key)
+        if q == 1:
+            gb.gdla_decode_fwd(dcfg[w], absorbed, x_new, cache, lens, y_new, dws, stream=st)
+        else:
+            gb.gdla_decode_multi_fwd(dcfg[w], absorbed, x_multi[q], cache, lens, y_multi[q], dws, stream=st)
+
     graphs = {}
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_pairs = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(args.steps)] for k, _, _ in dec_keys}
 
-    def step():
-        rec = {"prefill_ms": 0.0, "attn_ms": float("nan"), "down_ms": 0.0, "norm_ms": 0.0,
-               "up_ms": 0.0, "out_ms": 0.0}
-        if not args.skip_prefill:
-            flush.fill_(1)
-            prefill_once()
-            torch.cuda.synchronize(dev)
-            rec = {"prefill_ms": pev[0].elapsed_time(pev[5]), "attn_ms": pev[3].elapsed_time(pev[4]),
-                   "down_ms": pev[0].elapsed_time(pev[1]), "norm_ms": pev[1].elapsed_time(pev[2]),
-                   "up_ms": pev[2].elapsed_time(pev[3]), "out_ms": pev[4].elapsed_time(pev[5])}
-        for w in windows:
-            flush.fill_(1)
-            if w in graphs:          # whole decode step as one graph: events around the replay
-                g0.record(stream)
-                graphs[w].replay()
-                g1.record(stream)
-                torch.cuda.synchronize(dev)
-                rec[f"dec{w}_ms"] = g0.elapsed_time(g1)
-            else:                    # eager call: per-stage events from inside the library
-                decode_once(w)
-                torch.cuda.synchronize(dev)
-                e = dev_ev[w]
-                rec[f"dec{w}_ms"] = e[0].elapsed_time(e[4])
-                rec[f"dec{w}_attn_ms"] = e[1].elapsed_time(e[2])
-                rec[f"dec{w}_q_ms"] = e[0].elapsed_time(e[1])
-                rec[f"dec{w}_comb_ms"] = e[2].elapsed_time(e[3])
-        return rec
+    def prefill_step():
+        flush.fill_(1)
+        prefill_once()
+        torch.cuda.synchronize(dev)
+        return {"prefill_ms": pev[0].elapsed_time(pev[5]), "attn_ms": pev[3].elapsed_time(pev[4]),
+                "down_ms": pev[0].elapsed_time(pev[1]), "norm_ms": pev[1].elapsed_time(pev[2]),
+                "up_ms": pev[2].elapsed_time(pev[3]), "out_ms": pev[4].elapsed_time(pev[5])}
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    def decode_run(key, n, record=True):
+        for i in range(n):
+            if record:
+                ev_pairs[key][i][0].record(stream)
+            graphs[key].replay()
+            if record:
+                ev_pairs[key][i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return [a.elapsed_time(b) for a, b in ev_pairs[key][:n]] if record else []
+
+    for _ in range(0 if args.skip_prefill else max(3, args.warmup)):
+        prefill_step()
     assert gb.gdla_device_error(stream) == 0, "device error during warm-up"
-    eager_dec = {w: [] for w in windows}
-    eager_stage = {w: {"attn": [], "q": [], "comb": []} for w in windows}
+    eager_dec = {k: [] for k, _, _ in dec_keys}
+    eager_stage = {k: {"attn": [], "q": [], "comb": []} for k, _, _ in dec_keys}
     kernels_per_decode = {}
     for _ in range(5):
-        for w in windows:
+        for k, _, _ in dec_keys:
             flush.fill_(1)
             n0 = gb.gdla_kernel_launches()
-            decode_once(w)
-            kernels_per_decode[w] = gb.gdla_kernel_launches() - n0
+            gb.gdla_set_stage_events(dev_ev[k])
+            decode_call(k, stream)
+            kernels_per_decode[k] = gb.gdla_kernel_launches() - n0
             torch.cuda.synchronize(dev)
-            e = dev_ev[w]
-            eager_dec[w].append(e[0].elapsed_time(e[4]))
-            eager_stage[w]["attn"].append(e[1].elapsed_time(e[2]))
-            eager_stage[w]["q"].append(e[0].elapsed_time(e[1]))
-            eager_stage[w]["comb"].append(e[2].elapsed_time(e[3]))
+            e = dev_ev[k]
+            eager_dec[k].append(e[0].elapsed_time(e[4]))
+            eager_stage[k]["attn"].append(e[1].elapsed_time(e[2]))
+            eager_stage[k]["q"].append(e[0].elapsed_time(e[1]))
+            eager_stage[k]["comb"].append(e[2].elapsed_time(e[3]))
     gb.gdla_set_stage_events([])     # no event nodes inside the captured graphs
-    for w in windows:
+    for k, _, _ in dec_keys:
         g = torch.cuda.CUDAGraph()
         cs = torch.cuda.Stream(dev)
         cs.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(cs):
             with torch.cuda.graph(g, stream=cs):
-                gb.gdla_decode_fwd(dcfg[w], absorbed, x_new, cache, lens, y_new, dws, stream=cs)
+                decode_call(k, cs)
         torch.cuda.current_stream(dev).wait_stream(cs)
-        graphs[w] = g
-    for _ in range(2):
-        step()
+        graphs[k] = g
+    for k, _, _ in dec_keys:
+        decode_run(k, max(3, args.warmup), record=False)
     torch.cuda.synchronize(dev)
     assert gb.gdla_device_error(stream) == 0, "device error in graph warm-up"
 
@@ -311,15 +317,29 @@ def run_gpu(args):
     barrier()
     launches0 = gb.gdla_kernel_launches()
     recs = []
+    dec_ms = {}
+    # decode first (its graph warm-up just ran: the GPU is in its decode state), then prefill;
+    # clocks are sampled over each part and over the whole timed region
     with ClockSampler(local) as clk:
-        for _ in range(args.steps):
-            recs.append(step())
-        barrier()
+        with ClockSampler(local) as clk_dec:
+            for k, _, _ in dec_keys:
+                dec_ms[k] = decode_run(k, args.steps)
+            barrier()
+        with ClockSampler(local) as clk_pre:
+            for _ in range(0 if args.skip_prefill else args.steps):
+                recs.append(prefill_step())
+            barrier()
     # graph replays launch the captured kernels without passing through the library's counter
     launches = gb.gdla_kernel_launches() - launches0 + args.steps * sum(kernels_per_decode.values())
     gb.gdla_set_stage_events([])
     site = gb.gdla_device_error(stream)
     assert site == 0, f"device error site {site:#x} in the timed region"
+    if not recs:
+        recs = [{"prefill_ms": 0.0, "attn_ms": float("nan"), "down_ms": 0.0, "norm_ms": 0.0, "up_ms": 0.0,
+                 "out_ms": 0.0}]
+    for r in recs:
+        for k in dec_ms:
+            r[f"dec_{k}_ms"] = statistics.mean(dec_ms[k])
 
     def mean(k):
         return statistics.mean(r[k] for r in recs)
@@ -444,22 +464,27 @@ def run_gpu(args):
     e2e_val = world * tflops(layer_flop, e2e_t.item())
 
     decode = {}
-    for w in windows:
-        keys_read = dec_L + 1 if w == 0 else min(w, dec_L + 1)
-        kv_bytes = DECODE["B"] * keys_read * s.latent_row * 2
-        t_att = statistics.median(eager_stage[w]["attn"]) * 1e-3
-        t_all = st[f"dec{w}_ms"] * 1e-3
-        decode["causal" if w == 0 else f"swa{w}"] = {
-            "B": DECODE["B"], "cache_len": dec_L, "window": w,
-            "tok_per_s": world * DECODE["B"] / t_all, "ms": st[f"dec{w}_ms"],
-            "timing": "CUDA graph replay of one gdla_decode_fwd call",
-            "ms_eager": statistics.median(eager_dec[w]),
-            "latent_attention_ms": statistics.median(eager_stage[w]["attn"]),
-            "query_path_ms": statistics.median(eager_stage[w]["q"]),
-            "combine_ms": statistics.median(eager_stage[w]["comb"]),
+    for k, w, q in dec_keys:
+        keys_read = dec_L + q if w == 0 else min(w, dec_L + q)
+        kv_bytes = DECODE["B"] * keys_read * s.latent_row * 2        # each sequence's rows, once
+        t_att = statistics.median(eager_stage[k]["attn"]) * 1e-3
+        t_all = st[f"dec_{k}_ms"] * 1e-3
+        name = ("causal" if w == 0 else f"swa{w}") + ("" if q == 1 else f"_q{q}")
+        decode[name] = {
+            "B": DECODE["B"], "cache_len": dec_L, "window": w, "q_len": q,
+            "tok_per_s": world * DECODE["B"] * q / t_all, "ms": st[f"dec_{k}_ms"],
+            "timing": f"{args.steps} back-to-back CUDA graph replays of one decode call (mean)",
+            "ms_eager": statistics.median(eager_dec[k]),
+            "latent_attention_ms": statistics.median(eager_stage[k]["attn"]),
+            "query_path_ms": statistics.median(eager_stage[k]["q"]),
+            "combine_ms": statistics.median(eager_stage[k]["comb"]),
             "kv_bytes": kv_bytes, "kv_gbs": kv_bytes / t_att / 1e9,
             "kv_frac_of_hbm": kv_bytes / t_att / 1e9 / peaks["hbm_gbs"],
         }
+        if q > 1:
+            decode[name]["kv_note"] = ("kv_bytes counts each sequence's cache rows once: the rows of its "
+                                       f"{q} new tokens are consecutive query rows, whose CTAs read the same "
+                                       "tiles at about the same time (shared in L2)")
 
     traffic = None
     tf_path = os.path.join(ROOT, "profiles", "attn_prefill_t32768_causal.traffic.json")
@@ -474,7 +499,7 @@ def run_gpu(args):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": st["prefill_ms"] + sum(
-            st[f"dec{w}_ms"] for w in windows),
+            st[f"dec_{k}_ms"] for k, _, q in dec_keys if q == 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": (f"prefill_b1_t{T}_causal" + ("" if args.skip_decode else
@@ -482,7 +507,7 @@ def run_gpu(args):
                    "B": B, "seq_len": T, "mask": "causal", "d_model": s.d_model,
                    "heads": f"{s.n_signal} signal + {s.n_noise} noise, {s.n_kv_heads} KV",
                    "attn_operands": "fp16 (q, K^C, V, k^R, P); projections bf16; fp32 accumulate",
-                   "l2": "flushed (256 MiB write) before every timed call",
+                   "l2": "flushed (256 MiB write) before every timed prefill call; decode caches exceed L2",
                    "parallelism": f"replicas x{world}"},
         "prefill": {"layer_ms": st["prefill_ms"], "attention_ms": st["attn_ms"],
                     "down_proj_ms": st["down_ms"], "norm_rope_ms": st["norm_ms"],
@@ -505,6 +530,8 @@ def run_gpu(args):
                 "d2h_bytes_per_step": y.numel() * 2, "ms": e2e_t.item()},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
+        "clocks_decode_part": clk_dec.summary(),
+        "clocks_prefill_part": clk_pre.summary(),
     }
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.skip_prefill:
