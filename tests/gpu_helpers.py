@@ -35,6 +35,7 @@ def check(name, got, want, rel=REL_L2, mabs=MAX_ABS, errors=None):
     r, m = rel_l2(got, want), max_abs(got, want)
     ok = finite and r <= rel and m <= mabs
     msg = f"{name}: rel_l2={r:.3e} (<= {rel:.1e}) max_abs={m:.3e} (<= {mabs:.1e}) finite={finite}"
+    print(msg)     # shown with pytest -s: the measured errors beside their bounds
     if errors is not None:
         if not ok:
             errors.append(msg)
