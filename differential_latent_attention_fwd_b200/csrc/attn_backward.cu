@@ -13,14 +13,16 @@
 // accumulators in TMEM), in two kernels that each own their outputs (no atomics):
 //  * keys stationary (dK, dV): one CTA per (sequence, KV group j, 128 keys) keeps K = [K^C_j |
 //    k^R] and V_j of its keys in shared memory and loops over 64-query tiles x the group's five
-//    heads: S^T = K q^T and dP^T = V dH^T into TMEM; the softmax threads (thread = key) turn
-//    them into P^T and dS'^T (fp16, packed into the S^T slot) which are the A operands of
+//    heads: S^T = K q^T and dP^T = V dH^T into TMEM; the elementwise threads (two per key, each
+//    taking 32 of the 64 queries) turn them into P^T and dS'^T (fp16, packed into the S^T slot,
+//    each thread over the columns it has read) which are the A operands of
 //    dV += P^T dH and dK += dS'^T q.  TMEM: three rotating 64-column slots | dV 128 | dK 192.
 //    Unit u puts S^T in slot u % 3 and dP^T in slot (u + 1) % 3; the dP^T slot is free as soon
 //    as the elementwise threads have read it, so the tensor core computes S^T / dP^T of unit
 //    u + 1 (and dV / dK of unit u - 1) while they work on unit u.
 //  * queries stationary (dq): one CTA per (sequence, head, 128 queries) keeps q and dH and loops
-//    over 64-key tiles: S = q K^T, dP = dH V^T, dS' in place (thread = query), dq += dS' K.
+//    over 64-key tiles: S = q K^T, dP = dH V^T, dS' in place (two threads per query, 32 keys
+//    each), dq += dS' K.
 //    TMEM: two (S 64 | dP 64) buffers | dq 192 columns, so that the scores of the next key tile
 //    are computed while the elementwise threads work on this one.
 // Both recompute P from the saved log-sum-exp; the second recomputes S and dP, which costs
@@ -47,7 +49,7 @@ constexpr int A_V_OFF = A_K_OFF + 3 * BOX_BIG;
 constexpr int A_RING = A_V_OFF + 2 * BOX_BIG;
 constexpr int STAGE = 5 * BOX_SMALL;
 constexpr int A_LD_OFF = A_RING + NST * STAGE;
-constexpr int A_BAR_OFF = A_LD_OFF + 4 * 128 * 4;
+constexpr int A_BAR_OFF = A_LD_OFF + 8 * 64 * 4;
 constexpr int A_SMEM = A_BAR_OFF + 256 + 1024;
 // dq kernel: q block (3 boxes) | dH block (2) | ring of (K tile 3 boxes + V tile 2 boxes)
 constexpr int B_Q_OFF = 0;
@@ -93,21 +95,21 @@ __device__ __forceinline__ bool bwd_visible(int t, int s, int T, int W) {
   return t < T && s <= t && (W <= 0 || t - s < W);
 }
 
-__device__ __forceinline__ void bwd_init_bars(BwdBars* bars) {
+__device__ __forceinline__ void bwd_init_bars(BwdBars* bars, uint32_t n_el_warps) {
   mbar_init(&bars->fixed_full, 1);
   for (int s = 0; s < bwd::NST; ++s) {
     mbar_init(&bars->full[s], 1);
     mbar_init(&bars->empty[s], 1);
   }
   mbar_init(&bars->s_full, 1);
-  mbar_init(&bars->p_ready, 4);     // one arrival per elementwise warp
+  mbar_init(&bars->p_ready, n_el_warps);     // one arrival per elementwise warp
   mbar_init(&bars->acc_done, 1);
   mbar_init(&bars->mma_final, 1);
-  mbar_init(&bars->el_read, 4);     // one arrival per elementwise warp: S^T and dP^T read
+  mbar_init(&bars->el_read, n_el_warps);     // one arrival per elementwise warp: dP^T read
   mbar_init(&bars->dvdk_done, 1);
   for (int i = 0; i < 2; ++i) {
     mbar_init(&bars->s_full2[i], 1);
-    mbar_init(&bars->p_ready2[i], 4);
+    mbar_init(&bars->p_ready2[i], n_el_warps);
     mbar_init(&bars->buf_free2[i], 1);
   }
   fence_mbar_init();
@@ -115,9 +117,11 @@ __device__ __forceinline__ void bwd_init_bars(BwdBars* bars) {
 
 // =================================================================== keys stationary: dK, dV
 // Grid (KV group, key block, sequence): the heaviest causal blocks (first keys) launch first.
-// Roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5
-// elementwise (thread = key = TMEM lane 32 (warp % 4) + lane).
-__global__ void __launch_bounds__(192, 1)
+// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-9
+// elementwise: two threads per key (TMEM lane 32 (warp % 4) + lane), warps 2-5 taking queries
+// 0-31 of a unit and warps 6-9 queries 32-63, so that the elementwise step of a unit, which the
+// tensor core waits for, takes half as long.
+__global__ void __launch_bounds__(320, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                     const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mH,
                     const __grid_constant__ BwdTcParams p, KernelCtl ctl) {
@@ -135,7 +139,7 @@ __global__ void __launch_bounds__(192, 1)
   const int n_units = n_tiles * (g + 1);      // unit u: query tile u / (g + 1), head slot u % (g + 1)
 
   if (threadIdx.x == 0) {
-    bwd_init_bars(bars);
+    bwd_init_bars(bars, 8);
     tma_prefetch_desc(&mK);
     tma_prefetch_desc(&mV);
     tma_prefetch_desc(&mQ);
@@ -192,7 +196,10 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t v_lo = uint32_t(sdesc_sw128(smem_u32(smem + A_V_OFF), 16, 1024));
       const uint32_t r_lo = uint32_t(sdesc_sw128(smem_u32(smem + A_RING), 16, 1024));
       const uint32_t rmn_lo = uint32_t(sdesc_sw128(smem_u32(smem + A_RING), BOX_SMALL, 1024));
-      // dV += P^T dH and dK += dS'^T q of unit v (P^T | dS'^T in slot v % 3); then its stage is free
+      // dV += P^T dH and dK += dS'^T q of unit v; then its stage is free.  Slot v % 3 holds, for
+      // queries 32 h .. 32 h + 31 (h = 0, 1), P^T in columns 32 h .. 32 h + 15 and dS'^T in
+      // 32 h + 16 .. 32 h + 31 (fp16 pairs), so K step kk (16 queries) starts at column
+      // 32 (kk / 2) + 8 (kk % 2) (+ 16 for dS'^T)
       auto issue_dvdk = [&](int v) -> bool {
         if (!mbar_wait(&bars->p_ready, v & 1, ctl, SITE_BWD_MMA)) return false;
         tc_fence_after();
@@ -200,11 +207,11 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t stmn = rmn_lo + uint32_t((v % NST) * (STAGE / 16));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)       // K = 64 queries
-          mma_ts_w(tmem + T_DV, slot + 8 * kk, stmn + uint32_t(3 * (BOX_SMALL / 16) + kk * 128), hi, idesc_dv,
+          mma_ts_w(tmem + T_DV, slot + 32 * (kk >> 1) + 8 * (kk & 1), stmn + uint32_t(3 * (BOX_SMALL / 16) + kk * 128), hi, idesc_dv,
                    (v > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts_w(tmem + T_DK, slot + 32 + 8 * kk, stmn + uint32_t(kk * 128), hi, idesc_dk,
+          mma_ts_w(tmem + T_DK, slot + 32 * (kk >> 1) + 16 + 8 * (kk & 1), stmn + uint32_t(kk * 128), hi, idesc_dk,
                    (v > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty[v % NST]);
         mma_commit(&bars->dvdk_done);
@@ -239,24 +246,23 @@ __global__ void __launch_bounds__(192, 1)
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
   } else {
-    // ------------------------------------------------------------ elementwise (warps 2-5)
+    // ------------------------------------------------------------ elementwise (warps 2-9)
     const int q = warp & 3;
+    const int hq = (warp - 2) >> 2;            // which 32 queries of a unit: 32 hq .. 32 hq + 31
     const int r = 32 * q + lane;
     const int s_key = k0 + r;
     const uint32_t lane_off = uint32_t(q * 32) << 16;
-    // per warp: -lse and -Delta / sqrt(192) of the unit's 64 queries
-    float* ld = reinterpret_cast<float*>(smem + A_LD_OFF) + (warp - 2) * 128;
+    // per warp: -lse and -Delta / sqrt(192) of its 32 queries of the unit
+    float* ld = reinterpret_cast<float*>(smem + A_LD_OFF) + (warp - 2) * 64;
     bool ok = n_units > 0;
     for (int u = 0; u < n_units && ok; ++u) {
       const int h = head_of(u % (g + 1), j, p.n_signal, g);
       const int t0 = q_begin + (u / (g + 1)) * TQ;
       {
-        const long long o = ((long long)h * p.B + b) * p.Tpad + t0;
+        const long long o = ((long long)h * p.B + b) * p.Tpad + t0 + 32 * hq;
         __syncwarp();
         ld[lane] = -p.lseT[o + lane];
-        ld[32 + lane] = -p.lseT[o + 32 + lane];
-        ld[64 + lane] = -p.deltaT[o + lane] * p.scale;
-        ld[96 + lane] = -p.deltaT[o + 32 + lane] * p.scale;
+        ld[32 + lane] = -p.deltaT[o + lane] * p.scale;
         __syncwarp();
       }
       // every (query, key) pair of the unit visible: no per-element mask
@@ -265,65 +271,58 @@ __global__ void __launch_bounds__(192, 1)
       const bool w = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, u & 1, ctl, SITE_BWD_SOFTMAX));
       if (!w) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tS = tmem + 64 * uint32_t(u % 3) + lane_off, tD = tmem + 64 * uint32_t((u + 1) % 3) + lane_off;
-      // all of dP^T first: its slot is then free for the next unit's S^T (S^T's own slot
-      // receives P^T | dS'^T)
-      uint32_t dv[64];
+      // this thread's 32 columns of S^T and dP^T (the other half's warps take the other 32)
+      const uint32_t tS = tmem + 64 * uint32_t(u % 3) + 32 * hq + lane_off;
+      const uint32_t tD = tmem + 64 * uint32_t((u + 1) % 3) + 32 * hq + lane_off;
+      // dP^T first: once every warp has read it, its slot is free for the next unit's S^T (S^T's
+      // own slot receives P^T | dS'^T, each half writing only the columns it has read)
+      uint32_t dv[32], sv[32];
       GDLA_TMEM_LD32(tD, dv);
-      GDLA_TMEM_LD32(tD + 32, (dv + 32));
+      GDLA_TMEM_LD32(tS, sv);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->el_read);
-      uint32_t gk[2][16];
+      uint32_t pk[16], gk[16];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {          // 32 queries at a time
-        uint32_t sv[32];
-        GDLA_TMEM_LD32(tS + 32 * c, sv);
-        tmem_ld_wait();
-        uint32_t pk[16];
+      for (int k = 0; k < 8; ++k) {            // 4 queries: -lse and -Delta / sqrt(192) from the staging
+        const float4 l4 = *reinterpret_cast<const float4*>(ld + 4 * k);
+        const float4 d4 = *reinterpret_cast<const float4*>(ld + 32 + 4 * k);
+        const float nl[4] = {l4.x, l4.y, l4.z, l4.w}, nd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {        // 4 queries: -lse and -Delta / sqrt(192) from the staging
-          const float4 l4 = *reinterpret_cast<const float4*>(ld + 32 * c + 4 * k);
-          const float4 d4 = *reinterpret_cast<const float4*>(ld + 64 + 32 * c + 4 * k);
-          const float nl[4] = {l4.x, l4.y, l4.z, l4.w}, nd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int i = 2 * k + e;           // pair index within the chunk
-            float x0, x1, p0, p1, d0, d1, g0, g1;
-            ffma2vv(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), p.scale_log2, p.scale_log2,
-                    nl[2 * e], nl[2 * e + 1]);
-            if ((i & 3) == 3) {
-              exp2_poly2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            if (!interior) {
-              const int qi = 32 * c + 2 * i;
-              p0 = bwd_visible(t0 + qi, s_key, p.T, p.window) ? p0 : 0.f;
-              p1 = bwd_visible(t0 + qi + 1, s_key, p.T, p.window) ? p1 : 0.f;
-            }
-            pk[i] = pack_half2(p0, p1);
-            // dS' = P (dP - Delta) / sqrt(192)
-            ffma2vv(d0, d1, __uint_as_float(dv[32 * c + 2 * i]), __uint_as_float(dv[32 * c + 2 * i + 1]), p.scale,
-                    p.scale, nd[2 * e], nd[2 * e + 1]);
-            fmul2v(g0, g1, p0, p1, d0, d1);
-            gk[c][i] = pack_half2(g0, g1);
+        for (int e = 0; e < 2; ++e) {
+          const int i = 2 * k + e;             // pair index within the 32 queries
+          float x0, x1, p0, p1, d0, d1, g0, g1;
+          ffma2vv(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), p.scale_log2, p.scale_log2,
+                  nl[2 * e], nl[2 * e + 1]);
+          if ((i & 3) == 3) {
+            exp2_poly2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
           }
+          if (!interior) {
+            const int qi = 32 * hq + 2 * i;
+            p0 = bwd_visible(t0 + qi, s_key, p.T, p.window) ? p0 : 0.f;
+            p1 = bwd_visible(t0 + qi + 1, s_key, p.T, p.window) ? p1 : 0.f;
+          }
+          pk[i] = pack_half2(p0, p1);
+          // dS' = P (dP - Delta) / sqrt(192)
+          ffma2vv(d0, d1, __uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]), p.scale, p.scale,
+                  nd[2 * e], nd[2 * e + 1]);
+          fmul2v(g0, g1, p0, p1, d0, d1);
+          gk[i] = pack_half2(g0, g1);
         }
-        // P^T as fp16 pairs over the columns of the S^T slot already read
-        GDLA_TMEM_ST16(tS + 16 * c, pk);
       }
-      // dS'^T into the second half of the S^T slot (all of S^T has been read)
-      GDLA_TMEM_ST16(tS + 32, gk[0]);
-      GDLA_TMEM_ST16(tS + 48, gk[1]);
+      GDLA_TMEM_ST16(tS, pk);                  // P^T, 16 columns of fp16 pairs
+      GDLA_TMEM_ST16(tS + 16, gk);             // dS'^T
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);
     }
-    // ---- dV and dK of this CTA's keys
+    // ---- dV and dK of this CTA's keys: 128 dV columns, then 192 dK columns, five chunks of 32
+    // per half
     if (ok) {
       const bool w = __all_sync(0xffffffffu, mbar_wait(&bars->acc_done, 0, ctl, SITE_BWD_SOFTMAX));
       if (w) {
@@ -331,7 +330,7 @@ __global__ void __launch_bounds__(192, 1)
         const long long m = (long long)b * p.T + s_key;
         const bool row_ok = s_key < p.T;
 #pragma unroll 1
-        for (int c = 0; c < 10; ++c) {       // 128 dV columns, then 192 dK columns
+        for (int c = 5 * hq; c < 5 * hq + 5; ++c) {
           uint32_t v[32];
           GDLA_TMEM_LD32(tmem + T_DV + 32 * c + lane_off, v);
           tmem_ld_wait();
@@ -346,7 +345,6 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -358,7 +356,9 @@ __global__ void __launch_bounds__(192, 1)
 
 // =================================================================== queries stationary: dq
 // Grid (head, query block from the last, sequence): the heaviest causal blocks launch first.
-__global__ void __launch_bounds__(192, 1)
+// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-9
+// elementwise, two threads per query.
+__global__ void __launch_bounds__(320, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mH,
                   const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                   const __grid_constant__ BwdTcParams p, KernelCtl ctl) {
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(192, 1)
   const int n_units = s_hi > k_begin ? (s_hi - k_begin + TK - 1) / TK : 0;
 
   if (threadIdx.x == 0) {
-    bwd_init_bars(bars);
+    bwd_init_bars(bars, 8);
     tma_prefetch_desc(&mQ);
     tma_prefetch_desc(&mH);
     tma_prefetch_desc(&mK);
@@ -434,7 +434,8 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t r_lo = uint32_t(sdesc_sw128(smem_u32(smem + B_RING), 16, 1024));
       const uint32_t rmn_lo = uint32_t(sdesc_sw128(smem_u32(smem + B_RING), BOX_SMALL, 1024));
       // dq += dS'(v) K(v) once the elementwise threads have written dS'(v); then the key tile's
-      // stage and the S / dP buffer of v are free
+      // stage and the S / dP buffer of v are free.  dS' of keys 32 h .. 32 h + 31 (h = 0, 1) is in
+      // dP columns 32 h .. 32 h + 15 (fp16 pairs): K step kk starts at 32 (kk / 2) + 8 (kk % 2)
       auto issue_dq = [&](int v) -> bool {
         const int buf = v & 1;
         if (!mbar_wait(&bars->p_ready2[buf], (v >> 1) & 1, ctl, SITE_BWD_MMA)) return false;
@@ -442,7 +443,7 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t stmn = rmn_lo + uint32_t((v % NST) * (STAGE / 16));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)       // dq += dS' [K^C | k^R], K = 64 keys
-          mma_ts_w(tmem + T_DQ, tmem + T_DP + 128 * buf + 8 * kk, stmn + uint32_t(kk * 128), hi, idesc_dq,
+          mma_ts_w(tmem + T_DQ, tmem + T_DP + 128 * buf + 32 * (kk >> 1) + 8 * (kk & 1), stmn + uint32_t(kk * 128), hi, idesc_dq,
                    (v > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty[v % NST]);
         mma_commit(&bars->buf_free2[buf]);
@@ -474,8 +475,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
   } else {
-    // ------------------------------------------------------------ elementwise (warps 2-5)
+    // ------------------------------------------------------------ elementwise (warps 2-9)
+    // two threads per query: warps 2-5 take keys 0-31 of a tile, warps 6-9 keys 32-63
     const int q = warp & 3;
+    const int hk = (warp - 2) >> 2;
     const int r = 32 * q + lane;
     const int t = q0 + r;
     const uint32_t lane_off = uint32_t(q * 32) << 16;
@@ -490,35 +493,35 @@ __global__ void __launch_bounds__(192, 1)
       const bool w = __all_sync(0xffffffffu, mbar_wait(&bars->s_full2[buf], (u >> 1) & 1, ctl, SITE_BWD_SOFTMAX));
       if (!w) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tS = tmem + T_S + 128 * buf + lane_off, tD = tmem + T_DP + 128 * buf + lane_off;
+      // this half's 32 columns of S and dP; dS' (fp16 pairs) goes over the first 16 of those dP
+      // columns, which only this half reads
+      const uint32_t tS = tmem + T_S + 128 * buf + 32 * hk + lane_off;
+      const uint32_t tD = tmem + T_DP + 128 * buf + 32 * hk + lane_off;
+      uint32_t sv[32], dv[32];
+      GDLA_TMEM_LD32(tS, sv);
+      GDLA_TMEM_LD32(tD, dv);
+      tmem_ld_wait();
+      uint32_t gk[16];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sv[32], dv[32];
-        GDLA_TMEM_LD32(tS + 32 * c, sv);
-        GDLA_TMEM_LD32(tD + 32 * c, dv);
-        tmem_ld_wait();
-        uint32_t gk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0, x1, p0, p1, d0, d1, g0, g1;
-          ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), p.scale_log2, nl);
-          if ((i & 3) == 3) {
-            exp2_poly2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          if (!interior) {
-            const int ks = s0 + 32 * c + 2 * i;
-            p0 = bwd_visible(t, ks, p.T, p.window) ? p0 : 0.f;
-            p1 = bwd_visible(t, ks + 1, p.T, p.window) ? p1 : 0.f;
-          }
-          ffma2(d0, d1, __uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]), p.scale, nd);
-          fmul2v(g0, g1, p0, p1, d0, d1);
-          gk[i] = pack_half2(g0, g1);
+      for (int i = 0; i < 16; ++i) {
+        float x0, x1, p0, p1, d0, d1, g0, g1;
+        ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), p.scale_log2, nl);
+        if ((i & 3) == 3) {
+          exp2_poly2(x0, x1, p0, p1);
+        } else {
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
         }
-        GDLA_TMEM_ST16(tD + 16 * c, gk);
+        if (!interior) {
+          const int ks = s0 + 32 * hk + 2 * i;
+          p0 = bwd_visible(t, ks, p.T, p.window) ? p0 : 0.f;
+          p1 = bwd_visible(t, ks + 1, p.T, p.window) ? p1 : 0.f;
+        }
+        ffma2(d0, d1, __uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]), p.scale, nd);
+        fmul2v(g0, g1, p0, p1, d0, d1);
+        gk[i] = pack_half2(g0, g1);
       }
+      GDLA_TMEM_ST16(tD, gk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -530,7 +533,7 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const long long m = (long long)b * p.T + t;
 #pragma unroll 1
-        for (int c = 0; c < 6; ++c) {        // dq^C (128 columns), then dq^R (64)
+        for (int c = 3 * hk; c < 3 * hk + 3; ++c) {   // dq^C (128 columns), then dq^R (64)
           uint32_t v[32];
           GDLA_TMEM_LD32(tmem + T_DQ + 32 * c + lane_off, v);
           tmem_ld_wait();
@@ -545,7 +548,6 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -733,10 +735,10 @@ int launch_attn_bwd(const AttnBwdParams& a, const KernelCtlHost& ctlh, cudaStrea
   if (cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::A_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::B_SMEM) != cudaSuccess)
     return -4;
-  bwd_dkdv_kernel<<<dim3(ng, (a.T + bwd::BK - 1) / bwd::BK, a.B), 192, bwd::A_SMEM, st>>>(mK128, mV128, mQ64, mH64,
+  bwd_dkdv_kernel<<<dim3(ng, (a.T + bwd::BK - 1) / bwd::BK, a.B), 320, bwd::A_SMEM, st>>>(mK128, mV128, mQ64, mH64,
                                                                                            p, kc);
   if (cudaPeekAtLastError() != cudaSuccess) return -4;
-  bwd_dq_kernel<<<dim3(nH, (a.T + bwd::BQ - 1) / bwd::BQ, a.B), 192, bwd::B_SMEM, st>>>(mQ128, mH128, mK64, mV64, p,
+  bwd_dq_kernel<<<dim3(nH, (a.T + bwd::BQ - 1) / bwd::BQ, a.B), 320, bwd::B_SMEM, st>>>(mQ128, mH128, mK64, mV64, p,
                                                                                         kc);
   if (cudaPeekAtLastError() != cudaSuccess) return -4;
   const long long n_fin = M * ((long long)ng * 32 + 16);
