@@ -13,16 +13,16 @@
 // accumulators in TMEM), in two kernels that each own their outputs (no atomics):
 //  * keys stationary (dK, dV): one CTA per (sequence, KV group j, 128 keys) keeps K = [K^C_j |
 //    k^R] and V_j of its keys in shared memory and loops over 64-query tiles x the group's five
-//    heads: S^T = K q^T and dP^T = V dH^T into TMEM; the elementwise threads (two per key, each
-//    taking 32 of the 64 queries) turn them into P^T and dS'^T (fp16, packed into the S^T slot,
-//    each thread over the columns it has read) which are the A operands of
+//    heads: S^T = K q^T and dP^T = V dH^T into TMEM; the elementwise threads (EL_GROUPS per key,
+//    each taking QG of the 64 queries) turn them into P^T and dS'^T (fp16, packed into the S^T
+//    slot, each thread over the columns it has read) which are the A operands of
 //    dV += P^T dH and dK += dS'^T q.  TMEM: three rotating 64-column slots | dV 128 | dK 192.
 //    Unit u puts S^T in slot u % 3 and dP^T in slot (u + 1) % 3; the dP^T slot is free as soon
 //    as the elementwise threads have read it, so the tensor core computes S^T / dP^T of unit
 //    u + 1 (and dV / dK of unit u - 1) while they work on unit u.
 //  * queries stationary (dq): one CTA per (sequence, head, 128 queries) keeps q and dH and loops
-//    over 64-key tiles: S = q K^T, dP = dH V^T, dS' in place (two threads per query, 32 keys
-//    each), dq += dS' K.
+//    over 64-key tiles: S = q K^T, dP = dH V^T, dS' in place (EL_GROUPS threads per query, QG
+//    keys each), dq += dS' K.
 //    TMEM: two (S 64 | dP 64) buffers | dq 192 columns, so that the scores of the next key tile
 //    are computed while the elementwise threads work on this one.
 // Both recompute P from the saved log-sum-exp; the second recomputes S and dP, which costs
@@ -40,6 +40,12 @@ constexpr int BQ = 128;   // queries per dq CTA (TMEM lanes)
 constexpr int TQ = 64;    // query tile of the dK/dV loop
 constexpr int TK = 64;    // key tile of the dq loop
 constexpr int NST = 3;    // stages of the streamed operand ring
+// elementwise threads per key (dK/dV) or query (dq): group e of warps 2 + 4 e .. 5 + 4 e takes
+// the QG queries (keys) QG e .. QG e + QG - 1 of a 64-wide tile
+constexpr int EL_GROUPS = 4;
+constexpr int QG = 64 / EL_GROUPS;
+constexpr int EL_WARPS = 4 * EL_GROUPS;
+constexpr int THREADS = 64 + 32 * EL_WARPS;
 constexpr int BOX_BIG = 128 * 128;    // [128 rows][64 fp16] 128-byte-swizzled box
 constexpr int BOX_SMALL = 64 * 128;   // [64 rows][64 fp16]
 // dK/dV kernel: K block (3 boxes) | V block (2) | ring of (q tile 3 boxes + dH tile 2 boxes) |
@@ -49,7 +55,7 @@ constexpr int A_V_OFF = A_K_OFF + 3 * BOX_BIG;
 constexpr int A_RING = A_V_OFF + 2 * BOX_BIG;
 constexpr int STAGE = 5 * BOX_SMALL;
 constexpr int A_LD_OFF = A_RING + NST * STAGE;
-constexpr int A_BAR_OFF = A_LD_OFF + 8 * 64 * 4;
+constexpr int A_BAR_OFF = A_LD_OFF + EL_WARPS * 2 * QG * 4;
 constexpr int A_SMEM = A_BAR_OFF + 256 + 1024;
 // dq kernel: q block (3 boxes) | dH block (2) | ring of (K tile 3 boxes + V tile 2 boxes)
 constexpr int B_Q_OFF = 0;
@@ -91,6 +97,27 @@ __device__ __forceinline__ int head_of(int i, int j, int n_signal, int g) {
   return i == 0 ? n_signal + j : g * j + i - 1;
 }
 // Is query t allowed to see key s (causal, window W; both inside the sequence)?
+// The elementwise group's QG columns (32 lanes) out of TMEM, and half as many back.
+__device__ __forceinline__ void el_tmem_ld(uint32_t taddr, uint32_t* r) {
+  if constexpr (bwd::QG == 32) {
+    GDLA_TMEM_LD32(taddr, r);
+  } else {
+    static_assert(bwd::QG == 16, "elementwise group width");
+    GDLA_TMEM_LD16(taddr, r);
+  }
+}
+__device__ __forceinline__ void el_tmem_st_half(uint32_t taddr, const uint32_t* r) {
+  if constexpr (bwd::QG == 32) {
+    GDLA_TMEM_ST16(taddr, r);
+  } else {
+    GDLA_TMEM_ST8(taddr, r);
+  }
+}
+// First TMEM column of the fp16 pairs of queries (keys) 16 kk .. 16 kk + 15, written by
+// elementwise group 16 kk / QG at the start of its QG columns.
+__device__ __forceinline__ constexpr uint32_t el_col(int kk) {
+  return uint32_t(bwd::QG * ((16 * kk) / bwd::QG) + ((16 * kk) % bwd::QG) / 2);
+}
 __device__ __forceinline__ bool bwd_visible(int t, int s, int T, int W) {
   return t < T && s <= t && (W <= 0 || t - s < W);
 }
@@ -117,11 +144,11 @@ __device__ __forceinline__ void bwd_init_bars(BwdBars* bars, uint32_t n_el_warps
 
 // =================================================================== keys stationary: dK, dV
 // Grid (KV group, key block, sequence): the heaviest causal blocks (first keys) launch first.
-// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-9
-// elementwise: two threads per key (TMEM lane 32 (warp % 4) + lane), warps 2-5 taking queries
-// 0-31 of a unit and warps 6-9 queries 32-63, so that the elementwise step of a unit, which the
-// tensor core waits for, takes half as long.
-__global__ void __launch_bounds__(320, 1)
+// Roles (THREADS threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2 .. 1 +
+// EL_WARPS elementwise: EL_GROUPS threads per key (TMEM lane 32 (warp % 4) + lane), group e
+// (warps 2 + 4 e .. 5 + 4 e) taking the queries QG e .. QG e + QG - 1 of a unit, so that the
+// elementwise step of a unit, which the tensor core waits for, is split EL_GROUPS ways.
+__global__ void __launch_bounds__(bwd::THREADS, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                     const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mH,
                     const __grid_constant__ BwdTcParams p, KernelCtl ctl) {
@@ -139,7 +166,7 @@ __global__ void __launch_bounds__(320, 1)
   const int n_units = n_tiles * (g + 1);      // unit u: query tile u / (g + 1), head slot u % (g + 1)
 
   if (threadIdx.x == 0) {
-    bwd_init_bars(bars, 8);
+    bwd_init_bars(bars, bwd::EL_WARPS);
     tma_prefetch_desc(&mK);
     tma_prefetch_desc(&mV);
     tma_prefetch_desc(&mQ);
@@ -197,9 +224,8 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t r_lo = uint32_t(sdesc_sw128(smem_u32(smem + A_RING), 16, 1024));
       const uint32_t rmn_lo = uint32_t(sdesc_sw128(smem_u32(smem + A_RING), BOX_SMALL, 1024));
       // dV += P^T dH and dK += dS'^T q of unit v; then its stage is free.  Slot v % 3 holds, for
-      // queries 32 h .. 32 h + 31 (h = 0, 1), P^T in columns 32 h .. 32 h + 15 and dS'^T in
-      // 32 h + 16 .. 32 h + 31 (fp16 pairs), so K step kk (16 queries) starts at column
-      // 32 (kk / 2) + 8 (kk % 2) (+ 16 for dS'^T)
+      // the queries QG e .. QG e + QG - 1 of group e, P^T in columns QG e .. QG e + QG / 2 - 1
+      // and dS'^T in the next QG / 2 (fp16 pairs): K step kk starts at el_col(kk) (+ QG / 2)
       auto issue_dvdk = [&](int v) -> bool {
         if (!mbar_wait(&bars->p_ready, v & 1, ctl, SITE_BWD_MMA)) return false;
         tc_fence_after();
@@ -207,11 +233,11 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t stmn = rmn_lo + uint32_t((v % NST) * (STAGE / 16));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)       // K = 64 queries
-          mma_ts_w(tmem + T_DV, slot + 32 * (kk >> 1) + 8 * (kk & 1), stmn + uint32_t(3 * (BOX_SMALL / 16) + kk * 128), hi, idesc_dv,
+          mma_ts_w(tmem + T_DV, slot + el_col(kk), stmn + uint32_t(3 * (BOX_SMALL / 16) + kk * 128), hi, idesc_dv,
                    (v > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts_w(tmem + T_DK, slot + 32 * (kk >> 1) + 16 + 8 * (kk & 1), stmn + uint32_t(kk * 128), hi, idesc_dk,
+          mma_ts_w(tmem + T_DK, slot + el_col(kk) + QG / 2, stmn + uint32_t(kk * 128), hi, idesc_dk,
                    (v > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty[v % NST]);
         mma_commit(&bars->dvdk_done);
@@ -246,23 +272,23 @@ __global__ void __launch_bounds__(320, 1)
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
   } else {
-    // ------------------------------------------------------------ elementwise (warps 2-9)
+    // ------------------------------------------------------------ elementwise (warps 2 ..)
     const int q = warp & 3;
-    const int hq = (warp - 2) >> 2;            // which 32 queries of a unit: 32 hq .. 32 hq + 31
+    const int hq = (warp - 2) >> 2;            // group: queries QG hq .. QG hq + QG - 1 of a unit
     const int r = 32 * q + lane;
     const int s_key = k0 + r;
     const uint32_t lane_off = uint32_t(q * 32) << 16;
     // per warp: -lse and -Delta / sqrt(192) of its 32 queries of the unit
-    float* ld = reinterpret_cast<float*>(smem + A_LD_OFF) + (warp - 2) * 64;
+    float* ld = reinterpret_cast<float*>(smem + A_LD_OFF) + (warp - 2) * 2 * QG;
     bool ok = n_units > 0;
     for (int u = 0; u < n_units && ok; ++u) {
       const int h = head_of(u % (g + 1), j, p.n_signal, g);
       const int t0 = q_begin + (u / (g + 1)) * TQ;
       {
-        const long long o = ((long long)h * p.B + b) * p.Tpad + t0 + 32 * hq;
+        const long long o = ((long long)h * p.B + b) * p.Tpad + t0 + QG * hq;
         __syncwarp();
-        ld[lane] = -p.lseT[o + lane];
-        ld[32 + lane] = -p.deltaT[o + lane] * p.scale;
+#pragma unroll
+        for (int i = lane; i < 2 * QG; i += 32) ld[i] = i < QG ? -p.lseT[o + i] : -p.deltaT[o + i - QG] * p.scale;
         __syncwarp();
       }
       // every (query, key) pair of the unit visible: no per-element mask
@@ -271,23 +297,23 @@ __global__ void __launch_bounds__(320, 1)
       const bool w = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, u & 1, ctl, SITE_BWD_SOFTMAX));
       if (!w) { ok = false; break; }
       tc_fence_after();
-      // this thread's 32 columns of S^T and dP^T (the other half's warps take the other 32)
-      const uint32_t tS = tmem + 64 * uint32_t(u % 3) + 32 * hq + lane_off;
-      const uint32_t tD = tmem + 64 * uint32_t((u + 1) % 3) + 32 * hq + lane_off;
+      // this group's QG columns of S^T and dP^T
+      const uint32_t tS = tmem + 64 * uint32_t(u % 3) + QG * hq + lane_off;
+      const uint32_t tD = tmem + 64 * uint32_t((u + 1) % 3) + QG * hq + lane_off;
       // dP^T first: once every warp has read it, its slot is free for the next unit's S^T (S^T's
-      // own slot receives P^T | dS'^T, each half writing only the columns it has read)
-      uint32_t dv[32], sv[32];
-      GDLA_TMEM_LD32(tD, dv);
-      GDLA_TMEM_LD32(tS, sv);
+      // own slot receives P^T | dS'^T, each group writing only the columns it has read)
+      uint32_t dv[QG], sv[QG];
+      el_tmem_ld(tD, dv);
+      el_tmem_ld(tS, sv);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->el_read);
-      uint32_t pk[16], gk[16];
+      uint32_t pk[QG / 2], gk[QG / 2];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {            // 4 queries: -lse and -Delta / sqrt(192) from the staging
+      for (int k = 0; k < QG / 4; ++k) {            // 4 queries: -lse and -Delta / sqrt(192) from the staging
         const float4 l4 = *reinterpret_cast<const float4*>(ld + 4 * k);
-        const float4 d4 = *reinterpret_cast<const float4*>(ld + 32 + 4 * k);
+        const float4 d4 = *reinterpret_cast<const float4*>(ld + QG + 4 * k);
         const float nl[4] = {l4.x, l4.y, l4.z, l4.w}, nd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -302,7 +328,7 @@ __global__ void __launch_bounds__(320, 1)
             p1 = ex2_approx(x1);
           }
           if (!interior) {
-            const int qi = 32 * hq + 2 * i;
+            const int qi = QG * hq + 2 * i;
             p0 = bwd_visible(t0 + qi, s_key, p.T, p.window) ? p0 : 0.f;
             p1 = bwd_visible(t0 + qi + 1, s_key, p.T, p.window) ? p1 : 0.f;
           }
@@ -314,8 +340,8 @@ __global__ void __launch_bounds__(320, 1)
           gk[i] = pack_half2(g0, g1);
         }
       }
-      GDLA_TMEM_ST16(tS, pk);                  // P^T, 16 columns of fp16 pairs
-      GDLA_TMEM_ST16(tS + 16, gk);             // dS'^T
+      el_tmem_st_half(tS, pk);                 // P^T, QG / 2 columns of fp16 pairs
+      el_tmem_st_half(tS + QG / 2, gk);        // dS'^T
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -330,7 +356,7 @@ __global__ void __launch_bounds__(320, 1)
         const long long m = (long long)b * p.T + s_key;
         const bool row_ok = s_key < p.T;
 #pragma unroll 1
-        for (int c = 5 * hq; c < 5 * hq + 5; ++c) {
+        for (int c = hq; c < 10; c += EL_GROUPS) {
           uint32_t v[32];
           GDLA_TMEM_LD32(tmem + T_DV + 32 * c + lane_off, v);
           tmem_ld_wait();
@@ -356,9 +382,9 @@ __global__ void __launch_bounds__(320, 1)
 
 // =================================================================== queries stationary: dq
 // Grid (head, query block from the last, sequence): the heaviest causal blocks launch first.
-// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-9
-// elementwise, two threads per query.
-__global__ void __launch_bounds__(320, 1)
+// Roles (THREADS threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2 .. 1 +
+// EL_WARPS elementwise, EL_GROUPS threads per query.
+__global__ void __launch_bounds__(bwd::THREADS, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mH,
                   const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                   const __grid_constant__ BwdTcParams p, KernelCtl ctl) {
@@ -378,7 +404,7 @@ __global__ void __launch_bounds__(320, 1)
   const int n_units = s_hi > k_begin ? (s_hi - k_begin + TK - 1) / TK : 0;
 
   if (threadIdx.x == 0) {
-    bwd_init_bars(bars, 8);
+    bwd_init_bars(bars, bwd::EL_WARPS);
     tma_prefetch_desc(&mQ);
     tma_prefetch_desc(&mH);
     tma_prefetch_desc(&mK);
@@ -434,8 +460,8 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t r_lo = uint32_t(sdesc_sw128(smem_u32(smem + B_RING), 16, 1024));
       const uint32_t rmn_lo = uint32_t(sdesc_sw128(smem_u32(smem + B_RING), BOX_SMALL, 1024));
       // dq += dS'(v) K(v) once the elementwise threads have written dS'(v); then the key tile's
-      // stage and the S / dP buffer of v are free.  dS' of keys 32 h .. 32 h + 31 (h = 0, 1) is in
-      // dP columns 32 h .. 32 h + 15 (fp16 pairs): K step kk starts at 32 (kk / 2) + 8 (kk % 2)
+      // stage and the S / dP buffer of v are free.  dS' of the keys QG e .. QG e + QG - 1 of group
+      // e is in dP columns QG e .. QG e + QG / 2 - 1 (fp16 pairs): K step kk starts at el_col(kk)
       auto issue_dq = [&](int v) -> bool {
         const int buf = v & 1;
         if (!mbar_wait(&bars->p_ready2[buf], (v >> 1) & 1, ctl, SITE_BWD_MMA)) return false;
@@ -443,7 +469,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t stmn = rmn_lo + uint32_t((v % NST) * (STAGE / 16));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)       // dq += dS' [K^C | k^R], K = 64 keys
-          mma_ts_w(tmem + T_DQ, tmem + T_DP + 128 * buf + 32 * (kk >> 1) + 8 * (kk & 1), stmn + uint32_t(kk * 128), hi, idesc_dq,
+          mma_ts_w(tmem + T_DQ, tmem + T_DP + 128 * buf + el_col(kk), stmn + uint32_t(kk * 128), hi, idesc_dq,
                    (v > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->empty[v % NST]);
         mma_commit(&bars->buf_free2[buf]);
@@ -475,8 +501,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
   } else {
-    // ------------------------------------------------------------ elementwise (warps 2-9)
-    // two threads per query: warps 2-5 take keys 0-31 of a tile, warps 6-9 keys 32-63
+    // ------------------------------------------------------------ elementwise (warps 2 ..)
+    // EL_GROUPS threads per query: group e takes the keys QG e .. QG e + QG - 1 of a tile
     const int q = warp & 3;
     const int hk = (warp - 2) >> 2;
     const int r = 32 * q + lane;
@@ -493,17 +519,17 @@ __global__ void __launch_bounds__(320, 1)
       const bool w = __all_sync(0xffffffffu, mbar_wait(&bars->s_full2[buf], (u >> 1) & 1, ctl, SITE_BWD_SOFTMAX));
       if (!w) { ok = false; break; }
       tc_fence_after();
-      // this half's 32 columns of S and dP; dS' (fp16 pairs) goes over the first 16 of those dP
-      // columns, which only this half reads
-      const uint32_t tS = tmem + T_S + 128 * buf + 32 * hk + lane_off;
-      const uint32_t tD = tmem + T_DP + 128 * buf + 32 * hk + lane_off;
-      uint32_t sv[32], dv[32];
-      GDLA_TMEM_LD32(tS, sv);
-      GDLA_TMEM_LD32(tD, dv);
+      // this group's QG columns of S and dP; dS' (fp16 pairs) goes over the first QG / 2 of those
+      // dP columns, which only this group reads
+      const uint32_t tS = tmem + T_S + 128 * buf + QG * hk + lane_off;
+      const uint32_t tD = tmem + T_DP + 128 * buf + QG * hk + lane_off;
+      uint32_t sv[QG], dv[QG];
+      el_tmem_ld(tS, sv);
+      el_tmem_ld(tD, dv);
       tmem_ld_wait();
-      uint32_t gk[16];
+      uint32_t gk[QG / 2];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < QG / 2; ++i) {
         float x0, x1, p0, p1, d0, d1, g0, g1;
         ffma2(x0, x1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), p.scale_log2, nl);
         if ((i & 3) == 3) {
@@ -513,7 +539,7 @@ __global__ void __launch_bounds__(320, 1)
           p1 = ex2_approx(x1);
         }
         if (!interior) {
-          const int ks = s0 + 32 * hk + 2 * i;
+          const int ks = s0 + QG * hk + 2 * i;
           p0 = bwd_visible(t, ks, p.T, p.window) ? p0 : 0.f;
           p1 = bwd_visible(t, ks + 1, p.T, p.window) ? p1 : 0.f;
         }
@@ -521,7 +547,7 @@ __global__ void __launch_bounds__(320, 1)
         fmul2v(g0, g1, p0, p1, d0, d1);
         gk[i] = pack_half2(g0, g1);
       }
-      GDLA_TMEM_ST16(tD, gk);
+      el_tmem_st_half(tD, gk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -533,7 +559,7 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         const long long m = (long long)b * p.T + t;
 #pragma unroll 1
-        for (int c = 3 * hk; c < 3 * hk + 3; ++c) {   // dq^C (128 columns), then dq^R (64)
+        for (int c = hk; c < 6; c += EL_GROUPS) {   // dq^C (128 columns), then dq^R (64)
           uint32_t v[32];
           GDLA_TMEM_LD32(tmem + T_DQ + 32 * c + lane_off, v);
           tmem_ld_wait();
@@ -735,10 +761,10 @@ int launch_attn_bwd(const AttnBwdParams& a, const KernelCtlHost& ctlh, cudaStrea
   if (cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::A_SMEM) != cudaSuccess ||
       cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::B_SMEM) != cudaSuccess)
     return -4;
-  bwd_dkdv_kernel<<<dim3(ng, (a.T + bwd::BK - 1) / bwd::BK, a.B), 320, bwd::A_SMEM, st>>>(mK128, mV128, mQ64, mH64,
+  bwd_dkdv_kernel<<<dim3(ng, (a.T + bwd::BK - 1) / bwd::BK, a.B), bwd::THREADS, bwd::A_SMEM, st>>>(mK128, mV128, mQ64, mH64,
                                                                                            p, kc);
   if (cudaPeekAtLastError() != cudaSuccess) return -4;
-  bwd_dq_kernel<<<dim3(nH, (a.T + bwd::BQ - 1) / bwd::BQ, a.B), 320, bwd::B_SMEM, st>>>(mQ128, mH128, mK64, mV64, p,
+  bwd_dq_kernel<<<dim3(nH, (a.T + bwd::BQ - 1) / bwd::BQ, a.B), bwd::THREADS, bwd::B_SMEM, st>>>(mQ128, mH128, mK64, mV64, p,
                                                                                         kc);
   if (cudaPeekAtLastError() != cudaSuccess) return -4;
   const long long n_fin = M * ((long long)ng * 32 + 16);

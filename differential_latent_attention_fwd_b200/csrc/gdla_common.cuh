@@ -277,6 +277,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
         "r"(r[14]), "r"(r[15])                                                                   \
       : "memory")
 
+#define GDLA_TMEM_ST8(taddr, r)                                                                    \
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"            \
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),   \
+                 "r"(r[6]), "r"(r[7])                                                            \
+               : "memory")
+
 // 16-byte asynchronous global -> shared copy (all of a thread's copies stay in flight).
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
