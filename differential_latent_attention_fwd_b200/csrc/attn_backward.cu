@@ -281,16 +281,27 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     // per warp: -lse and -Delta / sqrt(192) of its 32 queries of the unit
     float* ld = reinterpret_cast<float*>(smem + A_LD_OFF) + (warp - 2) * 2 * QG;
     bool ok = n_units > 0;
-    for (int u = 0; u < n_units && ok; ++u) {
-      const int h = head_of(u % (g + 1), j, p.n_signal, g);
-      const int t0 = q_begin + (u / (g + 1)) * TQ;
-      {
-        const long long o = ((long long)h * p.B + b) * p.Tpad + t0 + QG * hq;
-        __syncwarp();
+    // -lse / -Delta of a unit's QG queries, lane i (and i + 32) holding entry i of the staging;
+    // the next unit's are loaded while this one is processed
+    constexpr int NPRE = 2 * QG / 32;
+    auto fetch_ld = [&](int uu, float* pre) {
+      const int hh = head_of(uu % (g + 1), j, p.n_signal, g);
+      const long long o = ((long long)hh * p.B + b) * p.Tpad + q_begin + (uu / (g + 1)) * TQ + QG * hq;
 #pragma unroll
-        for (int i = lane; i < 2 * QG; i += 32) ld[i] = i < QG ? -p.lseT[o + i] : -p.deltaT[o + i - QG] * p.scale;
-        __syncwarp();
+      for (int e = 0; e < NPRE; ++e) {
+        const int i = lane + 32 * e;
+        pre[e] = i < QG ? -p.lseT[o + i] : -p.deltaT[o + i - QG] * p.scale;
       }
+    };
+    float pre[NPRE];
+    if (n_units > 0) fetch_ld(0, pre);
+    for (int u = 0; u < n_units && ok; ++u) {
+      const int t0 = q_begin + (u / (g + 1)) * TQ;
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < NPRE; ++e) ld[lane + 32 * e] = pre[e];
+      __syncwarp();
+      if (u + 1 < n_units) fetch_ld(u + 1, pre);
       // every (query, key) pair of the unit visible: no per-element mask
       const bool interior = t0 >= k0 + BK - 1 && t0 + TQ <= p.T && k0 + BK <= p.T &&
                             (p.window <= 0 || t0 + TQ - 1 - k0 < p.window);
