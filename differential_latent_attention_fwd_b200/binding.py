@@ -46,7 +46,8 @@ class gdla_weights_t(ctypes.Structure):
 
 
 class gdla_absorbed_t(ctypes.Structure):
-    _fields_ = [("w", gdla_weights_t), ("W_UKt", ctypes.c_void_p), ("cfg", gdla_config_t),
+    _fields_ = [("w", gdla_weights_t), ("W_UKt", ctypes.c_void_p), ("W_a", ctypes.c_void_p),
+                ("W_bqg", ctypes.c_void_p), ("cfg", gdla_config_t),
                 ("magic", ctypes.c_uint32)]
 
 

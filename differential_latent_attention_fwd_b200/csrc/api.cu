@@ -79,9 +79,9 @@ static int varlen_max_units(long long total, long long n_docs) {
 // fp32 scratch of the split-K projections of a decode step (skinny M = B products).
 static long long decode_splitk_floats(const gdla_config_t* c, int B) {
   const int nH = c->n_signal + c->n_noise;
-  const int shapes[6][2] = {{c->q_rank, c->d_model}, {c->kv_rank + c->d_rope, c->d_model},
-                            {c->n_signal, c->d_model}, {nH * (c->d_nope + c->d_rope), c->q_rank},
-                            {c->n_signal * c->d_v, c->q_rank}, {c->d_model, c->n_signal * c->d_v}};
+  const int shapes[3][2] = {{c->q_rank + c->kv_rank + c->d_rope + c->n_signal, c->d_model},
+                            {nH * (c->d_nope + c->d_rope) + c->n_signal * c->d_v, c->q_rank},
+                            {c->d_model, c->n_signal * c->d_v}};
   long long m = 0;
   for (auto& sh : shapes) {
     const long long f = (long long)gemm_splitk_count(B, sh[0], sh[1]) * B * sh[0];
@@ -119,7 +119,8 @@ static void layout(const gdla_config_t* c, int B, int T, int mode, size_t off[WS
     // the attention's segments: one partial slot per (CTA, row) pair that can meet
     const long long slots = (long long)decode_cta_count() + M;
     sz[WS_LATENT] = 0;                                               // unused by decode
-    sz[WS_QQ] = M * qq * 4;                                          // fp32 q^C | q^R
+    sz[WS_QQ] = M * (qq + (long long)c->n_signal * c->d_v) * 4;      // fp32 q^C | q^R | G
+    sz[WS_G] = 0;                                                    // (G sits in the WS_QQ rows)
     sz[WS_KV] = M * (long long)nH * (c->kv_rank + c->d_rope) * 2;    // q~ rows
     sz[WS_ONOISE] = slots * nH * c->kv_rank * 4;                     // segment partials
     sz[WS_KR16] = slots * nH * 2 * 4;                                // segment (max, sum)
@@ -488,11 +489,27 @@ int gdla_workspace_offset(const gdla_config_t* cfg, int B, int T, int mode, int 
   return GDLA_OK;
 }
 
+// The absorbed tensors, in order: W_UKt, W_a, W_bqg (each rounded up to 256 bytes).
+static void absorbed_layout(const gdla_config_t* c, size_t off[4]) {
+  const int nH = c->n_signal + c->n_noise;
+  const size_t sz[3] = {(size_t)c->n_kv_heads * c->d_nope * c->kv_rank * 2,
+                        (size_t)c->d_model * (c->q_rank + c->kv_rank + c->d_rope + c->n_signal) * 2,
+                        (size_t)c->q_rank * ((size_t)nH * (c->d_nope + c->d_rope) + (size_t)c->n_signal * c->d_v) * 2};
+  size_t o = 0;
+  for (int i = 0; i < 3; ++i) {
+    off[i] = o;
+    o += (sz[i] + 255) & ~size_t(255);
+  }
+  off[3] = o;
+}
+
 int gdla_absorbed_size(const gdla_config_t* cfg, size_t* bytes) {
   int rc = check_config(cfg);
   if (rc) return rc;
   if (!bytes) return GDLA_ERR_INVALID_ARG;
-  *bytes = (size_t)cfg->n_kv_heads * cfg->d_nope * cfg->kv_rank * 2;
+  size_t off[4];
+  absorbed_layout(cfg, off);
+  *bytes = off[3];
   return GDLA_OK;
 }
 
@@ -707,11 +724,32 @@ int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void*
   size_t need;
   gdla_absorbed_size(cfg, &need);
   if (dst_bytes < need) return GDLA_ERR_WORKSPACE_TOO_SMALL;
-  if (launch_failed(launch_absorb_uk(w->W_bKV, dst, cfg->kv_rank, cfg->n_kv_heads, cfg->d_nope, cfg->d_v,
-                       static_cast<cudaStream_t>(stream))))
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  size_t off[4];
+  absorbed_layout(cfg, off);
+  uint8_t* base = static_cast<uint8_t*>(dst);
+  if (launch_failed(launch_absorb_uk(w->W_bKV, base + off[0], cfg->kv_rank, cfg->n_kv_heads, cfg->d_nope,
+                                     cfg->d_v, st)))
+    return GDLA_ERR_LAUNCH;
+  // W_a = [W_a^Q | W_a^KV | W^lambda] and W_bqg = [W_b^Q | W^G], so that each of the two
+  // products of the query path is one GEMM
+  const int nH = cfg->n_signal + cfg->n_noise;
+  const long long lda = cfg->q_rank + cfg->kv_rank + cfg->d_rope + cfg->n_signal;
+  const long long nqq = (long long)nH * (cfg->d_nope + cfg->d_rope);
+  const long long ldb = nqq + (long long)cfg->n_signal * cfg->d_v;
+  const int nkv = cfg->kv_rank + cfg->d_rope;
+  if (launch_failed(launch_copy_cols(w->W_aQ, cfg->q_rank, base + off[1], lda, 0, cfg->d_model, cfg->q_rank, st)) ||
+      launch_failed(launch_copy_cols(w->W_aKV, nkv, base + off[1], lda, cfg->q_rank, cfg->d_model, nkv, st)) ||
+      launch_failed(launch_copy_cols(w->W_lambda, cfg->n_signal, base + off[1], lda, cfg->q_rank + nkv,
+                                     cfg->d_model, cfg->n_signal, st)) ||
+      launch_failed(launch_copy_cols(w->W_bQ, nqq, base + off[2], ldb, 0, cfg->q_rank, int(nqq), st)) ||
+      launch_failed(launch_copy_cols(w->W_G, (long long)cfg->n_signal * cfg->d_v, base + off[2], ldb, int(nqq),
+                                     cfg->q_rank, cfg->n_signal * cfg->d_v, st)))
     return GDLA_ERR_LAUNCH;
   out->w = *w;
-  out->W_UKt = dst;
+  out->W_UKt = base + off[0];
+  out->W_a = base + off[1];
+  out->W_bqg = base + off[2];
   out->cfg = *cfg;
   out->magic = kAbsorbedMagic;
   return GDLA_OK;
@@ -731,7 +769,7 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   const int B = q_len * n_seq;   // query rows: token r % q_len of sequence r / q_len
   int rc = check_config(cfg);
   if (rc) return rc;
-  if (!ab || ab->magic != kAbsorbedMagic || !ab->W_UKt) return GDLA_ERR_INVALID_ARG;
+  if (!ab || ab->magic != kAbsorbedMagic || !ab->W_UKt || !ab->W_a || !ab->W_bqg) return GDLA_ERR_INVALID_ARG;
   if (ab->cfg.d_model != cfg->d_model || ab->cfg.n_noise != cfg->n_noise)
     return GDLA_ERR_INVALID_ARG;  // absorbed for another layer shape (the window may differ)
   const gdla_weights_t* w = &ab->w;
@@ -752,7 +790,6 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   void* cQ = ws + off[WS_CQ];
   float* lam = reinterpret_cast<float*>(ws + off[WS_LAM]);
   float* QQ = reinterpret_cast<float*>(ws + off[WS_QQ]);
-  void* G = ws + off[WS_G];
   void* qt = ws + off[WS_KV];
   float* part = reinterpret_cast<float*>(ws + off[WS_ONOISE]);
   float* ml = reinterpret_cast<float*>(ws + off[WS_KR16]);
@@ -768,14 +805,9 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   GemmEpi ep{};
   ep.ldc = ld1; ep.out_type = OUT_F32; ep.M = B; ep.pos_T = 1; ep.rope = rope;
   ep.splitk = splitk; ep.splitk_floats = splitk_n;
-  ep.C = D1; ep.N = cfg->q_rank;
-  if (launch_failed(launch_gemm(x_new, cfg->d_model, w->W_aQ, cfg->q_rank, false, B, ep.N, cfg->d_model, ep, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  ep.C = D1 + cfg->q_rank; ep.N = cfg->kv_rank + cfg->d_rope;
-  if (launch_failed(launch_gemm(x_new, cfg->d_model, w->W_aKV, ep.N, false, B, ep.N, cfg->d_model, ep, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  ep.C = D1 + cfg->q_rank + cfg->kv_rank + cfg->d_rope; ep.N = cfg->n_signal;
-  if (launch_failed(launch_gemm(x_new, cfg->d_model, w->W_lambda, ep.N, false, B, ep.N, cfg->d_model, ep, ctl, st)))
+  // [c^Q | c^KV | k^R | lambda logits] = x [W_a^Q | W_a^KV | W^lambda]: one product
+  ep.C = D1; ep.N = ld1;
+  if (launch_failed(launch_gemm(x_new, cfg->d_model, ab->W_a, ld1, false, B, ld1, cfg->d_model, ep, ctl, st)))
     return GDLA_ERR_LAUNCH;
 
   NormParams np{};
@@ -786,23 +818,20 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   np.rope = rope; np.err = err;
   if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
 
+  // [q^C | q^R (rotated at the token's position) | G] = c^Q [W_b^Q | W^G], fp32: one product
   const int nqq = nH * (cfg->d_nope + cfg->d_rope);
+  const int ldq = nqq + cfg->n_signal * cfg->d_v;
   GemmEpi eq{};
-  eq.C = QQ; eq.ldc = nqq; eq.out_type = OUT_F32; eq.M = B; eq.N = nqq;
+  eq.C = QQ; eq.ldc = ldq; eq.out_type = OUT_F32; eq.M = B; eq.N = ldq;
   eq.rope_lo = nH * cfg->d_nope; eq.rope_hi = nqq; eq.pos_T = 1; eq.pos_ptr = cache_len;
   eq.pos_div = q_len;
   eq.rope = rope; eq.splitk = splitk; eq.splitk_floats = splitk_n;
-  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_bQ, nqq, false, B, nqq, cfg->q_rank, eq, ctl, st)))
-    return GDLA_ERR_LAUNCH;
-  GemmEpi eg{};
-  eg.C = G; eg.ldc = cfg->n_signal * cfg->d_v; eg.out_type = OUT_BF16; eg.M = B; eg.N = eg.ldc;
-  eg.pos_T = 1; eg.splitk = splitk; eg.splitk_floats = splitk_n;
-  if (launch_failed(launch_gemm(cQ, cfg->q_rank, w->W_G, eg.N, false, B, eg.N, cfg->q_rank, eg, ctl, st)))
+  if (launch_failed(launch_gemm(cQ, cfg->q_rank, ab->W_bqg, ldq, false, B, ldq, cfg->q_rank, eq, ctl, st)))
     return GDLA_ERR_LAUNCH;
 
   DecQParams qp{};
   qp.B = B; qp.n_groups = cfg->n_noise; qp.n_signal = cfg->n_signal; qp.n_heads = nH;
-  qp.QQ = QQ; qp.qq_ld = nqq; qp.rope_col0 = nH * cfg->d_nope; qp.W_UKt = ab->W_UKt; qp.qt = qt;
+  qp.QQ = QQ; qp.qq_ld = ldq; qp.rope_col0 = nH * cfg->d_nope; qp.W_UKt = ab->W_UKt; qp.qt = qt;
   if (launch_failed(launch_qtilde(qp, st))) return GDLA_ERR_LAUNCH;
 
   DecAttnParams dp{};
@@ -823,7 +852,7 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   DecCombParams cp{};
   cp.B = B; cp.n_groups = cfg->n_noise; cp.n_signal = cfg->n_signal; cp.n_ctas = dp.n_ctas;
   cp.tstart = dp.tstart;
-  cp.part = part; cp.ml = ml; cp.lam = lam; cp.G = G; cp.W_bKV = w->W_bKV; cp.Dg = Dg;
+  cp.part = part; cp.ml = ml; cp.lam = lam; cp.G = QQ + nqq; cp.g_ld = ldq; cp.W_bKV = w->W_bKV; cp.Dg = Dg;
   if (launch_failed(launch_dec_combine(cp, st))) return GDLA_ERR_LAUNCH;
 
   stage(3, st);

@@ -41,6 +41,24 @@ int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int 
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
+__global__ void copy_cols_kernel(const uint4* __restrict__ src, long long ld_src8, uint4* __restrict__ dst,
+                                 long long ld_dst8, long long col0_8, int rows, int cols8) {
+  const long long total = (long long)rows * cols8;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / cols8, c = i % cols8;
+    dst[r * ld_dst8 + col0_8 + c] = src[r * ld_src8 + c];
+  }
+}
+
+int launch_copy_cols(const void* src, long long ld_src, void* dst, long long ld_dst, int col0, int rows,
+                     int cols, cudaStream_t st) {
+  if ((cols | col0) % 8 || ld_src % 8 || ld_dst % 8) return -1;
+  copy_cols_kernel<<<1024, 256, 0, st>>>(static_cast<const uint4*>(src), ld_src / 8, static_cast<uint4*>(dst),
+                                         ld_dst / 8, col0 / 8, rows, cols / 8);
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
+}
+
 // q~ rows: qt[b][h][0..511] = W_UK_j q^C_h, qt[b][h][512..575] = rotated q^R_h (bf16).
 // CTA (KV head j, QT_RB rows b): W_UK_j^T (128 x 512 bf16, 128 KB) is staged in shared memory
 // with asynchronous copies, then the 5 QT_RB query rows of the group's heads are projected in
@@ -277,13 +295,13 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
     if (row >= 4 * nb) continue;
     const int b = b0 + row / 4, s = row % 4, sig = 4 * j + s;
     const long long o = (long long)b * p.n_signal * 128 + sig * 128 + 8 * cg;
-    const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.G) + o);
-    const uint32_t gu[4] = {gv.x, gv.y, gv.z, gv.w};
+    const float* gp = p.G + (long long)b * p.g_ld + sig * 128 + 8 * cg;
+    const float4 g0 = *reinterpret_cast<const float4*>(gp), g1 = *reinterpret_cast<const float4*>(gp + 4);
+    const float gf[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
     uint32_t out[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      out[e] = pack_bf162(sigmoidf_fast(__uint_as_float(gu[e] << 16)) * acc[r][2 * e],
-                          sigmoidf_fast(__uint_as_float(gu[e] & 0xFFFF0000u)) * acc[r][2 * e + 1]);
+      out[e] = pack_bf162(sigmoidf_fast(gf[2 * e]) * acc[r][2 * e], sigmoidf_fast(gf[2 * e + 1]) * acc[r][2 * e + 1]);
     *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Dg) + o) = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }

@@ -41,13 +41,18 @@ struct DecCombParams {
   const float* part;           // segment partials, slot c + r for CTA c and row r
   const float* ml;
   const float* lam;       // [B][n_signal]
-  const void* G;          // bf16 [B][n_signal * 128]
+  const float* G;         // fp32 gate logits: row b at G + b * g_ld, [n_signal * 128]
+  long long g_ld;
   const void* W_bKV;      // bf16 [kv_rank][n_groups * 256]
   void* Dg;               // bf16 [B][n_signal * 128]
 };
 
 int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int d_nope, int d_v,
                      cudaStream_t st);
+// dst[r][col0 + c] = src[r][c] for r < rows, c < cols (bf16; cols, ld_src, ld_dst, col0
+// multiples of 8): concatenation of weight column blocks
+int launch_copy_cols(const void* src, long long ld_src, void* dst, long long ld_dst, int col0, int rows,
+                     int cols, cudaStream_t st);
 int launch_qtilde(const DecQParams& p, cudaStream_t st);
 int launch_dec_sched(const DecAttnParams& p, cudaStream_t st);
 int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t st);

@@ -84,6 +84,9 @@ typedef struct {
 typedef struct {
   gdla_weights_t w;          /* the original weights (pointers copied, not the data) */
   void* W_UKt;               /* bf16 [n_kv_heads][d_nope][kv_rank]: K^C blocks of W_b^KV, transposed */
+  void* W_a;                 /* bf16 [d_model][q_rank + kv_rank + d_rope + n_signal]: W_a^Q | W_a^KV |
+                                W^lambda side by side (one down-projection per decode step) */
+  void* W_bqg;               /* bf16 [q_rank][n_heads (d_nope + d_rope) + n_signal d_v]: W_b^Q | W^G */
   gdla_config_t cfg;
   uint32_t magic;
 } gdla_absorbed_t;
@@ -227,8 +230,11 @@ int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void*
  *   x_new [B, d_model] bf16.  kv_cache [B, cap, kv_rank + d_rope] bf16: rows 0..len[b]-1 hold
  *   the cached latent entries; the new token's entry is written at row len[b] (so
  *   len[b] < cap) and it attends to rows 0..len[b] (or the last `window` of them).
- *   Rows after len[b] up to the end of its 128-row block are read (and multiplied by zero
- *   weights), so they must hold finite values, e.g. a zero-initialised cache.
+ *   Rows after len[b] are never used: those up to the end of its 64-row tile are read but
+ *   replaced by zeros on chip before they meet the attention weights, so an unwritten tail
+ *   (even NaN or Inf) does not reach the output.
+ *   absorbed: from gdla_absorb_weights for this layer (the query path multiplies by its
+ *   concatenated W_a and W_bqg).
  *   cache_len [B] int32 (device).  y [B, d_model] bf16 (written).
  *   workspace: >= gdla_workspace_size(cfg, B, cap, GDLA_MODE_DECODE) bytes. */
 int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* absorbed, const void* x_new,

@@ -39,7 +39,10 @@ def test_workspace_size_and_offsets(L):
     assert gb.gdla_workspace_size(cfg, 2, 256, 0) > n
     d = gb.gdla_workspace_size(cfg, 64, 1, gb.GDLA_MODE_DECODE)
     assert d > 64 * 80 * 576 * 2
-    assert gb.gdla_absorbed_size(cfg) == 16 * 128 * 512 * 2
+    # W_UK^T, then [W_a^Q | W_a^KV | W^lambda] and [W_b^Q | W^G], each rounded up to 256 bytes
+    r256 = lambda b: (b + 255) // 256 * 256
+    assert gb.gdla_absorbed_size(cfg) == (r256(16 * 128 * 512 * 2) + r256(4096 * 1664 * 2) +
+                                          r256(1024 * (80 * 192 + 64 * 128) * 2))
 
 
 def test_host_validation_without_gpu(L):
