@@ -832,7 +832,7 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   DecQParams qp{};
   qp.B = B; qp.n_groups = cfg->n_noise; qp.n_signal = cfg->n_signal; qp.n_heads = nH;
   qp.QQ = QQ; qp.qq_ld = ldq; qp.rope_col0 = nH * cfg->d_nope; qp.W_UKt = ab->W_UKt; qp.qt = qt;
-  if (launch_failed(launch_qtilde(qp, st))) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_qtilde(qp, ctl, st))) return GDLA_ERR_LAUNCH;
 
   DecAttnParams dp{};
   dp.R = B; dp.n_seq = n_seq; dp.cap = cap; dp.window = cfg->window; dp.cache_len = cache_len;

@@ -21,8 +21,9 @@
 
 namespace gdla {
 
-// W_UKt[j][c][l] = W_bKV[l][j * (d_nope + d_v) + c]
-__global__ void absorb_uk_kernel(const __nv_bfloat16* __restrict__ W_bKV, __nv_bfloat16* __restrict__ W_UKt,
+// W_UKt[j][c][l] = W_bKV[l][j * (d_nope + d_v) + c], in fp16 (the operand type of the q~ MMAs;
+// exact for weights of magnitude >= 2^-14, the fp16 normal range)
+__global__ void absorb_uk_kernel(const __nv_bfloat16* __restrict__ W_bKV, __half* __restrict__ W_UKt,
                                  int kv_rank, int n_kv, int d_nope, int d_v) {
   const long long total = (long long)n_kv * d_nope * kv_rank;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -30,14 +31,14 @@ __global__ void absorb_uk_kernel(const __nv_bfloat16* __restrict__ W_bKV, __nv_b
     const int l = int(i % kv_rank);
     const int c = int((i / kv_rank) % d_nope);
     const int j = int(i / ((long long)kv_rank * d_nope));
-    W_UKt[i] = W_bKV[(long long)l * n_kv * (d_nope + d_v) + j * (d_nope + d_v) + c];
+    W_UKt[i] = __float2half_rn(__bfloat162float(W_bKV[(long long)l * n_kv * (d_nope + d_v) + j * (d_nope + d_v) + c]));
   }
 }
 
 int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int d_nope, int d_v,
                      cudaStream_t st) {
   absorb_uk_kernel<<<1024, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W_bKV),
-                                         static_cast<__nv_bfloat16*>(W_UKt), kv_rank, n_kv, d_nope, d_v);
+                                         static_cast<__half*>(W_UKt), kv_rank, n_kv, d_nope, d_v);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
@@ -59,82 +60,147 @@ int launch_copy_cols(const void* src, long long ld_src, void* dst, long long ld_
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 
-// q~ rows: qt[b][h][0..511] = W_UK_j q^C_h, qt[b][h][512..575] = rotated q^R_h (bf16).
-// CTA (KV head j, QT_RB rows b): W_UK_j^T (128 x 512 bf16, 128 KB) is staged in shared memory
-// with asynchronous copies, then the 5 QT_RB query rows of the group's heads are projected in
-// fp32.  Thread tile: 10 query rows x 8 latent columns, so that one 16-byte load of weights and
-// one broadcast 16-byte load of q^C feed 40 FMAs (the kernel is FMA-bound, not load-bound).
-constexpr int QT_RB = 8;
-__global__ void __launch_bounds__(256) qtilde_kernel(DecQParams p) {
-  constexpr int NR = 5 * QT_RB;                // query rows of a CTA
-  constexpr int TR = NR / 4;                   // rows per thread (4 row groups)
-  extern __shared__ uint8_t qt_smem[];
-  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(qt_smem);              // [128][512]
-  float (*qc)[128] = reinterpret_cast<float (*)[128]>(qt_smem + 128 * 512 * 2);  // [NR][128]
-  const int j = blockIdx.x, b0 = blockIdx.y * QT_RB, tid = threadIdx.x;
-  const int nb = min(QT_RB, p.B - b0);
-  const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_UKt) + (long long)j * 128 * 512;
-  for (int i = tid; i < 128 * 512 / 8; i += blockDim.x) cp_async16(wsm + i * 8, W + i * 8);
-  const int heads[5] = {p.n_signal + j, 4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3};
-  for (int i = tid; i < NR * 32; i += blockDim.x) {
-    const int r = i / 32, c4 = i % 32, bb = r / 5, hh = r % 5;
-    *reinterpret_cast<float4*>(&qc[r][4 * c4]) =
-        bb < nb ? *reinterpret_cast<const float4*>(p.QQ + (long long)(b0 + bb) * p.qq_ld + heads[hh] * 128 + 4 * c4)
-                : make_float4(0.f, 0.f, 0.f, 0.f);
+// q~ rows: qt[b][h][0..511] = W_UK_j q^C_h, qt[b][h][512..575] = rotated q^R_h (bf16), on the
+// tensor cores.  Per KV head j the rows (b, h) of its five heads form one product
+//   [5 B x 128] (q^C, fp16) x [128 x 512] (W_UK_j^T, fp16) -> fp32 in TMEM,
+// one CTA per (j, 128 rows): the q^C rows are converted to fp16 by the CTA's threads into a
+// 128-byte-swizzled K-major tile, W_UK_j^T (128 KB) arrives by TMA as eight [128][64] MN-major
+// boxes, and two tcgen05.mma chains (M 128, N 256, K 128) fill 512 TMEM columns, which the
+// four warps (thread = row) round to bf16.  Rows of the group: r = 5 b + hh, hh = 0 the noise
+// head n_signal + j, hh = 1..4 the signal heads 4 j + hh - 1.
+namespace qtc {
+constexpr int A_BOX = 128 * 128;              // [128 rows][64 fp16]
+constexpr int B_BOX = 128 * 128;              // [128 K rows][64 N fp16]
+constexpr int A_OFF = 0, B_OFF = 2 * A_BOX;
+constexpr int BAR_OFF = B_OFF + 8 * B_BOX;
+constexpr int SMEM = BAR_OFF + 64 + 1024;
+}  // namespace qtc
+
+__device__ __forceinline__ int qt_head(int hh, int j, int n_signal) {
+  return hh == 0 ? n_signal + j : 4 * j + hh - 1;
+}
+
+__global__ void __launch_bounds__(128, 1)
+    qtilde_tc_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ DecQParams p, KernelCtl ctl) {
+  using namespace qtc;
+  extern __shared__ uint8_t qt_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qt_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar_w = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* bar_mma = bar_w + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_w + 2);
+  const int j = blockIdx.x, t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int R = 5 * p.B;
+  const int gr = blockIdx.y * 128 + t;          // this thread's row of the group
+  const bool rv = gr < R;
+  const int b = gr / 5, h = qt_head(gr % 5, j, p.n_signal);
+
+  if (t == 0) {
+    mbar_init(bar_w, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&mapW);
+    mbar_expect_tx(bar_w, 8 * B_BOX);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) tma_load_2d(smem + B_OFF + c * B_BOX, &mapW, bar_w, 64 * c, j * 128);
   }
-  cp_async_wait_all();
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  // ---- A: row gr's q^C (fp32) -> fp16, chunk k8 (8 values) at swizzled position k8 ^ (t & 7)
+  bool bad = false;
+  {
+    const float* src = p.QQ + (long long)b * p.qq_ld + (long long)h * 128;
+#pragma unroll 4
+    for (int k8 = 0; k8 < 16; ++k8) {
+      float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+      if (rv) {
+        v0 = *reinterpret_cast<const float4*>(src + 8 * k8);
+        v1 = *reinterpret_cast<const float4*>(src + 8 * k8 + 4);
+      }
+      const uint4 pk = make_uint4(pack_half2_sat(v0.x, v0.y, bad), pack_half2_sat(v0.z, v0.w, bad),
+                                  pack_half2_sat(v1.x, v1.y, bad), pack_half2_sat(v1.z, v1.w, bad));
+      *reinterpret_cast<uint4*>(smem + A_OFF + (k8 >> 3) * A_BOX + t * 128 + (((k8 & 7) ^ (t & 7)) << 4)) = pk;
+    }
+  }
+  if (bad && ctl.err) atomicCAS(ctl.err, 0, SITE_FP16_RANGE);
+  fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
-  const int cg = tid & 63, rg = tid >> 6;      // latent columns 8 cg .. 8 cg + 7; rows rg, rg + 4, ...
-  float acc[TR][8];
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+  if (t == 0) {
+    ok = mbar_wait(bar_w, 0, ctl, SITE_DEC_MMA);
+    if (ok) {
+      tc_fence_after();
+      constexpr uint32_t idesc = make_idesc(128, 256, 0, 0, 1);
+      const uint64_t da = sdesc_sw128(smem_u32(smem + A_OFF), 16, 1024);
+      const uint64_t db = sdesc_sw128(smem_u32(smem + B_OFF), B_BOX, 1024);
 #pragma unroll
-  for (int r = 0; r < TR; ++r)
+      for (int nh = 0; nh < 2; ++nh)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + 256 * nh, da + uint64_t((kk >> 2) * (A_BOX >> 4) + (kk & 3) * 2),
+                 db + uint64_t(nh * 4 * (B_BOX >> 4) + kk * 128), idesc, kk > 0 ? 1u : 0u);
+      mma_commit(bar_mma);
+    }
+  }
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    // ---- epilogue: thread t = TMEM lane t = row gr
+    const bool w = __all_sync(0xffffffffu, mbar_wait(bar_mma, 0, ctl, SITE_DEC_MMA));
+    tc_fence_after();
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.qt) + ((long long)b * p.n_heads + h) * 576;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    if (w) {
 #pragma unroll 1
-  for (int c = 0; c < 128; c += 4) {
-    float w[4][8];
+      for (int c = 0; c < 16; ++c) {
+        uint32_t v[32];
+        GDLA_TMEM_LD32(tmem + 32 * c + lane_off, v);
+        tmem_ld_wait();
+        if (!rv) continue;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(wsm + (c + k) * 512 + 8 * cg);
-      const uint32_t u[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w[k][2 * e] = __uint_as_float(u[e] << 16);
-        w[k][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+        for (int e = 0; e < 32; e += 8)
+          *reinterpret_cast<uint4*>(dst + 32 * c + e) =
+              make_uint4(pack_bf162(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                         pack_bf162(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
+                         pack_bf162(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
+                         pack_bf162(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
+      }
+      if (rv) {
+        const float* qr = p.QQ + (long long)b * p.qq_ld + p.rope_col0 + (long long)h * 64;
+#pragma unroll 4
+        for (int e = 0; e < 64; e += 8) {
+          const float4 a0 = *reinterpret_cast<const float4*>(qr + e), a1 = *reinterpret_cast<const float4*>(qr + e + 4);
+          *reinterpret_cast<uint4*>(dst + 512 + e) = make_uint4(pack_bf162(a0.x, a0.y), pack_bf162(a0.z, a0.w),
+                                                                pack_bf162(a1.x, a1.y), pack_bf162(a1.z, a1.w));
+        }
       }
     }
-#pragma unroll
-    for (int r = 0; r < TR; ++r) {
-      const float4 q4 = *reinterpret_cast<const float4*>(&qc[rg + 4 * r][c]);
-      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(qv[k], w[k][e], acc[r][e]);
-    }
   }
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.qt);
-#pragma unroll
-  for (int r = 0; r < TR; ++r) {
-    const int row = rg + 4 * r, bb = row / 5, hh = row % 5;
-    if (bb >= nb) continue;
-    *reinterpret_cast<uint4*>(out + ((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 8 * cg) =
-        make_uint4(pack_bf162(acc[r][0], acc[r][1]), pack_bf162(acc[r][2], acc[r][3]),
-                   pack_bf162(acc[r][4], acc[r][5]), pack_bf162(acc[r][6], acc[r][7]));
+  if (t == 0) {
+    // before TMEM is released: the MMAs (if issued) are complete, the weight copy has landed
+    if (ok) mbar_drain(bar_mma, 0, ctl.err);
+    else mbar_drain(bar_w, 0, ctl.err);
   }
-  for (int i = tid; i < NR * 64; i += blockDim.x) {
-    const int r = i / 64, e = i % 64, bb = r / 5, hh = r % 5;
-    if (bb >= nb) continue;
-    out[((long long)(b0 + bb) * p.n_heads + heads[hh]) * 576 + 512 + e] =
-        __float2bfloat16_rn(p.QQ[(long long)(b0 + bb) * p.qq_ld + p.rope_col0 + heads[hh] * 64 + e]);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
-int launch_qtilde(const DecQParams& p, cudaStream_t st) {
-  const int smem = 128 * 512 * 2 + 5 * QT_RB * 128 * 4;
-  if (cudaFuncSetAttribute(qtilde_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+int launch_qtilde(const DecQParams& p, KernelCtlHost ctl, cudaStream_t st) {
+  CUtensorMap mw;
+  if (make_tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.W_UKt, 512, (uint64_t)p.n_groups * 128, 512 * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return -3;
+  if (cudaFuncSetAttribute(qtilde_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qtc::SMEM) != cudaSuccess)
     return -4;
-  qtilde_kernel<<<dim3(p.n_groups, (p.B + QT_RB - 1) / QT_RB), 256, smem, st>>>(p);
+  KernelCtl kc{ctl.err, ctl.limit_ns};
+  qtilde_tc_kernel<<<dim3(p.n_groups, (5 * p.B + 127) / 128), 128, qtc::SMEM, st>>>(mw, p, kc);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 

@@ -11,7 +11,7 @@ struct DecQParams {
   int B, n_groups, n_signal, n_heads;
   const float* QQ;        // [B, qq_ld] fp32: q^C (head-major) | rotated q^R (head-major)
   int qq_ld, rope_col0;
-  const void* W_UKt;      // bf16 [n_groups][128][512]
+  const void* W_UKt;      // fp16 [n_groups][128][512]
   void* qt;               // bf16 [B][n_heads][576]
 };
 
@@ -53,7 +53,7 @@ int launch_absorb_uk(const void* W_bKV, void* W_UKt, int kv_rank, int n_kv, int 
 // multiples of 8): concatenation of weight column blocks
 int launch_copy_cols(const void* src, long long ld_src, void* dst, long long ld_dst, int col0, int rows,
                      int cols, cudaStream_t st);
-int launch_qtilde(const DecQParams& p, cudaStream_t st);
+int launch_qtilde(const DecQParams& p, KernelCtlHost ctl, cudaStream_t st);
 int launch_dec_sched(const DecAttnParams& p, cudaStream_t st);
 int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t st);
 int decode_cta_count();

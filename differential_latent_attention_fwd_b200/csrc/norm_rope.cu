@@ -122,6 +122,101 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(const __grid_constant__ 
     p.lam[(long long)m * p.n_signal + c] = 1.0f / (1.0f + expf(-rl[c]));
 }
 
+// The same epilogue with one CTA of 256 threads per token (q_rank 1024, kv_rank 512): for the
+// few rows of a decode step, where one warp per token would leave the step waiting on a single
+// warp's chain of loads, reductions and stores.  Thread t owns c^Q columns 4t .. 4t + 3 and,
+// for t < 128, c^KV columns 4t .. 4t + 3; warp 0 rotates k^R (pair lane, lane + 32); threads
+// t < n_signal form lambda.
+__global__ void __launch_bounds__(256) norm_rope_row_kernel(const __grid_constant__ NormParams p) {
+  __shared__ float red[2][8];
+  const int m = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const float* row = p.D1 + (long long)m * p.ld1;
+  const __nv_bfloat16* g_q = static_cast<const __nv_bfloat16*>(p.g_q);
+  const __nv_bfloat16* g_kv = static_cast<const __nv_bfloat16*>(p.g_kv);
+  const int row_w = p.kv_rank + 64;
+  const float4 q4 = *reinterpret_cast<const float4*>(row + 4 * t);
+  const bool has_kv = t < 128;
+  const float4 kv4 = has_kv ? *reinterpret_cast<const float4*>(row + p.q_rank + 4 * t) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float* rkr = row + p.q_rank + p.kv_rank;
+  const float x1 = warp == 0 ? rkr[lane] : 0.f, x2 = warp == 0 ? rkr[lane + 32] : 0.f;
+  const float xl = t < p.n_signal ? rkr[64 + t] : 0.f;
+  float sq = q4.x * q4.x + q4.y * q4.y + q4.z * q4.z + q4.w * q4.w;
+  float sk = kv4.x * kv4.x + kv4.y * kv4.y + kv4.z * kv4.z + kv4.w * kv4.w;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+  }
+  if (lane == 0) {
+    red[0][warp] = sq;
+    red[1][warp] = sk;
+  }
+  __syncthreads();
+  float tq = 0.f, tk = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    tq += red[0][w];
+    tk += red[1][w];
+  }
+  const float rq = rsqrtf(tq / float(p.q_rank) + p.eps);
+  const float rkvn = rsqrtf(tk / float(p.kv_rank) + p.eps);
+  {
+    float g[4] = {1.f, 1.f, 1.f, 1.f};
+    if (g_q) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) g[e] = __bfloat162float(g_q[4 * t + e]);
+    }
+    uint2 pk;
+    pk.x = pack_bf162(q4.x * rq * g[0], q4.y * rq * g[1]);
+    pk.y = pack_bf162(q4.z * rq * g[2], q4.w * rq * g[3]);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.cQ) + (long long)m * p.q_rank + 4 * t) = pk;
+  }
+  const int qps = p.q_per_seq > 1 ? p.q_per_seq : 1;
+  int pos = (p.pos_ptr ? p.pos_ptr[m / qps] + m % qps : ((m + p.row_off) % p.pos_T)) + p.pos_off;
+  const int seq = p.pos_ptr ? m / qps : ((m + p.row_off) / p.pos_T);
+  bool cache_ok = p.cache != nullptr;
+  if (cache_ok && (pos < 0 || pos >= p.cache_cap)) {
+    if (t == 0 && p.err) atomicCAS(p.err, 0, SITE_BAD_CACHE_LEN);
+    cache_ok = false;
+    pos = 0;
+  }
+  __nv_bfloat16* dsts[2] = {p.latent ? static_cast<__nv_bfloat16*>(p.latent) + (long long)m * row_w : nullptr,
+                            cache_ok ? static_cast<__nv_bfloat16*>(p.cache) + ((long long)seq * p.cache_cap + pos) * row_w
+                                     : nullptr};
+  if (has_kv) {
+    float g[4] = {1.f, 1.f, 1.f, 1.f};
+    if (g_kv) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) g[e] = __bfloat162float(g_kv[4 * t + e]);
+    }
+    uint2 pk;
+    pk.x = pack_bf162(kv4.x * rkvn * g[0], kv4.y * rkvn * g[1]);
+    pk.y = pack_bf162(kv4.z * rkvn * g[2], kv4.w * rkvn * g[3]);
+#pragma unroll
+    for (int d = 0; d < 2; ++d)
+      if (dsts[d]) *reinterpret_cast<uint2*>(dsts[d] + 4 * t) = pk;
+  }
+  if (warp == 0) {
+    float cs, sn;
+    rope_cs(pos, p.rope.inv_freq[lane], &cs, &sn);
+    const float k1 = x1 * cs - x2 * sn, k2 = x2 * cs + x1 * sn;
+#pragma unroll
+    for (int d = 0; d < 2; ++d) {
+      if (!dsts[d]) continue;
+      dsts[d][p.kv_rank + lane] = __float2bfloat16_rn(k1);
+      dsts[d][p.kv_rank + lane + 32] = __float2bfloat16_rn(k2);
+    }
+    if (p.kR16) {
+      __half* kR16 = static_cast<__half*>(p.kR16);
+      bool bad = false;
+      kR16[(long long)m * 64 + lane] = half_sat(k1, bad);
+      kR16[(long long)m * 64 + lane + 32] = half_sat(k2, bad);
+      if (bad && p.err) atomicCAS(p.err, 0, SITE_FP16_RANGE);
+    }
+  }
+  if (t < p.n_signal) p.lam[(long long)m * p.n_signal + t] = 1.0f / (1.0f + expf(-xl));
+}
+
 // fp16 copy of the rotated k^R of bf16 latent rows (a key prefix handed in by the caller)
 __global__ void latent_to_kr16_kernel(const __nv_bfloat16* __restrict__ latent, int row_w,
                                       int kv_rank, long long rows, __half* __restrict__ kR16, int* err) {
@@ -146,7 +241,9 @@ int launch_norm_rope(const NormParams& p, cudaStream_t st) {
   if (p.M <= 0) return 0;
   const int threads = 256;
   const int blocks = (p.M * 32 + threads - 1) / threads;
-  if (p.q_rank == 1024 && p.kv_rank == 512)
+  if (p.q_rank == 1024 && p.kv_rank == 512 && p.M <= 4096 && p.n_signal <= 256)
+    norm_rope_row_kernel<<<p.M, 256, 0, st>>>(p);      // few rows: a CTA per token
+  else if (p.q_rank == 1024 && p.kv_rank == 512)
     norm_rope_kernel<32, 16><<<blocks, threads, 0, st>>>(p);
   else if (p.q_rank == 128 && p.kv_rank == 128)
     norm_rope_kernel<4, 4><<<blocks, threads, 0, st>>>(p);

@@ -83,7 +83,7 @@ typedef struct {
  * the caller; `base` is the caller's device buffer holding the derived tensors. */
 typedef struct {
   gdla_weights_t w;          /* the original weights (pointers copied, not the data) */
-  void* W_UKt;               /* bf16 [n_kv_heads][d_nope][kv_rank]: K^C blocks of W_b^KV, transposed */
+  void* W_UKt;               /* fp16 [n_kv_heads][d_nope][kv_rank]: K^C blocks of W_b^KV, transposed */
   void* W_a;                 /* bf16 [d_model][q_rank + kv_rank + d_rope + n_signal]: W_a^Q | W_a^KV |
                                 W^lambda side by side (one down-projection per decode step) */
   void* W_bqg;               /* bf16 [q_rank][n_heads (d_nope + d_rope) + n_signal d_v]: W_b^Q | W^G */
