@@ -107,20 +107,43 @@ __global__ void __launch_bounds__(128, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  // ---- A: row gr's q^C (fp32) -> fp16, chunk k8 (8 values) at swizzled position k8 ^ (t & 7)
-  bool bad = false;
+  // ---- rows of warp w: 32 w .. 32 w + 31 of the tile.  First the rotated q^R of each row
+  // (bf16) straight into q~ columns 512..575: lane l of load k serves row 2 k + l / 16, float4
+  // l % 16; then the q^C rows, one row per load (lane l: float4 l), as fp16 into the
+  // 128-byte-swizzled K-major A tile (8 values = 16 bytes per chunk, two lanes per chunk)
+  const int row0 = blockIdx.y * 128 + 32 * warp;
   {
-    const float* src = p.QQ + (long long)b * p.qq_ld + (long long)h * 128;
 #pragma unroll 4
-    for (int k8 = 0; k8 < 16; ++k8) {
-      float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-      if (rv) {
-        v0 = *reinterpret_cast<const float4*>(src + 8 * k8);
-        v1 = *reinterpret_cast<const float4*>(src + 8 * k8 + 4);
+    for (int k = 0; k < 16; ++k) {
+      const int rr = row0 + 2 * k + (lane >> 4);
+      if (rr < R) {
+        const int bb = rr / 5, hr = qt_head(rr % 5, j, p.n_signal);
+        const float4 a = *reinterpret_cast<const float4*>(p.QQ + (long long)bb * p.qq_ld + p.rope_col0 +
+                                                          (long long)hr * 64 + 4 * (lane & 15));
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.qt) + ((long long)bb * p.n_heads + hr) * 576 + 512 +
+                                  4 * (lane & 15)) = make_uint2(pack_bf162(a.x, a.y), pack_bf162(a.z, a.w));
       }
-      const uint4 pk = make_uint4(pack_half2_sat(v0.x, v0.y, bad), pack_half2_sat(v0.z, v0.w, bad),
-                                  pack_half2_sat(v1.x, v1.y, bad), pack_half2_sat(v1.z, v1.w, bad));
-      *reinterpret_cast<uint4*>(smem + A_OFF + (k8 >> 3) * A_BOX + t * 128 + (((k8 & 7) ^ (t & 7)) << 4)) = pk;
+    }
+  }
+  bool bad = false;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int rr = row0 + 16 * half + i;
+      v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (rr < R)
+        v[i] = *reinterpret_cast<const float4*>(p.QQ + (long long)(rr / 5) * p.qq_ld +
+                                                (long long)qt_head(rr % 5, j, p.n_signal) * 128 + 4 * lane);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int r = 32 * warp + 16 * half + i;        // row within the tile
+      const int k8 = lane >> 1;                        // 8-value chunk of the 128 columns
+      *reinterpret_cast<uint2*>(smem + A_OFF + (k8 >> 3) * A_BOX + r * 128 + (((k8 & 7) ^ (r & 7)) << 4) +
+                                8 * (lane & 1)) =
+          make_uint2(pack_half2_sat(v[i].x, v[i].y, bad), pack_half2_sat(v[i].z, v[i].w, bad));
     }
   }
   if (bad && ctl.err) atomicCAS(ctl.err, 0, SITE_FP16_RANGE);
@@ -167,15 +190,6 @@ __global__ void __launch_bounds__(128, 1)
                          pack_bf162(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
                          pack_bf162(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
                          pack_bf162(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
-      }
-      if (rv) {
-        const float* qr = p.QQ + (long long)b * p.qq_ld + p.rope_col0 + (long long)h * 64;
-#pragma unroll 4
-        for (int e = 0; e < 64; e += 8) {
-          const float4 a0 = *reinterpret_cast<const float4*>(qr + e), a1 = *reinterpret_cast<const float4*>(qr + e + 4);
-          *reinterpret_cast<uint4*>(dst + 512 + e) = make_uint4(pack_bf162(a0.x, a0.y), pack_bf162(a0.z, a0.w),
-                                                                pack_bf162(a1.x, a1.y), pack_bf162(a1.z, a1.w));
-        }
       }
     }
   }
@@ -352,7 +366,8 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
 #pragma unroll
       for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(dv[k], w[k][e], acc[r][e]);
+        for (int e = 0; e < 8; e += 2)       // packed f32x2 FMAs
+          ffma2vv(acc[r][e], acc[r][e + 1], w[k][e], w[k][e + 1], dv[k], dv[k], acc[r][e], acc[r][e + 1]);
     }
   }
 #pragma unroll
