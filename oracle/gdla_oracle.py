@@ -561,7 +561,9 @@ def gdla_prefill_packed(x_packed, cu_seqlens, weights: dict, cfg: OracleConfig, 
 # --------------------------------------------------------------------------------------
 # full layer: decode (one new token per sequence, keys = cached latent rows + itself)
 # --------------------------------------------------------------------------------------
-def _decode_common(x_new, weights, cache, cache_len, cfg, g_q, g_kv):
+def _decode_common(x_new, weights, cache, cache_len, cfg, g_q, g_kv, own_rows=None):
+    """own_rows [B, kv_rank + d_rope]: the new tokens' latent rows as the cache stores them
+    (e.g. after quantization), used as their own keys instead of the computed rows."""
     W = _weights64(weights)
     gq = None if g_q is None else f64(g_q)
     gkv = None if g_kv is None else f64(g_kv)
@@ -572,6 +574,9 @@ def _decode_common(x_new, weights, cache, cache_len, cfg, g_q, g_kv):
     cbar_new, kR_new = kv_latent(xn, W["W_aKV"], gkv, pos, cfg)
     lam = lambda_coeff(xn, W["W_lambda"])
     G = gate_logits(cQ, W["W_G"], cfg)
+    if own_rows is not None:
+        own = f64(own_rows)
+        cbar_new, kR_new = own[:, : cfg.kv_rank], own[:, cfg.kv_rank:]
     return W, lens, cQ, qC, qR, cbar_new, kR_new, lam, G
 
 
@@ -584,7 +589,7 @@ def _keys_of(cache, b, p, cbar_new, kR_new, cfg):
 
 
 def gdla_decode(x_new, weights: dict, cache, cache_len, cfg: OracleConfig, g_q=None, g_kv=None,
-                return_parts: bool = False):
+                return_parts: bool = False, own_rows=None):
     """Literal decode: the prefill definition applied to the new token at position cache_len[b].
 
     cache [B, cap, kv_rank + d_rope] holds (normalised c^KV | rotated k^R) per cached token.
@@ -592,7 +597,7 @@ def gdla_decode(x_new, weights: dict, cache, cache_len, cfg: OracleConfig, g_q=N
     Returns y [B, d] (and the new latent rows when ``return_parts``).
     """
     W, lens, cQ, qC, qR, cbar_new, kR_new, lam, G = _decode_common(
-        x_new, weights, cache, cache_len, cfg, g_q, g_kv)
+        x_new, weights, cache, cache_len, cfg, g_q, g_kv, own_rows)
     y = np.empty((len(lens), cfg.d_model))
     Dgs = []
     for b, p in enumerate(lens):
@@ -608,7 +613,7 @@ def gdla_decode(x_new, weights: dict, cache, cache_len, cfg: OracleConfig, g_q=N
 
 
 def gdla_decode_absorbed(x_new, weights: dict, cache, cache_len, cfg: OracleConfig, g_q=None,
-                         g_kv=None):
+                         g_kv=None, own_rows=None):
     """Weight-absorbed decode: attention runs in the latent space, K^C and V are never formed.
 
     With W_UK_j / W_UV_j the K^C / V column blocks of W_bKV for KV head j:
@@ -619,7 +624,7 @@ def gdla_decode_absorbed(x_new, weights: dict, cache, cache_len, cfg: OracleConf
     every cached row is too slow.
     """
     W, lens, cQ, qC, qR, cbar_new, kR_new, lam, G = _decode_common(
-        x_new, weights, cache, cache_len, cfg, g_q, g_kv)
+        x_new, weights, cache, cache_len, cfg, g_q, g_kv, own_rows)
     scale = 1.0 / np.sqrt(cfg.d_nope + cfg.d_rope)
     kvh = kv_head_of(cfg)
     nmap = noise_of_signal(cfg)
@@ -667,3 +672,123 @@ def gdla_decode_multi(x_new, weights: dict, cache, cache_len, cfg: OracleConfig,
         for i in range(q):
             y[b, i] = one(xn[b, i][None], weights, ext, [L + i], cfg, g_q=g_q, g_kv=g_kv)[0]
     return y
+
+
+# --------------------------------------------------------------------------------------
+# MXFP8 latent cache: decode over cache rows stored at 8 bits per value
+# --------------------------------------------------------------------------------------
+# The report's low-precision recipe stores tensors in MXFP8 (paperglide.net summary, the
+# low-precision training paragraph and the Figure 3 caption).  Written out here from the
+# format's definition (OCP microscaling: blocks of 32 values sharing one power-of-two scale,
+# stored as an 8-bit exponent E with scale 2^(E - 127); values in FP8 E4M3):
+#   E4M3 byte s.eeee.mmm: e = 0 -> (-1)^s 2^-6 (m / 8) (zero and subnormals); e > 0 ->
+#   (-1)^s 2^(e - 7) (1 + m / 8); s.1111.111 is NaN; no infinities; largest finite 448.
+# Readings where the pages say nothing (listed in the design notes):
+#   * a latent-cache row (576 values: normalised c^KV | rotated k^R) is 18 blocks of 32;
+#   * the block scale is the smallest power of two 2^k with max|v| <= 448 2^k (nothing is
+#     clipped), k in [-127, 127]; an all-zero block takes k = -127;
+#   * values v / 2^k are rounded to the nearest E4M3 value, ties to the even code;
+#   * a row of n values (n a multiple of 32) is stored as n E4M3 bytes, then its n / 32 scale
+#     bytes, then zero bytes up to a multiple of 16: 576 + 18 + 14 = 608 bytes for the layer's rows.
+FP8_BLOCK = 32
+E4M3_MAX = 448.0
+
+
+def fp8_row_bytes(n: int) -> int:
+    """Stored bytes of a row of n values."""
+    return (n + n // FP8_BLOCK + 15) // 16 * 16
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """float64 value of E4M3 codes (NaN for the two NaN codes), from the bit fields."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+_E4M3_POS = e4m3_value(np.arange(0x7F))          # codes 0x00..0x7E: the finite values >= 0, increasing
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Codes of the E4M3 values nearest to finite x (ties to the even code), saturating at
+    +-448.  By search over the 127 non-negative finite values."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 0x7E)       # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - _E4M3_POS[lo], _E4M3_POS[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(a == _E4M3_POS[hi], hi, code)
+    return (code | np.where((x < 0) & (code != 0), 0x80, 0)).astype(np.uint8)
+
+
+def mx_block_exponent(amax) -> np.ndarray:
+    """Smallest k with amax <= 448 * 2^k (k in [-127, 127]); -127 for an all-zero block."""
+    amax = np.asarray(amax, dtype=np.float64)
+    out = np.full(amax.shape, -127, dtype=np.int64)
+    nz = amax > 0
+    k = np.ceil(np.log2(np.where(nz, amax, 1.0) / E4M3_MAX)).astype(np.int64)
+    # log2 is a library routine with rounding: settle the boundary exactly
+    k = np.where(E4M3_MAX * np.exp2(k.astype(np.float64)) < amax, k + 1, k)
+    k = np.where(E4M3_MAX * np.exp2((k - 1).astype(np.float64)) >= amax, k - 1, k)
+    out[nz] = np.clip(k[nz], -127, 127)
+    return out
+
+
+def mxfp8_quantize_rows(rows) -> np.ndarray:
+    """Rows [N, n] (any float values; n a multiple of 32) -> stored bytes [N, fp8_row_bytes(n)]."""
+    v = f64(rows)
+    v = v.reshape(-1, v.shape[-1])
+    n = v.shape[1]
+    blk = v.reshape(v.shape[0], -1, FP8_BLOCK)
+    k = mx_block_exponent(np.abs(blk).max(axis=-1))                     # [N, n / 32]
+    q = e4m3_round(blk / np.exp2(k.astype(np.float64))[..., None]).reshape(v.shape[0], n)
+    out = np.zeros((v.shape[0], fp8_row_bytes(n)), dtype=np.uint8)
+    out[:, :n] = q
+    out[:, n: n + k.shape[1]] = (k + 127).astype(np.uint8)
+    return out
+
+
+def mxfp8_dequantize_rows(stored, n: int) -> np.ndarray:
+    """Stored bytes [N, fp8_row_bytes(n)] -> float64 rows [N, n]: each E4M3 value times its
+    block's 2^(E - 127)."""
+    b = np.asarray(stored, dtype=np.uint8).reshape(-1, fp8_row_bytes(n))
+    nblk = n // FP8_BLOCK
+    vals = e4m3_value(b[:, :n]).reshape(b.shape[0], nblk, FP8_BLOCK)
+    k = b[:, n: n + nblk].astype(np.int64) - 127
+    return (vals * np.exp2(k.astype(np.float64))[..., None]).reshape(b.shape[0], n)
+
+
+def gdla_decode_fp8(x_new, weights: dict, cache8, cache_len, cfg: OracleConfig, g_q=None, g_kv=None,
+                    route: str = "absorbed", q_len: int = 1):
+    """Decode over an MXFP8 latent cache cache8 [B, cap, fp8_row_bytes(kv_rank + d_rope)] (uint8).  Every key row the
+    attention reads is the dequantized stored row, the new tokens' own rows included: each new
+    token's latent row is quantized (it is what the cache receives) and read back.  With q_len > 1,
+    x_new is [B, q_len, d] and token i sits at position cache_len[b] + i.  Returns y [B, q_len, d]
+    (q_len > 1) or [B, d]."""
+    W = _weights64(weights)
+    gkv = None if g_kv is None else f64(g_kv)
+    one = gdla_decode if route == "literal" else gdla_decode_absorbed
+    xn = f64(x_new)
+    if q_len == 1 and xn.ndim == 2:
+        xn = xn[:, None, :]
+    B, q = xn.shape[0], xn.shape[1]
+    lens = [int(v) for v in (cache_len.tolist() if hasattr(cache_len, "tolist") else cache_len)]
+    y = np.empty((B, q, cfg.d_model))
+    for b in range(B):
+        L = lens[b]
+        n = cfg.kv_rank + cfg.d_rope
+        rows = mxfp8_dequantize_rows(np.asarray(cache8[b, :L]), n) if L else np.zeros((0, n))
+        cbar, kR = kv_latent(xn[b], W["W_aKV"], gkv, L + np.arange(q), cfg)
+        new = mxfp8_dequantize_rows(mxfp8_quantize_rows(np.concatenate([cbar, kR], -1)), n)
+        ext = np.concatenate([rows, new], 0)[None]
+        for i in range(q):
+            # keys: the cached rows, the earlier new tokens' stored rows, and its own stored row
+            y[b, i] = one(xn[b, i][None], weights, ext, [L + i], cfg, g_q=g_q, g_kv=g_kv,
+                          own_rows=ext[0, L + i][None])[0]
+    return y[:, 0] if q_len == 1 and np.asarray(x_new).ndim == 2 else y
