@@ -715,7 +715,8 @@ _E4M3_POS = e4m3_value(np.arange(0x7F))          # codes 0x00..0x7E: the finite 
 
 def e4m3_round(x) -> np.ndarray:
     """Codes of the E4M3 values nearest to finite x (ties to the even code), saturating at
-    +-448.  By search over the 127 non-negative finite values."""
+    +-448.  By search over the 127 non-negative finite values; the sign bit is x's sign (the
+    format is sign-magnitude: a negative x that rounds to zero gives -0, code 0x80)."""
     x = np.asarray(x, dtype=np.float64)
     a = np.minimum(np.abs(x), E4M3_MAX)
     hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 0x7E)       # first value >= a
@@ -724,7 +725,7 @@ def e4m3_round(x) -> np.ndarray:
     pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
     code = np.where(pick_hi, hi, lo)
     code = np.where(a == _E4M3_POS[hi], hi, code)
-    return (code | np.where((x < 0) & (code != 0), 0x80, 0)).astype(np.uint8)
+    return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
 
 
 def mx_block_exponent(amax) -> np.ndarray:

@@ -33,9 +33,10 @@ def test_e4m3_rounding_matches_torch():
     mids = (pos[1:] + pos[:-1]) / 2                  # exact ties: to the even code
     x = np.concatenate([np.random.default_rng(0).uniform(-460, 460, 200000), pos, -pos, mids, -mids,
                         np.random.default_rng(1).uniform(-2.0 ** -6, 2.0 ** -6, 20000)])
-    mine = O.e4m3_value(O.e4m3_round(x))
-    ref = torch.tensor(x).to(torch.float8_e4m3fn).double().numpy()
-    assert np.array_equal(mine, ref)
+    x = np.concatenate([x, [0.0, -0.0, -1e-5, 1e-5, -2.0 ** -10, 2.0 ** -10]])
+    mine = O.e4m3_round(x)
+    ref = torch.tensor(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(mine, ref)                  # the codes, sign of zero included
 
 
 def test_e4m3_saturates_at_448():
