@@ -87,6 +87,9 @@ def lib() -> ctypes.CDLL:
             "gdla_attn_train_workspace_size": [cfgp, I, I, ctypes.POINTER(SZ), ctypes.POINTER(SZ)],
             "gdla_attn_train_fwd": [cfgp, P, P, P, P, P, I, I, P, P, P, P, SZ, P],
             "gdla_attn_bwd": [cfgp, P, P, P, P, P, P, P, P, I, I, P, P, P, P, P, P, SZ, P],
+            "gdla_quantize_latent_fp8": [cfgp, P, ctypes.c_longlong, P, P],
+            "gdla_decode_fp8_fwd": [cfgp, abp, P, I, P, P, I, I, P, P, SZ, P],
+            "gdla_dequantize_latent_fp8": [cfgp, P, ctypes.c_longlong, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -245,6 +248,29 @@ def gdla_latent_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, pos_offset: int, la
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+FP8_ROW_BYTES = 608     # GDLA_FP8_ROW_BYTES
+
+
+def gdla_quantize_latent_fp8(cfg, latent: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """bf16 latent rows [..., 576] -> MXFP8 rows [..., 608] (uint8), same leading shape."""
+    rows = latent.numel() // (cfg.kv_rank + cfg.d_rope)
+    if out.numel() != rows * FP8_ROW_BYTES:
+        raise ValueError("out must hold rows x 608 bytes")
+    _check("gdla_quantize_latent_fp8", lib().gdla_quantize_latent_fp8(
+        ctypes.byref(cfg), _ptr(latent, torch.bfloat16, "latent"), rows, _ptr(out, torch.uint8, "out"),
+        _stream(stream)))
+
+
+def gdla_dequantize_latent_fp8(cfg, stored: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """MXFP8 rows [..., 608] (uint8) -> bf16 latent rows [..., 576]."""
+    rows = stored.numel() // FP8_ROW_BYTES
+    if out.numel() != rows * (cfg.kv_rank + cfg.d_rope):
+        raise ValueError("out must hold rows x 576 values")
+    _check("gdla_dequantize_latent_fp8", lib().gdla_dequantize_latent_fp8(
+        ctypes.byref(cfg), _ptr(stored, torch.uint8, "stored"), rows, _ptr(out, torch.bfloat16, "out"),
+        _stream(stream)))
+
+
 def gdla_prefill_context_fwd(cfg, w: gdla_weights_t, x: torch.Tensor, pos_offset: int,
                              prefix_latent: torch.Tensor | None, y: torch.Tensor,
                              workspace: torch.Tensor, latent_out: torch.Tensor | None = None,
@@ -288,6 +314,20 @@ def gdla_decode_multi_fwd(cfg, absorbed: gdla_absorbed_t, x_new: torch.Tensor, k
         ctypes.byref(cfg), ctypes.byref(absorbed), _ptr(x_new, torch.bfloat16, "x_new"), q_len,
         _ptr(kv_cache, torch.bfloat16, "kv_cache"), _ptr(cache_len, torch.int32, "cache_len"),
         kv_cache.shape[1], n_seq, _ptr(y, torch.bfloat16, "y"), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def gdla_decode_fp8_fwd(cfg, absorbed: gdla_absorbed_t, x_new: torch.Tensor, kv_cache8: torch.Tensor,
+                        cache_len: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor,
+                        stream=None) -> None:
+    """Decode over an MXFP8 cache kv_cache8 [n_seq, cap, 608] (uint8).  x_new [n_seq, d] (one new
+    token per sequence) or [n_seq, q_len, d]; y has the shape of x_new."""
+    n_seq = x_new.shape[0]
+    q_len = x_new.shape[1] if x_new.dim() == 3 else 1
+    _check("gdla_decode_fp8_fwd", lib().gdla_decode_fp8_fwd(
+        ctypes.byref(cfg), ctypes.byref(absorbed), _ptr(x_new, torch.bfloat16, "x_new"), q_len,
+        _ptr(kv_cache8, torch.uint8, "kv_cache8"), _ptr(cache_len, torch.int32, "cache_len"),
+        kv_cache8.shape[1], n_seq, _ptr(y, torch.bfloat16, "y"), _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

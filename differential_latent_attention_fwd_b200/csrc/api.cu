@@ -550,6 +550,32 @@ int gdla_prefill_varlen_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, c
                       static_cast<cudaStream_t>(stream), &vl);
 }
 
+static int check_fp8_rows(const gdla_config_t* cfg, const void* a, long long rows, const void* b) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (cfg->kv_rank + cfg->d_rope != 576) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  if (!a || !b || rows < 0 || !aligned16(a) || !aligned16(b)) return GDLA_ERR_INVALID_ARG;
+  return GDLA_OK;
+}
+
+int gdla_quantize_latent_fp8(const gdla_config_t* cfg, const void* latent, long long rows, void* out,
+                             void* stream) {
+  int rc = check_fp8_rows(cfg, latent, rows, out);
+  if (rc) return rc;
+  return launch_failed(launch_mxfp8_quantize(latent, rows, out, static_cast<cudaStream_t>(stream)))
+             ? GDLA_ERR_LAUNCH
+             : GDLA_OK;
+}
+
+int gdla_dequantize_latent_fp8(const gdla_config_t* cfg, const void* stored, long long rows, void* out,
+                               void* stream) {
+  int rc = check_fp8_rows(cfg, stored, rows, out);
+  if (rc) return rc;
+  return launch_failed(launch_mxfp8_dequantize(stored, rows, out, static_cast<cudaStream_t>(stream)))
+             ? GDLA_ERR_LAUNCH
+             : GDLA_OK;
+}
+
 int gdla_latent_fwd(const gdla_config_t* cfg, const gdla_weights_t* w, const void* x, int T,
                     int pos_offset, void* latent_out, void* workspace, size_t ws_bytes, void* stream) {
   int rc = check_config(cfg);
@@ -762,9 +788,11 @@ int gdla_decode_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const v
                                ws_bytes, stream);
 }
 
-int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const void* x_new,
-                          int q_len, void* kv_cache, const int* cache_len, int cap, int n_seq,
-                          void* y, void* workspace, size_t ws_bytes, void* stream) {
+// The decode step over a bf16 latent cache or an MXFP8 one (fp8): the same kernels, except
+// that the new rows are appended in MXFP8 form and the attention converts the cache tiles.
+static int decode_impl(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const void* x_new, int q_len,
+                       void* kv_cache, const int* cache_len, int cap, int n_seq, void* y, void* workspace,
+                       size_t ws_bytes, void* stream, bool fp8) {
   if (q_len <= 0 || n_seq <= 0 || (long long)q_len * n_seq > (1 << 20)) return GDLA_ERR_INVALID_ARG;
   const int B = q_len * n_seq;   // query rows: token r % q_len of sequence r / q_len
   int rc = check_config(cfg);
@@ -814,7 +842,7 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   np.D1 = D1; np.ld1 = ld1; np.M = B; np.q_rank = cfg->q_rank; np.kv_rank = cfg->kv_rank;
   np.n_signal = cfg->n_signal; np.g_q = w->g_q; np.g_kv = w->g_kv; np.eps = cfg->rms_eps;
   np.cQ = cQ; np.latent = nullptr; np.kR16 = nullptr; np.lam = lam; np.pos_T = 1;
-  np.pos_ptr = cache_len; np.q_per_seq = q_len; np.cache = kv_cache; np.cache_cap = cap;
+  np.pos_ptr = cache_len; np.q_per_seq = q_len; np.cache = kv_cache; np.cache_fp8 = fp8; np.cache_cap = cap;
   np.rope = rope; np.err = err;
   if (launch_failed(launch_norm_rope(np, st))) return GDLA_ERR_LAUNCH;
 
@@ -832,12 +860,13 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
   DecQParams qp{};
   qp.B = B; qp.n_groups = cfg->n_noise; qp.n_signal = cfg->n_signal; qp.n_heads = nH;
   qp.QQ = QQ; qp.qq_ld = ldq; qp.rope_col0 = nH * cfg->d_nope; qp.W_UKt = ab->W_UKt; qp.qt = qt;
+  qp.qt_f16 = fp8;
   if (launch_failed(launch_qtilde(qp, ctl, st))) return GDLA_ERR_LAUNCH;
 
   DecAttnParams dp{};
   dp.R = B; dp.n_seq = n_seq; dp.cap = cap; dp.window = cfg->window; dp.cache_len = cache_len;
   dp.q_len = q_len;
-  dp.cache = kv_cache; dp.qt = qt;
+  dp.cache = kv_cache; dp.cache_fp8 = fp8; dp.qt = qt;
   dp.scale_log2 = float(1.4426950408889634 / sqrt(double(cfg->d_nope + cfg->d_rope)));
   dp.tstart = reinterpret_cast<int*>(ws + off[WS_DSCHED]);
   dp.n_ctas = decode_cta_count();
@@ -864,6 +893,21 @@ int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, c
     return GDLA_ERR_LAUNCH;
   stage(4, st);
   return GDLA_OK;
+}
+
+int gdla_decode_multi_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const void* x_new,
+                          int q_len, void* kv_cache, const int* cache_len, int cap, int n_seq,
+                          void* y, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_impl(cfg, ab, x_new, q_len, kv_cache, cache_len, cap, n_seq, y, workspace, ws_bytes, stream,
+                     false);
+}
+
+int gdla_decode_fp8_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* ab, const void* x_new, int q_len,
+                        void* kv_cache8, const int* cache_len, int cap, int n_seq, void* y, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  if (cfg && cfg->kv_rank + cfg->d_rope != 576) return GDLA_ERR_UNSUPPORTED_SHAPE;
+  return decode_impl(cfg, ab, x_new, q_len, kv_cache8, cache_len, cap, n_seq, y, workspace, ws_bytes, stream,
+                     true);
 }
 
 int gdla_set_stage_events(void* const* events, int n) {

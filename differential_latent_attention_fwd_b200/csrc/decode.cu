@@ -120,8 +120,12 @@ __global__ void __launch_bounds__(128, 1)
         const int bb = rr / 5, hr = qt_head(rr % 5, j, p.n_signal);
         const float4 a = *reinterpret_cast<const float4*>(p.QQ + (long long)bb * p.qq_ld + p.rope_col0 +
                                                           (long long)hr * 64 + 4 * (lane & 15));
+        bool bad_r = false;
         *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.qt) + ((long long)bb * p.n_heads + hr) * 576 + 512 +
-                                  4 * (lane & 15)) = make_uint2(pack_bf162(a.x, a.y), pack_bf162(a.z, a.w));
+                                  4 * (lane & 15)) =
+            p.qt_f16 ? make_uint2(pack_half2_sat(a.x, a.y, bad_r), pack_half2_sat(a.z, a.w, bad_r))
+                     : make_uint2(pack_bf162(a.x, a.y), pack_bf162(a.z, a.w));
+        if (bad_r && ctl.err) atomicCAS(ctl.err, 0, SITE_FP16_RANGE);
       }
     }
   }
@@ -183,14 +187,17 @@ __global__ void __launch_bounds__(128, 1)
         GDLA_TMEM_LD32(tmem + 32 * c + lane_off, v);
         tmem_ld_wait();
         if (!rv) continue;
+        // bf16 q~, or fp16 (saturated, reported) for the fp16 MMAs over an MXFP8 cache
+        auto pk = [&](float a, float b) { return p.qt_f16 ? pack_half2_sat(a, b, bad) : pack_bf162(a, b); };
 #pragma unroll
         for (int e = 0; e < 32; e += 8)
           *reinterpret_cast<uint4*>(dst + 32 * c + e) =
-              make_uint4(pack_bf162(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
-                         pack_bf162(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
-                         pack_bf162(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
-                         pack_bf162(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
+              make_uint4(pk(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                         pk(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
+                         pk(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
+                         pk(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
       }
+      if (bad && ctl.err) atomicCAS(ctl.err, 0, SITE_FP16_RANGE);
     }
   }
   if (t == 0) {

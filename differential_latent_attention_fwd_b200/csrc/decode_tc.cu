@@ -40,6 +40,7 @@
 // never wrote (NaN, Inf) cannot reach the output through 0 * NaN.
 #include "gdla_common.cuh"
 #include "gdla_decode.h"
+#include "gdla_fp8.cuh"
 #include "gdla_internal.h"
 
 namespace gdla {
@@ -63,6 +64,14 @@ constexpr float RESCALE_THRESHOLD = 8.0f;
 constexpr int PREFETCH_AHEAD = 0;               // tiles of L2 prefetch ahead of the TMA loads (0: none;
                                                 // measured no faster at 3, slower at 6 and 12)
 static_assert(SMEM <= 232448, "shared memory");
+// MXFP8 cache rows (608 bytes: 576 E4M3 codes, 18 block scales, padding): a tile's raw rows
+// land by TMA in the upper half of each latent slot ([64 rows][128 codes], 8 KB) and after the
+// first 2 KB of its rope slot ([64 rows][96 bytes]: 64 rope codes + the 18 scales + 14 pad);
+// two converter warps turn them into fp16 in place, in the layout of the bf16 form.
+constexpr int LAT_RAW = LAT_SLOT / 2;
+constexpr int ROPE_RAW = 2048;
+constexpr int SMEM8 = SMEM;
+constexpr int C8_WARPS = 2;
 // The M = 128 score MMA reads 128 rows of each 80-row q~ box: the 48 rows past a box are the
 // next box, or (for the last box) the first 6 KB of P.  They only feed unused score rows.
 static_assert(P_OFF + 48 * 128 <= LAT_OFF, "q~ box over-read stays in the P buffer");
@@ -73,6 +82,7 @@ struct SkBars {
   uint64_t q_ready;                               // q~ (TMA part + TMEM part) of a segment
   uint64_t lat_full[dsk::NLAT], lat_empty[dsk::NLAT];
   uint64_t rope_full[dsk::NROPE], rope_empty[dsk::NROPE];
+  uint64_t lat_raw[dsk::NLAT], rope_raw[dsk::NROPE];  // MXFP8 cache: raw rows landed (TMA)
   uint64_t s_full, s_free, p_ready, pv_done, seg_done, mma_final;
   uint32_t tmem_base;
 };
@@ -132,9 +142,16 @@ struct DskWalk {
   }
 };
 
-__global__ void __launch_bounds__(192, 1)
+static_assert(sizeof(SkBars) <= 1024, "barrier block");
+
+// C8: the cache holds MXFP8 rows (mapC: their 128-code latent boxes, mapR: their rope codes and
+// scales); 64 more threads (warps 6-7) convert them, and q~, P and the cache tiles are fp16 MMA
+// operands instead of bf16.
+template <bool C8>
+__global__ void __launch_bounds__(C8 ? 256 : 192, 1)
     dec_attn_sk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapC,
-                       const __grid_constant__ DecAttnParams p, KernelCtl ctl) {
+                       const __grid_constant__ CUtensorMap mapR, const __grid_constant__ DecAttnParams p,
+                       KernelCtl ctl) {
   using namespace dsk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = dsk_align(smem_raw);
@@ -144,13 +161,16 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_ready, 5);          // producer's expect_tx + the four softmax warps
+    // full: the producer's expect_tx (bf16 tiles), or one arrival per converter warp (C8)
     for (int s = 0; s < NLAT; ++s) {
-      mbar_init(&bars->lat_full[s], 1);
+      mbar_init(&bars->lat_full[s], C8 ? C8_WARPS : 1);
       mbar_init(&bars->lat_empty[s], 1);
+      mbar_init(&bars->lat_raw[s], 1);
     }
     for (int s = 0; s < NROPE; ++s) {
-      mbar_init(&bars->rope_full[s], 1);
+      mbar_init(&bars->rope_full[s], C8 ? C8_WARPS : 1);
       mbar_init(&bars->rope_empty[s], 1);
+      mbar_init(&bars->rope_raw[s], 1);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, 4);           // one arrival per softmax warp: S read out of TMEM
@@ -161,6 +181,7 @@ __global__ void __launch_bounds__(192, 1)
     fence_mbar_init();
     tma_prefetch_desc(&mapQ);
     tma_prefetch_desc(&mapC);
+    if (C8) tma_prefetch_desc(&mapR);
   }
   if (warp == 5) {
     tmem_alloc(&bars->tmem_base, 512);
@@ -213,9 +234,15 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t ph = (gl / NLAT) & 1;
             if (gl >= NLAT && !mbar_wait(&bars->lat_empty[s], ph ^ 1, ctl, SITE_DEC_PRODUCER)) { ok = false; break; }
             uint8_t* dst = smem + LAT_OFF + s * LAT_SLOT;
-            mbar_expect_tx(&bars->lat_full[s], LAT_SLOT);
-            tma_load_2d(dst, &mapC, &bars->lat_full[s], 128 * u, y);
-            tma_load_2d(dst + LAT_SLOT / 2, &mapC, &bars->lat_full[s], 128 * u + 64, y);
+            if (C8) {
+              // [64 rows][128 codes] of the MXFP8 rows into the slot's upper half
+              mbar_expect_tx(&bars->lat_raw[s], LAT_SLOT / 2);
+              tma_load_2d(dst + LAT_RAW, &mapC, &bars->lat_raw[s], 128 * u, y);
+            } else {
+              mbar_expect_tx(&bars->lat_full[s], LAT_SLOT);
+              tma_load_2d(dst, &mapC, &bars->lat_full[s], 128 * u, y);
+              tma_load_2d(dst + LAT_SLOT / 2, &mapC, &bars->lat_full[s], 128 * u + 64, y);
+            }
             lat_issued |= 1u << s;
             lat_par = (lat_par & ~(1u << s)) | (ph << s);
           }
@@ -224,8 +251,14 @@ __global__ void __launch_bounds__(192, 1)
             const int s = J % NROPE;
             const uint32_t ph = (J / NROPE) & 1;
             if (J >= NROPE && !mbar_wait(&bars->rope_empty[s], ph ^ 1, ctl, SITE_DEC_PRODUCER)) { ok = false; break; }
-            mbar_expect_tx(&bars->rope_full[s], ROPE_SLOT);
-            tma_load_2d(smem + ROPE_OFF + s * ROPE_SLOT, &mapC, &bars->rope_full[s], 512, y);
+            if (C8) {
+              // [64 rows][96 bytes]: the rope codes, the 18 block scales and the padding
+              mbar_expect_tx(&bars->rope_raw[s], 64 * 96);
+              tma_load_2d(smem + ROPE_OFF + s * ROPE_SLOT + ROPE_RAW, &mapR, &bars->rope_raw[s], 512, y);
+            } else {
+              mbar_expect_tx(&bars->rope_full[s], ROPE_SLOT);
+              tma_load_2d(smem + ROPE_OFF + s * ROPE_SLOT, &mapC, &bars->rope_full[s], 512, y);
+            }
             rope_issued |= 1u << s;
             rope_par = (rope_par & ~(1u << s)) | (ph << s);
           }
@@ -239,17 +272,19 @@ __global__ void __launch_bounds__(192, 1)
         ++seg;
       }
       for (int s = 0; s < NLAT; ++s)
-        if (lat_issued & (1u << s)) mbar_drain(&bars->lat_full[s], (lat_par >> s) & 1, ctl.err);
+        if (lat_issued & (1u << s))
+          mbar_drain(C8 ? &bars->lat_raw[s] : &bars->lat_full[s], (lat_par >> s) & 1, ctl.err);
       for (int s = 0; s < NROPE; ++s)
-        if (rope_issued & (1u << s)) mbar_drain(&bars->rope_full[s], (rope_par >> s) & 1, ctl.err);
+        if (rope_issued & (1u << s))
+          mbar_drain(C8 ? &bars->rope_raw[s] : &bars->rope_full[s], (rope_par >> s) & 1, ctl.err);
       if (q_issued) mbar_drain(&bars->q_ready, (seg - 1) & 1, ctl.err);
     }
   } else if (warp == 5) {
     if (lane == 0) {
       // ============================================================ MMA issuer
       // Descriptors as (low, high) words; offsets below are in 16-byte units of the low word.
-      constexpr uint32_t idesc_s = make_idesc(128, TP, 1, 0, 0);
-      constexpr uint32_t idesc_o = make_idesc(128, NH, 1, 1, 0);
+      constexpr uint32_t idesc_s = make_idesc(128, TP, C8 ? 0 : 1, 0, 0);    // fp16 (C8) or bf16
+      constexpr uint32_t idesc_o = make_idesc(128, NH, C8 ? 0 : 1, 1, 0);
       const uint32_t hi = uint32_t(sdesc_sw128(smem_u32(smem), 16, 1024) >> 32);
       const uint32_t qs_lo = uint32_t(sdesc_sw128(smem_u32(smem + QS_OFF), 16, 1024));
       const uint32_t p_lo = uint32_t(sdesc_sw128(smem_u32(smem + P_OFF), 16, 1024));
@@ -333,6 +368,97 @@ __global__ void __launch_bounds__(192, 1)
       mma_commit(&bars->mma_final);
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
+  } else if (C8 && warp >= 6) {
+    // ============================================================ MXFP8 converters (warps 6-7)
+    // Thread c = row c of every tile.  Per tile: the rope box first (its bytes hold the row's
+    // 18 block scales, which the thread keeps for the latent units), then the four latent
+    // units; each unit: all 64 threads read their raw row, meet at a named barrier (the fp16
+    // output overwrites the raw bytes), convert E4M3 x 2^k -> fp16 into the 128-byte-swizzled
+    // K-major boxes and publish the slot.  Rows outside the row's key range become zeros, so an
+    // unwritten cache tail (NaN codes or scales) never reaches the MMAs.
+    const int r = threadIdx.x - 192;
+    const int sw = r & 7;
+    bool ok = true;
+    int J = 0;
+    bool fp16_bad = false;
+    // 16 E4M3 codes (one uint4) times 2^k -> 16 fp16 values (two uint4)
+    // (rows outside the key range are converted too, then replaced by zeros: only valid rows
+    // may report an fp16 range error)
+    auto convert16 = [&](const uint4 c, float s, uint4& o0, uint4& o1, bool valid) {
+      bool bad = false;
+      const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+      uint32_t h[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t x = f16x2_from_e4m3x2(uint16_t(w[i] >> (16 * e)));
+          const float lo = __half2float(__ushort_as_half(uint16_t(x & 0xFFFFu))) * s;
+          const float hi = __half2float(__ushort_as_half(uint16_t(x >> 16))) * s;
+          h[2 * i + e] = pack_half2_sat(lo, hi, bad);
+        }
+      }
+      fp16_bad |= bad && valid;
+      o0 = valid ? make_uint4(h[0], h[1], h[2], h[3]) : make_uint4(0u, 0u, 0u, 0u);
+      o1 = valid ? make_uint4(h[4], h[5], h[6], h[7]) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    while (ok && walk.next(p, &sg)) {
+      for (int j = 0; j < sg.g1 - sg.g0 && ok; ++j, ++J) {
+        const int pos = (sg.tile0 + j) * TP + r;
+        const bool valid = pos >= sg.lo && pos <= sg.hi;
+        // ---- rope box and scales
+        const int rs = J % NROPE;
+        const bool wr = mbar_wait(&bars->rope_raw[rs], (J / NROPE) & 1, ctl, SITE_DEC_CONVERT);
+        uint8_t* rslot = smem + ROPE_OFF + rs * ROPE_SLOT;
+        const uint8_t* raw = rslot + ROPE_RAW + r * 96;
+        uint4 rc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rc[i] = *reinterpret_cast<const uint4*>(raw + 16 * i);
+        const uint4 sc = *reinterpret_cast<const uint4*>(raw + 64);          // scales of blocks 0..15
+        const uint32_t sc2 = *reinterpret_cast<const uint32_t*>(raw + 80);   // blocks 16, 17
+        // every raw row read before any is overwritten (and a failed wait stops both warps)
+        if (named_bar_or(2, 64, !wr)) { ok = false; break; }
+        {
+          const float s16 = exp2i(int(sc2 & 0xFFu) - 127), s17 = exp2i(int((sc2 >> 8) & 0xFFu) - 127);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {       // codes 16 i .. 16 i + 15: chunks 2 i, 2 i + 1
+            uint4 o0, o1;
+            convert16(rc[i], i < 2 ? s16 : s17, o0, o1, valid);
+            *reinterpret_cast<uint4*>(rslot + r * 128 + (((2 * i) ^ sw) << 4)) = o0;
+            *reinterpret_cast<uint4*>(rslot + r * 128 + (((2 * i + 1) ^ sw) << 4)) = o1;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->rope_full[rs]);
+        // ---- latent units
+        const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll 1
+        for (int u = 0; u < 4; ++u) {
+          const int gl = 4 * J + u, s = gl % NLAT;
+          const bool wl = mbar_wait(&bars->lat_raw[s], (gl / NLAT) & 1, ctl, SITE_DEC_CONVERT);
+          uint8_t* slot = smem + LAT_OFF + s * LAT_SLOT;
+          uint4 c[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) c[i] = *reinterpret_cast<const uint4*>(slot + LAT_RAW + r * 128 + 16 * i);
+          if (named_bar_or(2, 64, !wl)) { ok = false; break; }
+          // codes 16 i .. 16 i + 15 of the unit: block 4 u + i / 2; box i / 4, chunks 2 (i % 4), +1
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float sk = exp2i(int((scw[u] >> (8 * (i >> 1))) & 0xFFu) - 127);
+            uint4 o0, o1;
+            convert16(c[i], sk, o0, o1, valid);
+            uint8_t* box = slot + (i >> 2) * (LAT_SLOT / 2) + r * 128;
+            *reinterpret_cast<uint4*>(box + (((2 * (i & 3)) ^ sw) << 4)) = o0;
+            *reinterpret_cast<uint4*>(box + (((2 * (i & 3) + 1) ^ sw) << 4)) = o1;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->lat_full[s]);
+        }
+      }
+    }
+    if (fp16_bad && p.err) atomicCAS(p.err, 0, SITE_FP16_RANGE);
   } else {
     // ============================================================ softmax / epilogue (warps 0-3)
     const int q = warp;                      // TMEM lane quarter
@@ -438,8 +564,9 @@ __global__ void __launch_bounds__(192, 1)
         // P has one buffer: PV(J - 1) must have read it (earlier segments' PVs are complete)
         const bool w3 = j == 0 || mbar_wait(&bars->pv_done, (J - 1) & 1, ctl, SITE_DEC_SOFTMAX);
         carried_fail = !w3;
-        if (edge && bnd < TP - 1) {
-          // rows past the row's last key: zero them in the four latent slots before the PV
+        if (!C8 && edge && bnd < TP - 1) {
+          // rows past the row's last key: zero them in the four latent slots before the PV (the
+          // MXFP8 converters have written such rows as zeros already)
           const int r0 = bnd + 1;
           const int nbytes = (TP - r0) * 128;
 #pragma unroll 1
@@ -472,9 +599,17 @@ __global__ void __launch_bounds__(192, 1)
                 p0 = (c >= a && c <= bnd) ? p0 : 0.f;
                 p1 = (c + 1 >= a && c + 1 <= bnd) ? p1 : 0.f;
               }
-              pk[e] = pack_bf162(p0, p1);
               // the row sum adds the rounded values the PV multiplies (weights summing to 1)
-              const float r0 = __uint_as_float(pk[e] << 16), r1 = __uint_as_float(pk[e] & 0xFFFF0000u);
+              float r0, r1;
+              if (C8) {
+                pk[e] = pack_half2(p0, p1);
+                r0 = __half2float(__ushort_as_half(uint16_t(pk[e] & 0xFFFFu)));
+                r1 = __half2float(__ushort_as_half(uint16_t(pk[e] >> 16)));
+              } else {
+                pk[e] = pack_bf162(p0, p1);
+                r0 = __uint_as_float(pk[e] << 16);
+                r1 = __uint_as_float(pk[e] & 0xFFFF0000u);
+              }
               if (e & 1) fadd2(ls2, ls3, r0, r1); else fadd2(ls0, ls1, r0, r1);
             }
             *reinterpret_cast<uint4*>(row + ((k ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -581,17 +716,36 @@ int launch_dec_sched(const DecAttnParams& p, cudaStream_t st) {
 }
 
 int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t st) {
-  CUtensorMap mq, mc;
-  if (make_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.qt, 576, (uint64_t)p.R * dsk::NH, 576 * 2,
-                   64, dsk::NH, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      make_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.cache, 576, (uint64_t)p.n_seq * p.cap, 576 * 2,
-                   64, dsk::TP, CU_TENSOR_MAP_SWIZZLE_128B))
+  CUtensorMap mq, mc, mr;
+  const bool c8 = p.cache_fp8 != 0;
+  if (make_tmap_2d(&mq, c8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.qt, 576,
+                   (uint64_t)p.R * dsk::NH, 576 * 2, 64, dsk::NH, CU_TENSOR_MAP_SWIZZLE_128B))
     return -3;
-  if (cudaFuncSetAttribute(dec_attn_sk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dsk::SMEM) != cudaSuccess)
-    return -4;
+  if (c8) {
+    // MXFP8 rows of 608 bytes: [64 rows][128 codes] latent boxes, [64 rows][96 bytes] rope + scales
+    if (make_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.cache, FP8_ROW_BYTES, (uint64_t)p.n_seq * p.cap,
+                     FP8_ROW_BYTES, 128, dsk::TP, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        make_tmap_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.cache, FP8_ROW_BYTES, (uint64_t)p.n_seq * p.cap,
+                     FP8_ROW_BYTES, 96, dsk::TP, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return -3;
+  } else {
+    if (make_tmap_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.cache, 576, (uint64_t)p.n_seq * p.cap, 576 * 2,
+                     64, dsk::TP, CU_TENSOR_MAP_SWIZZLE_128B))
+      return -3;
+    mr = mc;
+  }
   KernelCtl kc{ctl.err, ctl.limit_ns};
-  dec_attn_sk_kernel<<<p.n_ctas, 192, dsk::SMEM, st>>>(mq, mc, p, kc);
+  if (c8) {
+    if (cudaFuncSetAttribute(dec_attn_sk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dsk::SMEM8) != cudaSuccess)
+      return -4;
+    dec_attn_sk_kernel<true><<<p.n_ctas, 256, dsk::SMEM8, st>>>(mq, mc, mr, p, kc);
+  } else {
+    if (cudaFuncSetAttribute(dec_attn_sk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dsk::SMEM) != cudaSuccess)
+      return -4;
+    dec_attn_sk_kernel<false><<<p.n_ctas, 192, dsk::SMEM, st>>>(mq, mc, mr, p, kc);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 

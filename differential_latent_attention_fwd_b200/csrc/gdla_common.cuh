@@ -30,7 +30,7 @@ enum : int {
   SITE_GEMM_PRODUCER = 0x101, SITE_GEMM_MMA = 0x102, SITE_GEMM_EPI = 0x103,
   SITE_ATTN_PRODUCER = 0x201, SITE_ATTN_MMA = 0x202, SITE_ATTN_SOFTMAX = 0x203,
   SITE_DRAIN = 0x301, SITE_SELFTEST = 0x401,
-  SITE_DEC_PRODUCER = 0x501, SITE_DEC_MMA = 0x502, SITE_DEC_SOFTMAX = 0x503,
+  SITE_DEC_PRODUCER = 0x501, SITE_DEC_MMA = 0x502, SITE_DEC_SOFTMAX = 0x503, SITE_DEC_CONVERT = 0x504,
   SITE_BWD_PRODUCER = 0x511, SITE_BWD_MMA = 0x512, SITE_BWD_SOFTMAX = 0x513,
   SITE_BAD_CACHE_LEN = 0x601,  // a cache_len entry outside [0, cap): that sequence is skipped
   SITE_BAD_CU_SEQLENS = 0x602, // document offsets not 0..total non-decreasing: bad documents skipped

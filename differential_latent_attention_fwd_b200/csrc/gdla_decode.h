@@ -12,7 +12,8 @@ struct DecQParams {
   const float* QQ;        // [B, qq_ld] fp32: q^C (head-major) | rotated q^R (head-major)
   int qq_ld, rope_col0;
   const void* W_UKt;      // fp16 [n_groups][128][512]
-  void* qt;               // bf16 [B][n_heads][576]
+  void* qt;               // bf16 [B][n_heads][576], fp16 when qt_f16
+  int qt_f16;
 };
 
 // Upper bound of the decode attention grid (the merge kernel keeps one weight per segment of a
@@ -24,8 +25,9 @@ struct DecAttnParams {
   int n_seq, cap, window;
   int q_len;              // new tokens per sequence
   const int* cache_len;   // [n_seq] keys cached before the new tokens
-  const void* cache;      // bf16 [n_seq][cap][576]
-  const void* qt;         // bf16 [R][80][576]
+  const void* cache;      // bf16 [n_seq][cap][576], or MXFP8 rows [n_seq][cap][608] (cache_fp8)
+  int cache_fp8;
+  const void* qt;         // bf16 [R][80][576] (fp16 with an MXFP8 cache)
   float scale_log2;
   int* tstart;            // [R + 1] tile prefix over the rows (dec_sched_kernel)
   int n_ctas;             // grid of the attention kernel (G): slots = G + R - 1

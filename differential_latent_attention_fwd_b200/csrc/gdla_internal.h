@@ -82,7 +82,8 @@ struct NormParams {
   int pos_off;                // added to the position (a key prefix of pos_off tokens precedes row 0)
   int row_off;                // token index of row 0 in the full token matrix (row pieces)
   int q_per_seq;              // new tokens per sequence (0 is read as 1)
-  void* cache;                // optional bf16 [n_seq, cache_cap, kv_rank + 64]
+  void* cache;                // optional bf16 [n_seq, cache_cap, kv_rank + 64], or MXFP8 rows
+  int cache_fp8;              //   [n_seq, cache_cap, 608] when cache_fp8 (norm_rope_row_kernel only)
   long long cache_cap;
   int* err;                   // device error word (bad cache_len is reported here)
   RopeTable rope;
@@ -150,5 +151,9 @@ int launch_latent_to_kr16(const void* latent, int kv_rank, long long rows, void*
                           cudaStream_t st);
 int launch_attn_prefill(const void* QQ, int qq_ld, const void* KV, const void* kR16,
                         const AttnParams& p, KernelCtlHost ctl, cudaStream_t st);
+
+// MXFP8 latent-cache rows (gdla_fp8.cuh): bf16 rows [rows][576] <-> stored rows [rows][608]
+int launch_mxfp8_quantize(const void* in, long long rows, void* out, cudaStream_t st);
+int launch_mxfp8_dequantize(const void* in, long long rows, void* out, cudaStream_t st);
 
 }  // namespace gdla

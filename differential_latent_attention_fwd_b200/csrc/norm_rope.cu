@@ -9,6 +9,7 @@
 //   lambda   = sigmoid(x W^lambda), one per signal head  -> fp32
 // Position: prefill row m is token m % T of sequence m / T; decode row b is at pos_ptr[b].
 #include "gdla_common.cuh"
+#include "gdla_fp8.cuh"
 #include "gdla_internal.h"
 
 namespace gdla {
@@ -180,9 +181,32 @@ __global__ void __launch_bounds__(256) norm_rope_row_kernel(const __grid_constan
     cache_ok = false;
     pos = 0;
   }
+  const bool c8 = p.cache_fp8 != 0;
   __nv_bfloat16* dsts[2] = {p.latent ? static_cast<__nv_bfloat16*>(p.latent) + (long long)m * row_w : nullptr,
-                            cache_ok ? static_cast<__nv_bfloat16*>(p.cache) + ((long long)seq * p.cache_cap + pos) * row_w
-                                     : nullptr};
+                            cache_ok && !c8 ? static_cast<__nv_bfloat16*>(p.cache) + ((long long)seq * p.cache_cap + pos) * row_w
+                                            : nullptr};
+  // MXFP8 cache row (gdla_fp8.cuh): the bf16-rounded values, 32 per block (8 threads here)
+  uint8_t* row8 = cache_ok && c8 ? static_cast<uint8_t*>(p.cache) + ((long long)seq * p.cache_cap + pos) * FP8_ROW_BYTES
+                                 : nullptr;
+  if (row8 && t < 128) {
+    float g[4] = {1.f, 1.f, 1.f, 1.f};
+    if (g_kv) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) g[e] = __bfloat162float(g_kv[4 * t + e]);
+    }
+    const float b0 = __bfloat162float(__float2bfloat16_rn(kv4.x * rkvn * g[0]));
+    const float b1 = __bfloat162float(__float2bfloat16_rn(kv4.y * rkvn * g[1]));
+    const float b2 = __bfloat162float(__float2bfloat16_rn(kv4.z * rkvn * g[2]));
+    const float b3 = __bfloat162float(__float2bfloat16_rn(kv4.w * rkvn * g[3]));
+    float amax = fmaxf(fmaxf(fabsf(b0), fabsf(b1)), fmaxf(fabsf(b2), fabsf(b3)));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const int k = mx_block_exp(amax);
+    const float inv = exp2i(-k);
+    *reinterpret_cast<uint32_t*>(row8 + 4 * t) =
+        uint32_t(e4m3x2_from(b0 * inv, b1 * inv)) | (uint32_t(e4m3x2_from(b2 * inv, b3 * inv)) << 16);
+    if ((t & 7) == 0) row8[FP8_SCALE_OFF + (t >> 3)] = uint8_t(k + 127);
+  }
   if (has_kv) {
     float g[4] = {1.f, 1.f, 1.f, 1.f};
     if (g_kv) {
@@ -205,6 +229,24 @@ __global__ void __launch_bounds__(256) norm_rope_row_kernel(const __grid_constan
       if (!dsts[d]) continue;
       dsts[d][p.kv_rank + lane] = __float2bfloat16_rn(k1);
       dsts[d][p.kv_rank + lane + 32] = __float2bfloat16_rn(k2);
+    }
+    if (row8) {
+      // rope dims 0..31 form block 16 and 32..63 block 17 (one value per lane each)
+      const float r1 = __bfloat162float(__float2bfloat16_rn(k1)), r2 = __bfloat162float(__float2bfloat16_rn(k2));
+      float a1 = fabsf(r1), a2 = fabsf(r2);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, o));
+        a2 = fmaxf(a2, __shfl_xor_sync(0xffffffffu, a2, o));
+      }
+      const int k16 = mx_block_exp(a1), k17 = mx_block_exp(a2);
+      row8[p.kv_rank + lane] = uint8_t(e4m3x2_from(r1 * exp2i(-k16), 0.f) & 0xFFu);
+      row8[p.kv_rank + 32 + lane] = uint8_t(e4m3x2_from(r2 * exp2i(-k17), 0.f) & 0xFFu);
+      if (lane == 0) {
+        row8[FP8_SCALE_OFF + 16] = uint8_t(k16 + 127);
+        row8[FP8_SCALE_OFF + 17] = uint8_t(k17 + 127);
+      }
+      if (lane >= 1 && lane <= FP8_ROW_BYTES - FP8_SCALE_OFF - 18) row8[FP8_SCALE_OFF + 17 + lane] = 0;
     }
     if (p.kR16) {
       __half* kR16 = static_cast<__half*>(p.kR16);
@@ -241,8 +283,10 @@ int launch_norm_rope(const NormParams& p, cudaStream_t st) {
   if (p.M <= 0) return 0;
   const int threads = 256;
   const int blocks = (p.M * 32 + threads - 1) / threads;
-  if (p.q_rank == 1024 && p.kv_rank == 512 && p.M <= 4096 && p.n_signal <= 256)
-    norm_rope_row_kernel<<<p.M, 256, 0, st>>>(p);      // few rows: a CTA per token
+  if (p.q_rank == 1024 && p.kv_rank == 512 && (p.M <= 4096 || p.cache_fp8) && p.n_signal <= 256)
+    norm_rope_row_kernel<<<p.M, 256, 0, st>>>(p);      // few rows (or an MXFP8 cache): a CTA per token
+  else if (p.cache_fp8)
+    return -2;
   else if (p.q_rank == 1024 && p.kv_rank == 512)
     norm_rope_kernel<32, 16><<<blocks, threads, 0, st>>>(p);
   else if (p.q_rank == 128 && p.kv_rank == 128)

@@ -114,3 +114,27 @@ class GdlaLayer:
         gb.gdla_decode_multi_fwd(self.cfg, self.absorbed(stream), x_new, kv_cache, cache_len, y, ws,
                                  stream)
         return y
+
+    def decode_fp8(self, x_new: torch.Tensor, kv_cache8: torch.Tensor, cache_len: torch.Tensor,
+                   y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """Decode over an MXFP8 latent cache [n_seq, cap, 608] (uint8); x_new [n_seq, d] or
+        [n_seq, q_len, d]."""
+        if y is None:
+            y = torch.empty(x_new.shape, dtype=torch.bfloat16, device=self.device)
+        rows = x_new.shape[0] * (x_new.shape[1] if x_new.dim() == 3 else 1)
+        ws = self.workspace(rows, kv_cache8.shape[1], gb.GDLA_MODE_DECODE)
+        gb.gdla_decode_fp8_fwd(self.cfg, self.absorbed(stream), x_new, kv_cache8, cache_len, y, ws, stream)
+        return y
+
+    def quantize_latent_fp8(self, latent: torch.Tensor, stream=None) -> torch.Tensor:
+        """bf16 latent rows [..., 576] -> MXFP8 rows [..., 608] (uint8)."""
+        out = torch.empty(latent.shape[:-1] + (gb.FP8_ROW_BYTES,), dtype=torch.uint8, device=latent.device)
+        gb.gdla_quantize_latent_fp8(self.cfg, latent, out, stream)
+        return out
+
+    def dequantize_latent_fp8(self, stored: torch.Tensor, stream=None) -> torch.Tensor:
+        """MXFP8 rows [..., 608] (uint8) -> bf16 latent rows [..., 576]."""
+        out = torch.empty(stored.shape[:-1] + (self.cfg.kv_rank + self.cfg.d_rope,), dtype=torch.bfloat16,
+                          device=stored.device)
+        gb.gdla_dequantize_latent_fp8(self.cfg, stored, out, stream)
+        return out

@@ -226,6 +226,33 @@ int gdla_attn_bwd(const gdla_config_t* cfg, const void* qq, const void* kv, cons
 int gdla_absorb_weights(const gdla_config_t* cfg, const gdla_weights_t* w, void* dst,
                         size_t dst_bytes, gdla_absorbed_t* out, void* stream);
 
+/* MXFP8 latent cache (the report's low-precision format: MXFP8, i.e. blocks of 32 values
+ * sharing a power-of-two scale, each value in FP8 E4M3; paperglide.net summary, the
+ * low-precision paragraph and Figure 3).  A latent row of kv_rank + d_rope = 576 values is
+ * stored in GDLA_FP8_ROW_BYTES = 608 bytes: the 576 E4M3 codes of v / 2^k, then one byte k + 127
+ * per block of 32 values, then 14 zero bytes; k is the smallest integer with max|v| <= 448 2^k
+ * over the block (clamped to [-127, 127]; -127 for an all-zero block) and the codes are the
+ * nearest E4M3 values, ties to even.  Half the bytes of a bf16 row (1152).
+ *
+ * gdla_quantize_latent_fp8: bf16 rows [rows][576] (e.g. a prefill's kv_cache_out) -> stored
+ * rows [rows][608] (uint8).  gdla_dequantize_latent_fp8: stored rows -> bf16 rows (exact inside
+ * bf16's normal range: every stored value has 4 significant bits).  Both device memory; rows >= 0. */
+#define GDLA_FP8_ROW_BYTES 608
+int gdla_quantize_latent_fp8(const gdla_config_t* cfg, const void* latent, long long rows, void* out,
+                             void* stream);
+int gdla_dequantize_latent_fp8(const gdla_config_t* cfg, const void* stored, long long rows, void* out,
+                               void* stream);
+
+/* Decode over an MXFP8 latent cache: gdla_decode_multi_fwd with kv_cache8 [n_seq, cap, 608]
+ * (uint8, rows as gdla_quantize_latent_fp8 writes them; row cache_len[b] + i receives new token
+ * i's entry, quantized from its bf16 latent values).  The attention reads 608 bytes per cached
+ * position instead of 1152 and multiplies fp16 operands (q~, P and the converted tiles; fp32
+ * accumulation); a value outside the fp16 range is saturated and reported (site 0x701).
+ * Same workspace as gdla_decode_fwd. */
+int gdla_decode_fp8_fwd(const gdla_config_t* cfg, const gdla_absorbed_t* absorbed, const void* x_new,
+                        int q_len, void* kv_cache8, const int* cache_len, int cap, int n_seq, void* y,
+                        void* workspace, size_t ws_bytes, void* stream);
+
 /* Decode one new token per sequence.
  *   x_new [B, d_model] bf16.  kv_cache [B, cap, kv_rank + d_rope] bf16: rows 0..len[b]-1 hold
  *   the cached latent entries; the new token's entry is written at row len[b] (so

@@ -769,14 +769,16 @@ def gdla_decode_fp8(x_new, weights: dict, cache8, cache_len, cfg: OracleConfig, 
                     route: str = "absorbed", q_len: int = 1):
     """Decode over an MXFP8 latent cache cache8 [B, cap, fp8_row_bytes(kv_rank + d_rope)] (uint8).  Every key row the
     attention reads is the dequantized stored row, the new tokens' own rows included: each new
-    token's latent row is quantized (it is what the cache receives) and read back.  With q_len > 1,
+    token's latent row is rounded to bf16 and quantized (it is what the cache receives) and read
+    back.  With q_len > 1,
     x_new is [B, q_len, d] and token i sits at position cache_len[b] + i.  Returns y [B, q_len, d]
     (q_len > 1) or [B, d]."""
     W = _weights64(weights)
     gkv = None if g_kv is None else f64(g_kv)
     one = gdla_decode if route == "literal" else gdla_decode_absorbed
     xn = f64(x_new)
-    if q_len == 1 and xn.ndim == 2:
+    one_token = q_len == 1 and xn.ndim == 2
+    if one_token:
         xn = xn[:, None, :]
     B, q = xn.shape[0], xn.shape[1]
     lens = [int(v) for v in (cache_len.tolist() if hasattr(cache_len, "tolist") else cache_len)]
@@ -786,10 +788,14 @@ def gdla_decode_fp8(x_new, weights: dict, cache8, cache_len, cfg: OracleConfig, 
         n = cfg.kv_rank + cfg.d_rope
         rows = mxfp8_dequantize_rows(np.asarray(cache8[b, :L]), n) if L else np.zeros((0, n))
         cbar, kR = kv_latent(xn[b], W["W_aKV"], gkv, L + np.arange(q), cfg)
-        new = mxfp8_dequantize_rows(mxfp8_quantize_rows(np.concatenate([cbar, kR], -1)), n)
+        # what the cache receives: the MXFP8 form of the bf16 latent values (the row a bf16
+        # cache would hold; rounding to bf16 is a library step)
+        import torch
+        lat_bf16 = torch.tensor(np.concatenate([cbar, kR], -1)).to(torch.bfloat16).double().numpy()
+        new = mxfp8_dequantize_rows(mxfp8_quantize_rows(lat_bf16), n)
         ext = np.concatenate([rows, new], 0)[None]
         for i in range(q):
             # keys: the cached rows, the earlier new tokens' stored rows, and its own stored row
             y[b, i] = one(xn[b, i][None], weights, ext, [L + i], cfg, g_q=g_q, g_kv=g_kv,
                           own_rows=ext[0, L + i][None])[0]
-    return y[:, 0] if q_len == 1 and np.asarray(x_new).ndim == 2 else y
+    return y[:, 0] if one_token else y

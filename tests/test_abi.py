@@ -163,3 +163,8 @@ def test_binding_rejects_wrong_tensors_before_the_library():
     with pytest.raises(TypeError):
         gb._host_ptr(torch.zeros(8), torch.bfloat16, "x")
     assert gb._host_ptr(torch.zeros(8, dtype=torch.bfloat16), torch.bfloat16, "x").value is not None
+
+
+def test_fp8_row_bytes_matches_header():
+    from oracle import gdla_oracle as O
+    assert gb.FP8_ROW_BYTES == gb._header_define("GDLA_FP8_ROW_BYTES") == O.fp8_row_bytes(576)
