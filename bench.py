@@ -224,6 +224,9 @@ def run_gpu(args):
     x_multi = {q: torch.randn((DECODE["B"], q, s.d_model), generator=torch.Generator().manual_seed(6 + q))
                .bfloat16().to(dev) for q in multis}
     y_multi = {q: torch.empty_like(x_multi[q]) for q in multis}
+    # the same cache stored as MXFP8 rows (608 bytes a position instead of 1152)
+    cache8 = layer.quantize_latent_fp8(cache) if windows else None
+    y_new8 = torch.empty_like(x_new)
     absorbed = layer.absorbed()
     dcfg = {w: gb.make_config(s.with_window(w)) for w in (0, 2048)}
     dws = torch.empty(max(gb.gdla_workspace_size(dcfg[w], DECODE["B"] * qmax, cache.shape[1],
@@ -233,7 +236,7 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(dev)
     pev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     dev_ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-              for k in ["c", "w2048", "c_q2", "c_q3"]}
+              for k in ["c", "w2048", "c_q2", "c_q3", "c_fp8"]}
 
     def prefill_once():
         gb.gdla_set_stage_events(pev)
@@ -245,10 +248,14 @@ def run_gpu(args):
     # prefill, whose power draw would leave the decode at the prefill's reduced clocks; the
     # caches (2.4 GB causal, 151 MB for the 2048 window) exceed the 126 MB L2, so no flush.
     dec_keys = [("c" if w == 0 else f"w{w}", w, 1) for w in windows] + [(f"c_q{q}", 0, q) for q in multis]
+    if windows:
+        dec_keys.append(("c_fp8", 0, 1))
 
     def decode_call(key, st):
         _, w, q = next(d for d in dec_keys if d[0] == key)
-        if q == 1:
+        if key == "c_fp8":
+            gb.gdla_decode_fp8_fwd(dcfg[0], absorbed, x_new, cache8, lens, y_new8, dws, stream=st)
+        elif q == 1:
             gb.gdla_decode_fwd(dcfg[w], absorbed, x_new, cache, lens, y_new, dws, stream=st)
         else:
             gb.gdla_decode_multi_fwd(dcfg[w], absorbed, x_multi[q], cache, lens, y_multi[q], dws, stream=st)
@@ -472,10 +479,11 @@ def run_gpu(args):
     decode = {}
     for k, w, q in dec_keys:
         keys_read = dec_L + q if w == 0 else min(w, dec_L + q)
-        kv_bytes = DECODE["B"] * keys_read * s.latent_row * 2        # each sequence's rows, once
+        row_bytes = gb.FP8_ROW_BYTES if k == "c_fp8" else s.latent_row * 2
+        kv_bytes = DECODE["B"] * keys_read * row_bytes                # each sequence's rows, once
         t_att = statistics.median(eager_stage[k]["attn"]) * 1e-3
         t_all = st[f"dec_{k}_ms"] * 1e-3
-        name = ("causal" if w == 0 else f"swa{w}") + ("" if q == 1 else f"_q{q}")
+        name = ("causal" if w == 0 else f"swa{w}") + ("" if q == 1 else f"_q{q}") + ("_fp8" if k == "c_fp8" else "")
         decode[name] = {
             "B": DECODE["B"], "cache_len": dec_L, "window": w, "q_len": q,
             "tok_per_s": world * DECODE["B"] * q / t_all, "ms": st[f"dec_{k}_ms"],
@@ -487,6 +495,9 @@ def run_gpu(args):
             "kv_bytes": kv_bytes, "kv_gbs": kv_bytes / t_att / 1e9,
             "kv_frac_of_hbm": kv_bytes / t_att / 1e9 / peaks["hbm_gbs"],
         }
+        if k == "c_fp8":
+            decode[name]["kv_note"] = ("MXFP8 latent cache: 608 bytes per cached position (576 E4M3 "
+                                       "values, 18 block scales, padding) against 1152 in bf16")
         if q > 1:
             decode[name]["kv_note"] = ("kv_bytes counts each sequence's cache rows once: the rows of its "
                                        f"{q} new tokens are consecutive query rows, whose CTAs read the same "

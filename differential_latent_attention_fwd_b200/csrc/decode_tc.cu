@@ -71,7 +71,7 @@ static_assert(SMEM <= 232448, "shared memory");
 constexpr int LAT_RAW = LAT_SLOT / 2;
 constexpr int ROPE_RAW = 2048;
 constexpr int SMEM8 = SMEM;
-constexpr int C8_WARPS = 2;
+constexpr int C8_WARPS = 4;
 // The M = 128 score MMA reads 128 rows of each 80-row q~ box: the 48 rows past a box are the
 // next box, or (for the last box) the first 6 KB of P.  They only feed unused score rows.
 static_assert(P_OFF + 48 * 128 <= LAT_OFF, "q~ box over-read stays in the P buffer");
@@ -145,10 +145,10 @@ struct DskWalk {
 static_assert(sizeof(SkBars) <= 1024, "barrier block");
 
 // C8: the cache holds MXFP8 rows (mapC: their 128-code latent boxes, mapR: their rope codes and
-// scales); 64 more threads (warps 6-7) convert them, and q~, P and the cache tiles are fp16 MMA
+// scales); 128 more threads (warps 6-9) convert them, and q~, P and the cache tiles are fp16 MMA
 // operands instead of bf16.
 template <bool C8>
-__global__ void __launch_bounds__(C8 ? 256 : 192, 1)
+__global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
     dec_attn_sk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapC,
                        const __grid_constant__ CUtensorMap mapR, const __grid_constant__ DecAttnParams p,
                        KernelCtl ctl) {
@@ -229,39 +229,47 @@ __global__ void __launch_bounds__(C8 ? 256 : 192, 1)
         for (int j = 0; j < n_tiles && ok; ++j, ++J) {
           if (PREFETCH_AHEAD > 0 && j + PREFETCH_AHEAD < n_tiles) prefetch(j + PREFETCH_AHEAD);
           const int y = int(crow0 + (long long)(sg.tile0 + j) * TP);
-          for (int u = 0; u < 4 && ok; ++u) {
-            const int gl = 4 * J + u, s = gl % NLAT;
-            const uint32_t ph = (gl / NLAT) & 1;
-            if (gl >= NLAT && !mbar_wait(&bars->lat_empty[s], ph ^ 1, ctl, SITE_DEC_PRODUCER)) { ok = false; break; }
-            uint8_t* dst = smem + LAT_OFF + s * LAT_SLOT;
-            if (C8) {
-              // [64 rows][128 codes] of the MXFP8 rows into the slot's upper half
-              mbar_expect_tx(&bars->lat_raw[s], LAT_SLOT / 2);
-              tma_load_2d(dst + LAT_RAW, &mapC, &bars->lat_raw[s], 128 * u, y);
-            } else {
-              mbar_expect_tx(&bars->lat_full[s], LAT_SLOT);
-              tma_load_2d(dst, &mapC, &bars->lat_full[s], 128 * u, y);
-              tma_load_2d(dst + LAT_SLOT / 2, &mapC, &bars->lat_full[s], 128 * u + 64, y);
+          // the latent units and the rope box (for MXFP8 rows the rope box, which carries the
+          // rows' block scales, goes first: the converters need it before any latent unit)
+          auto load_lat = [&]() -> bool {
+            for (int u = 0; u < 4 && ok; ++u) {
+              const int gl = 4 * J + u, s = gl % NLAT;
+              const uint32_t ph = (gl / NLAT) & 1;
+              if (gl >= NLAT && !mbar_wait(&bars->lat_empty[s], ph ^ 1, ctl, SITE_DEC_PRODUCER)) return false;
+              uint8_t* dst = smem + LAT_OFF + s * LAT_SLOT;
+              if (C8) {
+                // [64 rows][128 codes] of the MXFP8 rows into the slot's upper half
+                mbar_expect_tx(&bars->lat_raw[s], LAT_SLOT / 2);
+                tma_load_2d(dst + LAT_RAW, &mapC, &bars->lat_raw[s], 128 * u, y);
+              } else {
+                mbar_expect_tx(&bars->lat_full[s], LAT_SLOT);
+                tma_load_2d(dst, &mapC, &bars->lat_full[s], 128 * u, y);
+                tma_load_2d(dst + LAT_SLOT / 2, &mapC, &bars->lat_full[s], 128 * u + 64, y);
+              }
+              lat_issued |= 1u << s;
+              lat_par = (lat_par & ~(1u << s)) | (ph << s);
             }
-            lat_issued |= 1u << s;
-            lat_par = (lat_par & ~(1u << s)) | (ph << s);
-          }
-          if (!ok) break;
-          {
-            const int s = J % NROPE;
-            const uint32_t ph = (J / NROPE) & 1;
-            if (J >= NROPE && !mbar_wait(&bars->rope_empty[s], ph ^ 1, ctl, SITE_DEC_PRODUCER)) { ok = false; break; }
-            if (C8) {
-              // [64 rows][96 bytes]: the rope codes, the 18 block scales and the padding
-              mbar_expect_tx(&bars->rope_raw[s], 64 * 96);
-              tma_load_2d(smem + ROPE_OFF + s * ROPE_SLOT + ROPE_RAW, &mapR, &bars->rope_raw[s], 512, y);
-            } else {
-              mbar_expect_tx(&bars->rope_full[s], ROPE_SLOT);
-              tma_load_2d(smem + ROPE_OFF + s * ROPE_SLOT, &mapC, &bars->rope_full[s], 512, y);
+            return true;
+          };
+          auto load_rope = [&]() -> bool {
+            {
+              const int s = J % NROPE;
+              const uint32_t ph = (J / NROPE) & 1;
+              if (J >= NROPE && !mbar_wait(&bars->rope_empty[s], ph ^ 1, ctl, SITE_DEC_PRODUCER)) return false;
+              if (C8) {
+                // [64 rows][96 bytes]: the rope codes, the 18 block scales and the padding
+                mbar_expect_tx(&bars->rope_raw[s], 64 * 96);
+                tma_load_2d(smem + ROPE_OFF + s * ROPE_SLOT + ROPE_RAW, &mapR, &bars->rope_raw[s], 512, y);
+              } else {
+                mbar_expect_tx(&bars->rope_full[s], ROPE_SLOT);
+                tma_load_2d(smem + ROPE_OFF + s * ROPE_SLOT, &mapC, &bars->rope_full[s], 512, y);
+              }
+              rope_issued |= 1u << s;
+              rope_par = (rope_par & ~(1u << s)) | (ph << s);
             }
-            rope_issued |= 1u << s;
-            rope_par = (rope_par & ~(1u << s)) | (ph << s);
-          }
+            return true;
+          };
+          if (C8 ? !(load_rope() && load_lat()) : !(load_lat() && load_rope())) { ok = false; break; }
           // q~ of this segment goes after its first tile: that tile's loads overlap the wait
           // for the previous segment to finish with the shared q~ boxes
           if (!q_done) {
@@ -369,14 +377,16 @@ __global__ void __launch_bounds__(C8 ? 256 : 192, 1)
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
   } else if (C8 && warp >= 6) {
-    // ============================================================ MXFP8 converters (warps 6-7)
-    // Thread c = row c of every tile.  Per tile: the rope box first (its bytes hold the row's
-    // 18 block scales, which the thread keeps for the latent units), then the four latent
-    // units; each unit: all 64 threads read their raw row, meet at a named barrier (the fp16
-    // output overwrites the raw bytes), convert E4M3 x 2^k -> fp16 into the 128-byte-swizzled
-    // K-major boxes and publish the slot.  Rows outside the row's key range become zeros, so an
-    // unwritten cache tail (NaN codes or scales) never reaches the MMAs.
-    const int r = threadIdx.x - 192;
+    // ============================================================ MXFP8 converters (warps 6-9)
+    // Two threads per row (half h of its codes).  Per tile: the rope box first (its bytes hold
+    // the row's 18 block scales, which the threads keep for the latent units), then the four
+    // latent units, thread h writing fp16 box h of the unit (64 of its 128 dims); each unit: all
+    // 128 threads read their raw half rows, meet at a named barrier (the fp16 output overwrites
+    // the raw bytes), convert E4M3 x 2^k -> fp16 into the 128-byte-swizzled K-major boxes and
+    // publish the slot.  Rows outside the row's key range become zeros, so an unwritten cache
+    // tail (NaN codes or scales) never reaches the MMAs.
+    const int c_id = threadIdx.x - 192;
+    const int r = c_id >> 1, hh = c_id & 1;
     const int sw = r & 7;
     bool ok = true;
     int J = 0;
@@ -384,18 +394,36 @@ __global__ void __launch_bounds__(C8 ? 256 : 192, 1)
     // 16 E4M3 codes (one uint4) times 2^k -> 16 fp16 values (two uint4)
     // (rows outside the key range are converted too, then replaced by zeros: only valid rows
     // may report an fp16 range error)
-    auto convert16 = [&](const uint4 c, float s, uint4& o0, uint4& o1, bool valid) {
+    // For a scale 2^k with k in [-14, 7] the product E4M3 x 2^k is an exact fp16 (at most
+    // 448 2^7 < 65504; the smallest, 2^-9 2^-14, is a multiple of the fp16 subnormal step 2^-24),
+    // so it is one fp16x2 multiply; other scales go through fp32 with a saturating check.
+    auto convert16 = [&](const uint4 c, int k, uint4& o0, uint4& o1, bool valid) {
       bool bad = false;
       const uint32_t w[4] = {c.x, c.y, c.z, c.w};
       uint32_t h[8];
+      if (k >= -14 && k <= 7) {
+        const uint32_t sh = uint32_t(k + 15) << 10;
+        const __half2 s2 = __halves2half2(__ushort_as_half(uint16_t(sh)), __ushort_as_half(uint16_t(sh)));
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4; ++i) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const uint32_t x = f16x2_from_e4m3x2(uint16_t(w[i] >> (16 * e)));
-          const float lo = __half2float(__ushort_as_half(uint16_t(x & 0xFFFFu))) * s;
-          const float hi = __half2float(__ushort_as_half(uint16_t(x >> 16))) * s;
-          h[2 * i + e] = pack_half2_sat(lo, hi, bad);
+          for (int e = 0; e < 2; ++e) {
+            uint32_t x = f16x2_from_e4m3x2(uint16_t(w[i] >> (16 * e)));
+            __half2 v = __hmul2(*reinterpret_cast<__half2*>(&x), s2);
+            h[2 * i + e] = *reinterpret_cast<uint32_t*>(&v);
+          }
+        }
+      } else {
+        const float s = exp2i(k);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const uint32_t x = f16x2_from_e4m3x2(uint16_t(w[i] >> (16 * e)));
+            const float lo = __half2float(__ushort_as_half(uint16_t(x & 0xFFFFu))) * s;
+            const float hi = __half2float(__ushort_as_half(uint16_t(x >> 16))) * s;
+            h[2 * i + e] = pack_half2_sat(lo, hi, bad);
+          }
         }
       }
       fp16_bad |= bad && valid;
@@ -411,21 +439,22 @@ __global__ void __launch_bounds__(C8 ? 256 : 192, 1)
         const bool wr = mbar_wait(&bars->rope_raw[rs], (J / NROPE) & 1, ctl, SITE_DEC_CONVERT);
         uint8_t* rslot = smem + ROPE_OFF + rs * ROPE_SLOT;
         const uint8_t* raw = rslot + ROPE_RAW + r * 96;
-        uint4 rc[4];
+        uint4 rc[2];                          // rope codes 32 hh .. 32 hh + 31
 #pragma unroll
-        for (int i = 0; i < 4; ++i) rc[i] = *reinterpret_cast<const uint4*>(raw + 16 * i);
+        for (int i = 0; i < 2; ++i) rc[i] = *reinterpret_cast<const uint4*>(raw + 32 * hh + 16 * i);
         const uint4 sc = *reinterpret_cast<const uint4*>(raw + 64);          // scales of blocks 0..15
         const uint32_t sc2 = *reinterpret_cast<const uint32_t*>(raw + 80);   // blocks 16, 17
         // every raw row read before any is overwritten (and a failed wait stops both warps)
-        if (named_bar_or(2, 64, !wr)) { ok = false; break; }
+        if (named_bar_or(2, 32 * C8_WARPS, !wr)) { ok = false; break; }
         {
-          const float s16 = exp2i(int(sc2 & 0xFFu) - 127), s17 = exp2i(int((sc2 >> 8) & 0xFFu) - 127);
+          const int sr = int((sc2 >> (8 * hh)) & 0xFFu) - 127;     // block 16 + hh
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {       // codes 16 i .. 16 i + 15: chunks 2 i, 2 i + 1
+          for (int i = 0; i < 2; ++i) {       // codes 32 hh + 16 i ..: chunks 4 hh + 2 i, + 1
+            const int ch = 4 * hh + 2 * i;
             uint4 o0, o1;
-            convert16(rc[i], i < 2 ? s16 : s17, o0, o1, valid);
-            *reinterpret_cast<uint4*>(rslot + r * 128 + (((2 * i) ^ sw) << 4)) = o0;
-            *reinterpret_cast<uint4*>(rslot + r * 128 + (((2 * i + 1) ^ sw) << 4)) = o1;
+            convert16(rc[i], sr, o0, o1, valid);
+            *reinterpret_cast<uint4*>(rslot + r * 128 + ((ch ^ sw) << 4)) = o0;
+            *reinterpret_cast<uint4*>(rslot + r * 128 + (((ch + 1) ^ sw) << 4)) = o1;
           }
         }
         fence_proxy_async_smem();
@@ -438,19 +467,19 @@ __global__ void __launch_bounds__(C8 ? 256 : 192, 1)
           const int gl = 4 * J + u, s = gl % NLAT;
           const bool wl = mbar_wait(&bars->lat_raw[s], (gl / NLAT) & 1, ctl, SITE_DEC_CONVERT);
           uint8_t* slot = smem + LAT_OFF + s * LAT_SLOT;
-          uint4 c[8];
+          uint4 c[4];                         // codes 64 hh .. 64 hh + 63 of the unit
 #pragma unroll
-          for (int i = 0; i < 8; ++i) c[i] = *reinterpret_cast<const uint4*>(slot + LAT_RAW + r * 128 + 16 * i);
-          if (named_bar_or(2, 64, !wl)) { ok = false; break; }
-          // codes 16 i .. 16 i + 15 of the unit: block 4 u + i / 2; box i / 4, chunks 2 (i % 4), +1
+          for (int i = 0; i < 4; ++i) c[i] = *reinterpret_cast<const uint4*>(slot + LAT_RAW + r * 128 + 64 * hh + 16 * i);
+          if (named_bar_or(2, 32 * C8_WARPS, !wl)) { ok = false; break; }
+          // codes 64 hh + 16 i ..: block 4 u + 2 hh + i / 2; box hh, chunks 2 i, 2 i + 1
+          uint8_t* box = slot + hh * (LAT_SLOT / 2) + r * 128;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float sk = exp2i(int((scw[u] >> (8 * (i >> 1))) & 0xFFu) - 127);
+          for (int i = 0; i < 4; ++i) {
+            const int sk = int((scw[u] >> (8 * (2 * hh + (i >> 1)))) & 0xFFu) - 127;
             uint4 o0, o1;
             convert16(c[i], sk, o0, o1, valid);
-            uint8_t* box = slot + (i >> 2) * (LAT_SLOT / 2) + r * 128;
-            *reinterpret_cast<uint4*>(box + (((2 * (i & 3)) ^ sw) << 4)) = o0;
-            *reinterpret_cast<uint4*>(box + (((2 * (i & 3) + 1) ^ sw) << 4)) = o1;
+            *reinterpret_cast<uint4*>(box + (((2 * i) ^ sw) << 4)) = o0;
+            *reinterpret_cast<uint4*>(box + (((2 * i + 1) ^ sw) << 4)) = o1;
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -739,7 +768,7 @@ int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t s
     if (cudaFuncSetAttribute(dec_attn_sk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsk::SMEM8) != cudaSuccess)
       return -4;
-    dec_attn_sk_kernel<true><<<p.n_ctas, 256, dsk::SMEM8, st>>>(mq, mc, mr, p, kc);
+    dec_attn_sk_kernel<true><<<p.n_ctas, 192 + 32 * dsk::C8_WARPS, dsk::SMEM8, st>>>(mq, mc, mr, p, kc);
   } else {
     if (cudaFuncSetAttribute(dec_attn_sk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsk::SMEM) != cudaSuccess)
