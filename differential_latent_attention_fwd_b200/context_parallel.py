@@ -18,6 +18,12 @@ Protocol for rank r holding tokens [start_r, start_r + T_r) of the sequence:
 `layer` needs `latent(x, pos_offset)`, `prefill_context(x, pos_offset, prefix_latent)` and
 `window` (0 = full causal); GdlaLayer provides them on the GPU.  The collectives are those of
 torch.distributed on the tensors' device (NCCL for CUDA tensors).
+
+With fp8=True the rows cross the network as MXFP8 rows (the report's low-precision format,
+paperglide.net summary, the low-precision paragraph and Figure 3: E4M3 values with one
+power-of-two scale per 32; 608 bytes instead of 1152): each rank quantizes its rows before the
+exchange (`layer.quantize_latent_fp8`) and the receiver dequantizes the prefix it gets
+(`layer.dequantize_latent_fp8`); a rank's own rows stay bf16.
 """
 from __future__ import annotations
 
@@ -77,11 +83,14 @@ def exchange_prefix(latent: torch.Tensor, lengths: list, rank: int, window: int,
     return torch.cat(blocks[:rank], 0)[-need:]
 
 
-def cp_prefill(layer, x_local: torch.Tensor, group=None) -> torch.Tensor:
+def cp_prefill(layer, x_local: torch.Tensor, group=None, fp8: bool = False) -> torch.Tensor:
     """y rows of this rank's tokens x_local [T_r, d] of a sequence split over the group."""
     rank = dist.get_rank(group)
     lengths = _lengths(x_local.shape[0], x_local.device, group)
     start = sum(lengths[:rank])
     latent = layer.latent(x_local, start)
-    prefix = exchange_prefix(latent, lengths, rank, int(layer.window), group)
+    send = layer.quantize_latent_fp8(latent) if fp8 else latent
+    prefix = exchange_prefix(send, lengths, rank, int(layer.window), group)
+    if fp8 and prefix is not None:
+        prefix = layer.dequantize_latent_fp8(prefix)
     return layer.prefill_context(x_local, start, prefix)

@@ -35,6 +35,13 @@ class OracleLayer:
         pre = None if prefix is None else prefix.numpy()
         return torch.from_numpy(O.gdla_prefill_after_prefix(x, pre, pos_offset, self.w, self.cfg))
 
+    def quantize_latent_fp8(self, latent):
+        self.sent_bytes = int(latent.shape[0]) * O.fp8_row_bytes(latent.shape[1])
+        return torch.from_numpy(O.mxfp8_quantize_rows(latent.numpy()))
+
+    def dequantize_latent_fp8(self, stored):
+        return torch.from_numpy(O.mxfp8_dequantize_rows(stored.numpy(), self.cfg.kv_rank + self.cfg.d_rope))
+
 
 def _worker(rank, world, port, window, lengths, seed, q):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -125,3 +132,60 @@ def test_cp_prefill_on_a_subgroup(window, lengths):
     y = O.gdla_prefill(inp.x, inp.weights, O.OracleConfig.from_shape(shape))[0]
     full = np.concatenate([got[r] for r in range(1, world)], 0)
     np.testing.assert_allclose(full, y, rtol=0, atol=1e-10)
+
+
+# latent rows of 28 + 4 = 32 values: one MXFP8 block per row
+SMALL8 = dict(SMALL, kv_rank=28)
+
+
+def _worker_fp8(rank, world, port, window, lengths, seed, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        shape = synth.GdlaShape(window=window, **SMALL8)
+        inp = synth.make_prefill_inputs(shape, 1, sum(lengths), seed)
+        start = sum(lengths[:rank])
+        x = inp.x[0, start: start + lengths[rank]]
+        lay = OracleLayer(shape, inp.weights)
+        y = cp_prefill(lay, x, fp8=True)
+        q.put((rank, y.numpy(), lay.sent_bytes))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("window,lengths", [(0, [7, 13, 10]), (6, [9, 8, 12])])
+def test_cp_prefill_fp8_exchange(window, lengths):
+    """Rows exchanged as MXFP8: each rank's result is the prefix computation over the
+    dequantized rows of the ranks before it (its own rows at full precision), and stays close
+    to the whole sequence."""
+    world = len(lengths)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_fp8, args=(r, world, port, window, lengths, 5, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {r: (y, nb) for r, y, nb in (q.get(timeout=240) for _ in range(world))}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    shape = synth.GdlaShape(window=window, **SMALL8)
+    cfg = O.OracleConfig.from_shape(shape)
+    inp = synth.make_prefill_inputs(shape, 1, sum(lengths), 5)
+    x = O.f64(inp.x[0])
+    T = sum(lengths)
+    cbar, kR = O.kv_latent(x, O.f64(inp.weights["W_aKV"]), None, np.arange(T), cfg)
+    rows = np.concatenate([cbar, kR], -1)
+    stored = O.mxfp8_dequantize_rows(O.mxfp8_quantize_rows(rows), rows.shape[1])
+    y_full = O.gdla_prefill(inp.x, inp.weights, cfg)[0]
+    for r in range(world):
+        start = sum(lengths[:r])
+        lo = 0 if window == 0 else max(0, start - (window - 1))
+        pre = stored[lo:start] if start > lo else None
+        want = O.gdla_prefill_after_prefix(inp.x[0, start: start + lengths[r]], pre, start, inp.weights, cfg)
+        y, nb = got[r]
+        np.testing.assert_allclose(y, want, rtol=1e-9, atol=1e-10)
+        assert nb == lengths[r] * O.fp8_row_bytes(32)      # 48 bytes a row instead of 64 in bf16
+        rel = np.linalg.norm(y - y_full[start: start + lengths[r]]) / np.linalg.norm(y_full[start: start + lengths[r]])
+        assert rel < 5e-2, rel
