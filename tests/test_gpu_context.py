@@ -88,3 +88,28 @@ def test_context_rejects_bad_offsets(cuda_ok):
     lat = layer.latent(x[0, :32].contiguous(), 0)
     with pytest.raises(gb.GdlaError):
         layer.prefill_context(x[0, 32:].contiguous(), 16, lat)     # 32 prefix rows before position 16
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_context_chunk_after_fp8_prefix(cuda_ok, window):
+    """The MXFP8 exchange of context parallelism on the GPU: the prefix rows are quantized and
+    dequantized by the library, and the chunk after them matches the oracle's prefix form over
+    the oracle's MXFP8 round trip of the (bf16) latent rows."""
+    from oracle import gdla_oracle as O
+    T0, T1 = 400, 300
+    shape, inp, layer, x = prefill_case(1, T0 + T1, window, seed=19)
+    lat0 = layer.latent(x[0, :T0].contiguous(), 0)
+    n = T0 if window == 0 else window - 1
+    stored = layer.quantize_latent_fp8(lat0[T0 - n:].contiguous())
+    assert stored.shape == (n, 608) and stored.dtype == torch.uint8
+    prefix = layer.dequantize_latent_fp8(stored)
+    y1 = layer.prefill_context(x[0, T0:].contiguous(), T0, prefix)
+    torch.cuda.synchronize()
+    assert gb.gdla_device_error() == 0
+    cfg = O.OracleConfig.from_shape(shape)
+    cbar, kR = O.kv_latent(O.f64(inp.x[0, :T0]), O.f64(inp.weights["W_aKV"]), O.f64(inp.g_kv), np.arange(T0), cfg)
+    rows_bf16 = torch.tensor(np.concatenate([cbar, kR], -1)[T0 - n:]).to(torch.bfloat16).double().numpy()
+    pre_o = O.mxfp8_dequantize_rows(O.mxfp8_quantize_rows(rows_bf16), 576)
+    rows = list(range(0, T1, 7)) + [T1 - 1]
+    yo = O.gdla_prefill_after_prefix(inp.x[0, T0:], pre_o, T0, inp.weights, cfg, g_q=inp.g_q, g_kv=inp.g_kv)
+    check(f"chunk after an MXFP8 prefix, W={window}", to_np(y1[rows]), yo[rows])
