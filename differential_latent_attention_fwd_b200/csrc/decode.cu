@@ -232,7 +232,7 @@ int launch_qtilde(const DecQParams& p, KernelCtlHost ctl, cudaStream_t st) {
 // differentials l_s - lambda_s l_noise of its 4 signal heads formed in shared memory (fp32);
 // then D = Dlat W_UV_j (4 CB rows x 128 columns, K = 512) and Dg = sigmoid(G) (.) D.
 // Row b's segments are the attention CTAs c_lo .. c_hi whose tile ranges meet the row's tiles
-// [tstart[b], tstart[b + 1]); CTA c wrote its piece to slot c + b.
+// [tstart[l], tstart[l + 1]) at list position l of row b; CTA c wrote its piece to slot c + l.
 constexpr int CB = 8;
 constexpr int MAXSEG = DEC_MAX_CTAS;
 __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
@@ -255,14 +255,14 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
   if (tid < CB) {
     int lo = 0, n = 0;
     if (tid < nb) {
-      const int b = b0 + tid;
-      const long long N = p.tstart[p.B], G = N < p.n_ctas ? N : p.n_ctas;
-      const long long t0 = p.tstart[b], t1 = p.tstart[b + 1];
+      const int b = b0 + tid, l = dec_list_pos(b, p.q_len, p.n_seq);
+      const long long N = p.tstart[p.B], G = dec_ctas_used(N, p.n_ctas, p.q_len);
+      const long long t0 = p.tstart[l], t1 = p.tstart[l + 1];
       if (t1 > t0) {
         // CTA c < G = min(grid, N) covers tiles [c N / G, (c + 1) N / G) (never empty): tile t
         // lies in CTA ((t + 1) G - 1) / N
         const int c_lo = int(((t0 + 1) * G - 1) / N), c_hi = int((t1 * G - 1) / N);
-        lo = c_lo + b;
+        lo = c_lo + l;
         n = c_hi - c_lo + 1;
       }
     }

@@ -15,12 +15,14 @@
 // a ring of nine 16 KB latent slots (two [64 positions][64 dims] boxes each) and two 8 KB
 // rotary slots (a tile takes four latent slots and one rotary slot): about 2.2 tiles.
 //
-// Work split ("stream-K"): the key tiles of all rows form one list, rows in order; CTA c of
-// G = min(grid, N) takes tiles [c N / G, (c + 1) N / G), i.e. one wave with equal work per SM
-// whatever the cache lengths.  The piece of a row inside one CTA's range is a segment: it gets its own online
-// softmax and writes a partial (m_h, l_h, O^T) to slot c + r; the merge kernel in decode.cu
-// combines a row's segments.  The rows of one sequence's q_len new tokens are consecutive, so
-// CTAs c and c + N_r G / N read the same cache tiles at about the same time (one DRAM read).
+// Work split ("stream-K"): the key tiles of all rows form one list, the rows in token-major
+// order (dec_list_pos: token 0 of every sequence, then token 1, ...); CTA c of G = min(grid, N)
+// takes tiles [c N / G, (c + 1) N / G), i.e. one wave with equal work per SM whatever the cache
+// lengths.  The piece of a row inside one CTA's range is a segment: it gets its own online
+// softmax and writes a partial (m_h, l_h, O^T) to slot c + l (l: the row's list position); the
+// merge kernel in decode.cu combines a row's segments.  With q_len new tokens per sequence the
+// list is q_len nearly equal parts with the same tile positions, so CTAs c and c + G / q_len
+// reach the same cache tiles at about the same time and the later reads hit L2.
 //
 // Roles (192 threads): warps 0-3 softmax and O^T epilogue (warp w reads TMEM lanes 32 w ..
 // 32 w + 31: thread = head h = 32 w + lane for h < 80, thread = latent row for O^T), warp 4 TMA
@@ -92,7 +94,8 @@ __device__ __forceinline__ uint8_t* dsk_align(uint8_t* p) {
 }
 
 // Key range of query row r: it is new token r % q_len of sequence r / q_len and sees the cache
-// rows 0 .. cache_len + r % q_len (the window keeps the last W of them).
+// rows 0 .. cache_len + r % q_len (the window keeps the last W of them).  (r: the query row,
+// not its position in the work list.)
 __device__ __forceinline__ void dsk_row_range(const DecAttnParams& p, int r, int* lo, int* hi) {
   const int ql = p.q_len > 1 ? p.q_len : 1;
   const int L = p.cache_len[r / ql] + r % ql;
@@ -100,9 +103,10 @@ __device__ __forceinline__ void dsk_row_range(const DecAttnParams& p, int r, int
   *lo = p.window > 0 ? max(0, L - p.window + 1) : 0;
 }
 
-// One segment: the tiles [g0, g1) of the global list, all in row r.
+// One segment: the tiles [g0, g1) of the global list, all in the row at list position r.
 struct DskSeg {
-  int r, g0, g1;        // row; global tile range
+  int r, g0, g1;        // list position of the row; global tile range
+  int q;                // the query row (token q % q_len of sequence q / q_len)
   int tile0;            // tile index (of TP positions) within the row of global tile g0
   int lo, hi;           // row's key range
 };
@@ -111,10 +115,10 @@ struct DskSeg {
 struct DskWalk {
   int t, t_end, r;
   __device__ void init(const DecAttnParams& p) {
-    // G = min(grid, N) CTAs share the N tiles, so that no CTA range is empty (the merge kernel
-    // relies on it); the CTAs beyond G have nothing to do
+    // G = min(grid, N) CTAs (a multiple of q_len) share the N tiles, so that no CTA range is
+    // empty (the merge kernel relies on it); the CTAs beyond G have nothing to do
     const long long N = p.tstart[p.R];
-    const long long G = N < (long long)gridDim.x ? N : (long long)gridDim.x;
+    const long long G = dec_ctas_used(N, gridDim.x, p.q_len > 1 ? p.q_len : 1);
     if ((long long)blockIdx.x >= G) {
       t = t_end = r = 0;
       return;
@@ -133,9 +137,10 @@ struct DskWalk {
     if (t >= t_end) return false;
     while (p.tstart[r + 1] <= t) ++r;
     s->r = r;
+    s->q = dec_row_of(r, p.q_len > 1 ? p.q_len : 1, p.n_seq);
     s->g0 = t;
     s->g1 = min(t_end, p.tstart[r + 1]);
-    dsk_row_range(p, r, &s->lo, &s->hi);
+    dsk_row_range(p, s->q, &s->lo, &s->hi);
     s->tile0 = s->lo / dsk::TP + (t - p.tstart[r]);
     t = s->g1;
     return true;
@@ -205,14 +210,14 @@ __global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
       int J = 0;            // CTA-local tile counter (over all segments)
       int seg = 0;
       while (ok && walk.next(p, &sg)) {
-        const long long crow0 = (long long)(sg.r / ql) * p.cap;
+        const long long crow0 = (long long)(sg.q / ql) * p.cap;
         bool q_done = false;
         auto load_q = [&]() -> bool {
           // the previous segment's score MMAs read the shared q~ boxes until it is done
           if (seg > 0 && !mbar_wait(&bars->seg_done, (seg - 1) & 1, ctl, SITE_DEC_PRODUCER)) return false;
           mbar_expect_tx(&bars->q_ready, 5 * QS_BOX);
           for (int c = 0; c < 5; ++c)
-            tma_load_2d(smem + QS_OFF + c * QS_BOX, &mapQ, &bars->q_ready, 256 + 64 * c, sg.r * NH);
+            tma_load_2d(smem + QS_OFF + c * QS_BOX, &mapQ, &bars->q_ready, 256 + 64 * c, sg.q * NH);
           q_issued = true;
           return true;
         };
@@ -505,7 +510,7 @@ __global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
       if (q < 3) {
         uint32_t v[32];
         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.qt) +
-                                                          ((long long)sg.r * NH + (hv ? h : 0)) * 576);
+                                                          ((long long)sg.q * NH + (hv ? h : 0)) * 576);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -687,9 +692,10 @@ __global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
   }
 }
 
-// Tile prefix over the query rows: tstart[r] = tiles of rows < r, tstart[R] = all tiles.  A row
-// whose cache_len entry is outside [0, cap - q_len] gets no tiles (its output is zero) and the
-// error word records SITE_BAD_CACHE_LEN.  One CTA of 1024 threads.
+// Tile prefix over the query rows in list order (dec_list_pos): tstart[l] = tiles of the rows
+// before list position l, tstart[R] = all tiles.  A row whose cache_len entry is outside
+// [0, cap - q_len] gets no tiles (its output is zero) and the error word records
+// SITE_BAD_CACHE_LEN.  One CTA of 1024 threads.
 __global__ void __launch_bounds__(1024) dec_sched_kernel(const int* __restrict__ cache_len, int R, int q_len,
                                                          int cap, int window, int* __restrict__ tstart,
                                                          int* err) {
@@ -700,9 +706,10 @@ __global__ void __launch_bounds__(1024) dec_sched_kernel(const int* __restrict__
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   for (int base = 0; base < R; base += blockDim.x) {
-    const int r = base + threadIdx.x;
+    const int l = base + threadIdx.x;           // list position (token-major order)
     int n = 0;
-    if (r < R) {
+    if (l < R) {
+      const int r = dec_row_of(l, ql, R / ql);
       const int L0 = cache_len[r / ql];
       if (L0 < 0 || L0 > cap - ql) {
         if (r % ql == 0) atomicCAS(err, 0, SITE_BAD_CACHE_LEN);
@@ -731,7 +738,7 @@ __global__ void __launch_bounds__(1024) dec_sched_kernel(const int* __restrict__
     }
     __syncthreads();
     const int incl = x + (warp > 0 ? wsum[warp - 1] : 0) + carry;
-    if (r < R) tstart[r] = incl - n;
+    if (l < R) tstart[l] = incl - n;
     __syncthreads();
     if (threadIdx.x == blockDim.x - 1) carry = incl;
     __syncthreads();

@@ -29,18 +29,40 @@ struct DecAttnParams {
   int cache_fp8;
   const void* qt;         // bf16 [R][80][576] (fp16 with an MXFP8 cache)
   float scale_log2;
-  int* tstart;            // [R + 1] tile prefix over the rows (dec_sched_kernel)
+  int* tstart;            // [R + 1] tile prefix over the rows in list order (dec_sched_kernel)
   int n_ctas;             // grid of the attention kernel (G): slots = G + R - 1
   float* part;            // [slots][80][512] latent accumulators of each segment
   float* ml;              // [slots][80][2]  (running max in log2 units, row sum)
   int* err;               // device error word
 };
 
+// Order of the query rows in the attention's work list: token-major, position l = (r % q_len)
+// * n_seq + r / q_len for query row r (token r % q_len of sequence r / q_len).  The q_len rows of
+// one sequence sit n_seq apart, so with the list split evenly over the CTAs the CTAs serving
+// them are about G / q_len apart and reach the same cache tiles at about the same time: the
+// second and later reads of a tile hit L2.
+__host__ __device__ __forceinline__ int dec_list_pos(int r, int q_len, int n_seq) {
+  return q_len > 1 ? (r % q_len) * n_seq + r / q_len : r;
+}
+__host__ __device__ __forceinline__ int dec_row_of(int l, int q_len, int n_seq) {
+  return q_len > 1 ? (l % n_seq) * q_len + l / n_seq : l;
+}
+
+// CTAs that take part in the attention's stream-K split of N tiles over a grid of `grid`:
+// min(grid, N), rounded down to a multiple of q_len (when that leaves at least q_len) so that
+// the q_len token parts of the list start on CTA boundaries.
+__host__ __device__ __forceinline__ long long dec_ctas_used(long long N, long long grid, int q_len) {
+  long long G = N < grid ? N : grid;
+  if (q_len > 1 && G >= q_len) G -= G % q_len;
+  return G;
+}
+
 struct DecCombParams {
   int B, n_groups, n_signal;   // B = query rows
+  int q_len, n_seq;            // (B = q_len * n_seq) for the list order of the rows
   int n_ctas;                  // G of the attention launch
-  const int* tstart;           // [B + 1] tile prefix over the rows
-  const float* part;           // segment partials, slot c + r for CTA c and row r
+  const int* tstart;           // [B + 1] tile prefix over the rows in list order
+  const float* part;           // segment partials, slot c + l for CTA c and list position l
   const float* ml;
   const float* lam;       // [B][n_signal]
   const float* G;         // fp32 gate logits: row b at G + b * g_ld, [n_signal * 128]
