@@ -179,44 +179,36 @@ def test_packed_documents_reject_bad_offsets(cuda_ok):
     assert gb.gdla_device_error() == 0x602
 
 
-def _stage_oracle_on_gpu_operands(ws, cfg, shape, T, window):
-    """The oracle's attention stage evaluated on the fp16/fp32 operands the GPU left in its
-    workspace (q, K^C, V, k^R, lambda, gate logits): isolates the attention kernel's arithmetic
-    from the rounding of its inputs."""
-    from oracle import gdla_oracle as O
-    nH = shape.n_heads
-    qq = to_np(ws_view(ws, cfg, 1, T, 0, WS_QQ, torch.float16, (T, nH * shape.d_qk)))
-    kv = to_np(ws_view(ws, cfg, 1, T, 0, WS_KV, torch.float16, (T, shape.n_kv_heads, 256)))
-    kr = to_np(ws_view(ws, cfg, 1, T, 0, 9, torch.float16, (T, shape.d_rope)))
-    lam = to_np(ws_view(ws, cfg, 1, T, 0, WS_LAM, torch.float32, (T, shape.n_signal)))
-    gate = to_np(ws_view(ws, cfg, 1, T, 0, WS_G, torch.bfloat16, (T, shape.n_signal, shape.d_v)))
-    ocfg = O.OracleConfig.from_shape(synth.GdlaShape(window=window))
-    Dg, _ = O.attention_stage(qq[:, : nH * 128].reshape(T, nH, 128), qq[:, nH * 128:].reshape(T, nH, 64),
-                              kv[..., :128], kv[..., 128:], kr, lam, gate, ocfg)
-    return Dg, max(np.abs(qq).max(), np.abs(kv).max(), np.abs(kr).max())
-
-
 def test_large_norm_gains_keep_fp16_operands_finite(cuda_ok):
-    """RMSNorm gains of 50 (q and KV latents): the fp16 attention operands grow 50x and stay
-    finite; no range error is reported, and the attention kernel matches the oracle's
-    attention stage on those operands."""
+    """RMSNorm gains of 50 on both latents: the fp16 attention operands grow about 50x and stay
+    finite, and no range error is reported.  Gains of 50 also scale the logits by 2500, where
+    the bf16 rounding of the latents alone moves the softmax by percents (measured: 4.9 % rel-L2
+    at gains 50, 5.1e-3 at gains 4), so parity against the oracle is checked with gains of 2
+    (operands x2, logits x4), at the layer bar."""
+    from oracle import gdla_oracle as O
+    from differential_latent_attention_fwd_b200.layer import GdlaLayer
     T, window = 200, 0
     shape = synth.GdlaShape(window=window)
     inp = synth.make_prefill_inputs(shape, 1, T, seed=13)
-    from differential_latent_attention_fwd_b200.layer import GdlaLayer
-    g50q = (torch.ones(shape.q_rank) * 50).bfloat16()
-    g50kv = (torch.ones(shape.kv_rank) * 50).bfloat16()
-    layer = GdlaLayer(shape, inp.weights, g50q, g50kv, device="cuda")
-    y = layer.prefill(inp.x.cuda())
-    torch.cuda.synchronize()
-    assert gb.gdla_device_error() == 0
-    assert bool(torch.isfinite(y).all())
-    Dg_o, amax = _stage_oracle_on_gpu_operands(layer._ws, layer.cfg, shape, T, window)
-    assert 10.0 < amax < 65504.0, amax
-    dg = to_np(ws_view(layer._ws, layer.cfg, 1, T, 0, WS_DG, torch.bfloat16, (T, 64, 128)))
-    # the gains scale V (hence D and Dg) by 50: the absolute bound scales with it, the relative
-    # one does not
-    check("Dg with gains x50 vs the oracle's stage on the same operands", dg, Dg_o, mabs=MAX_ABS * 50)
+    nH = shape.n_heads
+    for gain in (50.0, 2.0):
+        gq = (torch.ones(shape.q_rank) * gain).bfloat16()
+        gkv = (torch.ones(shape.kv_rank) * gain).bfloat16()
+        layer = GdlaLayer(shape, inp.weights, gq, gkv, device="cuda")
+        y = layer.prefill(inp.x.cuda())
+        torch.cuda.synchronize()
+        assert gb.gdla_device_error() == 0
+        assert bool(torch.isfinite(y).all())
+        qq = to_np(ws_view(layer._ws, layer.cfg, 1, T, 0, WS_QQ, torch.float16, (T, nH * shape.d_qk)))
+        kv = to_np(ws_view(layer._ws, layer.cfg, 1, T, 0, WS_KV, torch.float16, (T, shape.n_kv_heads, 256)))
+        amax = max(np.abs(qq).max(), np.abs(kv).max())
+        assert gain / 2 < amax < 65504.0, (gain, amax)
+        if gain == 2.0:
+            cfg = O.OracleConfig.from_shape(shape)
+            _, parts = O.gdla_prefill(inp.x, inp.weights, cfg, g_q=gq, g_kv=gkv, return_parts=True)
+            dg = to_np(ws_view(layer._ws, layer.cfg, 1, T, 0, WS_DG, torch.bfloat16, (T, 64, 128)))
+            # V (hence D and Dg) grows with the KV gain: the absolute bound scales with it
+            check("Dg with gains x2 vs the oracle with the same gains", dg, parts[0]["Dg"], mabs=MAX_ABS * gain)
 
 
 def test_fp16_operand_overflow_is_reported(cuda_ok):
