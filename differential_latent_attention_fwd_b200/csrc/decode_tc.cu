@@ -40,6 +40,13 @@
 // then rescaled), which is exact after the final division.  Rows of the last tile beyond the
 // row's last key are zeroed in shared memory before the PV, so that a cache tail the caller
 // never wrote (NaN, Inf) cannot reach the output through 0 * NaN.
+//
+// MXFP8 cache (template C8, rows of gdla_fp8.cuh): the producer loads a tile's rope codes and
+// block scales first, then its latent codes into the upper half of each ring slot; four more
+// warps (6-9, two threads per row) convert E4M3 x 2^k to fp16 in place, in the layout of the
+// bf16 tiles, and zero the rows outside the key range; q~, P and the tiles are fp16 MMA
+// operands.  The conversion adds to the per-tile chain above (slot freed -> codes loaded ->
+// converted -> scores), so the half-size cache is not faster than the bf16 one.
 #include "gdla_common.cuh"
 #include "gdla_decode.h"
 #include "gdla_fp8.cuh"
