@@ -63,16 +63,20 @@ int launch_copy_cols(const void* src, long long ld_src, void* dst, long long ld_
 // q~ rows: qt[b][h][0..511] = W_UK_j q^C_h, qt[b][h][512..575] = rotated q^R_h (bf16), on the
 // tensor cores.  Per KV head j the rows (b, h) of its five heads form one product
 //   [5 B x 128] (q^C, fp16) x [128 x 512] (W_UK_j^T, fp16) -> fp32 in TMEM,
-// one CTA per (j, 128 rows): the q^C rows are converted to fp16 by the CTA's threads into a
-// 128-byte-swizzled K-major tile, W_UK_j^T (128 KB) arrives by TMA as eight [128][64] MN-major
-// boxes, and two tcgen05.mma chains (M 128, N 256, K 128) fill 512 TMEM columns, which the
-// four warps (thread = row) round to bf16.  Rows of the group: r = 5 b + hh, hh = 0 the noise
-// head n_signal + j, hh = 1..4 the signal heads 4 j + hh - 1.
+// one CTA per (j, 128 rows, 128 of the 512 columns), so that a decode batch fills the SMs (three
+// CTAs fit on one): the q^C rows are converted to fp16 by the CTA's threads into a
+// 128-byte-swizzled K-major tile, the CTA's quarter of W_UK_j^T (32 KB) arrives by TMA as two
+// [128][64] MN-major boxes, and one tcgen05.mma chain (M 128, N 128, K 128) fills 128 TMEM
+// columns; while it runs the CTA copies its share of the rotated q^R rows.  The four warps
+// (thread = row) round the result to bf16 into shared memory, from where whole 256-byte row
+// pieces go out coalesced.  Rows of the group: r = 5 b + hh, hh = 0 the noise head n_signal + j,
+// hh = 1..4 the signal heads 4 j + hh - 1.
 namespace qtc {
+constexpr int NQ = 4;                         // column quarters of q~ (one CTA each)
 constexpr int A_BOX = 128 * 128;              // [128 rows][64 fp16]
 constexpr int B_BOX = 128 * 128;              // [128 K rows][64 N fp16]
 constexpr int A_OFF = 0, B_OFF = 2 * A_BOX;
-constexpr int BAR_OFF = B_OFF + 8 * B_BOX;
+constexpr int BAR_OFF = B_OFF + 2 * B_BOX;
 constexpr int SMEM = BAR_OFF + 64 + 1024;
 }  // namespace qtc
 
@@ -80,7 +84,7 @@ __device__ __forceinline__ int qt_head(int hh, int j, int n_signal) {
   return hh == 0 ? n_signal + j : 4 * j + hh - 1;
 }
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 3)
     qtilde_tc_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ DecQParams p, KernelCtl ctl) {
   using namespace qtc;
   extern __shared__ uint8_t qt_raw[];
@@ -88,47 +92,26 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* bar_w = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* bar_mma = bar_w + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_w + 2);
-  const int j = blockIdx.x, t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int j = blockIdx.x, nq = blockIdx.z, t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int R = 5 * p.B;
-  const int gr = blockIdx.y * 128 + t;          // this thread's row of the group
-  const bool rv = gr < R;
-  const int b = gr / 5, h = qt_head(gr % 5, j, p.n_signal);
+  const int tile0 = blockIdx.y * 128;           // first group row of the tile
 
   if (t == 0) {
     mbar_init(bar_w, 1);
     mbar_init(bar_mma, 1);
     fence_mbar_init();
     tma_prefetch_desc(&mapW);
-    mbar_expect_tx(bar_w, 8 * B_BOX);
+    mbar_expect_tx(bar_w, 2 * B_BOX);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) tma_load_2d(smem + B_OFF + c * B_BOX, &mapW, bar_w, 64 * c, j * 128);
+    for (int c = 0; c < 2; ++c) tma_load_2d(smem + B_OFF + c * B_BOX, &mapW, bar_w, 64 * (2 * nq + c), j * 128);
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, 128);
     tmem_relinquish();
   }
-  // ---- rows of warp w: 32 w .. 32 w + 31 of the tile.  First the rotated q^R of each row
-  // (bf16) straight into q~ columns 512..575: lane l of load k serves row 2 k + l / 16, float4
-  // l % 16; then the q^C rows, one row per load (lane l: float4 l), as fp16 into the
-  // 128-byte-swizzled K-major A tile (8 values = 16 bytes per chunk, two lanes per chunk)
-  const int row0 = blockIdx.y * 128 + 32 * warp;
-  {
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-      const int rr = row0 + 2 * k + (lane >> 4);
-      if (rr < R) {
-        const int bb = rr / 5, hr = qt_head(rr % 5, j, p.n_signal);
-        const float4 a = *reinterpret_cast<const float4*>(p.QQ + (long long)bb * p.qq_ld + p.rope_col0 +
-                                                          (long long)hr * 64 + 4 * (lane & 15));
-        bool bad_r = false;
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.qt) + ((long long)bb * p.n_heads + hr) * 576 + 512 +
-                                  4 * (lane & 15)) =
-            p.qt_f16 ? make_uint2(pack_half2_sat(a.x, a.y, bad_r), pack_half2_sat(a.z, a.w, bad_r))
-                     : make_uint2(pack_bf162(a.x, a.y), pack_bf162(a.z, a.w));
-        if (bad_r && ctl.err) atomicCAS(ctl.err, 0, SITE_FP16_RANGE);
-      }
-    }
-  }
+  // ---- A: the q^C rows of warp w (32 w .. 32 w + 31 of the tile), one row per load (lane l:
+  // float4 l), as fp16 into the 128-byte-swizzled K-major tile (two lanes per 16-byte chunk)
+  const int row0 = tile0 + 32 * warp;
   bool bad = false;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
@@ -151,65 +134,95 @@ __global__ void __launch_bounds__(128, 1)
     }
   }
   if (bad && ctl.err) atomicCAS(ctl.err, 0, SITE_FP16_RANGE);
+  bad = false;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  bool ok = true;
+  bool ok = true, issued = false;
   if (t == 0) {
     ok = mbar_wait(bar_w, 0, ctl, SITE_DEC_MMA);
     if (ok) {
       tc_fence_after();
-      constexpr uint32_t idesc = make_idesc(128, 256, 0, 0, 1);
+      issued = true;
+      constexpr uint32_t idesc = make_idesc(128, 128, 0, 0, 1);
       const uint64_t da = sdesc_sw128(smem_u32(smem + A_OFF), 16, 1024);
       const uint64_t db = sdesc_sw128(smem_u32(smem + B_OFF), B_BOX, 1024);
 #pragma unroll
-      for (int nh = 0; nh < 2; ++nh)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + 256 * nh, da + uint64_t((kk >> 2) * (A_BOX >> 4) + (kk & 3) * 2),
-                 db + uint64_t(nh * 4 * (B_BOX >> 4) + kk * 128), idesc, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss(tmem, da + uint64_t((kk >> 2) * (A_BOX >> 4) + (kk & 3) * 2), db + uint64_t(kk * 128), idesc,
+               kk > 0 ? 1u : 0u);
       mma_commit(bar_mma);
+    }
+  }
+  // ---- while the MMAs run: the rotated q^R of rows 32 nq .. 32 nq + 31 of the tile (bf16, or
+  // fp16 for the MXFP8 decode) straight into q~ columns 512..575, 16 lanes per row
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = 128 * i + t, rr = tile0 + 32 * nq + (idx >> 4), c4 = idx & 15;
+    if (rr < R) {
+      const int bb = rr / 5, hr = qt_head(rr % 5, j, p.n_signal);
+      const float4 a = *reinterpret_cast<const float4*>(p.QQ + (long long)bb * p.qq_ld + p.rope_col0 +
+                                                        (long long)hr * 64 + 4 * c4);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.qt) + ((long long)bb * p.n_heads + hr) * 576 + 512 +
+                                4 * c4) =
+          p.qt_f16 ? make_uint2(pack_half2_sat(a.x, a.y, bad), pack_half2_sat(a.z, a.w, bad))
+                   : make_uint2(pack_bf162(a.x, a.y), pack_bf162(a.z, a.w));
     }
   }
   ok = __syncthreads_and(ok);
   if (ok) {
-    // ---- epilogue: thread t = TMEM lane t = row gr
+    // ---- epilogue: thread t = TMEM lane t = tile row t; its 128 values are rounded into the
+    // (now free) A region as one 256-byte row, 16-byte chunk k at position k ^ (t & 15)
     const bool w = __all_sync(0xffffffffu, mbar_wait(bar_mma, 0, ctl, SITE_DEC_MMA));
     tc_fence_after();
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.qt) + ((long long)b * p.n_heads + h) * 576;
     const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    auto pk = [&](float a, float b) { return p.qt_f16 ? pack_half2_sat(a, b, bad) : pack_bf162(a, b); };
     if (w) {
-#pragma unroll 1
-      for (int c = 0; c < 16; ++c) {
-        uint32_t v[32];
-        GDLA_TMEM_LD32(tmem + 32 * c + lane_off, v);
-        tmem_ld_wait();
-        if (!rv) continue;
-        // bf16 q~, or fp16 (saturated, reported) for the fp16 MMAs over an MXFP8 cache
-        auto pk = [&](float a, float b) { return p.qt_f16 ? pack_half2_sat(a, b, bad) : pack_bf162(a, b); };
 #pragma unroll
-        for (int e = 0; e < 32; e += 8)
-          *reinterpret_cast<uint4*>(dst + 32 * c + e) =
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[64];
+        GDLA_TMEM_LD32(tmem + 64 * c + lane_off, v);
+        GDLA_TMEM_LD32(tmem + 64 * c + 32 + lane_off, (v + 32));
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 64; e += 8) {
+          const int k = (64 * c + e) >> 3;
+          *reinterpret_cast<uint4*>(smem + A_OFF + t * 256 + ((k ^ (t & 15)) << 4)) =
               make_uint4(pk(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
                          pk(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
                          pk(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
                          pk(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
+        }
       }
-      if (bad && ctl.err) atomicCAS(ctl.err, 0, SITE_FP16_RANGE);
+    }
+    ok = __syncthreads_and(w);
+    if (ok) {
+      // 16 lanes per row piece: columns 128 nq .. 128 nq + 127 of q~ row (b, h)
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int idx = 128 * i + t, r = idx >> 4, k = idx & 15, gr = tile0 + r;
+        if (gr < R) {
+          const int b = gr / 5, h = qt_head(gr % 5, j, p.n_signal);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.qt) + ((long long)b * p.n_heads + h) * 576 +
+                                    128 * nq + 8 * k) =
+              *reinterpret_cast<const uint4*>(smem + A_OFF + r * 256 + ((k ^ (r & 15)) << 4));
+        }
+      }
     }
   }
+  if (bad && ctl.err) atomicCAS(ctl.err, 0, SITE_FP16_RANGE);
   if (t == 0) {
     // before TMEM is released: the MMAs (if issued) are complete, the weight copy has landed
-    if (ok) mbar_drain(bar_mma, 0, ctl.err);
+    if (issued) mbar_drain(bar_mma, 0, ctl.err);
     else mbar_drain(bar_w, 0, ctl.err);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 128);
   }
 }
 
@@ -221,7 +234,7 @@ int launch_qtilde(const DecQParams& p, KernelCtlHost ctl, cudaStream_t st) {
   if (cudaFuncSetAttribute(qtilde_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qtc::SMEM) != cudaSuccess)
     return -4;
   KernelCtl kc{ctl.err, ctl.limit_ns};
-  qtilde_tc_kernel<<<dim3(p.n_groups, (5 * p.B + 127) / 128), 128, qtc::SMEM, st>>>(mw, p, kc);
+  qtilde_tc_kernel<<<dim3(p.n_groups, (5 * p.B + 127) / 128, qtc::NQ), 128, qtc::SMEM, st>>>(mw, p, kc);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 

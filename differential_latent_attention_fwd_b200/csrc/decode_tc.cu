@@ -81,6 +81,14 @@ constexpr int LAT_RAW = LAT_SLOT / 2;
 constexpr int ROPE_RAW = 2048;
 constexpr int SMEM8 = SMEM;
 constexpr int C8_WARPS = 4;
+// The MMA issuer is one thread whose issue rate bounds the kernel (52 MMAs a tile).  A warp
+// shares its scheduler with the warps of the same index mod 4; softmax warp 3 serves TMEM lanes
+// 96..127, beyond the 80 heads, and is nearly idle, so the bf16 kernel puts the issuer on warp 7
+// (warps 5 and 6 idle, 256 threads).  The MXFP8 kernel keeps it on warp 5 beside its converters.
+template <bool C8>
+constexpr int mma_warp() { return C8 ? 5 : 7; }
+template <bool C8>
+constexpr int block_threads() { return C8 ? 192 + 32 * C8_WARPS : 256; }
 // The M = 128 score MMA reads 128 rows of each 80-row q~ box: the 48 rows past a box are the
 // next box, or (for the last box) the first 6 KB of P.  They only feed unused score rows.
 static_assert(P_OFF + 48 * 128 <= LAT_OFF, "q~ box over-read stays in the P buffer");
@@ -160,7 +168,7 @@ static_assert(sizeof(SkBars) <= 1024, "barrier block");
 // scales); 128 more threads (warps 6-9) convert them, and q~, P and the cache tiles are fp16 MMA
 // operands instead of bf16.
 template <bool C8>
-__global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
+__global__ void __launch_bounds__(dsk::block_threads<C8>(), 1)
     dec_attn_sk_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapC,
                        const __grid_constant__ CUtensorMap mapR, const __grid_constant__ DecAttnParams p,
                        KernelCtl ctl) {
@@ -195,7 +203,7 @@ __global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
     tma_prefetch_desc(&mapC);
     if (C8) tma_prefetch_desc(&mapR);
   }
-  if (warp == 5) {
+  if (warp == mma_warp<C8>()) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -299,7 +307,7 @@ __global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
           mbar_drain(C8 ? &bars->rope_raw[s] : &bars->rope_full[s], (rope_par >> s) & 1, ctl.err);
       if (q_issued) mbar_drain(&bars->q_ready, (seg - 1) & 1, ctl.err);
     }
-  } else if (warp == 5) {
+  } else if (warp == mma_warp<C8>()) {
     if (lane == 0) {
       // ============================================================ MMA issuer
       // Descriptors as (low, high) words; offsets below are in 16-byte units of the low word.
@@ -500,7 +508,7 @@ __global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
       }
     }
     if (fp16_bad && p.err) atomicCAS(p.err, 0, SITE_FP16_RANGE);
-  } else {
+  } else if (warp < 4) {
     // ============================================================ softmax / epilogue (warps 0-3)
     const int q = warp;                      // TMEM lane quarter
     const int h = 32 * q + lane;             // head of this thread (h < 80), latent row in O^T
@@ -692,7 +700,7 @@ __global__ void __launch_bounds__(C8 ? 192 + 32 * dsk::C8_WARPS : 192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == mma_warp<C8>()) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -782,12 +790,12 @@ int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t s
     if (cudaFuncSetAttribute(dec_attn_sk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsk::SMEM8) != cudaSuccess)
       return -4;
-    dec_attn_sk_kernel<true><<<p.n_ctas, 192 + 32 * dsk::C8_WARPS, dsk::SMEM8, st>>>(mq, mc, mr, p, kc);
+    dec_attn_sk_kernel<true><<<p.n_ctas, dsk::block_threads<true>(), dsk::SMEM8, st>>>(mq, mc, mr, p, kc);
   } else {
     if (cudaFuncSetAttribute(dec_attn_sk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsk::SMEM) != cudaSuccess)
       return -4;
-    dec_attn_sk_kernel<false><<<p.n_ctas, 192, dsk::SMEM, st>>>(mq, mc, mr, p, kc);
+    dec_attn_sk_kernel<false><<<p.n_ctas, dsk::block_threads<false>(), dsk::SMEM, st>>>(mq, mc, mr, p, kc);
   }
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
