@@ -883,7 +883,7 @@ static int decode_impl(const gdla_config_t* cfg, const gdla_absorbed_t* ab, cons
   cp.q_len = q_len; cp.n_seq = n_seq;
   cp.tstart = dp.tstart;
   cp.part = part; cp.ml = ml; cp.lam = lam; cp.G = QQ + nqq; cp.g_ld = ldq; cp.W_bKV = w->W_bKV; cp.Dg = Dg;
-  if (launch_failed(launch_dec_combine(cp, st))) return GDLA_ERR_LAUNCH;
+  if (launch_failed(launch_dec_combine(cp, ctl, st))) return GDLA_ERR_LAUNCH;
 
   stage(3, st);
   GemmEpi eo{};

@@ -240,31 +240,70 @@ int launch_qtilde(const DecQParams& p, KernelCtlHost ctl, cudaStream_t st) {
 
 // ---------------------------------------------------------------- segment merge + combine + gate
 // CTA (KV group j, CB query rows b): while W_UV_j (the V column block of W_b^KV for KV head j,
-// 512 x 128 bf16) streams into shared memory, the key-range segments of the group's 5 heads are
-// merged (each segment's partial rescaled by 2^(m_seg - m), then normalised) and the latent
-// differentials l_s - lambda_s l_noise of its 4 signal heads formed in shared memory (fp32);
-// then D = Dlat W_UV_j (4 CB rows x 128 columns, K = 512) and Dg = sigmoid(G) (.) D.
+// 512 x 128 bf16) arrives by TMA, the key-range segments of the group's 5 heads are merged (each
+// segment's partial rescaled by 2^(m_seg - m), then normalised) and the latent differentials
+// l_s - lambda_s l_noise of its 4 signal heads formed (fp32); then D = Dlat W_UV_j on the tensor
+// cores and Dg = sigmoid(G) (.) D.  The fp32 differentials enter the bf16 MMA as two bf16 parts,
+// hi = bf16(x) and lo = bf16(x - hi) (rows 4 b + s and 32 + 4 b + s of the A tile), whose
+// products are added in fp32, so the product keeps about 16 bits of the differential.
 // Row b's segments are the attention CTAs c_lo .. c_hi whose tile ranges meet the row's tiles
 // [tstart[l], tstart[l + 1]) at list position l of row b; CTA c wrote its piece to slot c + l.
 constexpr int CB = 8;
 constexpr int MAXSEG = DEC_MAX_CTAS;
-__global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
+namespace dcb {
+constexpr int A_CHUNK = 64 * 128;                  // [64 rows][64 bf16], 128-byte swizzle
+constexpr int A_OFF = 0;                           // 8 chunks: K = 512
+constexpr int B_OFF = 8 * A_CHUNK;                 // [2 N chunks][512 K rows][64 bf16]
+constexpr int B_NCHUNK = 512 * 128;
+constexpr int SCR_OFF = B_OFF + 2 * B_NCHUNK;
+constexpr int SMEM = SCR_OFF + 5 * CB * MAXSEG * 4 + 5 * CB * 4 + 2 * CB * 4 + 64 + 1024;
+// the M = 128 MMA reads 128 rows of each 64-row A chunk: rows 64..127 are the next chunk (the
+// last chunk's: the first 8 KB of W_UV), which only feed TMEM lanes the epilogue never reads
+static_assert(B_OFF + A_CHUNK <= SCR_OFF, "A over-read stays in shared memory");
+}  // namespace dcb
+
+__global__ void __launch_bounds__(256, 1)
+    dec_combine_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ DecCombParams p,
+                       KernelCtl ctl) {
+  using namespace dcb;
   constexpr int NH = 80;
-  extern __shared__ uint8_t cb_smem[];
-  __nv_bfloat16* wsm = reinterpret_cast<__nv_bfloat16*>(cb_smem);                  // [512][128]
-  float (*dl)[512] = reinterpret_cast<float (*)[512]>(cb_smem + 512 * 128 * 2);     // [4 CB][512]
-  float (*wsp)[MAXSEG] = reinterpret_cast<float (*)[MAXSEG]>(cb_smem + 512 * 128 * 2 + 4 * CB * 512 * 4);
-  float* inv_L = reinterpret_cast<float*>(cb_smem + 512 * 128 * 2 + 4 * CB * 512 * 4 + 5 * CB * MAXSEG * 4);
+  extern __shared__ uint8_t cb_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(cb_raw) + 1023) & ~uintptr_t(1023));
+  float (*wsp)[MAXSEG] = reinterpret_cast<float (*)[MAXSEG]>(smem + SCR_OFF);
+  float* inv_L = reinterpret_cast<float*>(smem + SCR_OFF + 5 * CB * MAXSEG * 4);
   int* seg_lo = reinterpret_cast<int*>(inv_L + 5 * CB);
   int* seg_n = seg_lo + CB;
-  const int j = blockIdx.x, b0 = blockIdx.y * CB, tid = threadIdx.x;
+  uint64_t* bar_w = reinterpret_cast<uint64_t*>(seg_n + CB);
+  uint64_t* bar_mma = bar_w + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_w + 2);
+  const int j = blockIdx.x, b0 = blockIdx.y * CB, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nb = min(CB, p.B - b0);
-  const long long ldw = (long long)p.n_groups * 256;
-  const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(p.W_bKV) + j * 256 + 128;
-  for (int i = tid; i < 512 * 16; i += blockDim.x) {          // 16 x 16 bytes per 128-column row
-    const int l = i >> 4, q = i & 15;
-    cp_async16(wsm + l * 128 + q * 8, W + l * ldw + q * 8);
+  if (tid == 0) {
+    mbar_init(bar_w, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&mapW);
+    // W_UV_j = columns j 256 + 128 .. j 256 + 255 of W_b^KV: N chunk c, K half kh
+    mbar_expect_tx(bar_w, 2 * B_NCHUNK);
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int kh = 0; kh < 2; ++kh)
+        tma_load_2d(smem + B_OFF + c * B_NCHUNK + kh * (B_NCHUNK / 2), &mapW, bar_w, j * 256 + 128 + 64 * c, 256 * kh);
   }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  // the lambdas of this thread's rows, loaded now and used after the merge
+  constexpr int RB = CB / 2;
+  const int cq = tid & 127, rb = (tid >> 7) * RB;
+  float lamv[RB][4];
+#pragma unroll
+  for (int k = 0; k < RB; ++k)
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      lamv[k][s] = rb + k < nb ? p.lam[(long long)(b0 + rb + k) * p.n_signal + 4 * j + s] : 0.f;
   if (tid < CB) {
     int lo = 0, n = 0;
     if (tid < nb) {
@@ -287,13 +326,29 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
   if (tid < 5 * CB) {
     const int bb = tid / 5, h = heads[tid % 5];
     const int n = seg_n[bb], lo = seg_lo[bb];
+    // (m, l) of the segments, four loads in flight at a time
     float M = -INFINITY, Ls = 0.f;
-    for (int k = 0; k < n; ++k) M = fmaxf(M, p.ml[((long long)(lo + k) * NH + h) * 2]);
-    for (int k = 0; k < n; ++k) {
-      const float* ml = p.ml + ((long long)(lo + k) * NH + h) * 2;
-      const float w = ml[1] > 0.f ? ex2_approx(ml[0] - M) : 0.f;
-      wsp[tid][k] = w;
-      Ls += w * ml[1];
+    for (int k0 = 0; k0 < n; k0 += 4) {
+      float2 v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v[k] = k0 + k < n ? *reinterpret_cast<const float2*>(p.ml + ((long long)(lo + k0 + k) * NH + h) * 2)
+                          : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) M = fmaxf(M, v[k].x);
+    }
+    for (int k0 = 0; k0 < n; k0 += 4) {
+      float2 v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v[k] = k0 + k < n ? *reinterpret_cast<const float2*>(p.ml + ((long long)(lo + k0 + k) * NH + h) * 2)
+                          : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float w = v[k].y > 0.f ? ex2_approx(v[k].x - M) : 0.f;
+        if (k0 + k < n) wsp[tid][k0 + k] = w;
+        Ls += w * v[k].y;
+      }
     }
     inv_L[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
   }
@@ -302,8 +357,6 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
     // thread: latent columns 4 cq .. 4 cq + 3 of rows rb .. rb + CB / 2 - 1; segments outermost
     // so that a segment's 5 CB / 2 float4 loads are independent (rows with fewer segments load
     // nothing for the rest)
-    constexpr int RB = CB / 2;
-    const int cq = tid & 127, rb = (tid >> 7) * RB;
     int max_n = 0;
 #pragma unroll
     for (int k = 0; k < RB; ++k) max_n = max(max_n, seg_n[rb + k]);
@@ -337,82 +390,133 @@ __global__ void __launch_bounds__(256) dec_combine_kernel(DecCombParams p) {
           }
         }
     }
+    // differentials -> A tile: row 4 bb + s (hi part) and 32 + 4 bb + s (lo part), columns
+    // 4 cq .. 4 cq + 3 (8 bytes in the 16-byte unit (cq % 16) / 2 of K chunk cq / 16)
+    const int kc = cq >> 4, un = (cq & 15) >> 1, hb = 8 * (cq & 1);
 #pragma unroll
     for (int k = 0; k < RB; ++k) {
       const int bb = rb + k;
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
-        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
         if (bb < nb) {
-          const float lam = p.lam[(long long)(b0 + bb) * p.n_signal + 4 * j + s];
+          const float lam = lamv[k][s];
           const float iS = inv_L[5 * bb + 1 + s], iN = inv_L[5 * bb];
-          o.x = m4[k][1 + s].x * iS - lam * (m4[k][0].x * iN);
-          o.y = m4[k][1 + s].y * iS - lam * (m4[k][0].y * iN);
-          o.z = m4[k][1 + s].z * iS - lam * (m4[k][0].z * iN);
-          o.w = m4[k][1 + s].w * iS - lam * (m4[k][0].w * iN);
+          o[0] = m4[k][1 + s].x * iS - lam * (m4[k][0].x * iN);
+          o[1] = m4[k][1 + s].y * iS - lam * (m4[k][0].y * iN);
+          o[2] = m4[k][1 + s].z * iS - lam * (m4[k][0].z * iN);
+          o[3] = m4[k][1 + s].w * iS - lam * (m4[k][0].w * iN);
         }
-        *reinterpret_cast<float4*>(&dl[4 * bb + s][4 * cq]) = o;
+        uint32_t hi[2], lo[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          hi[e] = pack_bf162(o[2 * e], o[2 * e + 1]);
+          lo[e] = pack_bf162(o[2 * e] - __uint_as_float(hi[e] << 16),
+                             o[2 * e + 1] - __uint_as_float(hi[e] & 0xFFFF0000u));
+        }
+        const int r = 4 * bb + s;
+        *reinterpret_cast<uint2*>(smem + A_OFF + kc * A_CHUNK + r * 128 + ((un ^ (r & 7)) << 4) + hb) =
+            make_uint2(hi[0], hi[1]);
+        *reinterpret_cast<uint2*>(smem + A_OFF + kc * A_CHUNK + (r + 32) * 128 + ((un ^ (r & 7)) << 4) + hb) =
+            make_uint2(lo[0], lo[1]);
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // the gate logits of the CTA's 32 output rows, into the merge-weight area (free now): row
+  // r = 4 bb + s, 128 fp32; they land while the MMAs run
+  float* G_s = reinterpret_cast<float*>(smem + SCR_OFF);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = 256 * i + tid, r = idx >> 5, c4 = idx & 31, bb = r >> 2;
+    if (bb < nb)
+      cp_async16(G_s + r * 128 + 4 * c4, p.G + (long long)(b0 + bb) * p.g_ld + (4 * j + (r & 3)) * 128 + 4 * c4);
+  }
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true, issued = false;
+  if (tid == 0) {
+    ok = mbar_wait(bar_w, 0, ctl, SITE_DEC_MMA);
+    if (ok) {
+      tc_fence_after();
+      issued = true;
+      constexpr uint32_t idesc = make_idesc(128, 128, 1, 0, 1);
+      const uint64_t da = sdesc_sw128(smem_u32(smem + A_OFF), 16, 1024);
+      const uint64_t db = sdesc_sw128(smem_u32(smem + B_OFF), B_NCHUNK, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 32; ++kk)
+        mma_ss(tmem, da + uint64_t((kk >> 2) * (A_CHUNK >> 4) + (kk & 3) * 2), db + uint64_t(kk * 128), idesc,
+               kk > 0 ? 1u : 0u);
+      mma_commit(bar_mma);
+    }
+  }
+  ok = __syncthreads_and(ok);
+  // ---- epilogue.  Warp 0 holds the hi products (TMEM lanes 0..31 = rows 4 bb + s), warp 1 the
+  // lo products (lanes 32..63); both park them in the A tile (read by the completed MMAs) as
+  // [32 rows][32 float4], float4 c of row r at position c ^ r; then every thread finishes four
+  // float4 of the outputs, a warp per 256-byte output row.
+  float4* scr = reinterpret_cast<float4*>(smem + A_OFF);     // [2][32][32]
+  bool w = ok;
+  if (ok && warp < 2) {
+    w = __all_sync(0xffffffffu, mbar_wait(bar_mma, 0, ctl, SITE_DEC_MMA));
+    tc_fence_after();
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    if (w) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        GDLA_TMEM_LD32(tmem + 32 * c + lane_off, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          scr[(warp * 32 + lane) * 32 + ((8 * c + e) ^ lane)] =
+              make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
+                          __uint_as_float(v[4 * e + 3]));
       }
     }
   }
   cp_async_wait_all();
-  __syncthreads();
-  // D = Dlat W_UV_j: thread tile 2 rows x 8 columns (one 16-byte weight load and one broadcast
-  // 16-byte row load per 4 x 8 FMAs)
-  const int cg = tid & 15;          // columns 8 cg .. 8 cg + 7
-  const int r0 = (tid >> 4) * 2;    // rows r0, r0 + 1 of the 4 CB latent differentials
-  float acc[2][8];
+  w = __syncthreads_and(w);
+  if (w) {
 #pragma unroll
-  for (int r = 0; r < 2; ++r)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
-#pragma unroll 1
-  for (int l = 0; l < 512; l += 4) {
-    float w[4][8];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(wsm + (l + k) * 128 + 8 * cg);
-      const uint32_t u[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w[k][2 * e] = __uint_as_float(u[e] << 16);
-        w[k][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    for (int i = 0; i < 4; ++i) {
+      const int idx = 256 * i + tid, r = idx >> 5, c4 = idx & 31, bb = r >> 2;
+      if (bb < nb) {
+        const float4 hi = scr[r * 32 + (c4 ^ r)], lo = scr[(32 + r) * 32 + (c4 ^ r)];
+        const float4 g = *reinterpret_cast<const float4*>(G_s + r * 128 + 4 * c4);
+        const uint2 o = make_uint2(pack_bf162(sigmoidf_fast(g.x) * (hi.x + lo.x), sigmoidf_fast(g.y) * (hi.y + lo.y)),
+                                   pack_bf162(sigmoidf_fast(g.z) * (hi.z + lo.z), sigmoidf_fast(g.w) * (hi.w + lo.w)));
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.Dg) + (long long)(b0 + bb) * p.n_signal * 128 +
+                                  (4 * j + (r & 3)) * 128 + 4 * c4) = o;
       }
     }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const float4 d4 = *reinterpret_cast<const float4*>(&dl[r0 + r][l]);
-      const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int e = 0; e < 8; e += 2)       // packed f32x2 FMAs
-          ffma2vv(acc[r][e], acc[r][e + 1], w[k][e], w[k][e + 1], dv[k], dv[k], acc[r][e], acc[r][e + 1]);
-    }
   }
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int row = r0 + r;
-    if (row >= 4 * nb) continue;
-    const int b = b0 + row / 4, s = row % 4, sig = 4 * j + s;
-    const long long o = (long long)b * p.n_signal * 128 + sig * 128 + 8 * cg;
-    const float* gp = p.G + (long long)b * p.g_ld + sig * 128 + 8 * cg;
-    const float4 g0 = *reinterpret_cast<const float4*>(gp), g1 = *reinterpret_cast<const float4*>(gp + 4);
-    const float gf[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-    uint32_t out[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      out[e] = pack_bf162(sigmoidf_fast(gf[2 * e]) * acc[r][2 * e], sigmoidf_fast(gf[2 * e + 1]) * acc[r][2 * e + 1]);
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Dg) + o) = make_uint4(out[0], out[1], out[2], out[3]);
+  ok = w;
+  if (tid == 0) {
+    // before TMEM is released: the MMAs (if issued) are complete, the weight copy has landed
+    if (issued) mbar_drain(bar_mma, 0, ctl.err);
+    else mbar_drain(bar_w, 0, ctl.err);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 
-int launch_dec_combine(const DecCombParams& p, cudaStream_t st) {
+int launch_dec_combine(const DecCombParams& p, KernelCtlHost ctl, cudaStream_t st) {
   if (p.n_ctas > MAXSEG) return -1;
-  const int smem = 512 * 128 * 2 + 4 * CB * 512 * 4 + 5 * CB * MAXSEG * 4 + 5 * CB * 4 + 2 * CB * 4;
-  if (cudaFuncSetAttribute(dec_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  CUtensorMap mw;
+  if (make_tmap_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.W_bKV, (uint64_t)p.n_groups * 256, 512,
+                   (uint64_t)p.n_groups * 256 * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B))
+    return -3;
+  if (cudaFuncSetAttribute(dec_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dcb::SMEM) != cudaSuccess)
     return -4;
-  dec_combine_kernel<<<dim3(p.n_groups, (p.B + CB - 1) / CB), 256, smem, st>>>(p);
+  KernelCtl kc{ctl.err, ctl.limit_ns};
+  dec_combine_kernel<<<dim3(p.n_groups, (p.B + CB - 1) / CB), 256, dcb::SMEM, st>>>(mw, p, kc);
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -4;
 }
 

@@ -81,6 +81,6 @@ int launch_qtilde(const DecQParams& p, KernelCtlHost ctl, cudaStream_t st);
 int launch_dec_sched(const DecAttnParams& p, cudaStream_t st);
 int launch_dec_attn_tc(const DecAttnParams& p, KernelCtlHost ctl, cudaStream_t st);
 int decode_cta_count();
-int launch_dec_combine(const DecCombParams& p, cudaStream_t st);
+int launch_dec_combine(const DecCombParams& p, KernelCtlHost ctl, cudaStream_t st);
 
 }  // namespace gdla
