@@ -36,6 +36,7 @@ struct GemmEpi {
   // internal: set by launch_gemm for the split-K pass (raw fp32 partial tiles)
   float* partial_out;
   int kb_per_split;
+  int staged;            // internal: one-tile kernel drains through shared memory (coalesced stores)
   int* err;              // internal: device error word (fp16 outputs out of range are reported)
 };
 

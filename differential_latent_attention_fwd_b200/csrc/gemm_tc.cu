@@ -106,6 +106,93 @@ __device__ __forceinline__ void gemm_epilogue_row(uint32_t t_row, int row, int n
   }
 }
 
+// The same epilogue for a whole 128 x BN tile, staged through shared memory (the drained
+// operand ring): each thread rounds its accumulator row into a row of the staging tile (16-byte
+// pieces at position piece ^ (row % 8)), then the CTA stores whole output rows with
+// consecutive threads on consecutive 16-byte pieces.  Needs N % 64 == 0 and 16-byte aligned
+// output rows (checked by the launcher).  Called by all 128 threads.
+template <int BN>
+__device__ __forceinline__ void gemm_epilogue_staged(uint32_t tmem, int m0, int n0, bool ok, int split,
+                                                     const GemmEpi& ep, uint8_t* buf, const KernelCtl& ctl) {
+  const int t = threadIdx.x, warp = t >> 5;
+  const bool f32 = ep.partial_out != nullptr || ep.out_type == OUT_F32;
+  const int rowb = f32 ? BN * 4 : BN * 2;              // bytes of a staged row
+  const int row = m0 + t;
+  // an error raised before this epilogue (not its own fp16 overflow report below) stops the stores
+  const bool err_before = *reinterpret_cast<volatile int*>(ctl.err) != 0;
+  int pos = 0;
+  if (ep.rope_hi > ep.rope_lo && row < ep.M) {
+    const int dv = ep.pos_div > 1 ? ep.pos_div : 1;
+    pos = (ep.pos_ptr ? ep.pos_ptr[row / dv] + row % dv : ((row + ep.row_off) % ep.pos_T)) + ep.pos_off;
+  }
+  bool bad = false;
+  const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
+  uint8_t* my = buf + t * rowb;
+  const int sw = t & 7;
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    if (n0 + c0 >= ep.N) break;  // uniform
+    uint32_t r[64];
+    GDLA_TMEM_LD32(t_row + c0, r);
+    GDLA_TMEM_LD32(t_row + c0 + 32, (r + 32));
+    tmem_ld_wait();
+    float v[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+    const int col = n0 + c0;
+    if (!ep.partial_out && col >= ep.rope_lo && col < ep.rope_hi) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float cs, sn;
+        rope_cs(pos, ep.rope.inv_freq[i], &cs, &sn);
+        const float x1 = v[i], x2 = v[i + 32];
+        v[i] = x1 * cs - x2 * sn;
+        v[i + 32] = x2 * cs + x1 * sn;
+      }
+    }
+    if (f32) {
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        *reinterpret_cast<float4*>(my + 16 * ((c0 / 4 + q) ^ sw)) =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    } else {
+      uint32_t pk[32];
+      if (ep.out_type == OUT_BF16) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf162(v[2 * i], v[2 * i + 1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_half2_sat(v[2 * i], v[2 * i + 1], bad);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<uint4*>(my + 16 * ((c0 / 8 + q) ^ sw)) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    }
+  }
+  // only rows of the product report an fp16 overflow
+  if (bad && row < ep.M && ep.err) atomicCAS(ep.err, 0, SITE_FP16_RANGE);
+  if (__syncthreads_or(err_before) || !ok) return;
+  const int nrows = min(128, ep.M - m0);
+  const int ncols = min(BN, ep.N - n0);                 // a multiple of 64
+  const int ppr = ncols * (f32 ? 4 : 2) / 16;           // 16-byte pieces of an output row
+  uint8_t* base;
+  long long ld_bytes;
+  if (ep.partial_out) {
+    base = reinterpret_cast<uint8_t*>(ep.partial_out + ((long long)split * ep.M + m0) * ep.N + n0);
+    ld_bytes = (long long)ep.N * 4;
+  } else {
+    const int esz = f32 ? 4 : 2;
+    base = static_cast<uint8_t*>(ep.C) + ((long long)m0 * ep.ldc + n0) * esz;
+    ld_bytes = ep.ldc * esz;
+  }
+  for (int idx = t; idx < nrows * ppr; idx += 128) {
+    const int rr = idx / ppr, q = idx - rr * ppr;
+    *reinterpret_cast<uint4*>(base + rr * ld_bytes + 16 * q) =
+        *reinterpret_cast<const uint4*>(buf + rr * rowb + 16 * (q ^ (rr & 7)));
+  }
+}
+
 template <int BN, int STAGES, bool B_KMAJOR>
 __global__ void __launch_bounds__(128, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
@@ -196,9 +283,14 @@ __global__ void __launch_bounds__(128, 1)
   // ---------------- epilogue: thread = accumulator row
   const bool ok = mbar_wait(done, 0, ctl, SITE_GEMM_EPI) || mbar_drain(done, 0, ctl.err);
   tc_fence_after();
-  const int row = m0 + warp * 32 + lane;
-  const bool row_ok = ok && row < ep.M && *reinterpret_cast<volatile int*>(ctl.err) == 0;
-  gemm_epilogue_row<BN>(tmem + (uint32_t(warp * 32) << 16), row, n0, row_ok, int(blockIdx.z), ep);
+  if (ep.staged) {
+    // every MMA has completed, so every stage has landed and been read: the ring is free
+    gemm_epilogue_staged<BN>(tmem, m0, n0, ok, int(blockIdx.z), ep, smem, ctl);
+  } else {
+    const int row = m0 + warp * 32 + lane;
+    const bool row_ok = ok && row < ep.M && *reinterpret_cast<volatile int*>(ctl.err) == 0;
+    gemm_epilogue_row<BN>(tmem + (uint32_t(warp * 32) << 16), row, n0, row_ok, int(blockIdx.z), ep);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, BN);
@@ -500,6 +592,14 @@ int launch_gemm(const void* A, long long lda, const void* B, long long ldb, bool
       ep.kb_per_split = (nk + splits - 1) / splits;
       ep.partial_out = ep.splitk;
     }
+  }
+  {
+    // the staged epilogue of the one-tile kernel: whole 64-column chunks, 16-byte aligned rows
+    const bool f32 = ep.partial_out != nullptr || ep.out_type == OUT_F32;
+    const int esz = f32 ? 4 : 2;
+    const uintptr_t cb = ep.partial_out ? reinterpret_cast<uintptr_t>(ep.partial_out) : reinterpret_cast<uintptr_t>(ep.C);
+    const long long ldb_out = ep.partial_out ? (long long)N * 4 : ep.ldc * esz;
+    ep.staged = N % 64 == 0 && cb % 16 == 0 && ldb_out % 16 == 0;
   }
   CUtensorMap ma, mb;
   if (make_tmap_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, M, lda * 2, 64, 128,
