@@ -24,18 +24,18 @@
 // list is q_len nearly equal parts with the same tile positions, so CTAs c and c + G / q_len
 // reach the same cache tiles at about the same time and the later reads hit L2.
 //
-// Roles (192 threads): warps 0-3 softmax and O^T epilogue (warp w reads TMEM lanes 32 w ..
+// Roles (256 threads): warps 0-3 softmax and O^T epilogue (warp w reads TMEM lanes 32 w ..
 // 32 w + 31: thread = head h = 32 w + lane for h < 80, thread = latent row for O^T), warp 4 TMA
-// producer, warp 5 TMEM owner + MMA issuer.  The tensor core runs S(J), PV(J - 1), S(J + 1),
-// PV(J), ...: the softmax of tile J (read S, maximum, exponentials, P) overlaps PV(J - 1) and
-// S(J + 1), so the tensor core never waits for it.  The single S buffer is released as soon as
-// the softmax has read it into registers; the single P buffer is written once PV(J - 1) is done;
-// the ring holds tiles J - 1 and J plus one slot of J + 1.  The issuer steps through
-// precomputed descriptor words (rebuilding 64-bit descriptors per MMA had made the issue loop,
-// not the tensor core, the bound).  What bounds the kernel now: a tile's slots are held from its
-// S to its PV, about two tile periods in this order, so the ring's 2.25 tiles leave the loads of
-// tile J + 2 (issued as PV(J) frees tile J's slots) about one PV of lead against a load latency
-// of ~2300 cycles; the S MMAs of tile J + 2 wait for its last units.
+// producer, warp 7 TMEM owner + MMA issuer (warps 5, 6 idle; the MXFP8 form: warp 5 issues,
+// warps 6-9 convert).  The tensor core runs S(J), PV(J - 1), S(J + 1), PV(J), ...: the softmax
+// of tile J (read S, maximum, exponentials, P) overlaps PV(J - 1) and S(J + 1), so the tensor
+// core never waits for it.  The single S buffer is released as soon as the softmax has read it
+// into registers; the single P buffer is written once PV(J - 1) is done; the ring holds tiles
+// J - 1 and J plus one slot of J + 1.  The issuer steps through precomputed descriptor words
+// (rebuilding 64-bit descriptors per MMA had made the issue loop slower still).  What bounds the
+// kernel: the issue rate of that one thread, about 75 cycles per MMA here for the 52 MMAs of a
+// tile (36 score MMAs of N 64, 16 PV MMAs of N 80) plus the waits between them; traces show the
+// tile's units already landed when the issuer reaches them.
 // The running maximum m_h moves only when a score exceeds it by more than 2^8 (O^T and l_h are
 // then rescaled), which is exact after the final division.  Rows of the last tile beyond the
 // row's last key are zeroed in shared memory before the PV, so that a cache tail the caller
