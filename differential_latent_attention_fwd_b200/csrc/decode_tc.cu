@@ -87,6 +87,9 @@ constexpr int C8_WARPS = 4;
 // (warps 5 and 6 idle, 256 threads).  The MXFP8 kernel keeps it on warp 5 beside its converters.
 template <bool C8>
 constexpr int mma_warp() { return C8 ? 5 : 7; }
+// bf16 kernel: the PV MMAs have their own issuing thread (warp 6), so that the two chains (S on
+// warp 7, PV on warp 6) are issued in parallel; they touch disjoint TMEM columns and slots.
+constexpr int PV_WARP = 6;
 template <bool C8>
 constexpr int block_threads() { return C8 ? 192 + 32 * C8_WARPS : 256; }
 // The M = 128 score MMA reads 128 rows of each 80-row q~ box: the 48 rows past a box are the
@@ -196,8 +199,9 @@ __global__ void __launch_bounds__(dsk::block_threads<C8>(), 1)
     mbar_init(&bars->s_free, 4);           // one arrival per softmax warp: S read out of TMEM
     mbar_init(&bars->p_ready, 4);          // one arrival per softmax warp: P written
     mbar_init(&bars->pv_done, 1);
-    mbar_init(&bars->seg_done, 1);
-    mbar_init(&bars->mma_final, 1);
+    // (bf16: both issuing threads commit to these)
+    mbar_init(&bars->seg_done, C8 ? 1 : 2);
+    mbar_init(&bars->mma_final, C8 ? 1 : 2);
     fence_mbar_init();
     tma_prefetch_desc(&mapQ);
     tma_prefetch_desc(&mapC);
@@ -385,13 +389,49 @@ __global__ void __launch_bounds__(dsk::block_threads<C8>(), 1)
           rs = rs + 1 == NROPE ? 0 : rs + 1;
           ls += 4;
           if (ls >= NLAT) ls -= NLAT;
-          // ---- PV(J - 1) behind S(J): the softmax of tile J overlaps it
-          if (j > 0 && !issue_pv(J - 1, j == 1)) { ok = false; break; }
+          // ---- PV(J - 1) behind S(J): the softmax of tile J overlaps it (MXFP8 kernel; the
+          // bf16 kernel issues the PVs from their own thread)
+          if (C8 && j > 0 && !issue_pv(J - 1, j == 1)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!issue_pv(J - 1, sg.g1 - sg.g0 == 1)) { ok = false; break; }
+        if (C8 && !issue_pv(J - 1, sg.g1 - sg.g0 == 1)) { ok = false; break; }
         mma_commit(&bars->seg_done);
         ++seg;
+      }
+      mma_commit(&bars->mma_final);
+      mbar_drain(&bars->mma_final, 0, ctl.err);
+    }
+  } else if (!C8 && warp == PV_WARP) {
+    if (lane == 0) {
+      // ============================================================ PV issuer (bf16 kernel)
+      // PV(J): O^T += C(J)^T P^T as soon as the softmax has written P(J); the tile's slots are
+      // released block by block; the first PV of a segment starts O^T afresh
+      constexpr uint32_t idesc_o = make_idesc(128, NH, 1, 1, 0);
+      const uint32_t hi = uint32_t(sdesc_sw128(smem_u32(smem), 16, 1024) >> 32);
+      const uint32_t p_lo = uint32_t(sdesc_sw128(smem_u32(smem + P_OFF), 16, 1024));
+      const uint32_t latv_lo = uint32_t(sdesc_sw128(smem_u32(smem + LAT_OFF), LAT_SLOT / 2, 1024));  // MN-major
+      bool ok = true;
+      int J = 0;
+      while (ok && walk.next(p, &sg)) {
+        for (int j = 0; j < sg.g1 - sg.g0; ++j, ++J) {
+          if (!mbar_wait(&bars->p_ready, J & 1, ctl, SITE_DEC_MMA)) { ok = false; break; }
+          tc_fence_after();
+          int s0 = (4 * J) % NLAT;
+#pragma unroll
+          for (int mb = 0; mb < 4; ++mb) {
+            int s = s0 + mb;
+            if (s >= NLAT) s -= NLAT;
+            const uint32_t a = latv_lo + uint32_t(s) * (LAT_SLOT / 16);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss_w(tmem + O_COL + NH * mb, a + uint32_t(kk * 128), hi, p_lo + uint32_t(kk * 2), hi, idesc_o,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&bars->lat_empty[s]);
+          }
+          mma_commit(&bars->pv_done);
+        }
+        if (!ok) break;
+        mma_commit(&bars->seg_done);
       }
       mma_commit(&bars->mma_final);
       mbar_drain(&bars->mma_final, 0, ctl.err);
