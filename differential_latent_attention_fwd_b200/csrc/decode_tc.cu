@@ -26,16 +26,18 @@
 //
 // Roles (256 threads): warps 0-3 softmax and O^T epilogue (warp w reads TMEM lanes 32 w ..
 // 32 w + 31: thread = head h = 32 w + lane for h < 80, thread = latent row for O^T), warp 4 TMA
-// producer, warp 7 TMEM owner + MMA issuer (warps 5, 6 idle; the MXFP8 form: warp 5 issues,
-// warps 6-9 convert).  The tensor core runs S(J), PV(J - 1), S(J + 1), PV(J), ...: the softmax
-// of tile J (read S, maximum, exponentials, P) overlaps PV(J - 1) and S(J + 1), so the tensor
-// core never waits for it.  The single S buffer is released as soon as the softmax has read it
-// into registers; the single P buffer is written once PV(J - 1) is done; the ring holds tiles
-// J - 1 and J plus one slot of J + 1.  The issuer steps through precomputed descriptor words
+// producer, warp 7 TMEM owner + score (S) MMA issuer, warp 6 PV MMA issuer, warp 5 idle (the
+// MXFP8 form, 384 threads: warp 5 issues S, warp 11 PV, warps 6-9 convert).  Per tile J the
+// tensor core runs S(J) as its units land and PV(J) once the softmax has written P(J): the two
+// chains are issued by different threads, so the softmax of tile J overlaps PV(J - 1) and
+// S(J + 1).  The single S buffer is released as soon as the softmax has read it into
+// registers; the single P buffer is written once PV(J - 1) is done; the ring holds tiles J - 1
+// and J plus one slot of J + 1.  The issuers step through precomputed descriptor words
 // (rebuilding 64-bit descriptors per MMA had made the issue loop slower still).  What bounds the
-// kernel: the issue rate of that one thread, about 75 cycles per MMA here for the 52 MMAs of a
-// tile (36 score MMAs of N 64, 16 PV MMAs of N 80) plus the waits between them; traces show the
-// tile's units already landed when the issuer reaches them.
+// kernel: the issue rate of the issuing threads, about 75 cycles per MMA here (a tile takes 36
+// score MMAs of N 64 and 16 PV MMAs of N 80; one thread issuing all 52 was the bound before the
+// PV chain got its own thread); traces show the tile's units already landed when the issuer
+// reaches them.
 // The running maximum m_h moves only when a score exceeds it by more than 2^8 (O^T and l_h are
 // then rescaled), which is exact after the final division.  Rows of the last tile beyond the
 // row's last key are zeroed in shared memory before the PV, so that a cache tail the caller
@@ -81,17 +83,19 @@ constexpr int LAT_RAW = LAT_SLOT / 2;
 constexpr int ROPE_RAW = 2048;
 constexpr int SMEM8 = SMEM;
 constexpr int C8_WARPS = 4;
-// The MMA issuer is one thread whose issue rate bounds the kernel (52 MMAs a tile).  A warp
-// shares its scheduler with the warps of the same index mod 4; softmax warp 3 serves TMEM lanes
-// 96..127, beyond the 80 heads, and is nearly idle, so the bf16 kernel puts the issuer on warp 7
-// (warps 5 and 6 idle, 256 threads).  The MXFP8 kernel keeps it on warp 5 beside its converters.
+// The MMA issuing threads' issue rate bounds the kernel (52 MMAs a tile).  A warp shares its
+// scheduler with the warps of the same index mod 4; softmax warp 3 serves TMEM lanes 96..127,
+// beyond the 80 heads, and is nearly idle, so the bf16 kernel puts the score issuer on warp 7.
+// The MXFP8 kernel keeps it on warp 5 beside its converters.
 template <bool C8>
 constexpr int mma_warp() { return C8 ? 5 : 7; }
-// bf16 kernel: the PV MMAs have their own issuing thread (warp 6), so that the two chains (S on
-// warp 7, PV on warp 6) are issued in parallel; they touch disjoint TMEM columns and slots.
-constexpr int PV_WARP = 6;
+// The PV MMAs have their own issuing thread, so that the two chains (S, PV) are issued in
+// parallel; they touch disjoint TMEM columns and slots.  bf16: warp 6.  MXFP8: warp 11, on the
+// scheduler of the idle softmax warp 3 (warps 6-9 convert, warp 10 is idle).
 template <bool C8>
-constexpr int block_threads() { return C8 ? 192 + 32 * C8_WARPS : 256; }
+constexpr int pv_warp() { return C8 ? 11 : 6; }
+template <bool C8>
+constexpr int block_threads() { return C8 ? 384 : 256; }
 // The M = 128 score MMA reads 128 rows of each 80-row q~ box: the 48 rows past a box are the
 // next box, or (for the last box) the first 6 KB of P.  They only feed unused score rows.
 static_assert(P_OFF + 48 * 128 <= LAT_OFF, "q~ box over-read stays in the P buffer");
@@ -199,9 +203,9 @@ __global__ void __launch_bounds__(dsk::block_threads<C8>(), 1)
     mbar_init(&bars->s_free, 4);           // one arrival per softmax warp: S read out of TMEM
     mbar_init(&bars->p_ready, 4);          // one arrival per softmax warp: P written
     mbar_init(&bars->pv_done, 1);
-    // (bf16: both issuing threads commit to these)
-    mbar_init(&bars->seg_done, C8 ? 1 : 2);
-    mbar_init(&bars->mma_final, C8 ? 1 : 2);
+    // (both issuing threads commit to these)
+    mbar_init(&bars->seg_done, 2);
+    mbar_init(&bars->mma_final, 2);
     fence_mbar_init();
     tma_prefetch_desc(&mapQ);
     tma_prefetch_desc(&mapC);
@@ -313,41 +317,18 @@ __global__ void __launch_bounds__(dsk::block_threads<C8>(), 1)
     }
   } else if (warp == mma_warp<C8>()) {
     if (lane == 0) {
-      // ============================================================ MMA issuer
+      // ============================================================ score (S) issuer
       // Descriptors as (low, high) words; offsets below are in 16-byte units of the low word.
       constexpr uint32_t idesc_s = make_idesc(128, TP, C8 ? 0 : 1, 0, 0);    // fp16 (C8) or bf16
-      constexpr uint32_t idesc_o = make_idesc(128, NH, C8 ? 0 : 1, 1, 0);
       const uint32_t hi = uint32_t(sdesc_sw128(smem_u32(smem), 16, 1024) >> 32);
       const uint32_t qs_lo = uint32_t(sdesc_sw128(smem_u32(smem + QS_OFF), 16, 1024));
-      const uint32_t p_lo = uint32_t(sdesc_sw128(smem_u32(smem + P_OFF), 16, 1024));
       const uint32_t lat_lo = uint32_t(sdesc_sw128(smem_u32(smem + LAT_OFF), 16, 1024));        // K-major
-      const uint32_t latv_lo = uint32_t(sdesc_sw128(smem_u32(smem + LAT_OFF), LAT_SLOT / 2, 1024));  // MN-major
       const uint32_t rope_lo = uint32_t(sdesc_sw128(smem_u32(smem + ROPE_OFF), 16, 1024));
       const uint32_t tS = tmem + S_COL;
       bool ok = true;
       int J = 0, seg = 0;
       int ls = 0, rs = 0;                      // ring slot of the tile's first latent unit / its rope unit
       uint32_t lph = 0, rph = 0;               // parity of the next full-wait, per slot
-      // PV of the tile before: O^T += C(J)^T P^T once the softmax has written P (slots of the
-      // tile are released block by block)
-      auto issue_pv = [&](int Jp, bool first) -> bool {
-        if (!mbar_wait(&bars->p_ready, Jp & 1, ctl, SITE_DEC_MMA)) return false;
-        tc_fence_after();
-        int s0 = (4 * Jp) % NLAT;
-#pragma unroll
-        for (int mb = 0; mb < 4; ++mb) {
-          int s = s0 + mb;
-          if (s >= NLAT) s -= NLAT;
-          const uint32_t a = latv_lo + uint32_t(s) * (LAT_SLOT / 16);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss_w(tmem + O_COL + NH * mb, a + uint32_t(kk * 128), hi, p_lo + uint32_t(kk * 2), hi,
-                     idesc_o, (!first || kk > 0) ? 1u : 0u);
-          mma_commit(&bars->lat_empty[s]);
-        }
-        mma_commit(&bars->pv_done);
-        return true;
-      };
       while (ok && walk.next(p, &sg)) {
         if (!mbar_wait(&bars->q_ready, seg & 1, ctl, SITE_DEC_MMA)) { ok = false; break; }
         tc_fence_after();
@@ -389,24 +370,20 @@ __global__ void __launch_bounds__(dsk::block_threads<C8>(), 1)
           rs = rs + 1 == NROPE ? 0 : rs + 1;
           ls += 4;
           if (ls >= NLAT) ls -= NLAT;
-          // ---- PV(J - 1) behind S(J): the softmax of tile J overlaps it (MXFP8 kernel; the
-          // bf16 kernel issues the PVs from their own thread)
-          if (C8 && j > 0 && !issue_pv(J - 1, j == 1)) { ok = false; break; }
         }
         if (!ok) break;
-        if (C8 && !issue_pv(J - 1, sg.g1 - sg.g0 == 1)) { ok = false; break; }
         mma_commit(&bars->seg_done);
         ++seg;
       }
       mma_commit(&bars->mma_final);
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
-  } else if (!C8 && warp == PV_WARP) {
+  } else if (warp == pv_warp<C8>()) {
     if (lane == 0) {
-      // ============================================================ PV issuer (bf16 kernel)
+      // ============================================================ PV issuer
       // PV(J): O^T += C(J)^T P^T as soon as the softmax has written P(J); the tile's slots are
       // released block by block; the first PV of a segment starts O^T afresh
-      constexpr uint32_t idesc_o = make_idesc(128, NH, 1, 1, 0);
+      constexpr uint32_t idesc_o = make_idesc(128, NH, C8 ? 0 : 1, 1, 0);
       const uint32_t hi = uint32_t(sdesc_sw128(smem_u32(smem), 16, 1024) >> 32);
       const uint32_t p_lo = uint32_t(sdesc_sw128(smem_u32(smem + P_OFF), 16, 1024));
       const uint32_t latv_lo = uint32_t(sdesc_sw128(smem_u32(smem + LAT_OFF), LAT_SLOT / 2, 1024));  // MN-major
@@ -436,7 +413,7 @@ __global__ void __launch_bounds__(dsk::block_threads<C8>(), 1)
       mma_commit(&bars->mma_final);
       mbar_drain(&bars->mma_final, 0, ctl.err);
     }
-  } else if (C8 && warp >= 6) {
+  } else if (C8 && warp >= 6 && warp < 6 + C8_WARPS) {
     // ============================================================ MXFP8 converters (warps 6-9)
     // Two threads per row (half h of its codes).  Per tile: the rope box first (its bytes hold
     // the row's 18 block scales, which the threads keep for the latent units), then the four
