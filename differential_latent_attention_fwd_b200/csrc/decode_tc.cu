@@ -33,11 +33,10 @@
 // S(J + 1).  The single S buffer is released as soon as the softmax has read it into
 // registers; the single P buffer is written once PV(J - 1) is done; the ring holds tiles J - 1
 // and J plus one slot of J + 1.  The issuers step through precomputed descriptor words
-// (rebuilding 64-bit descriptors per MMA had made the issue loop slower still).  What bounds the
-// kernel: the issue rate of the issuing threads, about 75 cycles per MMA here (a tile takes 36
-// score MMAs of N 64 and 16 PV MMAs of N 80; one thread issuing all 52 was the bound before the
-// PV chain got its own thread); traces show the tile's units already landed when the issuer
-// reaches them.
+// (rebuilding 64-bit descriptors per MMA had made the issue loop slower still).  A tile takes 36
+// score MMAs of N 64 and 16 PV MMAs of N 80, about 75 cycles each to issue here; with one thread
+// issuing all 52 that issue rate was the bound (traces showed the tile's units already landed
+// when the issuer reached them), which is why the PV chain has its own thread.
 // The running maximum m_h moves only when a score exceeds it by more than 2^8 (O^T and l_h are
 // then rescaled), which is exact after the final division.  Rows of the last tile beyond the
 // row's last key are zeroed in shared memory before the PV, so that a cache tail the caller
